@@ -1,0 +1,162 @@
+/*
+ * kvq.h -- C ABI of the routed mixed-precision KV cache for NVIDIA B200 (sm_100a).
+ *
+ * The operations come from "TriRoute: Unified Learned Routing for Joint Adaptive
+ * Attention, Experts, and KV-Cache Allocation" (paper review page, section 3):
+ *   - Eq. 4 (KV-cache bit-width, asymmetric per-token group quantization): each
+ *     token's K and V are written at a width b in {2, 4, 8, 16}; for b < 16,
+ *     s = (max - min) / (2^b - 1), z = min, code = round((x - z) / s); b = 16 keeps
+ *     native fp16. The group is one (token, head) vector of head_dim values, and one b
+ *     covers a token's K and V (the equation quantizes the pair (k_t, v_t) together).
+ *   - Eq. 2 (attention resolution): each (token, head) query has a mode
+ *     skip -> 0, local-w -> attention over keys [t - w, t], full -> keys [0, t].
+ *   - Inference paragraph after Algorithm 1: skipped attention is never materialised
+ *     and each token's KV is stored at its chosen width.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor arguments are DEVICE pointers owned by the caller, except where marked
+ *     host. Element types: fp16 = IEEE binary16 (2 bytes), fp32 output.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) and never synchronize, except kvq_check().
+ *   - Return value: KVQ_OK, or a kvq_status code for errors detectable on the host
+ *     (null pointer, bad size, bad w, unsupported head_dim, CUDA launch failure); in that
+ *     case nothing was launched and kvq_last_error() describes the problem.
+ *   - Values that only the device sees (a bits entry outside {2,4,8,16}, a mode outside
+ *     {0,1,2}, a write that would exceed a sequence's capacity, cu_seqlens that are not
+ *     non-decreasing) never fault: the kernel skips the offending work, records the
+ *     error in the cache's device status word, and kvq_check() reports it.
+ *   - Calls that touch one cache must be ordered (same stream, or events); the cache
+ *     holds per-call scratch, so two calls on one cache that overlap on the GPU race.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *kvq_stream_t;
+
+/* Opaque cache handle; owned by the library (kvq_cache_create / kvq_cache_destroy). */
+typedef struct kvq_cache kvq_cache;
+
+typedef enum kvq_status {
+    KVQ_OK = 0,
+    KVQ_ERR_ARG = 1,          /* bad pointer, size, w or head_dim (host check) */
+    KVQ_ERR_BITS = 2,         /* a bits entry outside {2, 4, 8, 16} (device check) */
+    KVQ_ERR_MODE = 3,         /* a mode entry outside {0, 1, 2} (device check) */
+    KVQ_ERR_CAPACITY = 4,     /* a write past a sequence's capacity (device check) */
+    KVQ_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+    KVQ_ERR_DEVICE_CHECK = 6, /* any other device-side consistency check */
+    KVQ_ERR_NOMEM = 7         /* device allocation failed (create only) */
+} kvq_status;
+
+/* Query modes of Eq. 2. */
+enum { KVQ_MODE_SKIP = 0, KVQ_MODE_LOCAL = 1, KVQ_MODE_FULL = 2 };
+
+/*
+ * Create an empty cache for `batch` sequences of `heads` KV heads, head_dim in {64, 128}.
+ * capacity_tokens: HOST array [batch], the most tokens each sequence may ever hold
+ * (1 <= capacity <= 8388607). Device memory is allocated once here, at the worst case
+ * of b = 16 for every token (4 * head_dim bytes of records + 16 bytes of fp32 side
+ * entry + 4 bytes of record offset per (token, head)), plus the decode scheduler's work
+ * list and split-K partials. All lengths start at 0. `stream` orders the initialisation.
+ * On success *out receives the handle; on failure *out is NULL.
+ */
+int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
+                     const int64_t *capacity_tokens, kvq_stream_t stream);
+
+/* Free every device buffer of the cache (synchronizes the device first). NULL is a no-op. */
+int kvq_cache_destroy(kvq_cache *cache);
+
+/* Set every sequence's length to 0 and clear the device status word. */
+int kvq_cache_reset(kvq_cache *cache, kvq_stream_t stream);
+
+/*
+ * Roll sequences back: lengths is a DEVICE int32 array [batch]; sequence s keeps its
+ * first min(lengths[s], current length) tokens (a negative entry keeps the sequence
+ * unchanged). The dropped tokens' records are overwritten by later writes.
+ */
+int kvq_cache_truncate(kvq_cache *cache, const int32_t *lengths, kvq_stream_t stream);
+
+/* Copy the current lengths into a DEVICE int32 array [batch]. */
+int kvq_cache_lengths(const kvq_cache *cache, int32_t *lengths, kvq_stream_t stream);
+
+/*
+ * Quantize-on-write (Eq. 4): append n_tok tokens to the cache.
+ *   k, v:        fp16 [n_tok][heads][head_dim], tokens of sequence s are rows
+ *                cu_seqlens[s] .. cu_seqlens[s+1]-1 (ragged, packed).
+ *   bits:        uint8 [n_tok][heads], each in {2, 4, 8, 16}; one width covers the
+ *                token's K and V for that head.
+ *   cu_seqlens:  int32 [batch + 1], cu_seqlens[0] = 0, non-decreasing,
+ *                cu_seqlens[batch] = n_tok. Sequence s gets cu_seqlens[s+1]-cu_seqlens[s]
+ *                new tokens (possibly 0) appended after its current length.
+ *   n_tok:       host int, rows of k / v / bits (0 is a no-op).
+ * Per (token, head) and for each of K and V: mn/mx are the fp32 min/max of the
+ * head_dim values, s = fp32(mx - mn) / fp32(2^b - 1) (IEEE round-to-nearest-even),
+ * z = mn, code_i = rint(fp32(x_i - z) / s) clamped to [0, 2^b - 1], code 0 when s == 0.
+ * The codes are stored packed (code of channel c at bits [b*c, b*c + b) of the record
+ * part), (s, z) go to the fp32 side table; b = 16 stores the fp16 bits and side (1, 0).
+ * A sequence whose write would exceed its capacity is left unchanged (status
+ * KVQ_ERR_CAPACITY); a token-head with invalid bits rejects its sequence's write for
+ * that head (status KVQ_ERR_BITS).
+ */
+int kvq_write(const void *k, const void *v, const uint8_t *bits, const int32_t *cu_seqlens,
+              int64_t n_tok, kvq_cache *cache, kvq_stream_t stream);
+
+/*
+ * Routed causal prefill attention (Eq. 2) for tokens already written by kvq_write.
+ *   q:           fp16 [n_tok][heads][head_dim]; query i of sequence s (row
+ *                cu_seqlens[s] + i) sits at position t = len_s - n_s + i, where len_s is the
+ *                sequence's current length and n_s = cu_seqlens[s+1] - cu_seqlens[s]
+ *                (so: call kvq_write for the same tokens first).
+ *   modes:       uint8 [n_tok][heads], 0 skip, 1 local-w, 2 full.
+ *   w:           local window, >= 0; local reads keys max(0, t - w) .. t inclusive.
+ *   cu_seqlens:  int32 [batch + 1], as for kvq_write; n_tok host int.
+ *   out:         fp32 [n_tok][heads][head_dim]; skip rows are written as zeros.
+ * Logits are q . deq(k_j) / sqrt(head_dim); softmax over the mode's key set; the output
+ * is sum_j p_j deq(v_j), with deq = code * s + z (b = 16: the fp16 value).
+ */
+int routed_attn_prefill(const void *q, const kvq_cache *cache, const uint8_t *modes, int w,
+                        const int32_t *cu_seqlens, int64_t n_tok, float *out,
+                        kvq_stream_t stream);
+
+/*
+ * Routed decode attention (Eq. 2), one query per (sequence, head) at t = len_s - 1.
+ *   q:      fp16 [batch][heads][head_dim];  modes: uint8 [batch][heads];  w >= 0.
+ *   out:    fp32 [batch][heads][head_dim]; skip heads and empty sequences are zeros.
+ * Work is split over key chunks (split-K) by an on-device scheduler that drops skip
+ * heads and clamps local heads to their w + 1 keys, then merged by log-sum-exp.
+ */
+int routed_attn_decode(const void *q, const kvq_cache *cache, const uint8_t *modes, int w,
+                       float *out, kvq_stream_t stream);
+
+/*
+ * Read back stored records of one (sequence, head) for tokens first .. first+count-1
+ * (all below the current length; checked on the device).
+ *   k_codes, v_codes: uint16 [count][head_dim]: codes (b < 16) or raw fp16 bits (b = 16).
+ *   side:             fp32 [count][4] = (s_K, z_K, s_V, z_V).
+ *   bits:             uint8 [count].
+ * Any of the four may be NULL. Used to verify the stored bytes; not on the hot path.
+ */
+int kvq_cache_export(const kvq_cache *cache, int seq, int head, int64_t first, int64_t count,
+                     uint16_t *k_codes, uint16_t *v_codes, float *side, uint8_t *bits,
+                     kvq_stream_t stream);
+
+/*
+ * Synchronize `stream`, read the cache's device status word and clear it.
+ * Returns KVQ_OK or the first device-side error recorded since the last check.
+ */
+int kvq_check(kvq_cache *cache, kvq_stream_t stream);
+
+/* Text of the last host-side error on this thread ("" if none). */
+const char *kvq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */
