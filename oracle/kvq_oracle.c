@@ -79,8 +79,10 @@ int oracle_quantize(const uint16_t *x, int n, int b, uint16_t *codes, float *s_o
     }
     const unsigned top = (1u << b) - 1u;          /* 2^b - 1 */
     const float range = mx - mn;                  /* fp32, round to nearest even */
-    const float s = range / (float)top;           /* fp32 IEEE division */
-    const float z = mn;
+    /* "+ 0.0f" stores a zero as +0: min(x) and s are values, and -0 and +0 are one value
+       (which of the two a min scan meets first depends on the scan order) */
+    const float s = range / (float)top + 0.0f;    /* fp32 IEEE division */
+    const float z = mn + 0.0f;
     for (int i = 0; i < n; ++i) {
         unsigned c = 0;
         if (s != 0.0f) {

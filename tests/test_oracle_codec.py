@@ -144,3 +144,12 @@ def test_more_bits_never_worse_on_average():
 def test_rejects_bad_width():
     with pytest.raises(ValueError):
         oracle.quantize(np.zeros(8, np.float16), 3)
+
+
+def test_signed_zero_stored_as_plus_zero():
+    # -0 and +0 are one value; whichever the min scan meets first, z and s are stored as +0
+    for x in ([-0.0, 0.0, 0.0], [0.0, -0.0], [-0.0, -0.0], [-0.0, 1.0, 0.0]):
+        codes, s, z = oracle.quantize(np.array(x, np.float16), 4)
+        assert np.float32(z).view(np.uint32) == 0
+        if max(x) == 0.0:
+            assert np.float32(s).view(np.uint32) == 0 and np.all(codes == 0)
