@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the routed mixed-precision KV cache on B200.
+
+One step = one decode step of the 1.3B-like decode workload (batch 64, 16 heads,
+head_dim 128, 8192 cached tokens, w = 512): roll each sequence back to 8191 tokens,
+quantize-on-write the step's new token of every (sequence, head) (Eq. 4), then routed
+decode attention (Eq. 2: scheduler, split-K kernel, log-sum-exp combine) for the query at
+t = 8191. `value` = attended KV tokens per second (keys actually read; skip heads read
+none, local heads w + 1). The same line carries the HBM rate of the routed bytes, the
+roofline of the split-K kernel, the prefill workload (ragged prefill + write: TFLOP/s), an
+end-to-end figure through host buffers and the CPU oracle as a baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs the full workload on its own GPU (independent replicas, no
+collective on the data path; weak scaling); rank 0 prints the line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "decode attended-KV tokens/s & HBM GB/s (% of ~8 TB/s); prefill TFLOP/s"
+UNIT = "attended-KV tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples of one GPU while it runs."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            ident = str(device_index)
+        self.ident = ident
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        t0 = time.time()
+        while self.proc and time.time() - t0 < 5 and os.path.getsize(self.path) == 0:
+            time.sleep(0.05)
+
+    def mark(self):
+        return time.time()
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t_begin: float, t_end: float):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+                except Exception:
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        inside = [r for r in rows if t_begin - 1 <= r[0] <= t_end + 1] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ workload setup
+def decode_setup(wl, dev):
+    """Cache holding L - 1 tokens per sequence; the step's token, query and modes; the
+    exact keys and routed bytes one step reads."""
+    from mixed_precision_kv_write_b200 import kvq, synth
+    B, H, D, L, w = wl.batch, wl.heads, wl.head_dim, wl.seqlens[0], wl.w
+    cache = kvq.KVQCache(B, H, D, [L + 4] * B, device=dev)
+    q, modes = synth.decode_queries(wl, dev)
+    k_step = torch.empty((B, H, D), dtype=torch.float16, device=dev)
+    v_step = torch.empty_like(k_step)
+    b_step = torch.empty((B, H), dtype=torch.uint8, device=dev)
+    keys = 0
+    rec_bytes = 0
+    side_bytes = 0
+    idx = torch.arange(L, device=dev)
+    for s in range(B):
+        ks, vs, bs = synth.kv_sequence(wl, s, dev)
+        one = synth.cu_seqlens([L - 1 if i == s else 0 for i in range(B)], dev)
+        kvq.kvq_write(ks[:-1].contiguous(), vs[:-1].contiguous(), bs[:-1].contiguous(), one, cache)
+        k_step[s], v_step[s], b_step[s] = ks[-1], vs[-1], bs[-1]
+        m = modes[s].to(torch.int64)                                   # [H]
+        lo = torch.where(m == 1, torch.clamp(torch.tensor(L - 1 - w, device=dev), min=0),
+                         torch.zeros_like(m))
+        read = (idx[:, None] >= lo[None, :]) & (m[None, :] != 0)       # [L, H]
+        bf = bs.to(torch.int64)
+        keys += int(read.sum())
+        rec_bytes += int(((bf * D // 4) * read).sum())
+        side_bytes += int((16 * (bf < 16) * read).sum())
+        del ks, vs, bs
+    torch.cuda.synchronize(dev)
+    cache.check()
+    return dict(cache=cache, q=q, modes=modes, k_step=k_step, v_step=v_step, b_step=b_step,
+                cu_one=synth.cu_seqlens([1] * B, dev),
+                roll=torch.full((B,), L - 1, dtype=torch.int32, device=dev),
+                out=torch.empty((B, H, D), dtype=torch.float32, device=dev),
+                keys=keys, rec_bytes=rec_bytes, side_bytes=side_bytes,
+                q_bytes=B * H * D * 2, out_bytes=B * H * D * 4)
+
+
+def decode_step(st, w):
+    from mixed_precision_kv_write_b200 import kvq
+    c = st["cache"]
+    c.truncate(st["roll"])
+    kvq.kvq_write(st["k_step"], st["v_step"], st["b_step"], st["cu_one"], c)
+    kvq.routed_attn_decode(st["q"], c, st["modes"], w, out=st["out"])
+
+
+LAUNCHES_PER_DECODE_STEP = 6   # truncate, write scan, write quantize, sched, split-K, combine
+
+
+def prefill_measure(dev, reps=5, warm=2):
+    """Ragged prefill + quantize-on-write workload: lengths {1024, 3000, 8192, 5555},
+    16 heads, head_dim 128, w = 512."""
+    from mixed_precision_kv_write_b200 import kvq, synth
+    wl = synth.WORKLOADS["ragged_prefill"]
+    H, D = wl.heads, wl.head_dim
+    k, v, bits = synth.kv_tokens(wl, dev)
+    q, modes = synth.prefill_queries(wl, dev)
+    cu = synth.cu_seqlens(wl.seqlens, dev)
+    cache = kvq.KVQCache(wl.batch, H, D, list(wl.seqlens), device=dev)
+    out = torch.empty((wl.n_tok, H, D), dtype=torch.float32, device=dev)
+    # exact query-key pairs
+    pairs = 0
+    cul = synth.cu_seqlens(wl.seqlens).tolist()
+    for s in range(wl.batch):
+        L = wl.seqlens[s]
+        t = torch.arange(L, device=dev)[:, None]
+        m = modes[cul[s]:cul[s] + L].to(torch.int64)
+        n = torch.where(m == 2, t + 1, torch.where(m == 1, torch.clamp(t, max=wl.w) + 1, 0))
+        pairs += int(n.sum())
+    bf = bits.to(torch.int64)
+    write_bytes = wl.n_tok * H * D * 2 * 2 + int((bf * D // 4).sum()) + wl.n_tok * H * (16 + 4)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    tw, tp = [], []
+    for r in range(warm + reps):
+        flush.fill_(r & 255)
+        cache.reset()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        kvq.kvq_set_profile_events(e[0], e[1])
+        kvq.kvq_write(k, v, bits, cu, cache)
+        kvq.kvq_set_profile_events(e[2], e[3])
+        kvq.routed_attn_prefill(q, cache, modes, wl.w, cu, out=out)
+        kvq.kvq_set_profile_events(None, None)
+        stream.synchronize()
+        if r >= warm:
+            tw.append(e[0].elapsed_time(e[1]) * 1e-3)
+            tp.append(e[2].elapsed_time(e[3]) * 1e-3)
+    cache.check()
+    flops = 4.0 * D * pairs
+    t_p, t_w = statistics.median(tp), statistics.median(tw)
+    return dict(workload="ragged_prefill: lengths {1024,3000,8192,5555}, H=16, head_dim 128, w=512, "
+                "bits p=.3/.4/.2/.1, modes p=.2/.4/.4, 1% outlier channels x8",
+                pairs=pairs, flops=flops, prefill_s=t_p, tflops=flops / t_p / 1e12,
+                write_s=t_w, write_bytes=write_bytes, write_gbs=write_bytes / t_w / 1e9)
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_decode_sample(wl, budget_s=12.0, max_pairs=None):
+    """Time the CPU oracle on decode queries of the workload (skip heads excluded from the
+    sample: they do no work). Returns (keys/s, keys, seconds, description)."""
+    import oracle
+    from mixed_precision_kv_write_b200 import synth
+    q, modes = synth.decode_queries(wl, "cpu")
+    L, done_keys, t_total, n = wl.seqlens[0], 0, 0.0, 0
+    for s in range(wl.batch):
+        ks, vs, bs = synth.kv_sequence(wl, s, "cuda" if torch.cuda.is_available() else "cpu")
+        ks, vs, bs = ks.cpu(), vs.cpu(), bs.cpu()
+        for h in range(wl.heads):
+            m = int(modes[s, h])
+            if m == 0:
+                continue
+            kh, vh, bh = ks[:, h].contiguous().numpy(), vs[:, h].contiguous().numpy(), bs[:, h].numpy()
+            t0 = time.perf_counter()
+            oracle.routed_attention_head(q[s, h][None].numpy(), [L - 1], [m], wl.w, kh, vh, bh)
+            t_total += time.perf_counter() - t0
+            done_keys += L if m == 2 else min(L, wl.w + 1)
+            n += 1
+            if t_total >= budget_s or (max_pairs and n >= max_pairs):
+                desc = (f"oracle decode of {n} non-skip (sequence, head) queries of "
+                        f"{wl.name} in order, single-threaded C")
+                return done_keys / t_total, done_keys, t_total, desc
+    desc = f"oracle decode of all {n} non-skip queries of {wl.name}, single-threaded C"
+    return done_keys / t_total, done_keys, t_total, desc
+
+
+# ------------------------------------------------------------------ arms
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = False
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+        pg = True
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local, pg
+
+
+def max_over_ranks(x: float, pg: bool, dev) -> float:
+    if not pg:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg, dev):
+    if pg:
+        torch.distributed.barrier(device_ids=[dev.index])
+    torch.cuda.synchronize(dev)
+
+
+def run_ours(args):
+    from mixed_precision_kv_write_b200 import build as kbuild, kvq, synth
+    kbuild.build()
+    import oracle
+    oracle.build()
+    world, rank, local, pg = dist_setup()
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS["decode_1p3b"]
+    pk, pk_kind = peaks()
+
+    st = decode_setup(wl, dev)
+    stream = torch.cuda.current_stream(dev)
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(args.warmup):
+        decode_step(st, wl.w)
+    # per-step events around the split-K kernel (profiling hook of the C ABI)
+    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(pg, dev)
+    t_begin = time.time()
+    e0.record(stream)
+    for i in range(args.steps):
+        kvq.kvq_set_profile_events(*ev_k[i])
+        decode_step(st, wl.w)
+    e1.record(stream)
+    kvq.kvq_set_profile_events(None, None)
+    barrier(pg, dev)
+    t_end = time.time()
+    sampler.stop()
+    st["cache"].check()
+    elapsed = e0.elapsed_time(e1) * 1e-3
+    elapsed_max = max_over_ranks(elapsed, pg, dev)
+    k_times = [a.elapsed_time(b) * 1e-3 for a, b in ev_k]
+    k_avg = statistics.mean(k_times)
+    clocks = sampler.summary(t_begin, t_end)
+
+    keys = st["keys"]
+    routed = st["rec_bytes"] + st["side_bytes"]
+    value = keys * args.steps * world / elapsed_max
+    ms_step = elapsed_max / args.steps * 1e3
+    kernel_bytes = routed + st["q_bytes"]
+    hbm_peak = float(pk["hbm_gbs"])
+    achieved = kernel_bytes / k_avg / 1e9
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "decode_splitk_decode_1p3b.traffic.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                tj = json.load(f)
+            if tj.get("kernel_source_hash") == _src_hash():
+                traffic = tj.get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    # end to end through host buffers: per step H2D of the step inputs (pinned), D2H of out
+    host = {n: st[n].cpu().pin_memory() for n in ("k_step", "v_step", "b_step", "q", "modes")}
+    out_h = torch.empty(st["out"].shape, dtype=torch.float32, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * 4
+    from mixed_precision_kv_write_b200 import kvq as _k
+
+    def e2e_step():
+        for n, t in host.items():
+            st[n].copy_(t, non_blocking=True)
+        decode_step(st, wl.w)
+        out_h.copy_(st["out"], non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    barrier(pg, dev)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    barrier(pg, dev)
+    e2e_s = max_over_ranks(f0.elapsed_time(f1) * 1e-3, pg, dev)
+    e2e_value = keys * args.steps * world / e2e_s
+
+    pre = prefill_measure(dev) if not args.no_prefill else None
+    barrier(pg, dev)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) fp16 K/V/Q, i.i.d. widths and modes)",
+        "config": {
+            "workload": "decode_1p3b: batch 64, H=16, head_dim 128, cached context 8192, w=512, "
+                        "bits p(2/4/8/16)=.25/.45/.2/.1, modes p(skip/local/full)=.15/.45/.4",
+            "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
+            "context": wl.seqlens[0], "w": wl.w,
+            "step": "truncate to 8191, kvq_write of the step token, routed_attn_decode",
+            "l2": "no flush: each step reads %.0f MB of routed cache bytes > 126 MB L2" % (routed / 1e6),
+            "parallelism": f"{world} independent replica(s), no data-path collective",
+            "storage": "packed u2/u4/u8 codes + fp16, fp32 side table"},
+        "attended_keys_per_step": keys,
+        "routed_bytes_per_step": routed,
+        "hbm_gbs": routed / (elapsed_max / args.steps) / 1e9,
+        "hbm_frac_of_8tbs": routed / (elapsed_max / args.steps) / 1e9 / NOMINAL_HBM_GBS,
+        "roofline": {"kernel": "decode_splitk_kernel<128>", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm_peak, "peak_kind": pk_kind, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": kernel_bytes,
+                     "avg_launch_s": k_avg},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+        "gpu_launches": LAUNCHES_PER_DECODE_STEP * args.steps,
+    }
+    if pre:
+        bf16 = float(pk["bf16_tflops"])
+        line["prefill"] = {
+            "workload": pre["workload"], "tflops": pre["tflops"], "seconds": pre["prefill_s"],
+            "pairs": pre["pairs"], "flops": pre["flops"],
+            "roofline": {"kernel": "prefill attention", "bound": "tensor", "achieved": pre["tflops"],
+                         "peak": bf16, "peak_kind": pk_kind + " bf16 dense (burst)", "unit": "TFLOP/s",
+                         "frac": pre["tflops"] / bf16, "traffic": None},
+            "quantize": {"gbs": pre["write_gbs"], "bytes": pre["write_bytes"],
+                         "seconds": pre["write_s"], "frac_of_hbm": pre["write_gbs"] / hbm_peak}}
+    if rank == 0 and not args.no_cpu_baseline:
+        v_cpu, n_keys, secs, desc = oracle_decode_sample(wl, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": f"{desc}: {n_keys} keys in {secs:.1f} s"}
+    if pg:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args):
+    """The reference arm is the CPU oracle (no other implementation of this path exists):
+    each step decodes a bounded sample of the same workload on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from mixed_precision_kv_write_b200 import synth
+    oracle.build()
+    wl = synth.WORKLOADS["decode_1p3b"]
+    per_step = 4   # non-skip (sequence, head) queries per step
+    for _ in range(args.warmup):
+        oracle_decode_sample(wl, budget_s=1e9, max_pairs=1)
+    keys = 0
+    secs = 0.0
+    for _ in range(args.steps):
+        _, k, s, desc = oracle_decode_sample(wl, budget_s=1e9, max_pairs=per_step)
+        keys += k
+        secs += s
+    v = keys / secs
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "decode_1p3b (sampled: the first "
+                                            f"{per_step} non-skip queries per step)"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _src_hash():
+    import hashlib
+    h = hashlib.sha256()
+    p = os.path.join(ROOT, "mixed_precision_kv_write_b200", "csrc", "kvq_decode.cu")
+    with open(p, "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

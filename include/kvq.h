@@ -101,8 +101,8 @@ int kvq_cache_lengths(const kvq_cache *cache, int32_t *lengths, kvq_stream_t str
  * The codes are stored packed (code of channel c at bits [b*c, b*c + b) of the record
  * part), (s, z) go to the fp32 side table; b = 16 stores the fp16 bits and side (1, 0).
  * A sequence whose write would exceed its capacity is left unchanged (status
- * KVQ_ERR_CAPACITY); a token-head with invalid bits rejects its sequence's write for
- * that head (status KVQ_ERR_BITS).
+ * KVQ_ERR_CAPACITY); an invalid bits entry rejects its sequence's whole write, for
+ * every head (status KVQ_ERR_BITS).
  */
 int kvq_write(const void *k, const void *v, const uint8_t *bits, const int32_t *cu_seqlens,
               int64_t n_tok, kvq_cache *cache, kvq_stream_t stream);
@@ -151,6 +151,16 @@ int kvq_cache_export(const kvq_cache *cache, int seq, int head, int64_t first, i
  * Returns KVQ_OK or the first device-side error recorded since the last check.
  */
 int kvq_check(kvq_cache *cache, kvq_stream_t stream);
+
+/*
+ * Profiling hook for benchmarks. With non-NULL `before` / `after` (each a cudaEvent_t
+ * created by the caller), every following kvq_write, routed_attn_decode and
+ * routed_attn_prefill call records `before` on its stream immediately before its main
+ * kernel and `after` immediately after it (kvq_write: the quantize kernel; decode: the
+ * split-K kernel; prefill: the attention kernel), so the pair times that kernel alone.
+ * NULL, NULL turns recording off. Process-wide and not thread-safe.
+ */
+int kvq_set_profile_events(void *before, void *after);
 
 /* Text of the last host-side error on this thread ("" if none). */
 const char *kvq_last_error(void);

@@ -1,0 +1,361 @@
+// C ABI of the routed mixed-precision KV cache: argument checks, cache allocation,
+// small maintenance kernels (reset, truncate, lengths, export) and the status word.
+// The hot-path kernels live in kvq_write.cu, kvq_decode.cu and kvq_prefill.cu.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "kvq_internal.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int ok()
+{
+    g_err.clear();
+    return KVQ_OK;
+}
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+__global__ void truncate_kernel(kvq::CacheView c, const int32_t *__restrict__ lengths)
+{
+    const int sh = blockIdx.x * blockDim.x + threadIdx.x;
+    if (sh >= c.B * c.H) return;
+    const int s = sh / c.H, h = sh % c.H;
+    const int want = lengths[s];
+    const int have = c.len[sh];
+    if (want < 0 || want >= have) return;
+    c.end[sh] = c.meta[kvq::slot_of(c, s, h, want)] & ~15u;
+    c.len[sh] = want;
+}
+
+__global__ void lengths_kernel(kvq::CacheView c, int32_t *__restrict__ out)
+{
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s < c.B) out[s] = c.len[s * c.H];
+}
+
+// one warp per exported token
+__global__ void export_kernel(kvq::CacheView c, int s, int h, int64_t first, int64_t count,
+                              uint16_t *k_codes, uint16_t *v_codes, float *side, uint8_t *bits)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (i >= count) return;
+    const int64_t j = first + i;
+    if (j < 0 || j >= c.len[s * c.H + h]) {
+        if (lane == 0) kvq::set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+        return;
+    }
+    const int D = c.D;
+    const int64_t slot = kvq::slot_of(c, s, h, j);
+    const uint32_t mt = c.meta[slot];
+    const int b = 2 << (mt & 3u);
+    const uint8_t *rec = kvq::stream_of(c, s, h) + (mt & ~15u);
+    for (int part = 0; part < 2; ++part) {
+        uint16_t *dst = part == 0 ? k_codes : v_codes;
+        if (!dst) continue;
+        const uint8_t *p = rec + part * (b * D / 8);
+        for (int ch = lane; ch < D; ch += 32) {
+            uint16_t val;
+            if (b == 16) {
+                val = reinterpret_cast<const uint16_t *>(p)[ch];
+            } else {
+                const int bit = b * ch;
+                val = (uint16_t)((reinterpret_cast<const uint32_t *>(p)[bit >> 5] >> (bit & 31)) &
+                                 ((1u << b) - 1u));
+            }
+            dst[i * D + ch] = val;
+        }
+    }
+    if (lane == 0) {
+        if (side) reinterpret_cast<float4 *>(side)[i] = c.side[slot];
+        if (bits) bits[i] = (uint8_t)b;
+    }
+}
+
+__global__ void init_side_kernel(float4 *side, int64_t n)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        side[i] = make_float4(1.f, 0.f, 1.f, 0.f);
+}
+
+bool valid_cache(const kvq_cache *c) { return c && c->B > 0 && c->H > 0; }
+
+} // namespace
+
+namespace kvq {
+namespace {
+cudaEvent_t g_prof_before = nullptr, g_prof_after = nullptr;
+}
+void profile_before(cudaStream_t st)
+{
+    if (g_prof_before) cudaEventRecord(g_prof_before, st);
+}
+void profile_after(cudaStream_t st)
+{
+    if (g_prof_after) cudaEventRecord(g_prof_after, st);
+}
+
+int num_sms()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+} // namespace kvq
+
+extern "C" {
+
+const char *kvq_last_error(void) { return g_err.c_str(); }
+
+int kvq_set_profile_events(void *before, void *after)
+{
+    if ((before == nullptr) != (after == nullptr))
+        return fail(KVQ_ERR_ARG, "kvq_set_profile_events: pass two events or two NULLs");
+    kvq::g_prof_before = static_cast<cudaEvent_t>(before);
+    kvq::g_prof_after = static_cast<cudaEvent_t>(after);
+    return ok();
+}
+
+int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
+                     const int64_t *capacity_tokens, kvq_stream_t stream)
+{
+    if (!out) return fail(KVQ_ERR_ARG, "kvq_cache_create: out is NULL");
+    *out = nullptr;
+    if (batch <= 0 || heads <= 0) return fail(KVQ_ERR_ARG, "kvq_cache_create: batch and heads must be > 0");
+    if ((int64_t)batch * heads > (1 << 24)) return fail(KVQ_ERR_ARG, "kvq_cache_create: batch*heads too large");
+    if (head_dim != 64 && head_dim != 128)
+        return fail(KVQ_ERR_ARG, "kvq_cache_create: head_dim must be 64 or 128 (got %d)", head_dim);
+    if (!capacity_tokens) return fail(KVQ_ERR_ARG, "kvq_cache_create: capacity_tokens is NULL");
+    std::vector<int32_t> cap(batch), cap_pad(batch);
+    std::vector<int64_t> slot_base(batch);
+    int64_t slots = 0, max_items = 0;
+    int32_t max_cap = 0;
+    for (int s = 0; s < batch; ++s) {
+        const int64_t cp = capacity_tokens[s];
+        if (cp < 1 || cp > 8388607)
+            return fail(KVQ_ERR_ARG, "kvq_cache_create: capacity_tokens[%d] = %lld outside [1, 8388607]", s,
+                        (long long)cp);
+        cap[s] = (int32_t)cp;
+        cap_pad[s] = (int32_t)((cp + 4) & ~int64_t(3));    // >= cp + 1, multiple of 4
+        slot_base[s] = slots;
+        slots += (int64_t)heads * cap_pad[s];
+        max_items += (int64_t)heads * ((cp + kvq::kDecodeItemKeys - 1) / kvq::kDecodeItemKeys);
+        max_cap = std::max(max_cap, cap[s]);
+    }
+    if (max_items > INT32_MAX / 2) return fail(KVQ_ERR_ARG, "kvq_cache_create: too many decode items");
+
+    kvq_cache *c = new kvq_cache();
+    std::memset(c, 0, sizeof(*c));
+    c->B = batch;
+    c->H = heads;
+    c->D = head_dim;
+    c->total_slots = slots;
+    c->max_cap = max_cap;
+    cudaGetDevice(&c->device);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    auto alloc = [&](size_t bytes) -> void * {
+        void *p = nullptr;
+        if (cudaMalloc(&p, std::max<size_t>(bytes, 16)) != cudaSuccess) return nullptr;
+        c->allocs[c->n_allocs++] = p;
+        return p;
+    };
+    const int BH = batch * heads;
+    kvq::CacheView &v = c->view;
+    v.B = batch;
+    v.H = heads;
+    v.D = head_dim;
+    bool okk = true;
+    int32_t *cap_d = (int32_t *)alloc(sizeof(int32_t) * batch);
+    int32_t *cap_pad_d = (int32_t *)alloc(sizeof(int32_t) * batch);
+    int64_t *slot_base_d = (int64_t *)alloc(sizeof(int64_t) * batch);
+    v.rec = (uint8_t *)alloc((size_t)slots * 4 * head_dim);
+    v.meta = (uint32_t *)alloc(sizeof(uint32_t) * (size_t)slots);
+    v.side = (float4 *)alloc(sizeof(float4) * (size_t)slots);
+    v.len = (int32_t *)alloc(sizeof(int32_t) * BH);
+    v.end = (uint32_t *)alloc(sizeof(uint32_t) * BH);
+    v.wstart = (int32_t *)alloc(sizeof(int32_t) * BH);
+    v.status = (int32_t *)alloc(sizeof(int32_t));
+    kvq::DecodeWork &wk = c->work;
+    wk.max_items = max_items;
+    wk.items = (int4 *)alloc(sizeof(int4) * (size_t)max_items);
+    wk.count = (int32_t *)alloc(sizeof(int32_t));
+    wk.head_first = (int32_t *)alloc(sizeof(int32_t) * BH);
+    wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * BH);
+    wk.partials = (float *)alloc(sizeof(float) * (size_t)max_items * (head_dim + 4));
+    for (int i = 0; i < c->n_allocs; ++i) okk = okk && c->allocs[i];
+    if (!okk || c->n_allocs != 15) {
+        kvq_cache_destroy(c);
+        return fail(KVQ_ERR_NOMEM, "kvq_cache_create: cudaMalloc failed (%lld slots, %.2f GB of records)",
+                    (long long)slots, (double)slots * 4 * head_dim / 1e9);
+    }
+    v.cap = cap_d;
+    v.cap_pad = cap_pad_d;
+    v.slot_base = slot_base_d;
+    cudaError_t e = cudaSuccess;
+    e = e ? e : cudaMemcpyAsync(cap_d, cap.data(), sizeof(int32_t) * batch, cudaMemcpyHostToDevice, st);
+    e = e ? e : cudaMemcpyAsync(cap_pad_d, cap_pad.data(), sizeof(int32_t) * batch, cudaMemcpyHostToDevice, st);
+    e = e ? e : cudaMemcpyAsync(slot_base_d, slot_base.data(), sizeof(int64_t) * batch, cudaMemcpyHostToDevice, st);
+    e = e ? e : cudaMemsetAsync(v.len, 0, sizeof(int32_t) * BH, st);
+    e = e ? e : cudaMemsetAsync(v.end, 0, sizeof(uint32_t) * BH, st);
+    e = e ? e : cudaMemsetAsync(v.wstart, 0, sizeof(int32_t) * BH, st);
+    e = e ? e : cudaMemsetAsync(v.status, 0, sizeof(int32_t), st);
+    e = e ? e : cudaMemsetAsync(v.meta, 0, sizeof(uint32_t) * (size_t)slots, st);
+    e = e ? e : cudaMemsetAsync(wk.count, 0, sizeof(int32_t), st);
+    if (!e) {
+        init_side_kernel<<<1024, 256, 0, st>>>(v.side, slots);
+        e = cudaGetLastError();
+    }
+    // the host vectors above are pageable: finish the copies before they go out of scope
+    if (!e) e = cudaStreamSynchronize(st);
+    if (e) {
+        kvq_cache_destroy(c);
+        return cuda_fail(e, "kvq_cache_create");
+    }
+    *out = c;
+    return ok();
+}
+
+int kvq_cache_destroy(kvq_cache *c)
+{
+    if (!c) return ok();
+    cudaDeviceSynchronize();
+    for (int i = 0; i < c->n_allocs; ++i)
+        if (c->allocs[i]) cudaFree(c->allocs[i]);
+    delete c;
+    return ok();
+}
+
+int kvq_cache_reset(kvq_cache *c, kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_cache_reset: bad cache");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int BH = c->B * c->H;
+    cudaError_t e = cudaMemsetAsync(c->view.len, 0, sizeof(int32_t) * BH, st);
+    e = e ? e : cudaMemsetAsync(c->view.end, 0, sizeof(uint32_t) * BH, st);
+    e = e ? e : cudaMemsetAsync(c->view.status, 0, sizeof(int32_t), st);
+    return e ? cuda_fail(e, "kvq_cache_reset") : ok();
+}
+
+int kvq_cache_truncate(kvq_cache *c, const int32_t *lengths, kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_cache_truncate: bad cache");
+    if (!lengths) return fail(KVQ_ERR_ARG, "kvq_cache_truncate: lengths is NULL");
+    const int BH = c->B * c->H;
+    truncate_kernel<<<(BH + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c->view, lengths);
+    cudaError_t e = cudaGetLastError();
+    return e ? cuda_fail(e, "kvq_cache_truncate") : ok();
+}
+
+int kvq_cache_lengths(const kvq_cache *c, int32_t *lengths, kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_cache_lengths: bad cache");
+    if (!lengths) return fail(KVQ_ERR_ARG, "kvq_cache_lengths: lengths is NULL");
+    lengths_kernel<<<(c->B + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c->view, lengths);
+    cudaError_t e = cudaGetLastError();
+    return e ? cuda_fail(e, "kvq_cache_lengths") : ok();
+}
+
+int kvq_write(const void *k, const void *v, const uint8_t *bits, const int32_t *cu_seqlens,
+              int64_t n_tok, kvq_cache *c, kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_write: bad cache");
+    if (n_tok < 0 || n_tok > (int64_t)INT32_MAX / c->H)
+        return fail(KVQ_ERR_ARG, "kvq_write: n_tok = %lld out of range", (long long)n_tok);
+    if (!cu_seqlens) return fail(KVQ_ERR_ARG, "kvq_write: cu_seqlens is NULL");
+    if (n_tok > 0 && (!k || !v || !bits)) return fail(KVQ_ERR_ARG, "kvq_write: k, v or bits is NULL");
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15u)
+        return fail(KVQ_ERR_ARG, "kvq_write: k and v must be 16-byte aligned");
+    cudaError_t e = kvq::launch_write(c, static_cast<const __half *>(k), static_cast<const __half *>(v),
+                                      bits, cu_seqlens, n_tok, reinterpret_cast<cudaStream_t>(stream));
+    return e ? cuda_fail(e, "kvq_write") : ok();
+}
+
+int routed_attn_prefill(const void *q, const kvq_cache *c, const uint8_t *modes, int w,
+                        const int32_t *cu_seqlens, int64_t n_tok, float *out, kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "routed_attn_prefill: bad cache");
+    if (w < 0) return fail(KVQ_ERR_ARG, "routed_attn_prefill: w = %d < 0", w);
+    if (n_tok < 0 || n_tok > (int64_t)INT32_MAX / c->H)
+        return fail(KVQ_ERR_ARG, "routed_attn_prefill: n_tok = %lld out of range", (long long)n_tok);
+    if (!cu_seqlens) return fail(KVQ_ERR_ARG, "routed_attn_prefill: cu_seqlens is NULL");
+    if (n_tok > 0 && (!q || !modes || !out))
+        return fail(KVQ_ERR_ARG, "routed_attn_prefill: q, modes or out is NULL");
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15u)
+        return fail(KVQ_ERR_ARG, "routed_attn_prefill: q and out must be 16-byte aligned");
+    cudaError_t e = kvq::launch_prefill(c, static_cast<const __half *>(q), modes, w, cu_seqlens, n_tok, out,
+                                        reinterpret_cast<cudaStream_t>(stream));
+    return e ? cuda_fail(e, "routed_attn_prefill") : ok();
+}
+
+int routed_attn_decode(const void *q, const kvq_cache *c, const uint8_t *modes, int w, float *out,
+                       kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "routed_attn_decode: bad cache");
+    if (w < 0) return fail(KVQ_ERR_ARG, "routed_attn_decode: w = %d < 0", w);
+    if (!q || !modes || !out) return fail(KVQ_ERR_ARG, "routed_attn_decode: q, modes or out is NULL");
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15u)
+        return fail(KVQ_ERR_ARG, "routed_attn_decode: q and out must be 16-byte aligned");
+    cudaError_t e = kvq::launch_decode(c, static_cast<const __half *>(q), modes, w, out,
+                                       reinterpret_cast<cudaStream_t>(stream));
+    return e ? cuda_fail(e, "routed_attn_decode") : ok();
+}
+
+int kvq_cache_export(const kvq_cache *c, int seq, int head, int64_t first, int64_t count,
+                     uint16_t *k_codes, uint16_t *v_codes, float *side, uint8_t *bits, kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_cache_export: bad cache");
+    if (seq < 0 || seq >= c->B || head < 0 || head >= c->H)
+        return fail(KVQ_ERR_ARG, "kvq_cache_export: (seq, head) = (%d, %d) out of range", seq, head);
+    if (first < 0 || count < 0 || first + count > c->max_cap)
+        return fail(KVQ_ERR_ARG, "kvq_cache_export: token range out of capacity");
+    if (count == 0) return ok();
+    const int64_t threads = count * 32;
+    export_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        c->view, seq, head, first, count, k_codes, v_codes, side, bits);
+    cudaError_t e = cudaGetLastError();
+    return e ? cuda_fail(e, "kvq_cache_export") : ok();
+}
+
+int kvq_check(kvq_cache *c, kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_check: bad cache");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    cudaError_t e = cudaStreamSynchronize(st);
+    e = e ? e : cudaMemcpy(&h, c->view.status, sizeof(int32_t), cudaMemcpyDeviceToHost);
+    e = e ? e : cudaMemset(c->view.status, 0, sizeof(int32_t));
+    if (e) return cuda_fail(e, "kvq_check");
+    if (h) return fail(h, "device-side check failed with status %d", h);
+    return ok();
+}
+
+} // extern "C"

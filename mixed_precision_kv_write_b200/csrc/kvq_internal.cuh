@@ -1,0 +1,175 @@
+// Internal definitions of the routed mixed-precision KV cache (B200, sm_100a).
+//
+// Cache layout in HBM (per sequence s, head h, token j; "slot" = one (s, h, j)):
+//   records  one byte stream per (s, h), tokens in order; token j's record is
+//            [K part | V part], each part b*D/8 bytes: for b < 16 the codes are packed
+//            LSB-first (channel c occupies bits [b*c, b*c + b) of the part), for b = 16
+//            the part is the fp16 vector. Record size b*D/4 bytes, a multiple of 16.
+//            Stream (s, h) starts at byte slot(s, h, 0) * 4 * D, room for the worst case.
+//   meta     uint32 per slot: byte offset of the record inside its stream (a multiple of
+//            16) OR'ed with the width code (0, 1, 2, 3 for b = 2, 4, 8, 16).
+//   side     float4 per slot: (s_K, z_K, s_V, z_V) of Eq. 4; (1, 0, 1, 0) for b = 16.
+//   len/end  per (s, h): tokens held and the stream's end offset in bytes.
+// Slots: slot(s, h, j) = slot_base[s] + h * cap_pad[s] + j, cap_pad a multiple of 4 that
+// leaves at least one spare slot, so 16-byte bulk copies of meta may round to 4 slots.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+struct CacheView {
+    int B, H, D;
+    const int32_t *cap;       // [B] capacity in tokens
+    const int32_t *cap_pad;   // [B] slots per (s, h)
+    const int64_t *slot_base; // [B] first slot of sequence s
+    uint8_t *rec;             // record bytes
+    uint32_t *meta;           // [slots]
+    float4 *side;             // [slots]
+    int32_t *len;             // [B*H]
+    uint32_t *end;            // [B*H]
+    int32_t *wstart;          // [B*H] start position of the current write, -1 = rejected
+    int32_t *status;          // [1] first device-side error (kvq_status), 0 = none
+};
+
+__device__ __forceinline__ int64_t slot_of(const CacheView &c, int s, int h, int64_t j)
+{
+    return c.slot_base[s] + (int64_t)h * c.cap_pad[s] + j;
+}
+
+__device__ __forceinline__ uint8_t *stream_of(const CacheView &c, int s, int h)
+{
+    return c.rec + slot_of(c, s, h, 0) * (int64_t)(4 * c.D);
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ int width_code(int bits)
+{
+    return bits == 2 ? 0 : bits == 4 ? 1 : bits == 8 ? 2 : bits == 16 ? 3 : -1;
+}
+
+__device__ __forceinline__ void set_status(int32_t *status, int code)
+{
+    atomicCAS(status, 0, code);
+}
+
+// ---- scheduler work list (decode) ----------------------------------------------------
+constexpr int kDecodeItemKeys = 512;   // keys per split-K work item
+constexpr int kDecodeSubKeys = 64;     // keys per pipeline stage inside an item
+
+struct DecodeWork {
+    int4 *items;         // [max_items] (s*H + h, j0, j1, 0)
+    int32_t *count;      // [1]
+    int32_t *head_first; // [B*H]
+    int32_t *head_cnt;   // [B*H]
+    float *partials;     // [max_items][D + 4]: (m, l, -, -, o[D])
+    int64_t max_items;
+};
+
+// ---- PTX helpers -----------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait until the barrier's phase `parity` has completed. Bounded: gives up after about
+// two seconds, records KVQ_ERR_DEVICE_CHECK and returns false, so a logic error ends the
+// kernel with a status instead of hanging the GPU.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status)
+{
+    uint32_t addr = smem_u32(bar);
+    uint32_t done = 0;
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(done)
+                     : "r"(addr), "r"(parity)
+                     : "memory");
+        if (done) return true;
+        if ((it & 1023u) == 0) {
+            uint64_t t = global_ns();
+            if (t0 == 0) t0 = t;
+            else if (t - t0 > 2000000000ull) {
+                set_status(status, KVQ_ERR_DEVICE_CHECK);
+                return false;
+            }
+        }
+    }
+}
+
+// 1-D bulk copy global -> shared (TMA engine), completion counted on `bar` in bytes.
+// dst, src 16-byte aligned, bytes a multiple of 16. No multicast.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+} // namespace kvq
+
+// ---- launchers (implemented per kernel file, called by the C ABI) --------------------
+struct kvq_cache {
+    int B, H, D;
+    int device;
+    int64_t total_slots;
+    int32_t max_cap;
+    kvq::CacheView view;
+    kvq::DecodeWork work;
+    void *allocs[16];
+    int n_allocs;
+};
+
+namespace kvq {
+cudaError_t launch_write(const kvq_cache *c, const __half *k, const __half *v, const uint8_t *bits,
+                         const int32_t *cu, int64_t n_tok, cudaStream_t st);
+cudaError_t launch_decode(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,
+                          float *out, cudaStream_t st);
+cudaError_t launch_prefill(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,
+                           const int32_t *cu, int64_t n_tok, float *out, cudaStream_t st);
+int num_sms();
+// profiling hook (kvq_set_profile_events): record the caller's events around a main kernel
+void profile_before(cudaStream_t st);
+void profile_after(cudaStream_t st);
+} // namespace kvq

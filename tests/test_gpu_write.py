@@ -1,0 +1,125 @@
+"""GPU parity of quantize-on-write (Eq. 4): stored codes, scales, zeros and widths are
+bit-exact with the oracle, on every workload shape, plus the device-side error paths."""
+import numpy as np
+import pytest
+import torch
+
+from mixed_precision_kv_write_b200 import kvq, synth
+from kvq_testlib import build_cache, check_records
+
+pytestmark = pytest.mark.gpu
+W = synth.WORKLOADS
+
+
+@pytest.mark.parametrize("name,seqlens", [
+    ("tiny_prefill", None),
+    ("prefill_160m", (300, 1, 77, 2048)),
+    ("ragged_prefill", (1024, 3000, 17, 129)),
+    ("decode_1p3b", (513, 64, 1)),
+])
+def test_write_bit_exact(name, seqlens):
+    wl = W[name] if seqlens is None else synth.scaled(W[name], seqlens=seqlens)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cache = build_cache(wl, k, v, bits)
+    cache.check()
+    kc, vc, bc = k.cpu(), v.cpu(), bits.cpu()
+    pairs = [(s, h) for s in range(wl.batch) for h in range(wl.heads)]
+    check_records(cache, wl, kc, vc, bc, pairs)
+    assert cache.lengths().tolist() == list(wl.seqlens)
+
+
+def test_write_full_size_sampled():
+    # the full ragged-prefill workload (17771 tokens x 16 heads, head_dim 128), sampled heads
+    wl = W["ragged_prefill"]
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cache = build_cache(wl, k, v, bits)
+    cache.check()
+    rng = np.random.default_rng(0)
+    pairs = [(s, int(rng.integers(wl.heads))) for s in range(wl.batch)]
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), pairs)
+
+
+def test_write_in_chunks_equals_one_write():
+    # appending each sequence in pieces stores the same records as one write
+    wl = synth.scaled(W["prefill_160m"], seqlens=(200, 130))
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cache = kvq.KVQCache(wl.batch, wl.heads, wl.head_dim, list(wl.seqlens))
+    cu_all = synth.cu_seqlens(wl.seqlens).tolist()
+    for a, b in [(0, 1), (1, 70), (70, None)]:
+        idx, lens = [], []
+        for s in range(wl.batch):
+            L = wl.seqlens[s]
+            lo, hi = min(a, L), (L if b is None else min(b, L))
+            idx += list(range(cu_all[s] + lo, cu_all[s] + hi))
+            lens.append(hi - lo)
+        idx_t = torch.tensor(idx, device="cuda", dtype=torch.long)
+        kvq.kvq_write(k[idx_t].contiguous(), v[idx_t].contiguous(), bits[idx_t].contiguous(),
+                      synth.cu_seqlens(lens, "cuda"), cache)
+    cache.check()
+    assert cache.lengths().tolist() == [200, 130]
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(),
+                  [(s, h) for s in range(2) for h in range(wl.heads)])
+
+
+def test_constant_and_extreme_vectors():
+    wl = synth.Workload("edge", "prefill", (6,), 2, 128, 4, (0.25,) * 4, (1 / 3,) * 3, False, 7)
+    k = torch.zeros((6, 2, 128), dtype=torch.float16)
+    k[1] = 3.5                                        # constant: s = 0, codes 0
+    k[2, :, ::2] = 65504.0                            # fp16 extremes
+    k[2, :, 1::2] = -65504.0
+    k[3] = torch.linspace(-1, 1, 128, dtype=torch.float16)
+    k[4, :, 0] = -0.0                                 # signed zeros
+    k[5] = torch.randn((2, 128)).half() * 1e-4        # subnormal-scale values
+    v = k.flip(0).contiguous()
+    bits = torch.tensor([[2, 4], [8, 2], [2, 8], [4, 16], [16, 2], [8, 4]], dtype=torch.uint8)
+    cache = build_cache(wl, k.cuda(), v.cuda(), bits.cuda())
+    cache.check()
+    check_records(cache, wl, k, v, bits, [(0, 0), (0, 1)])
+
+
+def test_bad_bits_rejected_on_device():
+    wl = synth.scaled(W["tiny_prefill"], seqlens=(10,))
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    bits[3, 1] = 3
+    cache = kvq.KVQCache(1, wl.heads, wl.head_dim, [10])
+    kvq.kvq_write(k, v, bits, synth.cu_seqlens([10], "cuda"), cache)
+    with pytest.raises(kvq.KVQError) as e:
+        cache.check()
+    assert e.value.code == kvq.KVQ_ERR_BITS
+    cache.check()  # cleared
+    # the sequence's write was rejected for every head
+    assert cache.lengths().tolist() == [0]
+
+
+def test_capacity_overflow_rejected_on_device():
+    wl = synth.scaled(W["tiny_prefill"], seqlens=(10,))
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cache = kvq.KVQCache(1, wl.heads, wl.head_dim, [8])
+    kvq.kvq_write(k, v, bits, synth.cu_seqlens([10], "cuda"), cache)
+    with pytest.raises(kvq.KVQError) as e:
+        cache.check()
+    assert e.value.code == kvq.KVQ_ERR_CAPACITY
+    assert cache.lengths().tolist() == [0]
+
+
+def test_truncate_then_rewrite():
+    wl = synth.scaled(W["ragged_prefill"], seqlens=(100,), heads=3)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cache = build_cache(wl, k, v, bits)
+    cache.truncate(torch.tensor([60], dtype=torch.int32, device="cuda"))
+    assert cache.lengths().tolist() == [60]
+    # rewrite positions 60..99 with the same tokens: the cache equals a one-shot write
+    kvq.kvq_write(k[60:].contiguous(), v[60:].contiguous(), bits[60:].contiguous(),
+                  synth.cu_seqlens([40], "cuda"), cache)
+    cache.check()
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), [(0, h) for h in range(3)])
+
+
+def test_host_argument_errors():
+    cache = kvq.KVQCache(1, 2, 64, [4])
+    lib = kvq.load_library()
+    assert lib.routed_attn_decode(None, cache.handle, None, 0, None, None) == kvq.KVQ_ERR_ARG
+    q = torch.zeros((1, 2, 64), dtype=torch.float16, device="cuda")
+    m = torch.zeros((1, 2), dtype=torch.uint8, device="cuda")
+    with pytest.raises(kvq.KVQError):
+        kvq.routed_attn_decode(q, cache, m, -1)
