@@ -277,6 +277,8 @@ def run_ours(args):
     world, rank, local, pg = dist_setup()
     dev = torch.device("cuda", local)
     wl = synth.WORKLOADS["decode_1p3b"]
+    if args.decode_batch != wl.batch:     # smaller case for profiler captures
+        wl = synth.scaled(wl, seqlens=(wl.seqlens[0],) * args.decode_batch)
     pk, pk_kind = peaks()
 
     st = decode_setup(wl, dev)
@@ -451,6 +453,8 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--decode-batch", type=int, default=64,
+                    help="sequences of the decode workload (64; smaller only for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -83,7 +83,7 @@ def _stream(stream, device):
 def _check(t, name, dtype, device, shape=None):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda" or t.device != device:
+    if t.device.type != "cuda" or t.device.index != device.index:
         raise ValueError(f"{name} must be on {device} (got {t.device})")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
@@ -98,8 +98,11 @@ class KVQCache:
 
     def __init__(self, batch: int, heads: int, head_dim: int, capacity, device=None, stream=None):
         lib = load_library()
-        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
-            else torch.device(device)
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        if dev.type != "cuda":
+            raise ValueError(f"the cache lives on a CUDA device (got {dev})")
+        self.device = dev if dev.index is not None else \
+            torch.device("cuda", torch.cuda.current_device())
         cap = [int(capacity)] * batch if isinstance(capacity, int) else [int(x) for x in capacity]
         if len(cap) != batch:
             raise ValueError("capacity must be an int or have one entry per sequence")
@@ -158,6 +161,9 @@ class KVQCache:
 
 def kvq_set_profile_events(before=None, after=None):
     """Record torch.cuda.Event pairs around the main kernel of the following calls."""
+    for e in (before, after):
+        if e is not None and e.cuda_event == 0:
+            e.record()          # torch creates the CUDA event on first record
     b = None if before is None else ctypes.c_void_p(before.cuda_event)
     a = None if after is None else ctypes.c_void_p(after.cuda_event)
     _raise(load_library().kvq_set_profile_events(b, a))
