@@ -190,12 +190,16 @@ def prefill_measure(dev, reps=5, warm=2):
     for r in range(warm + reps):
         flush.fill_(r & 255)
         cache.reset()
+        if r >= warm:
+            torch.cuda.nvtx.range_push("prefill_timed")
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         kvq.kvq_set_profile_events(e[0], e[1])
         kvq.kvq_write(k, v, bits, cu, cache)
         kvq.kvq_set_profile_events(e[2], e[3])
         kvq.routed_attn_prefill(q, cache, modes, wl.w, cu, out=out)
         kvq.kvq_set_profile_events(None, None)
+        if r >= warm:
+            torch.cuda.nvtx.range_pop()
         stream.synchronize()
         if r >= warm:
             tw.append(e[0].elapsed_time(e[1]) * 1e-3)
@@ -293,11 +297,13 @@ def run_ours(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(pg, dev)
     t_begin = time.time()
+    torch.cuda.nvtx.range_push("decode_timed")
     e0.record(stream)
     for i in range(args.steps):
         kvq.kvq_set_profile_events(*ev_k[i])
         decode_step(st, wl.w)
     e1.record(stream)
+    torch.cuda.nvtx.range_pop()
     kvq.kvq_set_profile_events(None, None)
     barrier(pg, dev)
     t_end = time.time()

@@ -203,16 +203,18 @@ int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
     v.len = (int32_t *)alloc(sizeof(int32_t) * BH);
     v.end = (uint32_t *)alloc(sizeof(uint32_t) * BH);
     v.wstart = (int32_t *)alloc(sizeof(int32_t) * BH);
+    v.wend = (uint32_t *)alloc(sizeof(uint32_t) * BH);
+    v.bad = (uint32_t *)alloc(sizeof(uint32_t) * batch);
     v.status = (int32_t *)alloc(sizeof(int32_t));
     kvq::DecodeWork &wk = c->work;
     wk.max_items = max_items;
-    wk.items = (int4 *)alloc(sizeof(int4) * (size_t)max_items);
+    wk.items = (kvq::DecodeItem *)alloc(sizeof(kvq::DecodeItem) * (size_t)max_items);
     wk.count = (int32_t *)alloc(sizeof(int32_t));
     wk.head_first = (int32_t *)alloc(sizeof(int32_t) * BH);
     wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * BH);
     wk.partials = (float *)alloc(sizeof(float) * (size_t)max_items * (head_dim + 4));
     for (int i = 0; i < c->n_allocs; ++i) okk = okk && c->allocs[i];
-    if (!okk || c->n_allocs != 15) {
+    if (!okk || c->n_allocs != 17) {
         kvq_cache_destroy(c);
         return fail(KVQ_ERR_NOMEM, "kvq_cache_create: cudaMalloc failed (%lld slots, %.2f GB of records)",
                     (long long)slots, (double)slots * 4 * head_dim / 1e9);
@@ -227,6 +229,8 @@ int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
     e = e ? e : cudaMemsetAsync(v.len, 0, sizeof(int32_t) * BH, st);
     e = e ? e : cudaMemsetAsync(v.end, 0, sizeof(uint32_t) * BH, st);
     e = e ? e : cudaMemsetAsync(v.wstart, 0, sizeof(int32_t) * BH, st);
+    e = e ? e : cudaMemsetAsync(v.wend, 0, sizeof(uint32_t) * BH, st);
+    e = e ? e : cudaMemsetAsync(v.bad, 0, sizeof(uint32_t) * batch, st);
     e = e ? e : cudaMemsetAsync(v.status, 0, sizeof(int32_t), st);
     e = e ? e : cudaMemsetAsync(v.meta, 0, sizeof(uint32_t) * (size_t)slots, st);
     e = e ? e : cudaMemsetAsync(wk.count, 0, sizeof(int32_t), st);

@@ -4,14 +4,21 @@
 // Three launches:
 //   decode_sched_kernel   mode-aware scheduler: skip heads and empty sequences get no
 //                         work, local heads are clamped to keys [max(0, t - w), t], full
-//                         heads read [0, t]; each range is cut into items of up to 512
-//                         keys, listed on the device (no host round trip).
-//   decode_splitk_kernel  persistent CTAs: one producer warp streams each item's
-//                         contiguous record bytes, side entries and offsets into shared
-//                         memory with 1-D bulk copies (64-key stages, mbarrier pipeline);
-//                         eight consumer warps dequantize in registers and run an online
-//                         softmax; each item leaves a partial (m, l, o[D]).
-//   decode_combine_kernel log-sum-exp merge of an item list per (sequence, head).
+//                         heads read [0, t]; each range is cut into near-equal items of at
+//                         most 512 keys, listed on the device (no host round trip).
+//   decode_splitk_kernel  two CTAs per SM. A producer warp walks the CTA's items in
+//                         stages of at most 64 keys and 16 KB of records: it reads the
+//                         stage's record offsets, sorts the keys by width once (so the
+//                         consumers' 4-key steps rarely mix widths), and streams the stage's
+//                         contiguous record bytes, side entries and (for a new item) the
+//                         query into shared memory with 1-D bulk copies (4-stage mbarrier
+//                         pipeline). Eight consumer warps split each stage's keys: 8 lanes
+//                         per key, 16 channels per lane, K dot product -> logit -> online
+//                         softmax kept per 8-lane group -> V accumulation, all in registers;
+//                         the groups' states are merged once per item into a partial
+//                         (m, l, o[D]).
+//   decode_combine_kernel log-sum-exp merge of the item partials of each (sequence, head),
+//                         one thread per channel; zeros for skip heads and empty sequences.
 //
 // Arithmetic. With codes c, scale s and zero z (Eq. 4):
 //   q . deq(k_j) = s_j * (q . c_j) + z_j * sum(q)         (one dot product on integer codes)
@@ -29,9 +36,15 @@ namespace {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kStages = 4;
-constexpr int kSub = kDecodeSubKeys;              // 64 keys per stage
-
+constexpr int kStages = 3;                        // record stages in flight per CTA
+constexpr int kWin = kDecodeWindowKeys;           // keys per window of record offsets
+constexpr uint32_t kStageRecBytes = 24576;        // record bytes per stage, at most
+constexpr int kPermSlots = kWin + 32;             // width-sorted keys padded to whole chunks
+constexpr int kMetaSlots = 6;                     // windows of record offsets fetched ahead
+constexpr int kMetaWords = kWin + 8;
+constexpr int kNewItem = 1, kLastSub = 2;         // stage flags
+constexpr uint32_t kReadEndFromMeta = 0xFFFFFFFFu;
+constexpr uint32_t kValid = 0x80000000u;
 
 // q'_b[k] = q[k] * 2^(60 - pos_b(k)); the code field of channel k sits at pos_b(k) after
 // unpack: b = 2 -> 2*(k % 8), b = 4 -> 4*(k % 4), b = 8 -> 0. Dot products over codes
@@ -46,19 +59,33 @@ constexpr float kOUnscale = 562949953421312.0f;                    // 2^49
 
 template <int D>
 struct Stage {
-    uint32_t meta[kSub + 4];
-    float4 side[kSub];
-    alignas(16) uint8_t rec[kSub * 4 * D];
+    // width-sorted keys in class-pure chunks: kValid | (offset in rec << 9) |
+    // (width code << 7) | key; padding entries carry only their chunk's width code
+    uint32_t perm[kPermSlots];
+    int32_t info[4];         // item index, keys in the stage, flags, chunks
+    __half q[D];             // the item's query (copied with the item's first stage)
+    float4 side[kWin];       // (s_K, z_K, s_V, z_V) per key, token order
+    alignas(16) uint8_t rec[kStageRecBytes];
+};
+
+// one window of record offsets: meta of keys [ja, ...) of an item's stream
+struct alignas(16) MetaSlot {
+    uint32_t meta[kMetaWords];
+    int32_t it, j, j1, ja;
+    uint32_t end_off, first;
+    int64_t sbase;
+    int32_t sh, pad;
 };
 
 template <int D>
 struct DecodeSmem {
     Stage<D> st[kStages];
-    float logit[kStages][kSub];
-    uint8_t perm[kConsumerWarps][kSub];
-    float red[kConsumerWarps][D];
+    MetaSlot ms[kMetaSlots];
+    float red_o[kConsumerWarps][D];
+    float red_m[kConsumerWarps], red_l[kConsumerWarps], red_pz[kConsumerWarps];
     uint64_t full[kStages];
     uint64_t empty[kStages];
+    uint64_t mfull[kMetaSlots];
 };
 
 __device__ __forceinline__ float fld(uint32_t bits) { return __uint_as_float(bits); }
@@ -74,10 +101,10 @@ __global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ mod
     __syncthreads();
     for (int base = 0; base < BH; base += blockDim.x) {
         const int i = base + tid;
-        int cnt = 0, lo = 0, hi = 0;
+        int cnt = 0, lo = 0, hi = 0, L = 0;
         if (i < BH) {
             const int m = modes[i];
-            const int L = c.len[i];
+            L = c.len[i];
             if (m > KVQ_MODE_FULL) {
                 set_status(c.status, KVQ_ERR_MODE);
             } else if (m != KVQ_MODE_SKIP && L > 0) {
@@ -109,9 +136,24 @@ __global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ mod
         if (i < BH) {
             wk.head_first[i] = first;
             wk.head_cnt[i] = cnt;
-            for (int k = 0; k < cnt; ++k)
-                wk.items[first + k] = make_int4(i, lo + k * kDecodeItemKeys,
-                                                min(hi, lo + (k + 1) * kDecodeItemKeys), 0);
+            if (cnt > 0) {
+                const int s = i / c.H, h = i % c.H;
+                const int64_t sb = slot_of(c, s, h, 0);
+                const int n = hi - lo, per = n / cnt, rem = n % cnt;
+                int j0 = lo;
+                for (int k = 0; k < cnt; ++k) {               // near-equal, non-empty items
+                    DecodeItem it;
+                    it.sh = i;
+                    it.j0 = j0;
+                    it.j1 = j0 + per + (k < rem ? 1 : 0);
+                    j0 = it.j1;
+                    // the stream end for the item ending at the last token; else the
+                    // producer reads the offset of key j1 itself
+                    it.end_off = (it.j1 < L) ? kReadEndFromMeta : c.end[i];
+                    it.sbase = sb;
+                    wk.items[first + k] = it;
+                }
+            }
         }
         __syncthreads();
         if (tid == 0) carry_sh = carry + warp_tot[(blockDim.x >> 5) - 1];
@@ -128,56 +170,55 @@ struct QRegs {
 __device__ __forceinline__ float dot_codes2(const QRegs &q, uint32_t x)
 {
     const uint32_t y = x >> 16;
-    float a0 = 0.f, a1 = 0.f;
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-        a0 = fmaf(q.q2[k], fld(x & (3u << (2 * k))), a0);
-        a1 = fmaf(q.q2[k + 8], fld(y & (3u << (2 * k))), a1);
+        a[k & 1] = fmaf(q.q2[k], fld(x & (3u << (2 * k))), a[k & 1]);
+        a[2 + (k & 1)] = fmaf(q.q2[k + 8], fld(y & (3u << (2 * k))), a[2 + (k & 1)]);
     }
-    return a0 + a1;
+    return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 __device__ __forceinline__ float dot_codes4(const QRegs &q, uint2 x)
 {
-    float a0 = 0.f, a1 = 0.f;
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
     const uint32_t w[2] = {x.x, x.y};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const uint32_t lo = w[h], hi = w[h] >> 16;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            a0 = fmaf(q.q4[8 * h + k], fld(lo & (15u << (4 * k))), a0);
-            a1 = fmaf(q.q4[8 * h + 4 + k], fld(hi & (15u << (4 * k))), a1);
+            a[2 * h] = fmaf(q.q4[8 * h + k], fld(lo & (15u << (4 * k))), a[2 * h]);
+            a[2 * h + 1] = fmaf(q.q4[8 * h + 4 + k], fld(hi & (15u << (4 * k))), a[2 * h + 1]);
         }
     }
-    return a0 + a1;
+    return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 __device__ __forceinline__ float dot_codes8(const QRegs &q, uint4 x)
 {
-    float a0 = 0.f, a1 = 0.f;
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-        a0 = fmaf(q.q8[4 * h + 0], fld(__byte_perm(w[h], 0u, 0x4440)), a0);
-        a1 = fmaf(q.q8[4 * h + 1], fld(__byte_perm(w[h], 0u, 0x4441)), a1);
-        a0 = fmaf(q.q8[4 * h + 2], fld(__byte_perm(w[h], 0u, 0x4442)), a0);
-        a1 = fmaf(q.q8[4 * h + 3], fld(__byte_perm(w[h], 0u, 0x4443)), a1);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            a[e] = fmaf(q.q8[4 * h + e], fld(__byte_perm(w[h], 0u, 0x4440 + e)), a[e]);
     }
-    return a0 + a1;
+    return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 __device__ __forceinline__ float dot_native(const QRegs &q, uint4 x0, uint4 x1)
 {
     const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    float a0 = 0.f, a1 = 0.f;
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
         const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
-        a0 = fmaf(q.q8[2 * h], f.x, a0);
-        a1 = fmaf(q.q8[2 * h + 1], f.y, a1);
+        a[2 * (h & 1)] = fmaf(q.q8[2 * h], f.x, a[2 * (h & 1)]);
+        a[2 * (h & 1) + 1] = fmaf(q.q8[2 * h + 1], f.y, a[2 * (h & 1) + 1]);
     }
-    return a0 + a1;
+    return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 __device__ __forceinline__ void acc_codes2(float (&o)[16], float wv, uint32_t x)
@@ -227,15 +268,85 @@ __device__ __forceinline__ void acc_native(float (&o)[16], float wv, uint4 x0, u
     }
 }
 
+
+// merge the online-softmax state (m, l, pz, o) of this lane with the lane `mask` away
+__device__ __forceinline__ void merge_state(float &m, float &l, float &pz, float (&o)[16], int mask)
+{
+    const float mp = __shfl_xor_sync(0xffffffffu, m, mask);
+    const float lp = __shfl_xor_sync(0xffffffffu, l, mask);
+    const float zp = __shfl_xor_sync(0xffffffffu, pz, mask);
+    const float M = fmaxf(m, mp);
+    const float fa = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    const float fb = (mp == -INFINITY) ? 0.f : exp2f(mp - M);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float op = __shfl_xor_sync(0xffffffffu, o[k], mask);
+        o[k] = o[k] * fa + op * fb;
+    }
+    l = l * fa + lp * fb;
+    pz = pz * fa + zp * fb;
+    m = M;
+}
+
+struct KeyState {
+    float m, l, pz;
+    float o[16];
+};
+
+// One key per 8-lane group (16 lanes x 4 groups for head_dim 64: 4 lanes x 8 groups), all
+// of width class CLS (warp-uniform): K dot product on the codes, logit, online-softmax
+// update of the group's state, V accumulation. Lanes of invalid entries only take part in
+// the shuffles.
+template <int D, int CLS>
+__device__ __forceinline__ void process_key(KeyState &st, const QRegs &qr, float qsum, float qk_scale,
+                                            const Stage<D> &sg, uint32_t ent, int gl)
+{
+    constexpr int GROUP = D / 16;
+    const bool valid = (ent & kValid) != 0;
+    const uint8_t *r = sg.rec + ((ent >> 9) & 0x7FFFu);
+    float part = 0.f;
+    if (valid) {
+        if (CLS == 0) part = dot_codes2(qr, reinterpret_cast<const uint32_t *>(r)[gl]);
+        else if (CLS == 1) part = dot_codes4(qr, reinterpret_cast<const uint2 *>(r)[gl]);
+        else if (CLS == 2) part = dot_codes8(qr, reinterpret_cast<const uint4 *>(r)[gl]);
+        else part = dot_native(qr, reinterpret_cast<const uint4 *>(r)[2 * gl],
+                               reinterpret_cast<const uint4 *>(r)[2 * gl + 1]);
+    }
+#pragma unroll
+    for (int d = 1; d < GROUP; d <<= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
+    if (!valid) return;
+    const float4 sd = sg.side[ent & 127u];
+    const float dot = (CLS == 3) ? part * kDotNativeUnscale : fmaf(sd.x, part * kDotCodeUnscale, sd.y * qsum);
+    const float lg = dot * qk_scale;
+    if (lg > st.m) {                          // new running max of this key group
+        const float corr = exp2f(st.m - lg);
+        st.l *= corr;
+        st.pz *= corr;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) st.o[k] *= corr;
+        st.m = lg;
+    }
+    const float p = exp2f(lg - st.m);
+    st.l += p;
+    const uint8_t *rv = r + (D * (2 << CLS)) / 8;
+    if (CLS == 3) {
+        acc_native(st.o, p * kONativeScale, reinterpret_cast<const uint4 *>(rv)[2 * gl],
+                   reinterpret_cast<const uint4 *>(rv)[2 * gl + 1]);
+    } else {
+        st.pz = fmaf(p, sd.w, st.pz);
+        const float wv = p * sd.z * kWScale;
+        if (CLS == 0) acc_codes2(st.o, wv, reinterpret_cast<const uint32_t *>(rv)[gl]);
+        else if (CLS == 1) acc_codes4(st.o, wv, reinterpret_cast<const uint2 *>(rv)[gl]);
+        else acc_codes8(st.o, wv, reinterpret_cast<const uint4 *>(rv)[gl]);
+    }
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-decode_splitk_kernel(CacheView c, const __half *__restrict__ q, int w, DecodeWork wk)
+__global__ void __launch_bounds__(kThreads, 2)
+decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
 {
     constexpr int GROUP = D / 16;                 // lanes per key (16 channels per lane)
-    constexpr int KEYS_PER_STEP = 32 / GROUP;     // keys a warp handles at once
-    constexpr int KEYS_PER_WARP = kSub / kConsumerWarps;
-    constexpr int STEPS = KEYS_PER_WARP / KEYS_PER_STEP;
-    static_assert(STEPS * KEYS_PER_STEP == KEYS_PER_WARP, "sub-chunk split");
+    constexpr int KEYS_PER_STEP = 32 / GROUP;     // keys per chunk step of a warp
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     DecodeSmem<D> &sm = *reinterpret_cast<DecodeSmem<D> *>(smem_raw);
@@ -247,255 +358,323 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, int w, DecodeWor
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], kConsumerWarps);
         }
+        for (int i = 0; i < kMetaSlots; ++i) mbar_init(&sm.mfull[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
 
     if (warp == kConsumerWarps) {
         // ------------------------------ producer ---------------------------------
-        if (lane != 0) return;
-        int stage = 0;
+        // A filler cursor runs up to kMetaSlots windows ahead and bulk-copies each window of
+        // 128 record offsets into a shared ring; the record cursor reads a window from shared
+        // memory, cuts it into stages of at most kStageRecBytes, sorts each stage's keys by
+        // width and issues the stage's copies.
+        constexpr int KPL = kWin / 32;                // window keys per lane: lane + 32 r
+        int f_it = blockIdx.x;
+        if (f_it >= n_items) return;
+        DecodeItem f_d = wk.items[f_it];
+        int f_j = f_d.j0;
+        bool f_valid = true;
+        int filled = 0, consumed = 0, stage = 0;
         uint32_t phase = 0;
-        for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-            const int4 item = wk.items[it];
-            const int sh = item.x, s = sh / c.H, h = sh % c.H;
-            const int L = c.len[sh];
-            const int64_t sbase = slot_of(c, s, h, 0);
-            const uint8_t *stream = stream_of(c, s, h);
-            for (int j = item.y; j < item.z; j += kSub) {
-                const int je = min(j + kSub, item.z);
-                if (!mbar_wait(&sm.empty[stage], phase ^ 1u, c.status)) return;
-                const uint32_t off0 = c.meta[sbase + j] & ~15u;
-                const uint32_t off1 = (je < L) ? (c.meta[sbase + je] & ~15u) : c.end[sh];
-                const int ja = j & ~3, jb = (je + 3) & ~3;
-                const uint32_t meta_bytes = 4u * (uint32_t)(jb - ja);
-                const uint32_t side_bytes = 16u * (uint32_t)(je - j);
-                uint32_t rec_bytes = off1 - off0;
-                if (off1 < off0 || rec_bytes > (uint32_t)(kSub * 4 * D)) {   // corrupt offsets
-                    set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+        const uint32_t lt = (1u << lane) - 1u;
+        while (true) {
+            while (f_valid && filled < consumed + kMetaSlots) {
+                const int slot = filled % kMetaSlots;
+                MetaSlot &ms = sm.ms[slot];
+                const int ja = f_j & ~3;
+                const int jb = (min(f_j + kWin + 1, f_d.j1 + 1) + 3) & ~3;
+                if (lane == 0) {
+                    ms.it = f_it;
+                    ms.j = f_j;
+                    ms.j1 = f_d.j1;
+                    ms.ja = ja;
+                    ms.end_off = f_d.end_off;
+                    ms.first = (f_j == f_d.j0);
+                    ms.sbase = f_d.sbase;
+                    ms.sh = f_d.sh;
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    mbar_arrive_expect_tx(&sm.mfull[slot], 4u * (uint32_t)(jb - ja));
+                    bulk_g2s(ms.meta, c.meta + f_d.sbase + ja, 4u * (uint32_t)(jb - ja), &sm.mfull[slot]);
+                }
+                ++filled;
+                f_j += kWin;
+                if (f_j >= f_d.j1) {
+                    f_it += gridDim.x;
+                    if (f_it < n_items) {
+                        f_d = wk.items[f_it];
+                        f_j = f_d.j0;
+                    } else {
+                        f_valid = false;
+                    }
+                }
+            }
+            if (consumed == filled) break;
+            const int slot = consumed % kMetaSlots;
+            if (!mbar_wait(&sm.mfull[slot], (uint32_t)(consumed / kMetaSlots) & 1u, c.status)) return;
+            const MetaSlot &ms = sm.ms[slot];
+            const int j = ms.j, it = ms.it;
+            const int nwin = min(kWin, ms.j1 - j);
+            const bool lastwin = (j + nwin == ms.j1), first = ms.first != 0;
+            const uint32_t *mw = ms.meta + (j - ms.ja);
+            uint32_t m[KPL], nx[KPL];
+#pragma unroll
+            for (int r = 0; r < KPL; ++r) m[r] = (lane + 32 * r < nwin) ? mw[lane + 32 * r] : 0u;
+            const uint32_t bnd = ((!lastwin || ms.end_off == kReadEndFromMeta) ? mw[nwin] : ms.end_off) & ~15u;
+            const int64_t sbase = ms.sbase;
+            const int sh = ms.sh;
+            // nx[r]: offset right after key lane + 32 r (the next key's offset, or the bound)
+#pragma unroll
+            for (int r = 0; r < KPL; ++r) {
+                const uint32_t dn = __shfl_down_sync(0xffffffffu, m[r], 1) & ~15u;
+                const uint32_t wrap = (r + 1 < KPL) ? (__shfl_sync(0xffffffffu, m[(r + 1) % KPL], 0) & ~15u) : bnd;
+                nx[r] = (lane == 31) ? wrap : dn;
+                if (lane + 32 * r + 1 >= nwin) nx[r] = bnd;
+            }
+            ++consumed;
+
+            for (int w0 = 0; w0 < nwin;) {
+                // the stage: keys [w0, w1) of the window, at most kStageRecBytes of records
+                const uint32_t mstart = __shfl_sync(0xffffffffu, (w0 / 32 == 0) ? m[0] : (w0 / 32 == 1) ? m[1 % KPL]
+                                                                   : (w0 / 32 == 2) ? m[2 % KPL] : m[3 % KPL], w0 & 31);
+                const uint32_t off0 = mstart & ~15u;
+                int n = 0;
+#pragma unroll
+                for (int r = 0; r < KPL; ++r) {
+                    const int k = lane + 32 * r;
+                    n += __popc(__ballot_sync(0xffffffffu, k >= w0 && k < nwin && nx[r] - off0 <= kStageRecBytes));
+                }
+                if (n < 1) {          // only with corrupt offsets: flag it, keep making progress
+                    if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+                    n = 1;
+                }
+                const int w1 = w0 + n;
+                const int kl = w1 - 1;
+                const uint32_t nxl = __shfl_sync(0xffffffffu, (kl / 32 == 0) ? nx[0] : (kl / 32 == 1) ? nx[1 % KPL]
+                                                             : (kl / 32 == 2) ? nx[2 % KPL] : nx[3 % KPL], kl & 31);
+                const bool last = lastwin && w1 == nwin;
+                const bool new_item = first && w0 == 0;
+                uint32_t rec_bytes = nxl - off0;
+                if (nxl < off0 || rec_bytes > kStageRecBytes) {   // corrupt offsets
+                    if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
                     rec_bytes = 0;
                 }
+                // counting sort by width, each width's run padded to whole chunks of KEYS_PER_STEP
+                constexpr int PADL = KEYS_PER_STEP - 1;       // pad entries per width, at most
+                int cl_of[KPL], pos_of[KPL];
+#pragma unroll
+                for (int r = 0; r < KPL; ++r) {
+                    const int k = lane + 32 * r;
+                    cl_of[r] = (k >= w0 && k < w1) ? (int)(m[r] & 3u) : 4;
+                    pos_of[r] = 0;
+                }
+                int pstart = 0, pad_cls = -1, pad_pos = 0;
+#pragma unroll
+                for (int cl = 0; cl < 4; ++cl) {
+                    int before = 0;
+#pragma unroll
+                    for (int r = 0; r < KPL; ++r) {
+                        const uint32_t b = __ballot_sync(0xffffffffu, cl_of[r] == cl);
+                        if (cl_of[r] == cl) pos_of[r] = pstart + before + __popc(b & lt);
+                        before += __popc(b);
+                    }
+                    const int padded = (before + PADL) / KEYS_PER_STEP * KEYS_PER_STEP;
+                    if (lane / PADL == cl && before + lane % PADL < padded) {   // PADL lanes per width
+                        pad_cls = cl;
+                        pad_pos = pstart + before + lane % PADL;
+                    }
+                    pstart += padded;
+                }
+
+                if (!mbar_wait(&sm.empty[stage], phase ^ 1u, c.status)) return;
                 Stage<D> &sg = sm.st[stage];
-                mbar_arrive_expect_tx(&sm.full[stage], meta_bytes + side_bytes + rec_bytes);
-                bulk_g2s(sg.meta, c.meta + sbase + ja, meta_bytes, &sm.full[stage]);
-                bulk_g2s(sg.side, c.side + sbase + j, side_bytes, &sm.full[stage]);
-                if (rec_bytes) bulk_g2s(sg.rec, stream + off0, rec_bytes, &sm.full[stage]);
+#pragma unroll
+                for (int r = 0; r < KPL; ++r) {
+                    if (cl_of[r] < 4) {
+                        // offset inside the stage; the clamp only bites on corrupt offsets and
+                        // keeps every shared-memory read of the consumers inside the stage
+                        const uint32_t ro = min((m[r] & ~15u) - off0,
+                                                kStageRecBytes - (uint32_t)(D * (2 << cl_of[r])) / 4u);
+                        sg.perm[pos_of[r]] = kValid | (ro << 9) | ((uint32_t)cl_of[r] << 7) |
+                                             (uint32_t)(lane + 32 * r - w0);
+                    }
+                }
+                if (pad_cls >= 0) sg.perm[pad_pos] = (uint32_t)pad_cls << 7;
+                if (lane == 0) {
+                    sg.info[0] = it;
+                    sg.info[1] = n;
+                    sg.info[2] = (new_item ? kNewItem : 0) | (last ? kLastSub : 0);
+                    sg.info[3] = pstart / KEYS_PER_STEP;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    const uint32_t q_bytes = new_item ? 2u * D : 0u;
+                    mbar_arrive_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
+                    bulk_g2s(sg.side, c.side + sbase + j + w0, 16u * n, &sm.full[stage]);
+                    if (rec_bytes)
+                        bulk_g2s(sg.rec, c.rec + sbase * (int64_t)(4 * D) + off0, rec_bytes, &sm.full[stage]);
+                    if (q_bytes) bulk_g2s(sg.q, q + (int64_t)sh * D, q_bytes, &sm.full[stage]);
+                }
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1u;
                 }
+                w0 = w1;
             }
         }
         return;
     }
 
     // -------------------------------- consumers -------------------------------------
-    const int g = lane / GROUP;          // key slot within a step
+    const int g = lane / GROUP;          // key slot within a chunk step
     const int gl = lane % GROUP;         // channel block: channels [16 gl, 16 gl + 16)
     const float qk_scale = kLog2e * rsqrtf((float)D);   // logits in log2 units
-    int stage = 0;
+    int stage = 0, rot = 0;
     uint32_t phase = 0;
+    QRegs qr;
+    float qsum = 0.f;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-        const int4 item = wk.items[it];
-        const int sh = item.x;
-
-        // query: this lane's 16 channels, scaled per width; sum(q) over all D
-        QRegs qr;
-        float qsum = 0.f;
-        {
-            const uint4 *qp = reinterpret_cast<const uint4 *>(q + (int64_t)sh * D + 16 * gl);
-            const uint4 a = qp[0], bq = qp[1];
-            const uint32_t hw[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+        KeyState ks;
+        ks.m = -INFINITY;
+        ks.l = 0.f;
+        ks.pz = 0.f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hw[e]));
-                const float fv[2] = {f.x, f.y};
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int k = 2 * e + u;
-                    qsum += fv[u];
-                    qr.q8[k] = fv[u] * kQScale;
-                    qr.q4[k] = qr.q8[k] * __uint_as_float((127u - 4u * (k % 4)) << 23);
-                    qr.q2[k] = qr.q8[k] * __uint_as_float((127u - 2u * (k % 8)) << 23);
-                }
-            }
-#pragma unroll
-            for (int d = 1; d < GROUP; d <<= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, d);
-        }
-
-        float m_run = -INFINITY, l_run = 0.f, pz_run = 0.f;
-        float o[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) o[k] = 0.f;
-
-        for (int j = item.y; j < item.z; j += kSub) {
-            const int n = min(kSub, item.z - j);
+        for (int k = 0; k < 16; ++k) ks.o[k] = 0.f;
+        bool last = false;
+        while (!last) {
             if (!mbar_wait(&sm.full[stage], phase, c.status)) return;
             Stage<D> &sg = sm.st[stage];
-            const int mo = j & 3;                      // meta copy starts at j & ~3
-            const uint32_t off0 = sg.meta[mo] & ~15u;
-
-            // order the stage's keys by width (warp-redundant counting sort via ballots)
-            {
-                const int k0 = lane, k1 = lane + 32;
-                const int c0 = (k0 < n) ? (int)(sg.meta[mo + k0] & 3u) : 4;
-                const int c1 = (k1 < n) ? (int)(sg.meta[mo + k1] & 3u) : 4;
-                const uint32_t lt = (1u << lane) - 1u;
-                int base = 0, p0 = 0, p1 = 0;
+            const int flags = sg.info[2];
+            const int n_chunks = sg.info[3];
+            last = (flags & kLastSub) != 0;
+            if (flags & kNewItem) {
+                // query: this lane's 16 channels, scaled per width; sum(q) over all D
+                const uint4 a = reinterpret_cast<const uint4 *>(sg.q + 16 * gl)[0];
+                const uint4 bq = reinterpret_cast<const uint4 *>(sg.q + 16 * gl)[1];
+                const uint32_t hw[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+                qsum = 0.f;
 #pragma unroll
-                for (int cl = 0; cl < 4; ++cl) {
-                    const uint32_t b0 = __ballot_sync(0xffffffffu, c0 == cl);
-                    const uint32_t b1 = __ballot_sync(0xffffffffu, c1 == cl);
-                    if (c0 == cl) p0 = base + __popc(b0 & lt);
-                    if (c1 == cl) p1 = base + __popc(b0) + __popc(b1 & lt);
-                    base += __popc(b0) + __popc(b1);
-                }
-                if (k0 < n) sm.perm[warp][p0] = (uint8_t)k0;
-                if (k1 < n) sm.perm[warp][p1] = (uint8_t)k1;
-                __syncwarp();
-            }
-
-            // K pass: logits of this warp's keys
+                for (int e = 0; e < 8; ++e) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hw[e]));
+                    const float fv[2] = {f.x, f.y};
 #pragma unroll
-            for (int stp = 0; stp < STEPS; ++stp) {
-                const int pos = warp * KEYS_PER_WARP + stp * KEYS_PER_STEP + g;
-                float part = 0.f;
-                int key = -1;
-                int cls = 0;
-                if (pos < n) {
-                    key = sm.perm[warp][pos];
-                    const uint32_t mt = sg.meta[mo + key];
-                    cls = mt & 3u;
-                    const uint8_t *r = sg.rec + ((mt & ~15u) - off0);
-                    if (cls == 0) part = dot_codes2(qr, reinterpret_cast<const uint32_t *>(r)[gl]);
-                    else if (cls == 1) part = dot_codes4(qr, reinterpret_cast<const uint2 *>(r)[gl]);
-                    else if (cls == 2) part = dot_codes8(qr, reinterpret_cast<const uint4 *>(r)[gl]);
-                    else part = dot_native(qr, reinterpret_cast<const uint4 *>(r)[2 * gl],
-                                           reinterpret_cast<const uint4 *>(r)[2 * gl + 1]);
-                }
-#pragma unroll
-                for (int d = 1; d < GROUP; d <<= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
-                if (key >= 0 && gl == 0) {
-                    const float4 sd = sg.side[key];
-                    float dot;
-                    if (cls == 3) dot = part * kDotNativeUnscale;
-                    else dot = fmaf(sd.x, part * kDotCodeUnscale, sd.y * qsum);
-                    sm.logit[stage][key] = dot * qk_scale;
-                }
-            }
-            named_bar_sync(1, 32 * kConsumerWarps);
-
-            // softmax over the stage (every warp redundantly, so no second barrier)
-            const float l0 = (lane < n) ? sm.logit[stage][lane] : -INFINITY;
-            const float l1 = (lane + 32 < n) ? sm.logit[stage][lane + 32] : -INFINITY;
-            float cmax = fmaxf(l0, l1);
-#pragma unroll
-            for (int d = 16; d >= 1; d >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, d));
-            const float m_new = fmaxf(m_run, cmax);
-            const float corr = exp2f(m_run - m_new);
-            const float p0 = (lane < n) ? exp2f(l0 - m_new) : 0.f;
-            const float p1 = (lane + 32 < n) ? exp2f(l1 - m_new) : 0.f;
-            float psum = p0 + p1;
-            float pz = 0.f;
-            if (lane < n && (sg.meta[mo + lane] & 3u) != 3u) pz = p0 * sg.side[lane].w;
-            if (lane + 32 < n && (sg.meta[mo + lane + 32] & 3u) != 3u) pz = fmaf(p1, sg.side[lane + 32].w, pz);
-#pragma unroll
-            for (int d = 16; d >= 1; d >>= 1) {
-                psum += __shfl_xor_sync(0xffffffffu, psum, d);
-                pz += __shfl_xor_sync(0xffffffffu, pz, d);
-            }
-            l_run = fmaf(l_run, corr, psum);
-            pz_run = fmaf(pz_run, corr, pz);
-            m_run = m_new;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] *= corr;
-
-            // V pass
-#pragma unroll
-            for (int stp = 0; stp < STEPS; ++stp) {
-                const int pos = warp * KEYS_PER_WARP + stp * KEYS_PER_STEP + g;
-                const int key = (pos < n) ? sm.perm[warp][pos] : 0;
-                const float pa = __shfl_sync(0xffffffffu, p0, key & 31);
-                const float pb = __shfl_sync(0xffffffffu, p1, key & 31);
-                if (pos < n) {
-                    const float p = (key < 32) ? pa : pb;
-                    const uint32_t mt = sg.meta[mo + key];
-                    const int cls = mt & 3u;
-                    const uint8_t *r = sg.rec + ((mt & ~15u) - off0) + (D * (2 << cls)) / 8;
-                    if (cls == 3) {
-                        acc_native(o, p * kONativeScale, reinterpret_cast<const uint4 *>(r)[2 * gl],
-                                   reinterpret_cast<const uint4 *>(r)[2 * gl + 1]);
-                    } else {
-                        const float wv = p * sg.side[key].z * kWScale;
-                        if (cls == 0) acc_codes2(o, wv, reinterpret_cast<const uint32_t *>(r)[gl]);
-                        else if (cls == 1) acc_codes4(o, wv, reinterpret_cast<const uint2 *>(r)[gl]);
-                        else acc_codes8(o, wv, reinterpret_cast<const uint4 *>(r)[gl]);
+                    for (int u = 0; u < 2; ++u) {
+                        const int k = 2 * e + u;
+                        qsum += fv[u];
+                        qr.q8[k] = fv[u] * kQScale;
+                        qr.q4[k] = qr.q8[k] * __uint_as_float((127u - 4u * (k % 4)) << 23);
+                        qr.q2[k] = qr.q8[k] * __uint_as_float((127u - 2u * (k % 8)) << 23);
                     }
                 }
+#pragma unroll
+                for (int d = 1; d < GROUP; d <<= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, d);
+            }
+            // class-pure chunks, dealt to the warps round-robin (rotated every stage)
+            for (int ch = (warp + kConsumerWarps - rot) % kConsumerWarps; ch < n_chunks; ch += kConsumerWarps) {
+                const uint32_t ent = sg.perm[KEYS_PER_STEP * ch + g];
+                const int cls = (ent >> 7) & 3u;           // the same for the whole chunk
+                if (cls == 0) process_key<D, 0>(ks, qr, qsum, qk_scale, sg, ent, gl);
+                else if (cls == 1) process_key<D, 1>(ks, qr, qsum, qk_scale, sg, ent, gl);
+                else if (cls == 2) process_key<D, 2>(ks, qr, qsum, qk_scale, sg, ent, gl);
+                else process_key<D, 3>(ks, qr, qsum, qk_scale, sg, ent, gl);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);
+            rot = (rot + 1) % kConsumerWarps;
             if (++stage == kStages) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
 
-        // reduce o over the key slots of the warp, then over the consumer warps
+        // merge the key groups of the warp, then the warps, into the item's partial
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-#pragma unroll
-            for (int d = GROUP; d < 32; d <<= 1) o[k] += __shfl_xor_sync(0xffffffffu, o[k], d);
-        }
+        for (int mask = GROUP; mask < 32; mask <<= 1) merge_state(ks.m, ks.l, ks.pz, ks.o, mask);
         if (g == 0) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) sm.red[warp][16 * gl + k] = o[k];
+            for (int k = 0; k < 16; ++k) sm.red_o[warp][16 * gl + k] = ks.o[k];
+            if (gl == 0) {
+                sm.red_m[warp] = ks.m;
+                sm.red_l[warp] = ks.l;
+                sm.red_pz[warp] = ks.pz;
+            }
         }
         named_bar_sync(1, 32 * kConsumerWarps);
-        float *part = wk.partials + (int64_t)it * (D + 4);
-        for (int ch = tid; ch < D; ch += 32 * kConsumerWarps) {
-            float acc = 0.f;
+        if (warp == 0) {
+            float M = -INFINITY;
 #pragma unroll
-            for (int wv = 0; wv < kConsumerWarps; ++wv) acc += sm.red[wv][ch];
-            part[4 + ch] = fmaf(acc, kOUnscale, pz_run);
+            for (int wv = 0; wv < kConsumerWarps; ++wv) M = fmaxf(M, sm.red_m[wv]);
+            float f[kConsumerWarps];
+            float L = 0.f, PZ = 0.f;
+#pragma unroll
+            for (int wv = 0; wv < kConsumerWarps; ++wv) {
+                f[wv] = (sm.red_m[wv] == -INFINITY) ? 0.f : exp2f(sm.red_m[wv] - M);
+                L = fmaf(sm.red_l[wv], f[wv], L);
+                PZ = fmaf(sm.red_pz[wv], f[wv], PZ);
+            }
+            float *part = wk.partials + (int64_t)it * (D + 4);
+            for (int chn = lane; chn < D; chn += 32) {
+                float acc = 0.f;
+#pragma unroll
+                for (int wv = 0; wv < kConsumerWarps; ++wv) acc = fmaf(sm.red_o[wv][chn], f[wv], acc);
+                part[4 + chn] = fmaf(acc, kOUnscale, PZ);
+            }
+            if (lane == 0) {
+                part[0] = M;
+                part[1] = L;
+            }
         }
-        if (tid == 0) {
-            part[0] = m_run;
-            part[1] = l_run;
-        }
-        named_bar_sync(1, 32 * kConsumerWarps);   // red[] is reused by the next item
+        named_bar_sync(1, 32 * kConsumerWarps);   // red_* are reused by the next item
     }
 }
 
+// One CTA of D threads per (sequence, head): thread = channel.
 template <int D>
-__global__ void decode_combine_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
+__global__ void __launch_bounds__(D)
+decode_combine_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
 {
-    constexpr int PER_LANE = D / 32;
-    const int lane = threadIdx.x & 31;
-    const int sh = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (sh >= c.B * c.H) return;
+    __shared__ float red[D / 32];
+    const int sh = blockIdx.x, ch = threadIdx.x, lane = ch & 31, wid = ch >> 5;
     const int first = wk.head_first[sh], cnt = wk.head_cnt[sh];
-    float acc[PER_LANE];
-#pragma unroll
-    for (int e = 0; e < PER_LANE; ++e) acc[e] = 0.f;
+    const float *P = wk.partials + (int64_t)first * (D + 4);
+    float res = 0.f;
     if (cnt > 0) {
         float M = -INFINITY;
-        for (int i = 0; i < cnt; ++i) M = fmaxf(M, wk.partials[(int64_t)(first + i) * (D + 4)]);
-        float L = 0.f;
-        for (int i = 0; i < cnt; ++i) {
-            const float *p = wk.partials + (int64_t)(first + i) * (D + 4);
+        for (int i = ch; i < cnt; i += D) M = fmaxf(M, P[(int64_t)i * (D + 4)]);
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+        if (lane == 0) red[wid] = M;
+        __syncthreads();
+        M = red[0];
+#pragma unroll
+        for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
+        float L = 0.f, acc = 0.f;
+        int i = 0;
+        for (; i + 4 <= cnt; i += 4) {
+            float mm[4], ll[4], oo[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float *p = P + (int64_t)(i + u) * (D + 4);
+                mm[u] = p[0];
+                ll[u] = p[1];
+                oo[u] = p[4 + ch];
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float f = exp2f(mm[u] - M);
+                L = fmaf(ll[u], f, L);
+                acc = fmaf(oo[u], f, acc);
+            }
+        }
+        for (; i < cnt; ++i) {
+            const float *p = P + (int64_t)i * (D + 4);
             const float f = exp2f(p[0] - M);
             L = fmaf(p[1], f, L);
-#pragma unroll
-            for (int e = 0; e < PER_LANE; ++e) acc[e] = fmaf(p[4 + lane + 32 * e], f, acc[e]);
+            acc = fmaf(p[4 + ch], f, acc);
         }
-        const float inv = 1.0f / L;
-#pragma unroll
-        for (int e = 0; e < PER_LANE; ++e) acc[e] *= inv;
+        res = acc / L;
     }
-    float *o = out + (int64_t)sh * D;
-#pragma unroll
-    for (int e = 0; e < PER_LANE; ++e) o[lane + 32 * e] = acc[e];
+    out[(int64_t)sh * D + ch] = res;
 }
 
 template <int D>
@@ -512,12 +691,11 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const __half *q, const uint8
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    const int grid = (int)std::min<int64_t>(cache->work.max_items, (int64_t)num_sms());
+    const int grid = (int)std::min<int64_t>(cache->work.max_items, 2 * (int64_t)num_sms());
     profile_before(st);
-    decode_splitk_kernel<D><<<grid, kThreads, smem, st>>>(c, q, w, cache->work);
+    decode_splitk_kernel<D><<<grid, kThreads, smem, st>>>(c, q, cache->work);
     profile_after(st);
-    const int BH = c.B * c.H;
-    decode_combine_kernel<D><<<(BH * 32 + 255) / 256, 256, 0, st>>>(c, cache->work, out);
+    decode_combine_kernel<D><<<c.B * c.H, D, 0, st>>>(c, cache->work, out);
     return cudaGetLastError();
 }
 

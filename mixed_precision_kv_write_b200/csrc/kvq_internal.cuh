@@ -33,6 +33,8 @@ struct CacheView {
     int32_t *len;             // [B*H]
     uint32_t *end;            // [B*H]
     int32_t *wstart;          // [B*H] start position of the current write, -1 = rejected
+    uint32_t *wend;           // [B*H] stream end after the current write
+    uint32_t *bad;            // [B] id of the last write call that saw a bad width
     int32_t *status;          // [1] first device-side error (kvq_status), 0 = none
 };
 
@@ -60,10 +62,17 @@ __device__ __forceinline__ void set_status(int32_t *status, int code)
 
 // ---- scheduler work list (decode) ----------------------------------------------------
 constexpr int kDecodeItemKeys = 512;   // keys per split-K work item
-constexpr int kDecodeSubKeys = 64;     // keys per pipeline stage inside an item
+constexpr int kDecodeWindowKeys = 128; // keys per window of record offsets inside an item
+
+struct __align__(16) DecodeItem {
+    int32_t sh, j0, j1;  // (sequence, head) and key range [j0, j1)
+    uint32_t end_off;    // byte offset of key j1 in the stream (the stream end if j1 = len)
+    int64_t sbase;       // slot of key 0 of (sequence, head)
+    int64_t pad;
+};
 
 struct DecodeWork {
-    int4 *items;         // [max_items] (s*H + h, j0, j1, 0)
+    DecodeItem *items;   // [max_items]
     int32_t *count;      // [1]
     int32_t *head_first; // [B*H]
     int32_t *head_cnt;   // [B*H]
@@ -157,12 +166,13 @@ struct kvq_cache {
     int32_t max_cap;
     kvq::CacheView view;
     kvq::DecodeWork work;
-    void *allocs[16];
+    uint32_t write_gen;       // id of the last kvq_write call
+    void *allocs[24];
     int n_allocs;
 };
 
 namespace kvq {
-cudaError_t launch_write(const kvq_cache *c, const __half *k, const __half *v, const uint8_t *bits,
+cudaError_t launch_write(kvq_cache *c, const __half *k, const __half *v, const uint8_t *bits,
                          const int32_t *cu, int64_t n_tok, cudaStream_t st);
 cudaError_t launch_decode(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,
                           float *out, cudaStream_t st);

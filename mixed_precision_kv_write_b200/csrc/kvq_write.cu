@@ -1,32 +1,44 @@
 // Quantize-on-write (TriRoute paper review page, section 3, Eq. 4).
 //
 // Two launches per kvq_write call:
-//   write_scan_kernel   one warp per (sequence, head): validates capacity and widths (a
-//                       bad width rejects the sequence's write for every head),
-//                       assigns each new token's record offset (prefix sum of record
-//                       sizes b*D/4 in token order) and advances the stream's length/end.
+//   write_scan_kernel   a warp (short appends) or a block (long ones) per (sequence, head):
+//                       validates capacity and widths (a bad width rejects the sequence's
+//                       write for every head) and assigns each new token's record offset
+//                       (prefix sum of record sizes b*D/4 in token order).
 //   write_quant_kernel  one warp per (token, head): for K and for V, min/max over the
 //                       head_dim values, s = (max - min)/(2^b - 1), z = min, codes
 //                       rint((x - z)/s) in IEEE fp32 round-to-nearest-even (s == 0 -> 0),
-//                       packed LSB-first into the record; (s, z) into the side table.
+//                       packed LSB-first into the record; (s, z) into the side table;
+//                       commits the new length and stream end of accepted sequences.
 // HBM traffic per (token, head): reads 2*D*2 bytes, writes b*D/4 + 16 + 4 bytes.
 #include "kvq_internal.cuh"
 
 namespace kvq {
 namespace {
 
-__global__ void write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits,
-                                  const int32_t *__restrict__ cu, int64_t n_tok)
+// TPS threads per (sequence, head): validates the call's widths of its head (a bad entry
+// marks the sequence bad for this call, so no head of it is written), checks capacity,
+// and assigns the new tokens' record offsets with a parallel prefix sum of the record
+// sizes b*D/4. The new length/end are committed by the quantize kernel, which sees the
+// per-sequence verdict of every head.
+template <int TPS>
+__global__ void __launch_bounds__(256)
+write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *__restrict__ cu,
+                  int64_t n_tok, uint32_t gen)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    constexpr int PER = 8;                       // tokens per thread per pass
+    constexpr int WARPS = TPS / 32;
+    __shared__ uint32_t wsum[256 / 32];
+    const int tid = threadIdx.x % TPS, lane = threadIdx.x & 31;
+    const int grp = threadIdx.x / TPS, wig = tid >> 5;     // group in block, warp in group
+    const int64_t gsh = (int64_t)blockIdx.x * (256 / TPS) + grp;
     const int H = c.H;
-    if (warp >= (int64_t)c.B * H) return;
-    const int s = (int)(warp / H), h = (int)(warp % H), sh = s * H + h;
+    if (gsh >= (int64_t)c.B * H) return;         // whole group exits together
+    const int s = (int)(gsh / H), h = (int)(gsh % H), sh = s * H + h;
 
     const int64_t t0 = cu[s], t1 = cu[s + 1];
     if (t0 < 0 || t1 < t0 || t1 > n_tok || (s == 0 && t0 != 0)) {
-        if (lane == 0) {
+        if (tid == 0) {
             set_status(c.status, KVQ_ERR_DEVICE_CHECK);
             c.wstart[sh] = -1;
         }
@@ -35,49 +47,74 @@ __global__ void write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits,
     const int n = (int)(t1 - t0);
     const int L0 = c.len[sh];
     if ((int64_t)L0 + n > c.cap[s]) {
-        if (lane == 0) {
+        if (tid == 0) {
             set_status(c.status, KVQ_ERR_CAPACITY);
-            c.wstart[sh] = -1;
-        }
-        return;
-    }
-    // every head of the sequence validates all of the sequence's new widths, so an invalid
-    // entry rejects the sequence's write for all heads alike (lengths stay equal)
-    bool bad = false;
-    for (int64_t e = (int64_t)t0 * H + lane; e < (int64_t)t1 * H; e += 32)
-        bad |= width_code(bits[e]) < 0;
-    bad = __any_sync(0xffffffffu, bad);
-    if (bad) {
-        if (lane == 0) {
-            set_status(c.status, KVQ_ERR_BITS);
             c.wstart[sh] = -1;
         }
         return;
     }
     const int64_t slot0 = slot_of(c, s, h, L0);
     uint32_t off = c.end[sh];
-    for (int i0 = 0; i0 < n; i0 += 32) {
-        const int i = i0 + lane;
-        uint32_t size = 0;
-        int wc = 0;
-        if (i < n) {
-            const int b = bits[(t0 + i) * H + h];
-            wc = width_code(b);
-            size = (uint32_t)(b * c.D / 4);
+    bool bad = false;
+    for (int base = 0; base < n; base += TPS * PER) {
+        uint32_t sz[PER];
+        uint32_t wcs[PER];
+        uint32_t mine = 0;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int i = base + tid * PER + e;
+            sz[e] = 0;
+            wcs[e] = 0;
+            if (i < n) {
+                const int b = bits[(t0 + i) * H + h];
+                const int wc = width_code(b);
+                if (wc < 0) bad = true;
+                else {
+                    wcs[e] = (uint32_t)wc;
+                    sz[e] = (uint32_t)(b * c.D / 4);
+                }
+            }
+            mine += sz[e];
         }
-        uint32_t incl = size;
+        uint32_t incl = mine;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
             if (lane >= d) incl += y;
         }
-        if (i < n) c.meta[slot0 + i] = (off + incl - size) | (uint32_t)wc;
-        off += __shfl_sync(0xffffffffu, incl, 31);
+        uint32_t before = incl - mine, total;
+        if (WARPS > 1) {
+            if (lane == 31) wsum[grp * WARPS + wig] = incl;
+            __syncthreads();
+            uint32_t wpre = 0, wtot = 0;
+#pragma unroll
+            for (int q = 0; q < WARPS; ++q) {
+                const uint32_t t = wsum[grp * WARPS + q];
+                if (q < wig) wpre += t;
+                wtot += t;
+            }
+            __syncthreads();
+            before += wpre;
+            total = wtot;
+        } else {
+            total = __shfl_sync(0xffffffffu, incl, 31);
+        }
+        uint32_t o = off + before;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int i = base + tid * PER + e;
+            if (i < n) c.meta[slot0 + i] = o | wcs[e];
+            o += sz[e];
+        }
+        off += total;
     }
-    if (lane == 0) {
+    if (bad) {
+        c.bad[s] = gen;                          // same value from every writer
+        set_status(c.status, KVQ_ERR_BITS);
+    }
+    if (tid == 0) {
         c.wstart[sh] = L0;
-        c.len[sh] = L0 + n;
-        c.end[sh] = off;
+        c.wend[sh] = off;
     }
 }
 
@@ -86,7 +123,7 @@ __global__ void write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits,
 template <int D>
 __global__ void write_quant_kernel(CacheView c, const __half *__restrict__ k,
                                    const __half *__restrict__ v, const uint8_t *__restrict__ bits,
-                                   const int32_t *__restrict__ cu, int64_t n_tok)
+                                   const int32_t *__restrict__ cu, int64_t n_tok, uint32_t gen)
 {
     constexpr int VL = D / 4;            // lanes per vector
     constexpr int PER_ITER = 32 / VL;    // vectors per warp iteration
@@ -108,7 +145,11 @@ __global__ void write_quant_kernel(CacheView c, const __half *__restrict__ k,
     const int s = lo;
     if (tk >= cu[s + 1]) return;     // cu_seqlens violated its contract (flagged by the scan)
     const int start = c.wstart[s * H + h];
-    if (start < 0) return;           // this sequence's write was rejected
+    if (start < 0 || c.bad[s] == gen) return;     // this sequence's write was rejected
+    if (tk == cu[s] && lane == 0) {               // commit the new length and stream end
+        c.len[s * H + h] = start + (cu[s + 1] - cu[s]);
+        c.end[s * H + h] = c.wend[s * H + h];
+    }
     const int64_t j = start + (tk - cu[s]);
     const int64_t slot = slot_of(c, s, h, j);
     const uint32_t meta = c.meta[slot];
@@ -178,27 +219,32 @@ __global__ void write_quant_kernel(CacheView c, const __half *__restrict__ k,
 
 } // namespace
 
-cudaError_t launch_write(const kvq_cache *cache, const __half *k, const __half *v,
+cudaError_t launch_write(kvq_cache *cache, const __half *k, const __half *v,
                          const uint8_t *bits, const int32_t *cu, int64_t n_tok, cudaStream_t st)
 {
     const CacheView &c = cache->view;
+    const uint32_t gen = ++cache->write_gen;
+    profile_before(st);
     {
-        const int64_t warps = (int64_t)c.B * c.H;
-        const int threads = 128;
-        const int64_t blocks = (warps * 32 + threads - 1) / threads;
-        write_scan_kernel<<<(unsigned)blocks, threads, 0, st>>>(c, bits, cu, n_tok);
+        const int64_t groups = (int64_t)c.B * c.H;
+        // a warp per (sequence, head) for short appends (decode steps), a block for long ones
+        if (n_tok <= 64 * (int64_t)c.B) {
+            const int64_t blocks = (groups + 7) / 8;
+            write_scan_kernel<32><<<(unsigned)blocks, 256, 0, st>>>(c, bits, cu, n_tok, gen);
+        } else {
+            write_scan_kernel<256><<<(unsigned)groups, 256, 0, st>>>(c, bits, cu, n_tok, gen);
+        }
     }
     if (n_tok > 0) {
         const int64_t warps = n_tok * c.H;
         const int threads = 256;
         const int64_t blocks = (warps * 32 + threads - 1) / threads;
-        profile_before(st);
         if (c.D == 128)
-            write_quant_kernel<128><<<(unsigned)blocks, threads, 0, st>>>(c, k, v, bits, cu, n_tok);
+            write_quant_kernel<128><<<(unsigned)blocks, threads, 0, st>>>(c, k, v, bits, cu, n_tok, gen);
         else
-            write_quant_kernel<64><<<(unsigned)blocks, threads, 0, st>>>(c, k, v, bits, cu, n_tok);
-        profile_after(st);
+            write_quant_kernel<64><<<(unsigned)blocks, threads, 0, st>>>(c, k, v, bits, cu, n_tok, gen);
     }
+    profile_after(st);
     return cudaGetLastError();
 }
 
