@@ -135,6 +135,28 @@ int routed_attn_decode(const void *q, const kvq_cache *cache, const uint8_t *mod
                        float *out, kvq_stream_t stream);
 
 /*
+ * Allocation-free variant of routed_attn_decode (no counterpart in the paper).
+ * Same arguments, same arithmetic and the same kernels, but the per-call scratch (the
+ * scheduler's work list and the split-K partials) lives in a 16 MiB array in the library's
+ * static device memory instead of the cache's workspace, and the call allocates nothing:
+ * no cudaMalloc or cudaFree. It is meant for callers that cannot allocate device memory at
+ * the point of the call: code whose allocations are owned by a host framework's own pool,
+ * code that must not trigger the implicit synchronization of an allocation, or code
+ * running where allocation is not permitted.
+ *   - Every GPU that loads the library holds the 16 MiB array until the process exits.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents (nothing in it
+ *     needs clearing: each call rewrites its work list). Calls that overlap on the GPU, from
+ *     any stream or thread, race on it: order them.
+ *   - A cache whose worst case (every head full at capacity) needs more scratch than the
+ *     array holds is rejected with KVQ_ERR_ARG before anything is launched; use
+ *     routed_attn_decode for it.
+ */
+int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache, const uint8_t *modes, int w,
+                               float *out, kvq_stream_t stream);
+
+/*
  * Read back stored records of one (sequence, head) for tokens first .. first+count-1
  * (all below the current length; checked on the device).
  *   k_codes, v_codes: uint16 [count][head_dim]: codes (b < 16) or raw fp16 bits (b = 16).

@@ -118,6 +118,12 @@ void profile_after(cudaStream_t st)
     if (g_prof_after) cudaEventRecord(g_prof_after, st);
 }
 
+int report_error(int code, const char *msg)
+{
+    if (code == KVQ_OK) return ok();
+    return fail(code, "%s", msg);
+}
+
 int num_sms()
 {
     static int n = 0;

@@ -29,6 +29,9 @@
 // folded into the other operand (q for K, the softmax weight for V), which keeps the
 // unpack at one LOP3 per code. fp32 subnormals must not be flushed: build without
 // -ftz / fast-math.
+#include <cstdio>
+#include <mutex>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -709,3 +712,106 @@ cudaError_t launch_decode(const kvq_cache *cache, const __half *q, const uint8_t
 }
 
 } // namespace kvq
+
+// ---- allocation-free decode -------------------------------------------------------------
+// routed_attn_decode_noalloc runs the same three kernels as routed_attn_decode, but its
+// per-call scratch (the scheduler's work list and the split-K partials) lives in the
+// file-scope array below instead of the cache's workspace, and the call allocates
+// nothing. Host code must never hand `g_decode_scratch` itself to a kernel: on the host
+// that name is only a stand-in. The device address is looked up once per device, with that
+// device current, by cudaGetSymbolAddress.
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB on every device
+}
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+namespace kvq {
+namespace {
+
+std::mutex g_scratch_mu;
+void *g_scratch_addr[256] = {};   // device address of g_decode_scratch, per device ordinal
+
+cudaError_t static_scratch(int dev, unsigned char **out)
+{
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = p;
+    }
+    *out = static_cast<unsigned char *>(g_scratch_addr[dev]);
+    return cudaSuccess;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <int D>
+cudaError_t launch_decode_static(const kvq_cache *cache, const DecodeWork &wk, const __half *q,
+                                 const uint8_t *modes, int w, float *out, cudaStream_t st)
+{
+    const CacheView &c = cache->view;
+    decode_sched_kernel<<<1, 1024, 0, st>>>(c, modes, w, wk);
+    const size_t smem = sizeof(DecodeSmem<D>);
+    cudaError_t e = cudaFuncSetAttribute(decode_splitk_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(wk.max_items, 2 * (int64_t)num_sms());
+    decode_splitk_kernel<D><<<grid, kThreads, smem, st>>>(c, q, wk);
+    decode_combine_kernel<D><<<c.B * c.H, D, 0, st>>>(c, wk, out);
+    return cudaGetLastError();
+}
+
+} // namespace
+} // namespace kvq
+
+extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache, const uint8_t *modes,
+                                          int w, float *out, kvq_stream_t stream)
+{
+    using namespace kvq;
+    if (!cache || cache->B <= 0 || cache->H <= 0)
+        return report_error(KVQ_ERR_ARG, "routed_attn_decode_noalloc: bad cache");
+    if (w < 0) return report_error(KVQ_ERR_ARG, "routed_attn_decode_noalloc: w < 0");
+    if (!q || !modes || !out) return report_error(KVQ_ERR_ARG, "routed_attn_decode_noalloc: q, modes or out is NULL");
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15u)
+        return report_error(KVQ_ERR_ARG, "routed_attn_decode_noalloc: q and out must be 16-byte aligned");
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return report_error(KVQ_ERR_CUDA, "routed_attn_decode_noalloc: cudaGetDevice failed");
+    if (dev != cache->device)
+        return report_error(KVQ_ERR_ARG, "routed_attn_decode_noalloc: the cache's device is not the current device");
+
+    // scratch layout: count | head_first | head_cnt | items | partials, each 256-byte aligned,
+    // sized for the cache's worst case (every head full at capacity)
+    const int BH = cache->B * cache->H;
+    const int64_t items = cache->work.max_items;
+    const size_t o_first = 256;
+    const size_t o_cnt = o_first + align256(sizeof(int32_t) * (size_t)BH);
+    const size_t o_items = o_cnt + align256(sizeof(int32_t) * (size_t)BH);
+    const size_t o_part = o_items + align256(sizeof(DecodeItem) * (size_t)items);
+    const size_t need = o_part + sizeof(float) * (size_t)items * (cache->D + 4);
+    if (need > kStaticScratchBytes) {
+        char msg[256];
+        snprintf(msg, sizeof(msg),
+                 "routed_attn_decode_noalloc: this cache needs %zu bytes of scratch, more than the %zu "
+                 "bytes of static scratch; use routed_attn_decode",
+                 need, kStaticScratchBytes);
+        return report_error(KVQ_ERR_ARG, msg);
+    }
+    unsigned char *base = nullptr;
+    e = static_scratch(dev, &base);
+    if (e != cudaSuccess) return report_error(KVQ_ERR_CUDA, "routed_attn_decode_noalloc: cudaGetSymbolAddress failed");
+    DecodeWork wk;
+    wk.count = reinterpret_cast<int32_t *>(base);
+    wk.head_first = reinterpret_cast<int32_t *>(base + o_first);
+    wk.head_cnt = reinterpret_cast<int32_t *>(base + o_cnt);
+    wk.items = reinterpret_cast<DecodeItem *>(base + o_items);
+    wk.partials = reinterpret_cast<float *>(base + o_part);
+    wk.max_items = items;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    e = (cache->D == 128) ? launch_decode_static<128>(cache, wk, static_cast<const __half *>(q), modes, w, out, st)
+                          : launch_decode_static<64>(cache, wk, static_cast<const __half *>(q), modes, w, out, st);
+    if (e != cudaSuccess) return report_error(KVQ_ERR_CUDA, "routed_attn_decode_noalloc: kernel launch failed");
+    return report_error(KVQ_OK, "");
+}

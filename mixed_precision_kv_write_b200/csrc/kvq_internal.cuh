@@ -179,6 +179,8 @@ cudaError_t launch_decode(const kvq_cache *c, const __half *q, const uint8_t *mo
 cudaError_t launch_prefill(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,
                            const int32_t *cu, int64_t n_tok, float *out, cudaStream_t st);
 int num_sms();
+// records a host-side status for kvq_last_error() and returns `code`
+int report_error(int code, const char *msg);
 // profiling hook (kvq_set_profile_events): record the caller's events around a main kernel
 void profile_before(cudaStream_t st);
 void profile_after(cudaStream_t st);

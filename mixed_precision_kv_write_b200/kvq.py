@@ -22,7 +22,8 @@ MODE_SKIP, MODE_LOCAL, MODE_FULL = 0, 1, 2
 # every symbol include/kvq.h declares
 EXPORTS = ("kvq_cache_create", "kvq_cache_destroy", "kvq_cache_reset", "kvq_cache_truncate",
            "kvq_cache_lengths", "kvq_write", "routed_attn_prefill", "routed_attn_decode",
-           "kvq_cache_export", "kvq_check", "kvq_set_profile_events", "kvq_last_error")
+           "routed_attn_decode_noalloc", "kvq_cache_export", "kvq_check", "kvq_set_profile_events",
+           "kvq_last_error")
 
 _lib = None
 
@@ -52,6 +53,7 @@ def load_library(path: str = LIB_PATH):
         "kvq_write": ([vp, vp, vp, vp, i64, vp, vp], i32),
         "routed_attn_prefill": ([vp, vp, vp, i32, vp, i64, vp, vp], i32),
         "routed_attn_decode": ([vp, vp, vp, i32, vp, vp], i32),
+        "routed_attn_decode_noalloc": ([vp, vp, vp, i32, vp, vp], i32),
         "kvq_cache_export": ([vp, i32, i32, i64, i64, vp, vp, vp, vp, vp], i32),
         "kvq_check": ([vp, vp], i32),
         "kvq_set_profile_events": ([vp, vp], i32),
@@ -207,4 +209,21 @@ def routed_attn_decode(q, cache: KVQCache, modes, w: int, out=None, stream=None)
     _check(out, "out", torch.float32, dev, shape)
     _raise(load_library().routed_attn_decode(_ptr(q), cache.handle, _ptr(modes), int(w), _ptr(out),
                                              _stream(stream, dev)))
+    return out
+
+
+def routed_attn_decode_noalloc(q, cache: KVQCache, modes, w: int, out=None, stream=None):
+    """routed_attn_decode without any device allocation in the call: its scratch is the
+    library's static device array (see include/kvq.h). Pass a preallocated `out` to keep
+    the whole call allocation-free; the first call on a device should precede any stream
+    capture, and calls that overlap on the GPU race on the shared scratch."""
+    dev = cache.device
+    shape = (cache.batch, cache.heads, cache.head_dim)
+    _check(q, "q", torch.float16, dev, shape)
+    _check(modes, "modes", torch.uint8, dev, shape[:2])
+    if out is None:
+        out = torch.empty(shape, dtype=torch.float32, device=dev)
+    _check(out, "out", torch.float32, dev, shape)
+    _raise(load_library().routed_attn_decode_noalloc(_ptr(q), cache.handle, _ptr(modes), int(w),
+                                                     _ptr(out), _stream(stream, dev)))
     return out
