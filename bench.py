@@ -322,16 +322,7 @@ def run_ours(args):
     kernel_bytes = routed + st["q_bytes"]
     hbm_peak = float(pk["hbm_gbs"])
     achieved = kernel_bytes / k_avg / 1e9
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "decode_splitk_decode_1p3b.traffic.json")
-    if os.path.exists(prof):
-        try:
-            with open(prof) as f:
-                tj = json.load(f)
-            if tj.get("kernel_source_hash") == _src_hash():
-                traffic = tj.get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = _profiled_traffic("decode_splitk_decode_1p3b.md", "kvq_decode.cu")
 
     # end to end through host buffers: per step H2D of the step inputs (pinned), D2H of out
     host = {n: st[n].cpu().pin_memory() for n in ("k_step", "v_step", "b_step", "q", "modes")}
@@ -441,13 +432,23 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def _src_hash():
+def _src_hash(name):
     import hashlib
-    h = hashlib.sha256()
-    p = os.path.join(ROOT, "mixed_precision_kv_write_b200", "csrc", "kvq_decode.cu")
-    with open(p, "rb") as f:
-        h.update(f.read())
-    return h.hexdigest()[:16]
+    with open(os.path.join(ROOT, "mixed_precision_kv_write_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _profiled_traffic(summary, source):
+    """DRAM bytes per launch from an ncu summary in profiles/, if the summary's
+    `<!-- traffic: bytes=N source=HASH -->` line matches the current kernel source."""
+    import re
+    p = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(p):
+        return None
+    m = re.search(r"<!-- traffic: bytes=(\d+) source=([0-9a-f]+) -->", open(p).read())
+    if not m or m.group(2) != _src_hash(source):
+        return None
+    return int(m.group(1))
 
 
 def main():
