@@ -219,8 +219,12 @@ int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
     wk.head_first = (int32_t *)alloc(sizeof(int32_t) * BH);
     wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * BH);
     wk.partials = (float *)alloc(sizeof(float) * (size_t)max_items * (head_dim + 4));
+    c->pf_max_tiles = slots / 128 + 2LL * BH;
+    c->pf_tiles = alloc(sizeof(int32_t) * 4 * (size_t)c->pf_max_tiles);
+    c->pf_count = (int32_t *)alloc(sizeof(int32_t));
+    c->pf_qidx = (int32_t *)alloc(sizeof(int32_t) * (size_t)slots);
     for (int i = 0; i < c->n_allocs; ++i) okk = okk && c->allocs[i];
-    if (!okk || c->n_allocs != 17) {
+    if (!okk || c->n_allocs != 20) {
         kvq_cache_destroy(c);
         return fail(KVQ_ERR_NOMEM, "kvq_cache_create: cudaMalloc failed (%lld slots, %.2f GB of records)",
                     (long long)slots, (double)slots * 4 * head_dim / 1e9);
@@ -321,8 +325,10 @@ int routed_attn_prefill(const void *q, const kvq_cache *c, const uint8_t *modes,
         return fail(KVQ_ERR_ARG, "routed_attn_prefill: q, modes or out is NULL");
     if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15u)
         return fail(KVQ_ERR_ARG, "routed_attn_prefill: q and out must be 16-byte aligned");
-    cudaError_t e = kvq::launch_prefill(c, static_cast<const __half *>(q), modes, w, cu_seqlens, n_tok, out,
-                                        reinterpret_cast<cudaStream_t>(stream));
+    if (n_tok * c->H > c->total_slots)
+        return fail(KVQ_ERR_ARG, "routed_attn_prefill: n_tok = %lld exceeds the cache's capacity", (long long)n_tok);
+    cudaError_t e = kvq::launch_prefill_tc(c, static_cast<const __half *>(q), modes, w, cu_seqlens, n_tok, out,
+                                           reinterpret_cast<cudaStream_t>(stream));
     return e ? cuda_fail(e, "routed_attn_prefill") : ok();
 }
 

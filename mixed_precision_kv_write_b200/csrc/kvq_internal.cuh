@@ -167,6 +167,10 @@ struct kvq_cache {
     kvq::CacheView view;
     kvq::DecodeWork work;
     uint32_t write_gen;       // id of the last kvq_write call
+    void *pf_tiles;           // prefill tile list (PfTile = 4 x int32), pf_max_tiles entries
+    int32_t *pf_count;        // [1]
+    int32_t *pf_qidx;         // [total_slots] per-(sequence, head) query lists
+    int64_t pf_max_tiles;
     void *allocs[24];
     int n_allocs;
 };
@@ -176,8 +180,8 @@ cudaError_t launch_write(kvq_cache *c, const __half *k, const __half *v, const u
                          const int32_t *cu, int64_t n_tok, cudaStream_t st);
 cudaError_t launch_decode(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,
                           float *out, cudaStream_t st);
-cudaError_t launch_prefill(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,
-                           const int32_t *cu, int64_t n_tok, float *out, cudaStream_t st);
+cudaError_t launch_prefill_tc(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,
+                              const int32_t *cu, int64_t n_tok, float *out, cudaStream_t st);
 int num_sms();
 // records a host-side status for kvq_last_error() and returns `code`
 int report_error(int code, const char *msg);

@@ -1,0 +1,579 @@
+// Routed causal prefill attention (TriRoute paper review page, section 3, Eq. 2) over the
+// mixed-precision cache of Eq. 4, on the sm_100a tensor cores (tcgen05 + TMEM).
+//
+// Two launches per call:
+//   prefill_sched_kernel  one CTA per (sequence, head): compacts the call's queries by
+//                         mode into a local list and a full list, cuts each into tiles of
+//                         at most 128 queries, and writes zeros for skip queries. A local
+//                         tile reads keys [min(t) - w, max(t)], a full tile [0, max(t)],
+//                         so local rows do not pay for a full tile's range.
+//   prefill_tc_kernel     one CTA per tile:
+//     - warps 0-3 (one thread per query row): Q row -> shared (fp16, 128B-swizzled
+//       K-major); per key tile, S row from TMEM -> logits (s_K * (q.c) + z_K * sum(q)) /
+//       sqrt(D) with the row's causal/window mask -> online softmax -> P' = p * s_V split
+//       into fp16 hi + lo (fp16 rounding of P alone would cost ~1e-2 on outlier channels)
+//       -> shared; rescale the O row in TMEM when the row max grows; final O / l.
+//     - warps 4-7: unpack each 64-key tile's K and V codes into exact fp16 operands (codes
+//       are integers <= 255; b = 16 keys are the fp16 values) in shared memory, double
+//       buffered; K 128B-swizzled K-major, V 128B-swizzled MN-major.
+//     - warp 8: owns 256 TMEM columns (S double buffer: 2 x 64, O: D) and issues the MMAs
+//       from one lane: S = Q C_K^T (M128 N64 K16 steps) one key tile ahead, then
+//       O += P'_hi V and O += P'_lo V (M128 ND K16) once P' of the tile is in shared memory.
+//   All mbarrier waits are bounded; on a timeout the CTA records KVQ_ERR_DEVICE_CHECK,
+//   leaves its loops, waits (bounded) for its MMAs and frees its TMEM before returning.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kQRows = 128;     // queries per tile (MMA M)
+constexpr int kKeys = 64;       // keys per key tile (QK MMA N, PV MMA K)
+constexpr int kTcThreads = 288; // 9 warps
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemS = 0, kTmemO = 128;   // S double buffer at columns 0 and 64
+
+// ---- tcgen05 / UMMA helpers -------------------------------------------------------
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), descriptor version 1.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp16 A/B, fp32 accumulator, M = 128.
+__host__ __device__ constexpr uint32_t umma_idesc(int n, bool b_mn_major)
+{
+    return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, bool acc)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)acc)
+                 : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+                   "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+                   "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+                 "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+                   "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+                   "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+                   "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+                   "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+                   "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+                   "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+                   "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+                   "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+                   "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+                   "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+                 : "memory");
+}
+
+// byte offset of the 16-byte chunk `cc` (0..7) of row r inside a 128B-swizzled K-major
+// block of rows (rows of 128 bytes, 8-row atoms of 1024 bytes)
+__device__ __forceinline__ uint32_t kmajor_off(int r, int cc)
+{
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((cc ^ (r & 7)) << 4));
+}
+
+// fp16 operands holding integer codes: two codes c0, c1 -> half2 (c0, c1), exact
+__device__ __forceinline__ uint32_t codes_to_h2(uint32_t lo, uint32_t hi)
+{
+    const uint32_t h = lo | (hi << 16) | 0x64006400u;          // (1024 + c0, 1024 + c1)
+    const __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&h), __floats2half2_rn(1024.f, 1024.f));
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// 8 channels starting at channel 8*chunk of a packed part -> 16 bytes of fp16
+__device__ __forceinline__ uint4 unpack8(const uint8_t *part, int bits, int chunk)
+{
+    uint4 o;
+    uint32_t *w = reinterpret_cast<uint32_t *>(&o);
+    if (bits == 16) {
+        return reinterpret_cast<const uint4 *>(part)[chunk];
+    } else if (bits == 8) {
+        const uint2 x = reinterpret_cast<const uint2 *>(part)[chunk];
+        const uint32_t xs[2] = {x.x, x.y};
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            w[2 * i] = codes_to_h2(xs[i] & 0xFFu, (xs[i] >> 8) & 0xFFu);
+            w[2 * i + 1] = codes_to_h2((xs[i] >> 16) & 0xFFu, xs[i] >> 24);
+        }
+    } else if (bits == 4) {
+        const uint32_t x = reinterpret_cast<const uint32_t *>(part)[chunk];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = codes_to_h2((x >> (8 * i)) & 0xFu, (x >> (8 * i + 4)) & 0xFu);
+    } else {
+        const uint32_t x = reinterpret_cast<const uint16_t *>(part)[chunk];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = codes_to_h2((x >> (4 * i)) & 3u, (x >> (4 * i + 2)) & 3u);
+    }
+    return o;
+}
+
+struct PfTile {
+    int32_t sh, mode, start, count;   // (sequence, head), mode, first list entry, queries
+};
+
+template <int D>
+struct alignas(1024) PfSmem {
+    __half q[kQRows * D];             // K-major SW128, D/64 blocks of 128 rows x 128 B
+    __half k[2][kKeys * D];           // K-major SW128, D/64 blocks of 64 rows x 128 B
+    __half v[2][kKeys * D];           // MN-major SW128: atom (8 keys x 64 ch) at (key/8)*(D/64)+ch/64
+    __half p_hi[kQRows * kKeys];      // K-major SW128, 128 rows x 128 B
+    __half p_lo[kQRows * kKeys];
+    float side[2][4][kKeys];          // s_K, z_K, s_V, z_V per key of a buffer
+    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full, pv_done, drain;
+    uint32_t tmem_base;
+    int32_t klo, khi, abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_t *__restrict__ cu,
+                  const PfTile *__restrict__ tiles, const int32_t *__restrict__ tile_count,
+                  const int32_t *__restrict__ qidx, float *__restrict__ out)
+{
+    if ((int)blockIdx.x >= *tile_count) return;
+    extern __shared__ uint8_t smem_raw[];
+    PfSmem<D> &sm = *reinterpret_cast<PfSmem<D> *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const PfTile tile = tiles[blockIdx.x];
+    const int H = c.H, sh = tile.sh, s = sh / H, h = sh % H;
+    const int n_s = cu[s + 1] - cu[s];
+    const int pos0 = c.len[sh] - n_s;
+    const int64_t sbase = slot_of(c, s, h, 0);
+    const uint8_t *stream = stream_of(c, s, h);
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.kv_full[i], 128);
+            mbar_init(&sm.kv_empty[i], 1);
+        }
+        mbar_init(&sm.s_full[0], 1);
+        mbar_init(&sm.s_full[1], 1);
+        mbar_init(&sm.p_full, 128);
+        mbar_init(&sm.pv_done, 1);
+        mbar_init(&sm.drain, 1);
+        sm.klo = INT32_MAX;
+        sm.khi = -1;
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&sm.tmem_base)), "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    __syncthreads();
+
+    // ---- prologue: query rows (warps 0-3) ----
+    int row_t = -1, row_lo = 0, row_i = -1;
+    float qsum = 0.f;
+    if (tid < kQRows) {
+        const int r = tid;
+        const bool valid = r < tile.count;
+        if (valid) {
+            row_i = qidx[tile.start + r];
+            row_t = pos0 + row_i;
+            row_lo = (tile.mode == KVQ_MODE_LOCAL) ? max(0, row_t - w) : 0;
+            atomicMin(&sm.klo, row_lo);
+            atomicMax(&sm.khi, row_t);
+        }
+        const uint4 *src = reinterpret_cast<const uint4 *>(q + ((int64_t)(cu[s] + max(row_i, 0)) * H + h) * D);
+#pragma unroll
+        for (int ch = 0; ch < D / 8; ++ch) {
+            uint4 x = valid ? src[ch] : make_uint4(0, 0, 0, 0);
+            const __half2 *hx = reinterpret_cast<const __half2 *>(&x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(hx[e]);
+                qsum += f.x + f.y;
+            }
+            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(sm.q) + (ch >> 3) * (kQRows * 128) +
+                                       kmajor_off(r, ch & 7)) = x;
+        }
+        fence_async_smem();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const int klo = sm.klo, khi = sm.khi;
+    const int n_kt = (khi >= klo) ? (khi - klo + kKeys) / kKeys : 0;
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 8) {
+        // ------------------------------- MMA issuer --------------------------------
+        // order: QK(0), then per tile t: QK(t+1) into the other S buffer, wait P(t), PV(t)
+        const uint32_t q0 = smem_u32(sm.q), p_hi0 = smem_u32(sm.p_hi), p_lo0 = smem_u32(sm.p_lo);
+        constexpr uint32_t idesc_qk = umma_idesc(kKeys, false);
+        constexpr uint32_t idesc_pv = umma_idesc(D, true);
+        constexpr uint32_t v_sbo = (D / 64) * 1024;       // next 8 keys
+        auto issue_qk = [&](int t) -> bool {
+            const int b = t & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.kv_full[b], (t >> 1) & 1, c.status))) return false;
+            tc_fence_after();
+            const uint32_t k0 = smem_u32(sm.k[b]);
+            if (lane == 0) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t da = umma_desc(q0 + (kk >> 2) * (kQRows * 128) + (kk & 3) * 32, 16, 1024);
+                    const uint64_t db = umma_desc(k0 + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
+                    umma_f16(tmem + kTmemS + 64 * b, da, db, idesc_qk, kk > 0);
+                }
+                umma_commit(&sm.s_full[b]);
+            }
+            __syncwarp();
+            return true;
+        };
+        bool alive = n_kt > 0 && issue_qk(0);
+        for (int t = 0; alive && t < n_kt; ++t) {
+            if (t + 1 < n_kt && !issue_qk(t + 1)) {
+                alive = false;
+                break;
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_full, t & 1, c.status))) {
+                alive = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t v0 = smem_u32(sm.v[t & 1]);
+            if (lane == 0) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const uint32_t pb = half ? p_lo0 : p_hi0;
+#pragma unroll
+                    for (int kk = 0; kk < kKeys / 16; ++kk) {
+                        const uint64_t da = umma_desc(pb + kk * 32, 16, 1024);
+                        const uint64_t db = umma_desc(v0 + 2 * kk * v_sbo, 1024, v_sbo);
+                        umma_f16(tmem + kTmemO, da, db, idesc_pv, half > 0 || t > 0 || kk > 0);
+                    }
+                }
+                umma_commit(&sm.pv_done);
+                umma_commit(&sm.kv_empty[t & 1]);
+            }
+            __syncwarp();
+        }
+        if (!alive) sm.abort_flag = 1;
+        // every MMA this CTA issued has completed before its TMEM is freed (bounded wait)
+        if (lane == 0) umma_commit(&sm.drain);
+        __syncwarp();
+        mbar_wait(&sm.drain, 0, c.status);
+    } else if (warp >= 4) {
+        // ------------------------------ K/V unpack -----------------------------------
+        const int u = tid - 128;
+        const int kj = u >> 1, half = u & 1;
+        constexpr int CH = D / 2;                    // channels per thread
+        for (int t = 0; t < n_kt; ++t) {
+            const int b = t & 1;
+            if (!mbar_wait(&sm.kv_empty[b], ((t >> 1) & 1) ^ 1, c.status) ||
+                *reinterpret_cast<volatile int *>(&sm.abort_flag)) {
+                sm.abort_flag = 1;
+                break;
+            }
+            const int j = klo + t * kKeys + kj;
+            uint8_t *kb = reinterpret_cast<uint8_t *>(sm.k[b]);
+            uint8_t *vb = reinterpret_cast<uint8_t *>(sm.v[b]);
+            if (j <= khi) {
+                const uint32_t mt = c.meta[sbase + j];
+                const int bits = 2 << (mt & 3u);
+                const uint8_t *rk = stream + (mt & ~15u);
+                const uint8_t *rv = rk + bits * D / 8;
+                if (half == 0) {
+                    const float4 sd = c.side[sbase + j];
+                    sm.side[b][0][kj] = sd.x;
+                    sm.side[b][1][kj] = sd.y;
+                    sm.side[b][2][kj] = sd.z;
+                    sm.side[b][3][kj] = sd.w;
+                }
+#pragma unroll
+                for (int cc = 0; cc < CH / 8; ++cc) {
+                    const int chunk = half * (CH / 8) + cc;   // 8-channel chunk index
+                    const uint4 kx = unpack8(rk, bits, chunk);
+                    const uint4 vx = unpack8(rv, bits, chunk);
+                    *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(kj, chunk & 7)) = kx;
+                    const int n = chunk * 8;
+                    const int atom = (kj >> 3) * (D / 64) + (n >> 6);
+                    *reinterpret_cast<uint4 *>(vb + atom * 1024 + (kj & 7) * 128 + ((((n & 63) >> 3) ^ (kj & 7)) << 4)) = vx;
+                }
+            } else {
+                if (half == 0) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sm.side[b][e][kj] = 0.f;
+                }
+#pragma unroll
+                for (int cc = 0; cc < CH / 8; ++cc) {
+                    const int chunk = half * (CH / 8) + cc;
+                    *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(kj, chunk & 7)) =
+                        make_uint4(0, 0, 0, 0);
+                    const int n = chunk * 8;
+                    const int atom = (kj >> 3) * (D / 64) + (n >> 6);
+                    *reinterpret_cast<uint4 *>(vb + atom * 1024 + (kj & 7) * 128 + ((((n & 63) >> 3) ^ (kj & 7)) << 4)) =
+                        make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(&sm.kv_full[b]);
+        }
+    } else {
+        // ------------------------------ softmax rows ---------------------------------
+        const int r = tid;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float scale = kLog2e * rsqrtf((float)D);
+        float m_run = -INFINITY, l_run = 0.f, pz_run = 0.f;
+        uint8_t *ph = reinterpret_cast<uint8_t *>(sm.p_hi);
+        uint8_t *pl = reinterpret_cast<uint8_t *>(sm.p_lo);
+        bool ok = true;
+        for (int t = 0; t < n_kt; ++t) {
+            const int b = t & 1;
+            // warp-uniform outcome: the TMEM accesses below are .sync.aligned
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (t >> 1) & 1, c.status) &&
+                                             !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
+                sm.abort_flag = 1;
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int kt0 = klo + t * kKeys;
+            float lg[kKeys];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float sv[32];
+                tmem_ld32(tmem + lane_base + kTmemS + 64 * b + 32 * hf, sv);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int cidx = 32 * hf + e;
+                    const int j = kt0 + cidx;
+                    const bool valid = (row_t >= 0) && j >= row_lo && j <= row_t;
+                    const float v = fmaf(sm.side[b][0][cidx], sv[e], sm.side[b][1][cidx] * qsum);
+                    lg[cidx] = valid ? v * scale : -INFINITY;
+                    mx = fmaxf(mx, lg[cidx]);
+                }
+            }
+            const float m_new = fmaxf(m_run, mx);
+            const float corr = (m_run == -INFINITY) ? ((m_new == -INFINITY) ? 1.f : 0.f) : exp2f(m_run - m_new);
+            float psum = 0.f, pz = 0.f;
+#pragma unroll
+            for (int cidx = 0; cidx < kKeys; ++cidx) {
+                const float p = (lg[cidx] == -INFINITY) ? 0.f : exp2f(lg[cidx] - m_new);
+                psum += p;
+                pz = fmaf(p, sm.side[b][3][cidx], pz);
+                lg[cidx] = p * sm.side[b][2][cidx];            // P' = p * s_V
+            }
+            l_run = fmaf(l_run, corr, psum);
+            pz_run = fmaf(pz_run, corr, pz);
+            m_run = m_new;
+            if (t > 0) {
+                // PV(t-1) must be done: it reads P and accumulates into O
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (t - 1) & 1, c.status))) {
+                    sm.abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, corr != 1.f)) {        // rescale this warp's O rows
+#pragma unroll
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        float ov[32];
+                        tmem_ld32(tmem + lane_base + kTmemO + cb * 32, ov);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ov[e] *= corr;
+                        tmem_st32(tmem + lane_base + kTmemO + cb * 32, ov);
+                    }
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                }
+            }
+            // P' = hi + lo, both fp16, row r of the two K-major P tiles
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float a = lg[8 * cc + 2 * e], bq = lg[8 * cc + 2 * e + 1];
+                    const __half2 hv = __floats2half2_rn(a, bq);
+                    const float2 hf = __half22float2(hv);
+                    const __half2 lv = __floats2half2_rn(a - hf.x, bq - hf.y);
+                    hw[e] = *reinterpret_cast<const uint32_t *>(&hv);
+                    lw[e] = *reinterpret_cast<const uint32_t *>(&lv);
+                }
+                *reinterpret_cast<uint4 *>(ph + kmajor_off(r, cc)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(pl + kmajor_off(r, cc)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&sm.p_full);
+        }
+        if (ok && n_kt > 0 && __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (n_kt - 1) & 1, c.status))) {
+            tc_fence_after();
+            const bool write = row_t >= 0;
+            const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
+            float *dst = out + ((int64_t)(cu[s] + max(row_i, 0)) * H + h) * D;
+#pragma unroll
+            for (int cb = 0; cb < D / 32; ++cb) {
+                float ov[32];
+                tmem_ld32(tmem + lane_base + kTmemO + cb * 32, ov);
+                if (write) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(dst + cb * 32 + e) =
+                            make_float4((ov[e] + pz_run) * inv, (ov[e + 1] + pz_run) * inv,
+                                        (ov[e + 2] + pz_run) * inv, (ov[e + 3] + pz_run) * inv);
+                }
+            }
+        } else if (row_t >= 0) {
+            sm.abort_flag = 1;
+        }
+    }
+
+    // ---- teardown: every role ends here; TMEM is freed even after an abort ----
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+// One CTA per (sequence, head): compaction of the call's queries by mode.
+__global__ void __launch_bounds__(256)
+prefill_sched_kernel(CacheView c, const uint8_t *__restrict__ modes, const int32_t *__restrict__ cu,
+                     int64_t n_tok, int D, float *__restrict__ out, PfTile *__restrict__ tiles,
+                     int32_t *__restrict__ tile_count, int32_t *__restrict__ qidx)
+{
+    __shared__ int wl[8], wf[8];
+    __shared__ int tot_l, tot_f;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int H = c.H, sh = blockIdx.x, s = sh / H, h = sh % H;
+    const int64_t t0 = cu[s], t1 = cu[s + 1];
+    if (t0 < 0 || t1 < t0 || t1 > n_tok) return;      // flagged by the write's checks
+    const int n = (int)(t1 - t0);
+    if (n == 0) return;
+    if (c.len[sh] - n < 0) {
+        if (tid == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+        return;
+    }
+    int32_t *region = qidx + t0 * H + (int64_t)h * n;    // local from the front, full from the back
+    if (tid == 0) {
+        tot_l = 0;
+        tot_f = 0;
+    }
+    __syncthreads();
+    for (int base = 0; base < n; base += 256) {
+        const int i = base + tid;
+        int m = -1;
+        if (i < n) {
+            m = modes[(t0 + i) * H + h];
+            if (m > KVQ_MODE_FULL) {
+                set_status(c.status, KVQ_ERR_MODE);
+                m = KVQ_MODE_SKIP;
+            }
+            if (m == KVQ_MODE_SKIP) {
+                float4 *dst = reinterpret_cast<float4 *>(out + ((t0 + i) * H + h) * D);
+                for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        const uint32_t bl = __ballot_sync(0xffffffffu, m == KVQ_MODE_LOCAL);
+        const uint32_t bf = __ballot_sync(0xffffffffu, m == KVQ_MODE_FULL);
+        if (lane == 0) {
+            wl[wid] = __popc(bl);
+            wf[wid] = __popc(bf);
+        }
+        __syncthreads();
+        int pl = tot_l, pf = tot_f;
+        for (int q2 = 0; q2 < wid; ++q2) {
+            pl += wl[q2];
+            pf += wf[q2];
+        }
+        const uint32_t lt = (1u << lane) - 1u;
+        if (m == KVQ_MODE_LOCAL) region[pl + __popc(bl & lt)] = i;
+        if (m == KVQ_MODE_FULL) region[n - 1 - (pf + __popc(bf & lt))] = i;
+        __syncthreads();
+        if (tid == 0) {
+            for (int q2 = 0; q2 < 8; ++q2) {
+                tot_l += wl[q2];
+                tot_f += wf[q2];
+            }
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+        const int ntl = (tot_l + kQRows - 1) / kQRows, ntf = (tot_f + kQRows - 1) / kQRows;
+        const int first = atomicAdd(tile_count, ntl + ntf);
+        const int32_t off = (int32_t)(t0 * H + (int64_t)h * n);
+        for (int k = 0; k < ntl; ++k)
+            tiles[first + k] = PfTile{sh, KVQ_MODE_LOCAL, off + k * kQRows, min(kQRows, tot_l - k * kQRows)};
+        for (int k = 0; k < ntf; ++k)
+            tiles[first + ntl + k] = PfTile{sh, KVQ_MODE_FULL, off + n - tot_f + k * kQRows,
+                                            min(kQRows, tot_f - k * kQRows)};
+    }
+}
+
+template <int D>
+cudaError_t run_tc(const kvq_cache *cache, const __half *q, const uint8_t *modes, int w, const int32_t *cu,
+                   int64_t n_tok, float *out, cudaStream_t st)
+{
+    const CacheView &c = cache->view;
+    PfTile *tiles = reinterpret_cast<PfTile *>(cache->pf_tiles);
+    cudaError_t e = cudaMemsetAsync(cache->pf_count, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return e;
+    prefill_sched_kernel<<<c.B * c.H, 256, 0, st>>>(c, modes, cu, n_tok, D, out, tiles, cache->pf_count,
+                                                     cache->pf_qidx);
+    const int64_t max_tiles = n_tok * c.H / kQRows + 2LL * c.B * c.H;
+    const size_t smem = sizeof(PfSmem<D>) + 1024;
+    static bool attr_done = false;
+    if (!attr_done) {
+        e = cudaFuncSetAttribute(prefill_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    profile_before(st);
+    prefill_tc_kernel<D><<<(unsigned)max_tiles, kTcThreads, smem, st>>>(c, q, w, cu, tiles, cache->pf_count,
+                                                                        cache->pf_qidx, out);
+    profile_after(st);
+    return cudaGetLastError();
+}
+
+} // namespace
+
+cudaError_t launch_prefill_tc(const kvq_cache *cache, const __half *q, const uint8_t *modes, int w,
+                              const int32_t *cu, int64_t n_tok, float *out, cudaStream_t st)
+{
+    if (n_tok == 0) return cudaSuccess;
+    if (cache->D == 128) return run_tc<128>(cache, q, modes, w, cu, n_tok, out, st);
+    return run_tc<64>(cache, q, modes, w, cu, n_tok, out, st);
+}
+
+} // namespace kvq
