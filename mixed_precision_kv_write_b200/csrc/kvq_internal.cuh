@@ -115,24 +115,27 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
-// Wait until the barrier's phase `parity` has completed. Bounded: gives up after about
-// two seconds, records KVQ_ERR_DEVICE_CHECK and returns false, so a logic error ends the
-// kernel with a status instead of hanging the GPU.
+// Wait until the barrier's phase `parity` has completed. The waiting thread may be
+// suspended by the hardware for up to ~0.1 ms per try (woken when the phase completes),
+// so waiting warps do not spin on issue slots. Bounded: gives up after about two seconds,
+// records KVQ_ERR_DEVICE_CHECK and returns false, so a logic error ends the kernel with a
+// status instead of hanging the GPU.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status)
 {
-    uint32_t addr = smem_u32(bar);
+    const uint32_t addr = smem_u32(bar);
+    const uint32_t suspend_ns = 100000;
     uint32_t done = 0;
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         asm volatile("{\n\t.reg .pred p;\n\t"
-                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
                      "selp.u32 %0, 1, 0, p;\n\t}"
                      : "=r"(done)
-                     : "r"(addr), "r"(parity)
+                     : "r"(addr), "r"(parity), "r"(suspend_ns)
                      : "memory");
         if (done) return true;
-        if ((it & 1023u) == 0) {
-            uint64_t t = global_ns();
+        if ((it & 15u) == 0) {
+            const uint64_t t = global_ns();
             if (t0 == 0) t0 = t;
             else if (t - t0 > 2000000000ull) {
                 set_status(status, KVQ_ERR_DEVICE_CHECK);
@@ -140,6 +143,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_
             }
         }
     }
+}
+
+// Non-blocking test of a barrier phase (no suspension).
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(done)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return done != 0;
 }
 
 // 1-D bulk copy global -> shared (TMA engine), completion counted on `bar` in bytes.

@@ -15,10 +15,12 @@
 //       -> shared; rescale the O row in TMEM when the row max grows; final O / l.
 //     - warps 4-7: unpack each 64-key tile's K and V codes into exact fp16 operands (codes
 //       are integers <= 255; b = 16 keys are the fp16 values) in shared memory, double
-//       buffered; K 128B-swizzled K-major, V 128B-swizzled MN-major.
+//       buffered; K 128B-swizzled K-major, V 128B-swizzled MN-major. The packed bytes are
+//       fetched one tile ahead with cp.async and the record offsets three tiles ahead.
 //     - warp 8: owns 256 TMEM columns (S double buffer: 2 x 64, O: D) and issues the MMAs
-//       from one lane: S = Q C_K^T (M128 N64 K16 steps) one key tile ahead, then
-//       O += P'_hi V and O += P'_lo V (M128 ND K16) once P' of the tile is in shared memory.
+//       from one lane: S = Q C_K^T (M128 N64 K16 steps) as soon as a K tile is unpacked
+//       (up to one tile ahead), O += P'_hi V and O += P'_lo V (M128 ND K16) as soon as P' of
+//       the tile is in shared memory, whichever is ready first.
 //   All mbarrier waits are bounded; on a timeout the CTA records KVQ_ERR_DEVICE_CHECK,
 //   leaves its loops, waits (bounded) for its MMAs and frees its TMEM before returning.
 #include "kvq_internal.cuh"
@@ -108,39 +110,60 @@ __device__ __forceinline__ uint32_t kmajor_off(int r, int cc)
     return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((cc ^ (r & 7)) << 4));
 }
 
-// fp16 operands holding integer codes: two codes c0, c1 -> half2 (c0, c1), exact
-__device__ __forceinline__ uint32_t codes_to_h2(uint32_t lo, uint32_t hi)
+// fp16 operands holding integer codes. A word whose two halves are 0x64cc (the fp16
+// number 1024 + c for a code c < 1024) minus (1024, 1024) is the half2 (c0, c1), exactly.
+__device__ __forceinline__ uint32_t h2_minus_1024(uint32_t h)
 {
-    const uint32_t h = lo | (hi << 16) | 0x64006400u;          // (1024 + c0, 1024 + c1)
-    const __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&h), __floats2half2_rn(1024.f, 1024.f));
-    return *reinterpret_cast<const uint32_t *>(&v);
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64006400u));
+    return r;
 }
 
-// 8 channels starting at channel 8*chunk of a packed part -> 16 bytes of fp16
+// two codes sitting in bytes 0 and 2 of `t` (other bits arbitrary) -> half2 (c0, c1)
+__device__ __forceinline__ uint32_t bytes02_to_h2(uint32_t t, uint32_t mask)
+{
+    return h2_minus_1024((t & mask) | 0x64006400u);
+}
+
+// 8 channels starting at channel 8*chunk of a packed part -> 16 bytes of fp16 (registers only)
 __device__ __forceinline__ uint4 unpack8(const uint8_t *part, int bits, int chunk)
 {
-    uint4 o;
-    uint32_t *w = reinterpret_cast<uint32_t *>(&o);
-    if (bits == 16) {
-        return reinterpret_cast<const uint4 *>(part)[chunk];
-    } else if (bits == 8) {
+    if (bits == 16) return reinterpret_cast<const uint4 *>(part)[chunk];
+    uint32_t w0, w1, w2, w3;
+    if (bits == 8) {
         const uint2 x = reinterpret_cast<const uint2 *>(part)[chunk];
-        const uint32_t xs[2] = {x.x, x.y};
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            w[2 * i] = codes_to_h2(xs[i] & 0xFFu, (xs[i] >> 8) & 0xFFu);
-            w[2 * i + 1] = codes_to_h2((xs[i] >> 16) & 0xFFu, xs[i] >> 24);
-        }
+        // bytes (c0, 0x64, c1, 0x64) via byte permutes, then - 1024
+        w0 = h2_minus_1024(__byte_perm(x.x, 0x64646464u, 0x5140));
+        w1 = h2_minus_1024(__byte_perm(x.x, 0x64646464u, 0x5342));
+        w2 = h2_minus_1024(__byte_perm(x.y, 0x64646464u, 0x5140));
+        w3 = h2_minus_1024(__byte_perm(x.y, 0x64646464u, 0x5342));
     } else if (bits == 4) {
         const uint32_t x = reinterpret_cast<const uint32_t *>(part)[chunk];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) w[i] = codes_to_h2((x >> (8 * i)) & 0xFu, (x >> (8 * i + 4)) & 0xFu);
+        const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;   // even / odd channels
+        // pair k = (lo byte k, hi byte k) placed in bytes 0 and 2
+        w0 = bytes02_to_h2(__byte_perm(lo, hi, 0x0400), 0x00FF00FFu);
+        w1 = bytes02_to_h2(__byte_perm(lo, hi, 0x0501), 0x00FF00FFu);
+        w2 = bytes02_to_h2(__byte_perm(lo, hi, 0x0602), 0x00FF00FFu);
+        w3 = bytes02_to_h2(__byte_perm(lo, hi, 0x0703), 0x00FF00FFu);
     } else {
         const uint32_t x = reinterpret_cast<const uint16_t *>(part)[chunk];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) w[i] = codes_to_h2((x >> (4 * i)) & 3u, (x >> (4 * i + 2)) & 3u);
+        // channel 2k at bits 4k, channel 2k+1 at bits 4k+2: move the odd ones up by 14
+        const uint32_t y = (x & 0x3333u) | ((x & 0xCCCCu) << 14);        // even: bits 4k, odd: bits 16+4k
+        w0 = bytes02_to_h2(y, 0x00030003u);
+        w1 = bytes02_to_h2(y >> 4, 0x00030003u);
+        w2 = bytes02_to_h2(y >> 8, 0x00030003u);
+        w3 = bytes02_to_h2(y >> 12, 0x00030003u);
     }
-    return o;
+    return make_uint4(w0, w1, w2, w3);
+}
+
+// 2^x with the hardware's approximate exp2 (relative error of a few ulp), used for the
+// softmax weights; 2^-inf = 0.
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 struct PfTile {
@@ -154,7 +177,10 @@ struct alignas(1024) PfSmem {
     __half v[2][kKeys * D];           // MN-major SW128: atom (8 keys x 64 ch) at (key/8)*(D/64)+ch/64
     __half p_hi[kQRows * kKeys];      // K-major SW128, 128 rows x 128 B
     __half p_lo[kQRows * kKeys];
-    float side[2][4][kKeys];          // s_K, z_K, s_V, z_V per key of a buffer
+    float2 side_k[2][kKeys];          // (s_K * c, z_K * c) per key, c = log2(e)/sqrt(D)
+    float2 side_v[2][kKeys];          // (s_V, z_V) per key
+    uint8_t raw[2][kKeys * 2][2 * D + 16]; // packed K and V bytes of each (key, half), by cp.async
+                                           // (16 bytes of padding spread the slots over the banks)
     uint64_t kv_full[2], kv_empty[2], s_full[2], p_full, pv_done, drain;
     uint32_t tmem_base;
     int32_t klo, khi, abort_flag;
@@ -241,9 +267,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         constexpr uint32_t idesc_qk = umma_idesc(kKeys, false);
         constexpr uint32_t idesc_pv = umma_idesc(D, true);
         constexpr uint32_t v_sbo = (D / 64) * 1024;       // next 8 keys
-        auto issue_qk = [&](int t) -> bool {
+        auto issue_qk = [&](int t) {
             const int b = t & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.kv_full[b], (t >> 1) & 1, c.status))) return false;
             tc_fence_after();
             const uint32_t k0 = smem_u32(sm.k[b]);
             if (lane == 0) {
@@ -256,18 +281,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 umma_commit(&sm.s_full[b]);
             }
             __syncwarp();
-            return true;
         };
-        bool alive = n_kt > 0 && issue_qk(0);
-        for (int t = 0; alive && t < n_kt; ++t) {
-            if (t + 1 < n_kt && !issue_qk(t + 1)) {
-                alive = false;
-                break;
-            }
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_full, t & 1, c.status))) {
-                alive = false;
-                break;
-            }
+        auto issue_pv = [&](int t) {
             tc_fence_after();
             const uint32_t v0 = smem_u32(sm.v[t & 1]);
             if (lane == 0) {
@@ -285,6 +300,35 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 umma_commit(&sm.kv_empty[t & 1]);
             }
             __syncwarp();
+        };
+        // Issue QK(t) as soon as K(t) is unpacked and PV(t) as soon as P(t) is written,
+        // whichever comes first. QK may run one tile ahead of PV (S is double buffered).
+        bool alive = true;
+        int next_qk = 0, next_pv = 0;
+        uint64_t t_start = global_ns();
+        while (next_pv < n_kt) {
+            bool progressed = false;
+            if (next_qk < n_kt && next_qk <= next_pv + 1 &&
+                __all_sync(0xffffffffu, mbar_test(&sm.kv_full[next_qk & 1], (next_qk >> 1) & 1))) {
+                issue_qk(next_qk++);
+                progressed = true;
+            }
+            if (next_pv < next_qk && __all_sync(0xffffffffu, mbar_test(&sm.p_full, next_pv & 1))) {
+                issue_pv(next_pv++);
+                progressed = true;
+            }
+            if (progressed) {
+                t_start = global_ns();
+            } else if (global_ns() - t_start > 2000000000ull) {   // bounded: about two seconds
+                set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+                alive = false;
+                break;
+            } else if (*reinterpret_cast<volatile int *>(&sm.abort_flag)) {
+                alive = false;
+                break;
+            } else {
+                __nanosleep(64);          // leave the issue slots to the warps doing the work
+            }
         }
         if (!alive) sm.abort_flag = 1;
         // every MMA this CTA issued has completed before its TMEM is freed (bounded wait)
@@ -293,65 +337,91 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         mbar_wait(&sm.drain, 0, c.status);
     } else if (warp >= 4) {
         // ------------------------------ K/V unpack -----------------------------------
+        // Thread = (key of the tile, half of the channels). Two-deep prefetch: record offset
+        // and side entry of tile t+2 in registers, packed record bytes of tile t+1 copied by
+        // cp.async into this thread's own staging slot, tile t converted to fp16 operands.
         const int u = tid - 128;
         const int kj = u >> 1, half = u & 1;
         constexpr int CH = D / 2;                    // channels per thread
+        constexpr uint32_t kNone = 0xFFFFFFFFu;
+        auto load_meta = [&](int t, uint32_t &mt, float4 &sd) {
+            const int j = klo + t * kKeys + kj;
+            if (t < n_kt && j <= khi) {
+                mt = c.meta[sbase + j];
+                sd = c.side[sbase + j];
+            } else {
+                mt = kNone;
+                sd = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        };
+        auto issue_records = [&](int t, uint32_t mt) {
+            if (t < n_kt && mt != kNone) {
+                const int bits = 2 << (mt & 3u);
+                const uint32_t part = (uint32_t)(CH * bits / 8);          // bytes of this half
+                const uint8_t *rk = stream + (mt & ~15u) + half * part;
+                const uint8_t *rv = stream + (mt & ~15u) + (uint32_t)(bits * D / 8) + half * part;
+                uint8_t *dst = sm.raw[t & 1][u];
+                if (part >= 16) {
+                    for (uint32_t o = 0; o < part; o += 16) {
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + o)), "l"(rk + o) : "memory");
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + D + o)), "l"(rv + o) : "memory");
+                    }
+                } else {                                                   // 8 bytes (head_dim 64, b = 2)
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(rk) : "memory");
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst + D)), "l"(rv) : "memory");
+                }
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+        uint32_t m_cur, m_n1, m_n2, m_n3;
+        float4 sd_cur, sd_n1, sd_n2, sd_n3;
+        load_meta(0, m_cur, sd_cur);
+        load_meta(1, m_n1, sd_n1);
+        load_meta(2, m_n2, sd_n2);
+        issue_records(0, m_cur);
         for (int t = 0; t < n_kt; ++t) {
             const int b = t & 1;
+            issue_records(t + 1, m_n1);
+            load_meta(t + 3, m_n3, sd_n3);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
             if (!mbar_wait(&sm.kv_empty[b], ((t >> 1) & 1) ^ 1, c.status) ||
                 *reinterpret_cast<volatile int *>(&sm.abort_flag)) {
                 sm.abort_flag = 1;
                 break;
             }
-            const int j = klo + t * kKeys + kj;
             uint8_t *kb = reinterpret_cast<uint8_t *>(sm.k[b]);
             uint8_t *vb = reinterpret_cast<uint8_t *>(sm.v[b]);
-            if (j <= khi) {
-                const uint32_t mt = c.meta[sbase + j];
-                const int bits = 2 << (mt & 3u);
-                const uint8_t *rk = stream + (mt & ~15u);
-                const uint8_t *rv = rk + bits * D / 8;
-                if (half == 0) {
-                    const float4 sd = c.side[sbase + j];
-                    sm.side[b][0][kj] = sd.x;
-                    sm.side[b][1][kj] = sd.y;
-                    sm.side[b][2][kj] = sd.z;
-                    sm.side[b][3][kj] = sd.w;
-                }
+            if (half == 0) {
+                const float lsc = kLog2e * rsqrtf((float)D);
+                sm.side_k[b][kj] = make_float2(sd_cur.x * lsc, sd_cur.y * lsc);
+                sm.side_v[b][kj] = make_float2(sd_cur.z, sd_cur.w);
+            }
+            const uint8_t *src = sm.raw[b][u];
+            const int bits = (m_cur == kNone) ? 0 : (2 << (m_cur & 3u));
 #pragma unroll
-                for (int cc = 0; cc < CH / 8; ++cc) {
-                    const int chunk = half * (CH / 8) + cc;   // 8-channel chunk index
-                    const uint4 kx = unpack8(rk, bits, chunk);
-                    const uint4 vx = unpack8(rv, bits, chunk);
-                    *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(kj, chunk & 7)) = kx;
-                    const int n = chunk * 8;
-                    const int atom = (kj >> 3) * (D / 64) + (n >> 6);
-                    *reinterpret_cast<uint4 *>(vb + atom * 1024 + (kj & 7) * 128 + ((((n & 63) >> 3) ^ (kj & 7)) << 4)) = vx;
-                }
-            } else {
-                if (half == 0) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) sm.side[b][e][kj] = 0.f;
-                }
-#pragma unroll
-                for (int cc = 0; cc < CH / 8; ++cc) {
-                    const int chunk = half * (CH / 8) + cc;
-                    *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(kj, chunk & 7)) =
-                        make_uint4(0, 0, 0, 0);
-                    const int n = chunk * 8;
-                    const int atom = (kj >> 3) * (D / 64) + (n >> 6);
-                    *reinterpret_cast<uint4 *>(vb + atom * 1024 + (kj & 7) * 128 + ((((n & 63) >> 3) ^ (kj & 7)) << 4)) =
-                        make_uint4(0, 0, 0, 0);
-                }
+            for (int cc = 0; cc < CH / 8; ++cc) {
+                const int chunk = half * (CH / 8) + cc;       // 8-channel chunk of the row
+                const uint4 kx = bits ? unpack8(src, bits, cc) : make_uint4(0, 0, 0, 0);
+                const uint4 vx = bits ? unpack8(src + D, bits, cc) : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(kj, chunk & 7)) = kx;
+                const int n = chunk * 8;
+                const int atom = (kj >> 3) * (D / 64) + (n >> 6);
+                *reinterpret_cast<uint4 *>(vb + atom * 1024 + (kj & 7) * 128 + ((((n & 63) >> 3) ^ (kj & 7)) << 4)) = vx;
             }
             fence_async_smem();
             mbar_arrive(&sm.kv_full[b]);
+            m_cur = m_n1;
+            sd_cur = sd_n1;
+            m_n1 = m_n2;
+            sd_n1 = sd_n2;
+            m_n2 = m_n3;
+            sd_n2 = sd_n3;
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
         // ------------------------------ softmax rows ---------------------------------
         const int r = tid;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const float scale = kLog2e * rsqrtf((float)D);
         float m_run = -INFINITY, l_run = 0.f, pz_run = 0.f;
         uint8_t *ph = reinterpret_cast<uint8_t *>(sm.p_hi);
         uint8_t *pl = reinterpret_cast<uint8_t *>(sm.p_lo);
@@ -368,6 +438,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             tc_fence_after();
             const int kt0 = klo + t * kKeys;
             float lg[kKeys];
+            // the row's keys in this tile: [max(row_lo, kt0), min(row_t, kt0 + 63)]
+            const int c_lo = max(row_lo - kt0, 0), c_hi = min(row_t - kt0, kKeys - 1);
             float mx = -INFINITY;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -376,22 +448,27 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int cidx = 32 * hf + e;
-                    const int j = kt0 + cidx;
-                    const bool valid = (row_t >= 0) && j >= row_lo && j <= row_t;
-                    const float v = fmaf(sm.side[b][0][cidx], sv[e], sm.side[b][1][cidx] * qsum);
-                    lg[cidx] = valid ? v * scale : -INFINITY;
+                    const float2 sd = sm.side_k[b][cidx];
+                    const float v = fmaf(sd.x, sv[e], sd.y * qsum);      // logit in log2 units
+                    lg[cidx] = (cidx >= c_lo && cidx <= c_hi) ? v : -INFINITY;
                     mx = fmaxf(mx, lg[cidx]);
                 }
             }
-            const float m_new = fmaxf(m_run, mx);
-            const float corr = (m_run == -INFINITY) ? ((m_new == -INFINITY) ? 1.f : 0.f) : exp2f(m_run - m_new);
+            // Lazy rescaling: the row keeps its running max until a new key exceeds it by
+            // more than 8 (so p <= 2^8 fits fp16 after the s_V scale); then O, l and pz are
+            // rescaled. The final O / l uses the same max, so the result is unchanged.
+            const bool bump = mx > m_run + 8.f;
+            const float m_new = bump ? mx : m_run;
+            const float corr = bump ? ((m_run == -INFINITY) ? 0.f : ex2(m_run - m_new)) : 1.f;
             float psum = 0.f, pz = 0.f;
+            const float shift = (m_new == -INFINITY) ? 0.f : m_new;   // all keys masked so far
 #pragma unroll
             for (int cidx = 0; cidx < kKeys; ++cidx) {
-                const float p = (lg[cidx] == -INFINITY) ? 0.f : exp2f(lg[cidx] - m_new);
+                const float2 sd = sm.side_v[b][cidx];
+                const float p = ex2(lg[cidx] - shift);                  // 2^-inf = 0 for masked keys
                 psum += p;
-                pz = fmaf(p, sm.side[b][3][cidx], pz);
-                lg[cidx] = p * sm.side[b][2][cidx];            // P' = p * s_V
+                pz = fmaf(p, sd.y, pz);
+                lg[cidx] = p * sd.x;                                   // P' = p * s_V
             }
             l_run = fmaf(l_run, corr, psum);
             pz_run = fmaf(pz_run, corr, pz);
@@ -404,7 +481,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                     break;
                 }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, corr != 1.f)) {        // rescale this warp's O rows
+                if (__any_sync(0xffffffffu, bump)) {        // rescale this warp's O rows
 #pragma unroll
                     for (int cb = 0; cb < D / 32; ++cb) {
                         float ov[32];
