@@ -5,12 +5,15 @@
 //                       validates capacity and widths (a bad width rejects the sequence's
 //                       write for every head) and assigns each new token's record offset
 //                       (prefix sum of record sizes b*D/4 in token order).
-//   write_quant_kernel  one warp per (token, head): for K and for V, min/max over the
-//                       head_dim values, s = (max - min)/(2^b - 1), z = min, codes
+//   write_quant_kernel  one CTA per tile of tokens x heads staged by bulk copies: for K
+//                       and for V of every (token, head), min/max over the head_dim
+//                       values, s = (max - min)/(2^b - 1), z = min, codes
 //                       rint((x - z)/s) in IEEE fp32 round-to-nearest-even (s == 0 -> 0),
 //                       packed LSB-first into the record; (s, z) into the side table;
 //                       commits the new length and stream end of accepted sequences.
 // HBM traffic per (token, head): reads 2*D*2 bytes, writes b*D/4 + 16 + 4 bytes.
+#include <algorithm>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -118,103 +121,180 @@ write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *
     }
 }
 
-// D/4 lanes quantize one vector (4 channels per lane); a warp covers K and V of one
-// (token, head): sequentially for D = 128, side by side for D = 64.
-template <int D>
-__global__ void write_quant_kernel(CacheView c, const __half *__restrict__ k,
-                                   const __half *__restrict__ v, const uint8_t *__restrict__ bits,
-                                   const int32_t *__restrict__ cu, int64_t n_tok, uint32_t gen)
+// Staging of the quantize kernel: each CTA copies the fp16 K and V rows of T tokens x HG
+// heads (at most kWqHalves values per tensor) into shared memory with two bulk copies.
+constexpr int kWqThreads = 256;
+constexpr int kWqHalves = 8192;          // 16 KB of K and 16 KB of V per CTA
+constexpr int kWqMaxPairs = kWqHalves / 64;
+
+struct WqPair {                          // one (token, head) of the CTA
+    int64_t slot;                        // side-table slot
+    int64_t rec;                         // byte offset of the record in the record array
+    uint32_t meta;                       // width code in bits 0-1
+    int32_t ok;                          // 0: not written (rejected write or bad call)
+};
+
+// Codes are rint(fl(u / s)) with u = fl(x - z), clamped at 0 (u >= 0 and u <= fl(max - min),
+// so a finite code never exceeds 2^b - 1; a NaN gives 0). The quotient is first formed as
+// q = fl(u * fl(1 / s)). Standard rounding-error analysis bounds |q - u/s| by
+// (2 * 2^-24 + 2^-48) |u/s| and |fl(u/s) - u/s| by 2^-24 |u/s|; with |u/s| <= 256 the two
+// quotients differ by less than 2^-14. So unless q lies within 2^-13 of a half-integer,
+// both round to the same integer; a lane holding such a q recomputes its codes with the
+// IEEE division. The codes are therefore those of the correctly rounded quotient.
+__device__ __forceinline__ void quant8(const float (&x)[8], float z, float sc, uint32_t (&cd)[8])
 {
-    constexpr int VL = D / 4;            // lanes per vector
-    constexpr int PER_ITER = 32 / VL;    // vectors per warp iteration
-    const int lane = threadIdx.x & 31;
-    const int li = lane % VL;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int H = c.H;
-    if (warp >= n_tok * H) return;
-    const int64_t tk = warp / H;
-    const int h = (int)(warp % H);
-
-    // sequence of token tk: last s with cu[s] <= tk
-    int lo = 0, hi = c.B;            // invariant: cu[lo] <= tk < cu[hi]
-    while (hi - lo > 1) {
-        int mid = (lo + hi) >> 1;
-        if (cu[mid] <= tk) lo = mid;
-        else hi = mid;
-    }
-    const int s = lo;
-    if (tk >= cu[s + 1]) return;     // cu_seqlens violated its contract (flagged by the scan)
-    const int start = c.wstart[s * H + h];
-    if (start < 0 || c.bad[s] == gen) return;     // this sequence's write was rejected
-    if (tk == cu[s] && lane == 0) {               // commit the new length and stream end
-        c.len[s * H + h] = start + (cu[s + 1] - cu[s]);
-        c.end[s * H + h] = c.wend[s * H + h];
-    }
-    const int64_t j = start + (tk - cu[s]);
-    const int64_t slot = slot_of(c, s, h, j);
-    const uint32_t meta = c.meta[slot];
-    const int wc = meta & 3u;
-    const int b = 2 << wc;           // 2, 4, 8, 16
-    uint8_t *rec = stream_of(c, s, h) + (meta & ~15u);
-    const int part_bytes = b * D / 8;
-
-    float s_part[2] = {1.0f, 1.0f}, z_part[2] = {0.0f, 0.0f};
+    const float r = __frcp_rn(sc);
+    bool near_half = false;
 #pragma unroll
-    for (int it = 0; it < 2 / PER_ITER; ++it) {
-        const int part = it * PER_ITER + lane / VL;   // 0 = K, 1 = V
-        const __half *src = (part == 0 ? k : v) + (tk * H + h) * D + 4 * li;
-        const uint2 raw = *reinterpret_cast<const uint2 *>(src);
-        uint8_t *dst = rec + part * part_bytes;
-        if (b == 16) {
-            *reinterpret_cast<uint2 *>(dst + 8 * li) = raw;
-            continue;
+    for (int e = 0; e < 8; ++e) {
+        const float q = __fmul_rn(__fsub_rn(x[e], z), r);
+        const float c = rintf(q);
+        near_half |= fabsf(q - c) > 0.4998779296875f;       // 0.5 - 2^-13
+        cd[e] = __float2uint_rz(fmaxf(c, 0.0f));
+    }
+    if (near_half) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            cd[e] = __float2uint_rz(fmaxf(rintf(__fdiv_rn(__fsub_rn(x[e], z), sc)), 0.0f));
+    }
+}
+
+// One CTA per tile of T tokens x HG heads. Warp 0 starts two bulk copies (the tile's K and
+// V rows are contiguous when HG = H, else one copy per token and tensor); meanwhile every
+// thread resolves the destination of one (token, head): its sequence (binary search of
+// cu_seqlens), the call's verdict, the write start, and the record offset the scan kernel
+// assigned. Then each vector of D values is quantized by D/8 lanes from shared memory.
+template <int D>
+__global__ void __launch_bounds__(kWqThreads)
+write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__restrict__ v,
+                   const int32_t *__restrict__ cu, int64_t n_tok, uint32_t gen, int T, int HG)
+{
+    constexpr int VL = D / 8;                // lanes per vector, 8 values per lane
+    constexpr int VPW = 32 / VL;             // vectors per warp pass
+    extern __shared__ __align__(128) uint8_t wq_smem[];
+    __shared__ uint64_t bar;
+    __shared__ WqPair pairs[kWqMaxPairs];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = c.H;
+    const int64_t t0 = (int64_t)blockIdx.x * T;
+    const int h0 = blockIdx.y * HG;
+    const int Tc = (int)(n_tok - t0 < T ? n_tok - t0 : T);
+    const int HGc = min(HG, H - h0);
+    const uint32_t tensor_bytes = (uint32_t)(Tc * HGc * D * 2);
+    __half *sk = reinterpret_cast<__half *>(wq_smem);
+    __half *sv = sk + kWqHalves;
+
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        if (lane == 0) mbar_arrive_expect_tx(&bar, 2 * tensor_bytes);
+        __syncwarp();
+        if (HGc == H) {
+            if (lane < 2)
+                bulk_g2s(lane ? sv : sk, (lane ? v : k) + t0 * H * D, tensor_bytes, &bar);
+        } else {
+            for (int i = lane; i < 2 * Tc; i += 32) {
+                const int j = i >> 1;
+                bulk_g2s((i & 1 ? sv : sk) + j * HGc * D,
+                         (i & 1 ? v : k) + ((t0 + j) * H + h0) * D, HGc * D * 2, &bar);
+            }
         }
-        const __half2 h01 = *reinterpret_cast<const __half2 *>(&raw.x);
-        const __half2 h23 = *reinterpret_cast<const __half2 *>(&raw.y);
-        float x[4] = {__low2float(h01), __high2float(h01), __low2float(h23), __high2float(h23)};
-        float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
-        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    }
+
+    for (int i = tid; i < Tc * HGc; i += kWqThreads) {
+        const int64_t tk = t0 + i / HGc;
+        const int h = h0 + i % HGc;
+        WqPair pr;
+        pr.slot = 0;
+        pr.rec = 0;
+        pr.meta = 0;
+        pr.ok = 0;
+        int lo = 0, hi = c.B;                // cu[lo] <= tk < cu[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (cu[mid] <= tk) lo = mid;
+            else hi = mid;
+        }
+        const int s = lo;
+        if (tk < cu[s + 1] && c.bad[s] != gen) {
+            const int st = c.wstart[s * H + h];
+            if (st >= 0) {
+                const int64_t t_in_seq = tk - cu[s];
+                pr.slot = slot_of(c, s, h, st + t_in_seq);
+                pr.meta = c.meta[pr.slot];
+                pr.rec = slot_of(c, s, h, 0) * (int64_t)(4 * D) + (pr.meta & ~15u);
+                pr.ok = 1;
+                if (t_in_seq == 0) {          // commit the new length and stream end
+                    c.len[s * H + h] = st + (cu[s + 1] - cu[s]);
+                    c.end[s * H + h] = c.wend[s * H + h];
+                }
+            }
+        }
+        pairs[i] = pr;
+    }
+    __syncthreads();
+    if (!mbar_wait(&bar, 0, c.status)) return;
+
+    const int n_vec = 2 * Tc * HGc;          // vector vi: pair vi / 2, K (even) or V (odd)
+    const int li = lane % VL;
+    for (int vb = warp * VPW; vb < n_vec; vb += (kWqThreads / 32) * VPW) {
+        const int vi = vb + lane / VL;
+        const bool in_range = vi < n_vec;
+        const int pi = vi >> 1, part = vi & 1;
+        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+        if (in_range) raw = *reinterpret_cast<const uint4 *>((part ? sv : sk) + pi * D + 8 * li);
+        float x[8];
+        {
+            const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x[2 * e] = __low2float(h2[e]);
+                x[2 * e + 1] = __high2float(h2[e]);
+            }
+        }
+        float mn = x[0], mx = x[0];
+#pragma unroll
+        for (int e = 1; e < 8; ++e) {
+            mn = fminf(mn, x[e]);
+            mx = fmaxf(mx, x[e]);
+        }
 #pragma unroll
         for (int d = VL / 2; d >= 1; d >>= 1) {
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, d));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
         }
-        const float top = (float)((1u << b) - 1u);
-        // zeros are stored as +0 (the min scan may meet -0 or +0 first)
-        const float sc = __fadd_rn(__fdiv_rn(__fsub_rn(mx, mn), top), 0.0f);
-        const float z = __fadd_rn(mn, 0.0f);
-        uint32_t packed = 0;
+        if (!in_range) continue;
+        const WqPair pr = pairs[pi];
+        if (!pr.ok) continue;
+        const int b = 2 << (pr.meta & 3u);
+        uint8_t *dst = c.rec + pr.rec + part * (b * D / 8);
+        float sc = 1.0f, z = 0.0f;
+        if (b == 16) {
+            reinterpret_cast<uint4 *>(dst)[li] = raw;
+        } else {
+            const float top = (float)((1u << b) - 1u);
+            // zeros are stored as +0 (the min scan may meet -0 or +0 first)
+            sc = __fadd_rn(__fdiv_rn(__fsub_rn(mx, mn), top), 0.0f);
+            z = __fadd_rn(mn, 0.0f);
+            uint32_t cd[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            if (sc != 0.0f) quant8(x, z, sc, cd);
+            if (b == 8) {
+                const uint32_t w0 = cd[0] | cd[1] << 8 | cd[2] << 16 | cd[3] << 24;
+                const uint32_t w1 = cd[4] | cd[5] << 8 | cd[6] << 16 | cd[7] << 24;
+                reinterpret_cast<uint2 *>(dst)[li] = make_uint2(w0, w1);
+            } else {
+                uint32_t w = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            uint32_t code = 0;
-            if (sc != 0.0f) {
-                float r = rintf(__fdiv_rn(__fsub_rn(x[e], z), sc));
-                r = fminf(fmaxf(r, 0.0f), top);
-                code = (uint32_t)r;
+                for (int e = 0; e < 8; ++e) w |= cd[e] << (e * b);
+                if (b == 4) reinterpret_cast<uint32_t *>(dst)[li] = w;
+                else reinterpret_cast<uint16_t *>(dst)[li] = (uint16_t)w;
             }
-            packed |= code << (e * b);
         }
-        if (b == 2) dst[li] = (uint8_t)packed;
-        else if (b == 4) reinterpret_cast<uint16_t *>(dst)[li] = (uint16_t)packed;
-        else reinterpret_cast<uint32_t *>(dst)[li] = packed;
-        s_part[it] = sc;
-        z_part[it] = z;
+        if (li == 0) reinterpret_cast<float2 *>(&c.side[pr.slot])[part] = make_float2(sc, z);
     }
-    // side entry (s_K, z_K, s_V, z_V): K values live in lane 0, V values in lane 0 (D = 128,
-    // second iteration) or lane VL (D = 64)
-    float sK, zK, sV, zV;
-    if (PER_ITER == 1) {
-        sK = s_part[0];
-        zK = z_part[0];
-        sV = s_part[1 % (2 / PER_ITER)];
-        zV = z_part[1 % (2 / PER_ITER)];
-    } else {
-        sK = __shfl_sync(0xffffffffu, s_part[0], 0);
-        zK = __shfl_sync(0xffffffffu, z_part[0], 0);
-        sV = __shfl_sync(0xffffffffu, s_part[0], VL);
-        zV = __shfl_sync(0xffffffffu, z_part[0], VL);
-    }
-    if (lane == 0) c.side[slot] = make_float4(sK, zK, sV, zV);
 }
 
 } // namespace
@@ -236,13 +316,17 @@ cudaError_t launch_write(kvq_cache *cache, const __half *k, const __half *v,
         }
     }
     if (n_tok > 0) {
-        const int64_t warps = n_tok * c.H;
-        const int threads = 256;
-        const int64_t blocks = (warps * 32 + threads - 1) / threads;
+        // tiles of T tokens x HG heads, at most kWqHalves values per tensor; one token per
+        // tile when the call is too short to give every SM a few tiles
+        const int HG = std::min(c.H, kWqHalves / c.D);
+        int T = std::max(1, kWqHalves / (HG * c.D));
+        if (n_tok < (int64_t)T * 2 * num_sms()) T = 1;
+        const dim3 grid((unsigned)((n_tok + T - 1) / T), (unsigned)((c.H + HG - 1) / HG));
+        const size_t smem = 2 * kWqHalves * sizeof(__half);
         if (c.D == 128)
-            write_quant_kernel<128><<<(unsigned)blocks, threads, 0, st>>>(c, k, v, bits, cu, n_tok, gen);
+            write_quant_kernel<128><<<grid, kWqThreads, smem, st>>>(c, k, v, cu, n_tok, gen, T, HG);
         else
-            write_quant_kernel<64><<<(unsigned)blocks, threads, 0, st>>>(c, k, v, bits, cu, n_tok, gen);
+            write_quant_kernel<64><<<grid, kWqThreads, smem, st>>>(c, k, v, cu, n_tok, gen, T, HG);
     }
     profile_after(st);
     return cudaGetLastError();
