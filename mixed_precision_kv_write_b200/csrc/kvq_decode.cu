@@ -6,13 +6,14 @@
 //                         work, local heads are clamped to keys [max(0, t - w), t], full
 //                         heads read [0, t]; each range is cut into near-equal items of at
 //                         most 512 keys, listed on the device (no host round trip).
-//   decode_splitk_kernel  two CTAs per SM. A producer warp walks the CTA's items in
-//                         stages of at most 64 keys and 16 KB of records: it reads the
-//                         stage's record offsets, sorts the keys by width once (so the
+//   decode_splitk_kernel  three CTAs per SM. A producer warp walks the CTA's items in
+//                         stages of at most 128 keys and 24 KB of records: it keeps a ring
+//                         of record-offset windows fetched ahead, cuts each stage at the
+//                         byte budget, sorts the stage's keys by width once (so the
 //                         consumers' 4-key steps rarely mix widths), and streams the stage's
 //                         contiguous record bytes, side entries and (for a new item) the
-//                         query into shared memory with 1-D bulk copies (4-stage mbarrier
-//                         pipeline). Eight consumer warps split each stage's keys: 8 lanes
+//                         query into shared memory with 1-D bulk copies (2-stage mbarrier
+//                         pipeline). Five consumer warps split each stage's keys: 8 lanes
 //                         per key, 16 channels per lane, K dot product -> logit -> online
 //                         softmax kept per 8-lane group -> V accumulation, all in registers;
 //                         the groups' states are merged once per item into a partial
@@ -37,9 +38,9 @@
 namespace kvq {
 namespace {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 5;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kStages = 3;                        // record stages in flight per CTA
+constexpr int kStages = 2;                        // record stages in flight per CTA
 constexpr int kWin = kDecodeWindowKeys;           // keys per window of record offsets
 constexpr uint32_t kStageRecBytes = 24576;        // record bytes per stage, at most
 constexpr int kPermSlots = kWin + 32;             // width-sorted keys padded to whole chunks
@@ -345,7 +346,7 @@ __device__ __forceinline__ void process_key(KeyState &st, const QRegs &qr, float
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
 decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
 {
     constexpr int GROUP = D / 16;                 // lanes per key (16 channels per lane)
@@ -694,7 +695,7 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const __half *q, const uint8
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    const int grid = (int)std::min<int64_t>(cache->work.max_items, 2 * (int64_t)num_sms());
+    const int grid = (int)std::min<int64_t>(cache->work.max_items, 3 * (int64_t)num_sms());
     profile_before(st);
     decode_splitk_kernel<D><<<grid, kThreads, smem, st>>>(c, q, cache->work);
     profile_after(st);

@@ -134,28 +134,78 @@ struct WqPair {                          // one (token, head) of the CTA
     int32_t ok;                          // 0: not written (rejected write or bad call)
 };
 
-// Codes are rint(fl(u / s)) with u = fl(x - z), clamped at 0 (u >= 0 and u <= fl(max - min),
-// so a finite code never exceeds 2^b - 1; a NaN gives 0). The quotient is first formed as
-// q = fl(u * fl(1 / s)). Standard rounding-error analysis bounds |q - u/s| by
-// (2 * 2^-24 + 2^-48) |u/s| and |fl(u/s) - u/s| by 2^-24 |u/s|; with |u/s| <= 256 the two
-// quotients differ by less than 2^-14. So unless q lies within 2^-13 of a half-integer,
-// both round to the same integer; a lane holding such a q recomputes its codes with the
-// IEEE division. The codes are therefore those of the correctly rounded quotient.
-__device__ __forceinline__ void quant8(const float (&x)[8], float z, float sc, uint32_t (&cd)[8])
+// Codes are rint(fl(u / s)) with u = fl(x - z), clamped to [0, 2^b - 1].
+// The correctly rounded quotient fl(u / s) is formed with Markstein's correction
+// (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): with y = RN(1/s) and the faithful q0 = RN(u y),
+// the remainder r = u - s q0 is exact in one FMA, and RN(q0 + r y) = RN(u / s). Because
+// 0 <= u <= fl(max - min) the quotient lies in [0, 2^b - 1 + 2^-14], so rint never leaves the
+// code range. rint is taken by adding 1.5 * 2^23: for 0 <= q < 2^22 the sum is
+// 1.5 * 2^23 + rint(q) exactly (round-to-nearest-even), the integer in the low mantissa bits.
+// A NaN quotient (NaN or infinite inputs) is caught by a running sum and the lane falls
+// back to the plain clamped formula, which maps it to code 0.
+constexpr float kRoundMagic = 12582912.0f;          // 1.5 * 2^23
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+
+// Quantizes a lane's NC chunks of 8 fp16 values to BITS-bit codes. Chunk j holds channels
+// 8 * (j * VL + li) .. + 7 of the vector, so its 8 codes fill BITS bytes of the part at byte
+// BITS * (j * VL + li), and the VL lanes of a vector store adjacent chunks.
+template <int BITS, int NC, int VL>
+__device__ __forceinline__ void quant_store(const uint4 (&raw)[NC], float z, float sc,
+                                            uint8_t *dst, int li)
 {
-    const float r = __frcp_rn(sc);
-    bool near_half = false;
+    uint32_t w[NC][2];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float q = __fmul_rn(__fsub_rn(x[e], z), r);
-        const float c = rintf(q);
-        near_half |= fabsf(q - c) > 0.4998779296875f;       // 0.5 - 2^-13
-        cd[e] = __float2uint_rz(fmaxf(c, 0.0f));
+    for (int j = 0; j < NC; ++j) w[j][0] = w[j][1] = 0u;
+    if (sc != 0.0f) {
+        const float y = __frcp_rn(sc);
+        float nan_probe = 0.0f;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+            const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[j]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float x = (e & 1) ? __high2float(h2[e >> 1]) : __low2float(h2[e >> 1]);
+                const float u = __fsub_rn(x, z);
+                const float q0 = __fmul_rn(u, y);
+                const float r = __fmaf_rn(-sc, q0, u);
+                const float q = __fmaf_rn(r, y, q0);
+                const float t = __fadd_rn(q, kRoundMagic);
+                nan_probe = __fadd_rn(nan_probe, q);
+                // code << shift; the 1.5 * 2^23 bits are taken off below
+                w[j][(e * BITS) >> 5] += __float_as_uint(t) << ((e * BITS) & 31);
+            }
+        }
+        constexpr int kWordBits = BITS * 8 < 32 ? BITS * 8 : 32;   // code bits per word
+        uint32_t magic = 0u;
+#pragma unroll
+        for (int sh = 0; sh < kWordBits; sh += BITS) magic += kRoundMagicBits << sh;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+            w[j][0] -= magic;
+            if (BITS == 8) w[j][1] -= magic;
+        }
+        if (nan_probe != nan_probe) {
+            const float top = (float)((1u << BITS) - 1u);
+#pragma unroll
+            for (int j = 0; j < NC; ++j) {
+                const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[j]);
+                w[j][0] = w[j][1] = 0u;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float x = (e & 1) ? __high2float(h2[e >> 1]) : __low2float(h2[e >> 1]);
+                    const float c = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x, z), sc)), 0.0f), top);
+                    w[j][(e * BITS) >> 5] |= __float2uint_rz(c) << ((e * BITS) & 31);
+                }
+            }
+        }
     }
-    if (near_half) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            cd[e] = __float2uint_rz(fmaxf(rintf(__fdiv_rn(__fsub_rn(x[e], z), sc)), 0.0f));
+    for (int j = 0; j < NC; ++j) {
+        const int chunk = j * VL + li;
+        if (BITS == 8) reinterpret_cast<uint2 *>(dst)[chunk] = make_uint2(w[j][0], w[j][1]);
+        else if (BITS == 4) reinterpret_cast<uint32_t *>(dst)[chunk] = w[j][0];
+        else reinterpret_cast<uint16_t *>(dst)[chunk] = (uint16_t)w[j][0];
     }
 }
 
@@ -163,17 +213,20 @@ __device__ __forceinline__ void quant8(const float (&x)[8], float z, float sc, u
 // V rows are contiguous when HG = H, else one copy per token and tensor); meanwhile every
 // thread resolves the destination of one (token, head): its sequence (binary search of
 // cu_seqlens), the call's verdict, the write start, and the record offset the scan kernel
-// assigned. Then each vector of D values is quantized by D/8 lanes from shared memory.
+// assigned. Then each vector of D values is quantized by D/32 lanes from shared memory.
 template <int D>
 __global__ void __launch_bounds__(kWqThreads)
 write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__restrict__ v,
                    const int32_t *__restrict__ cu, int64_t n_tok, uint32_t gen, int T, int HG)
 {
-    constexpr int VL = D / 8;                // lanes per vector, 8 values per lane
+    constexpr int NC = 4;                    // chunks of 8 values per lane
+    constexpr int VL = D / (8 * NC);         // lanes per vector
     constexpr int VPW = 32 / VL;             // vectors per warp pass
     extern __shared__ __align__(128) uint8_t wq_smem[];
     __shared__ uint64_t bar;
     __shared__ WqPair pairs[kWqMaxPairs];
+    __shared__ uint8_t order[kWqMaxPairs];   // written pairs sorted by width
+    __shared__ int n_written;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = c.H;
     const int64_t t0 = (int64_t)blockIdx.x * T;
@@ -236,62 +289,70 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
         pairs[i] = pr;
     }
     __syncthreads();
+    // Sort the written pairs by width, so the lanes of a warp pass mostly share one code path.
+    if (warp == 0) {
+        const int n_pairs = Tc * HGc;
+        int base = 0;
+        for (int cls = 0; cls < 4; ++cls) {
+            for (int i0 = 0; i0 < n_pairs; i0 += 32) {
+                const int i = i0 + lane;
+                const bool in = i < n_pairs && pairs[i].ok && (int)(pairs[i].meta & 3u) == cls;
+                const uint32_t m = __ballot_sync(0xffffffffu, in);
+                if (in) order[base + __popc(m & ((1u << lane) - 1u))] = (uint8_t)i;
+                base += __popc(m);
+            }
+        }
+        if (lane == 0) n_written = base;
+    }
+    __syncthreads();
     if (!mbar_wait(&bar, 0, c.status)) return;
 
-    const int n_vec = 2 * Tc * HGc;          // vector vi: pair vi / 2, K (even) or V (odd)
+    const int n_vec = 2 * n_written;         // vector vi: pair order[vi / 2], K (even) or V (odd)
     const int li = lane % VL;
     for (int vb = warp * VPW; vb < n_vec; vb += (kWqThreads / 32) * VPW) {
         const int vi = vb + lane / VL;
         const bool in_range = vi < n_vec;
-        const int pi = vi >> 1, part = vi & 1;
-        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-        if (in_range) raw = *reinterpret_cast<const uint4 *>((part ? sv : sk) + pi * D + 8 * li);
-        float x[8];
-        {
-            const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw);
+        const int pi = in_range ? order[vi >> 1] : 0, part = vi & 1;
+        uint4 raw[NC];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                x[2 * e] = __low2float(h2[e]);
-                x[2 * e + 1] = __high2float(h2[e]);
-            }
-        }
-        float mn = x[0], mx = x[0];
+        for (int j = 0; j < NC; ++j) raw[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (in_range) {
+            const uint4 *src = reinterpret_cast<const uint4 *>((part ? sv : sk) + pi * D);
 #pragma unroll
-        for (int e = 1; e < 8; ++e) {
-            mn = fminf(mn, x[e]);
-            mx = fmaxf(mx, x[e]);
+            for (int j = 0; j < NC; ++j) raw[j] = src[j * VL + li];
         }
+        const __half2 (&h2)[4 * NC] = *reinterpret_cast<const __half2 (*)[4 * NC]>(raw);
+        // min and max in fp16 (exact); (min, -max) travel as one half2 through the shuffles
+        __half2 lo2 = h2[0], hi2 = h2[0];
+#pragma unroll
+        for (int e = 1; e < 4 * NC; ++e) {
+            lo2 = __hmin2(lo2, h2[e]);
+            hi2 = __hmax2(hi2, h2[e]);
+        }
+        __half2 mm = __halves2half2(__hmin(__low2half(lo2), __high2half(lo2)),
+                                    __hneg(__hmax(__low2half(hi2), __high2half(hi2))));
 #pragma unroll
         for (int d = VL / 2; d >= 1; d >>= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, d));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+            const uint32_t o = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t *>(&mm), d);
+            mm = __hmin2(mm, *reinterpret_cast<const __half2 *>(&o));
         }
         if (!in_range) continue;
         const WqPair pr = pairs[pi];
-        if (!pr.ok) continue;
         const int b = 2 << (pr.meta & 3u);
         uint8_t *dst = c.rec + pr.rec + part * (b * D / 8);
         float sc = 1.0f, z = 0.0f;
         if (b == 16) {
-            reinterpret_cast<uint4 *>(dst)[li] = raw;
+#pragma unroll
+            for (int j = 0; j < NC; ++j) reinterpret_cast<uint4 *>(dst)[j * VL + li] = raw[j];
         } else {
+            const float mn = __low2float(mm), mx = -__high2float(mm);
             const float top = (float)((1u << b) - 1u);
             // zeros are stored as +0 (the min scan may meet -0 or +0 first)
             sc = __fadd_rn(__fdiv_rn(__fsub_rn(mx, mn), top), 0.0f);
             z = __fadd_rn(mn, 0.0f);
-            uint32_t cd[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-            if (sc != 0.0f) quant8(x, z, sc, cd);
-            if (b == 8) {
-                const uint32_t w0 = cd[0] | cd[1] << 8 | cd[2] << 16 | cd[3] << 24;
-                const uint32_t w1 = cd[4] | cd[5] << 8 | cd[6] << 16 | cd[7] << 24;
-                reinterpret_cast<uint2 *>(dst)[li] = make_uint2(w0, w1);
-            } else {
-                uint32_t w = 0;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) w |= cd[e] << (e * b);
-                if (b == 4) reinterpret_cast<uint32_t *>(dst)[li] = w;
-                else reinterpret_cast<uint16_t *>(dst)[li] = (uint16_t)w;
-            }
+            if (b == 8) quant_store<8, NC, VL>(raw, z, sc, dst, li);
+            else if (b == 4) quant_store<4, NC, VL>(raw, z, sc, dst, li);
+            else quant_store<2, NC, VL>(raw, z, sc, dst, li);
         }
         if (li == 0) reinterpret_cast<float2 *>(&c.side[pr.slot])[part] = make_float2(sc, z);
     }
