@@ -3,7 +3,7 @@
 //
 // Two launches per call:
 //   prefill_sched_kernel  one CTA per (sequence, head): compacts the call's queries by
-//                         mode into a local list and a full list, cuts each into tiles of
+//                         mode (stable) into a local list and a full list, cuts each into tiles of
 //                         at most 128 queries, and writes zeros for skip queries. A local
 //                         tile reads keys [min(t) - w, max(t)], a full tile [0, max(t)],
 //                         so local rows do not pay for a full tile's range.
@@ -544,14 +544,18 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     }
 }
 
-// One CTA per (sequence, head): compaction of the call's queries by mode.
-__global__ void __launch_bounds__(256)
+// One CTA per (sequence, head): stable compaction of the call's queries by mode, 4096
+// queries per pass (4 consecutive queries per thread, block prefix sum of the per-thread
+// counts packed as local | full << 16). Skip rows are zeroed a whole row per warp store.
+constexpr int kSchedThreads = 1024, kSchedPer = 4;
+
+__global__ void __launch_bounds__(kSchedThreads)
 prefill_sched_kernel(CacheView c, const uint8_t *__restrict__ modes, const int32_t *__restrict__ cu,
                      int64_t n_tok, int D, float *__restrict__ out, PfTile *__restrict__ tiles,
                      int32_t *__restrict__ tile_count, int32_t *__restrict__ qidx)
 {
-    __shared__ int wl[8], wf[8];
-    __shared__ int tot_l, tot_f;
+    __shared__ int wsum[kSchedThreads / 32];
+    __shared__ int carry_l, carry_f;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int H = c.H, sh = blockIdx.x, s = sh / H, h = sh % H;
     const int64_t t0 = cu[s], t1 = cu[s + 1];
@@ -564,49 +568,74 @@ prefill_sched_kernel(CacheView c, const uint8_t *__restrict__ modes, const int32
     }
     int32_t *region = qidx + t0 * H + (int64_t)h * n;    // local from the front, full from the back
     if (tid == 0) {
-        tot_l = 0;
-        tot_f = 0;
+        carry_l = 0;
+        carry_f = 0;
     }
-    __syncthreads();
-    for (int base = 0; base < n; base += 256) {
-        const int i = base + tid;
-        int m = -1;
-        if (i < n) {
-            m = modes[(t0 + i) * H + h];
-            if (m > KVQ_MODE_FULL) {
-                set_status(c.status, KVQ_ERR_MODE);
-                m = KVQ_MODE_SKIP;
+    constexpr int kPass = kSchedThreads * kSchedPer;
+    for (int base = 0; base < n; base += kPass) {
+        int m[kSchedPer];
+        int cnt = 0;                                     // local | full << 16
+#pragma unroll
+        for (int k = 0; k < kSchedPer; ++k) {
+            const int i = base + tid * kSchedPer + k;
+            m[k] = -1;
+            if (i < n) {
+                m[k] = modes[(t0 + i) * H + h];
+                if (m[k] > KVQ_MODE_FULL) {
+                    set_status(c.status, KVQ_ERR_MODE);
+                    m[k] = KVQ_MODE_SKIP;
+                }
             }
-            if (m == KVQ_MODE_SKIP) {
-                float4 *dst = reinterpret_cast<float4 *>(out + ((t0 + i) * H + h) * D);
-                for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            cnt += (m[k] == KVQ_MODE_LOCAL) ? 1 : (m[k] == KVQ_MODE_FULL) ? (1 << 16) : 0;
         }
-        const uint32_t bl = __ballot_sync(0xffffffffu, m == KVQ_MODE_LOCAL);
-        const uint32_t bf = __ballot_sync(0xffffffffu, m == KVQ_MODE_FULL);
-        if (lane == 0) {
-            wl[wid] = __popc(bl);
-            wf[wid] = __popc(bf);
+        int incl = cnt;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        if (lane == 31) wsum[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            const int x = wsum[lane];
+            int y = x;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, y, d);
+                if (lane >= d) y += o;
+            }
+            wsum[lane] = y - x;                          // exclusive prefix of the warps
         }
         __syncthreads();
-        int pl = tot_l, pf = tot_f;
-        for (int q2 = 0; q2 < wid; ++q2) {
-            pl += wl[q2];
-            pf += wf[q2];
+        const int pre = wsum[wid] + incl - cnt;
+        int pl = carry_l + (pre & 0xFFFF), pf = carry_f + (pre >> 16);
+#pragma unroll
+        for (int k = 0; k < kSchedPer; ++k) {
+            const int i = base + tid * kSchedPer + k;
+            if (m[k] == KVQ_MODE_LOCAL) region[pl++] = i;
+            if (m[k] == KVQ_MODE_FULL) region[n - 1 - (pf++)] = i;
         }
-        const uint32_t lt = (1u << lane) - 1u;
-        if (m == KVQ_MODE_LOCAL) region[pl + __popc(bl & lt)] = i;
-        if (m == KVQ_MODE_FULL) region[n - 1 - (pf + __popc(bf & lt))] = i;
-        __syncthreads();
-        if (tid == 0) {
-            for (int q2 = 0; q2 < 8; ++q2) {
-                tot_l += wl[q2];
-                tot_f += wf[q2];
+        // zeros for skip rows: one row of D floats per warp store
+#pragma unroll
+        for (int k = 0; k < kSchedPer; ++k) {
+            uint32_t skip = __ballot_sync(0xffffffffu, m[k] == KVQ_MODE_SKIP);
+            while (skip) {
+                const int src = __ffs(skip) - 1;
+                skip &= skip - 1;
+                const int64_t row = (t0 + base + (wid * 32 + src) * kSchedPer + k) * H + h;
+                if (lane < D / 4)
+                    reinterpret_cast<float4 *>(out + row * D)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
+        }
+        __syncthreads();
+        if (tid == kSchedThreads - 1) {                  // its pl, pf are the pass totals
+            carry_l = pl;
+            carry_f = pf;
         }
         __syncthreads();
     }
     if (tid == 0) {
+        const int tot_l = carry_l, tot_f = carry_f;
         const int ntl = (tot_l + kQRows - 1) / kQRows, ntf = (tot_f + kQRows - 1) / kQRows;
         const int first = atomicAdd(tile_count, ntl + ntf);
         const int32_t off = (int32_t)(t0 * H + (int64_t)h * n);
@@ -626,7 +655,7 @@ cudaError_t run_tc(const kvq_cache *cache, const __half *q, const uint8_t *modes
     PfTile *tiles = reinterpret_cast<PfTile *>(cache->pf_tiles);
     cudaError_t e = cudaMemsetAsync(cache->pf_count, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return e;
-    prefill_sched_kernel<<<c.B * c.H, 256, 0, st>>>(c, modes, cu, n_tok, D, out, tiles, cache->pf_count,
+    prefill_sched_kernel<<<c.B * c.H, kSchedThreads, 0, st>>>(c, modes, cu, n_tok, D, out, tiles, cache->pf_count,
                                                      cache->pf_qidx);
     const int64_t max_tiles = n_tok * c.H / kQRows + 2LL * c.B * c.H;
     const size_t smem = sizeof(PfSmem<D>) + 1024;

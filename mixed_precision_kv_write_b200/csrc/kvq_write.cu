@@ -24,17 +24,17 @@ namespace {
 // and assigns the new tokens' record offsets with a parallel prefix sum of the record
 // sizes b*D/4. The new length/end are committed by the quantize kernel, which sees the
 // per-sequence verdict of every head.
-template <int TPS>
-__global__ void __launch_bounds__(256)
+template <int TPS, int BS = (TPS < 256 ? 256 : TPS)>
+__global__ void __launch_bounds__(BS)
 write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *__restrict__ cu,
                   int64_t n_tok, uint32_t gen)
 {
     constexpr int PER = 8;                       // tokens per thread per pass
     constexpr int WARPS = TPS / 32;
-    __shared__ uint32_t wsum[256 / 32];
+    __shared__ uint32_t wsum[BS / 32];
     const int tid = threadIdx.x % TPS, lane = threadIdx.x & 31;
     const int grp = threadIdx.x / TPS, wig = tid >> 5;     // group in block, warp in group
-    const int64_t gsh = (int64_t)blockIdx.x * (256 / TPS) + grp;
+    const int64_t gsh = (int64_t)blockIdx.x * (BS / TPS) + grp;
     const int H = c.H;
     if (gsh >= (int64_t)c.B * H) return;         // whole group exits together
     const int s = (int)(gsh / H), h = (int)(gsh % H), sh = s * H + h;
@@ -373,7 +373,7 @@ cudaError_t launch_write(kvq_cache *cache, const __half *k, const __half *v,
             const int64_t blocks = (groups + 7) / 8;
             write_scan_kernel<32><<<(unsigned)blocks, 256, 0, st>>>(c, bits, cu, n_tok, gen);
         } else {
-            write_scan_kernel<256><<<(unsigned)groups, 256, 0, st>>>(c, bits, cu, n_tok, gen);
+            write_scan_kernel<1024><<<(unsigned)groups, 1024, 0, st>>>(c, bits, cu, n_tok, gen);
         }
     }
     if (n_tok > 0) {
