@@ -167,114 +167,115 @@ __global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ mod
 }
 
 // ---- per-width dot products and accumulations for one lane's 16 channels ----------
+// Channels c and c + 8 of the lane travel as one float2, so every FMA is a packed FFMA2
+// (two fp32 FMAs, each with the rounding of fmaf, subnormal operands kept).
 struct QRegs {
-    float q2[16], q4[16], q8[16];   // q * 2^(60 - pos_b)
+    float2 q2[8], q4[8], q8[8];   // (q[j], q[j + 8]) * 2^(60 - pos_b)
 };
+
+__device__ __forceinline__ float2 fpair(uint32_t a, uint32_t b) { return make_float2(fld(a), fld(b)); }
+__device__ __forceinline__ float2 bcast(float a) { return make_float2(a, a); }
 
 __device__ __forceinline__ float dot_codes2(const QRegs &q, uint32_t x)
 {
-    const uint32_t y = x >> 16;
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t y = x >> 16;                 // channels 8..15
+    float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-        a[k & 1] = fmaf(q.q2[k], fld(x & (3u << (2 * k))), a[k & 1]);
-        a[2 + (k & 1)] = fmaf(q.q2[k + 8], fld(y & (3u << (2 * k))), a[2 + (k & 1)]);
+        const uint32_t m = 3u << (2 * k);
+        a[k & 1] = __ffma2_rn(q.q2[k], fpair(x & m, y & m), a[k & 1]);
     }
-    return (a[0] + a[1]) + (a[2] + a[3]);
+    return (a[0].x + a[1].x) + (a[0].y + a[1].y);
 }
 
 __device__ __forceinline__ float dot_codes4(const QRegs &q, uint2 x)
 {
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t w[2] = {x.x, x.y};
+    const uint32_t lo0 = x.x, hi0 = x.x >> 16, lo1 = x.y, hi1 = x.y >> 16;
+    float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const uint32_t lo = w[h], hi = w[h] >> 16;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            a[2 * h] = fmaf(q.q4[8 * h + k], fld(lo & (15u << (4 * k))), a[2 * h]);
-            a[2 * h + 1] = fmaf(q.q4[8 * h + 4 + k], fld(hi & (15u << (4 * k))), a[2 * h + 1]);
-        }
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t m = 15u << (4 * k);
+        a[0] = __ffma2_rn(q.q4[k], fpair(lo0 & m, lo1 & m), a[0]);          // channels k, 8 + k
+        a[1] = __ffma2_rn(q.q4[4 + k], fpair(hi0 & m, hi1 & m), a[1]);      // 4 + k, 12 + k
     }
-    return (a[0] + a[1]) + (a[2] + a[3]);
+    return (a[0].x + a[1].x) + (a[0].y + a[1].y);
 }
 
 __device__ __forceinline__ float dot_codes8(const QRegs &q, uint4 x)
 {
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            a[e] = fmaf(q.q8[4 * h + e], fld(__byte_perm(w[h], 0u, 0x4440 + e)), a[e]);
+    for (int e = 0; e < 4; ++e) {
+        const uint32_t sel = 0x4440 + e;
+        a[0] = __ffma2_rn(q.q8[e], fpair(__byte_perm(x.x, 0u, sel), __byte_perm(x.z, 0u, sel)), a[0]);
+        a[1] = __ffma2_rn(q.q8[4 + e], fpair(__byte_perm(x.y, 0u, sel), __byte_perm(x.w, 0u, sel)), a[1]);
     }
-    return (a[0] + a[1]) + (a[2] + a[3]);
+    return (a[0].x + a[1].x) + (a[0].y + a[1].y);
 }
 
 __device__ __forceinline__ float dot_native(const QRegs &q, uint4 x0, uint4 x1)
 {
     const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
+    for (int h = 0; h < 4; ++h) {               // word h: channels 2h, 2h + 1; word h + 4: + 8
         const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
-        a[2 * (h & 1)] = fmaf(q.q8[2 * h], f.x, a[2 * (h & 1)]);
-        a[2 * (h & 1) + 1] = fmaf(q.q8[2 * h + 1], f.y, a[2 * (h & 1) + 1]);
+        const float2 g = __half22float2(*reinterpret_cast<const __half2 *>(&w[h + 4]));
+        a[0] = __ffma2_rn(q.q8[2 * h], make_float2(f.x, g.x), a[0]);
+        a[1] = __ffma2_rn(q.q8[2 * h + 1], make_float2(f.y, g.y), a[1]);
     }
-    return (a[0] + a[1]) + (a[2] + a[3]);
+    return (a[0].x + a[1].x) + (a[0].y + a[1].y);
 }
 
-__device__ __forceinline__ void acc_codes2(float (&o)[16], float wv, uint32_t x)
+__device__ __forceinline__ void acc_codes2(float2 (&o)[8], float wv, uint32_t x)
 {
     const uint32_t y = x >> 16;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
         const float wk = wv * __uint_as_float((127u - 2u * k) << 23);   // wv * 2^-2k
-        o[k] = fmaf(wk, fld(x & (3u << (2 * k))), o[k]);
-        o[k + 8] = fmaf(wk, fld(y & (3u << (2 * k))), o[k + 8]);
+        const uint32_t m = 3u << (2 * k);
+        o[k] = __ffma2_rn(bcast(wk), fpair(x & m, y & m), o[k]);
     }
 }
 
-__device__ __forceinline__ void acc_codes4(float (&o)[16], float wv, uint2 x)
+__device__ __forceinline__ void acc_codes4(float2 (&o)[8], float wv, uint2 x)
 {
-    const uint32_t w[2] = {x.x, x.y};
+    const uint32_t hi0 = x.x >> 16, hi1 = x.y >> 16;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const float wk = wv * __uint_as_float((127u - 4u * k) << 23);   // wv * 2^-4k
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            o[8 * h + k] = fmaf(wk, fld(w[h] & (15u << (4 * k))), o[8 * h + k]);
-            o[8 * h + 4 + k] = fmaf(wk, fld((w[h] >> 16) & (15u << (4 * k))), o[8 * h + 4 + k]);
-        }
+        const float2 wk = bcast(wv * __uint_as_float((127u - 4u * k) << 23));   // wv * 2^-4k
+        const uint32_t m = 15u << (4 * k);
+        o[k] = __ffma2_rn(wk, fpair(x.x & m, x.y & m), o[k]);
+        o[4 + k] = __ffma2_rn(wk, fpair(hi0 & m, hi1 & m), o[4 + k]);
     }
 }
 
-__device__ __forceinline__ void acc_codes8(float (&o)[16], float wv, uint4 x)
+__device__ __forceinline__ void acc_codes8(float2 (&o)[8], float wv, uint4 x)
 {
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    const float2 w2 = bcast(wv);
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            o[4 * h + e] = fmaf(wv, fld(__byte_perm(w[h], 0u, 0x4440 + e)), o[4 * h + e]);
+    for (int e = 0; e < 4; ++e) {
+        const uint32_t sel = 0x4440 + e;
+        o[e] = __ffma2_rn(w2, fpair(__byte_perm(x.x, 0u, sel), __byte_perm(x.z, 0u, sel)), o[e]);
+        o[4 + e] = __ffma2_rn(w2, fpair(__byte_perm(x.y, 0u, sel), __byte_perm(x.w, 0u, sel)), o[4 + e]);
     }
 }
 
-__device__ __forceinline__ void acc_native(float (&o)[16], float wv, uint4 x0, uint4 x1)
+__device__ __forceinline__ void acc_native(float2 (&o)[8], float wv, uint4 x0, uint4 x1)
 {
     const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    const float2 w2 = bcast(wv);
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
+    for (int h = 0; h < 4; ++h) {
         const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
-        o[2 * h] = fmaf(wv, f.x, o[2 * h]);
-        o[2 * h + 1] = fmaf(wv, f.y, o[2 * h + 1]);
+        const float2 g = __half22float2(*reinterpret_cast<const __half2 *>(&w[h + 4]));
+        o[2 * h] = __ffma2_rn(w2, make_float2(f.x, g.x), o[2 * h]);
+        o[2 * h + 1] = __ffma2_rn(w2, make_float2(f.y, g.y), o[2 * h + 1]);
     }
 }
 
-
 // merge the online-softmax state (m, l, pz, o) of this lane with the lane `mask` away
-__device__ __forceinline__ void merge_state(float &m, float &l, float &pz, float (&o)[16], int mask)
+__device__ __forceinline__ void merge_state(float &m, float &l, float &pz, float2 (&o)[8], int mask)
 {
     const float mp = __shfl_xor_sync(0xffffffffu, m, mask);
     const float lp = __shfl_xor_sync(0xffffffffu, l, mask);
@@ -283,9 +284,10 @@ __device__ __forceinline__ void merge_state(float &m, float &l, float &pz, float
     const float fa = (m == -INFINITY) ? 0.f : exp2f(m - M);
     const float fb = (mp == -INFINITY) ? 0.f : exp2f(mp - M);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const float op = __shfl_xor_sync(0xffffffffu, o[k], mask);
-        o[k] = o[k] * fa + op * fb;
+    for (int k = 0; k < 8; ++k) {
+        const float2 op = make_float2(__shfl_xor_sync(0xffffffffu, o[k].x, mask),
+                                      __shfl_xor_sync(0xffffffffu, o[k].y, mask));
+        o[k] = __ffma2_rn(op, bcast(fb), __fmul2_rn(o[k], bcast(fa)));
     }
     l = l * fa + lp * fb;
     pz = pz * fa + zp * fb;
@@ -294,7 +296,7 @@ __device__ __forceinline__ void merge_state(float &m, float &l, float &pz, float
 
 struct KeyState {
     float m, l, pz;
-    float o[16];
+    float2 o[8];      // (o[j], o[j + 8]) of the lane's 16 channels
 };
 
 // One key per 8-lane group (16 lanes x 4 groups for head_dim 64: 4 lanes x 8 groups), all
@@ -327,7 +329,7 @@ __device__ __forceinline__ void process_key(KeyState &st, const QRegs &qr, float
         st.l *= corr;
         st.pz *= corr;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) st.o[k] *= corr;
+        for (int k = 0; k < 8; ++k) st.o[k] = __fmul2_rn(st.o[k], bcast(corr));
         st.m = lg;
     }
     const float p = exp2f(lg - st.m);
@@ -543,7 +545,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         ks.l = 0.f;
         ks.pz = 0.f;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) ks.o[k] = 0.f;
+        for (int k = 0; k < 8; ++k) ks.o[k] = make_float2(0.f, 0.f);
         bool last = false;
         while (!last) {
             if (!mbar_wait(&sm.full[stage], phase, c.status)) return;
@@ -563,11 +565,20 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     const float fv[2] = {f.x, f.y};
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int k = 2 * e + u;
+                        const int k = 2 * e + u;        // channel 16 gl + k -> pair k % 8, half k / 8
                         qsum += fv[u];
-                        qr.q8[k] = fv[u] * kQScale;
-                        qr.q4[k] = qr.q8[k] * __uint_as_float((127u - 4u * (k % 4)) << 23);
-                        qr.q2[k] = qr.q8[k] * __uint_as_float((127u - 2u * (k % 8)) << 23);
+                        const float v8 = fv[u] * kQScale;
+                        const float v4 = v8 * __uint_as_float((127u - 4u * (k % 4)) << 23);
+                        const float v2 = v8 * __uint_as_float((127u - 2u * (k % 8)) << 23);
+                        if (k < 8) {
+                            qr.q8[k].x = v8;
+                            qr.q4[k].x = v4;
+                            qr.q2[k].x = v2;
+                        } else {
+                            qr.q8[k - 8].y = v8;
+                            qr.q4[k - 8].y = v4;
+                            qr.q2[k - 8].y = v2;
+                        }
                     }
                 }
 #pragma unroll
@@ -596,7 +607,10 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         for (int mask = GROUP; mask < 32; mask <<= 1) merge_state(ks.m, ks.l, ks.pz, ks.o, mask);
         if (g == 0) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) sm.red_o[warp][16 * gl + k] = ks.o[k];
+            for (int k = 0; k < 8; ++k) {
+                sm.red_o[warp][16 * gl + k] = ks.o[k].x;
+                sm.red_o[warp][16 * gl + 8 + k] = ks.o[k].y;
+            }
             if (gl == 0) {
                 sm.red_m[warp] = ks.m;
                 sm.red_l[warp] = ks.l;
