@@ -63,10 +63,11 @@ constexpr float kOUnscale = 562949953421312.0f;                    // 2^49
 
 template <int D>
 struct Stage {
-    // width-sorted keys in class-pure chunks: kValid | (offset in rec << 9) |
-    // (width code << 7) | key; padding entries carry only their chunk's width code
+    // width-sorted keys in class-pure chunks: kValid | (key << 16) | offset in rec;
+    // padding entries are 0
     uint32_t perm[kPermSlots];
     int32_t info[4];         // item index, keys in the stage, flags, chunks
+    int32_t cls_chunk[8];    // first chunk of each width class (b = 2, 4, 8, 16), [4] = chunks
     __half q[D];             // the item's query (copied with the item's first stage)
     float4 side[kWin];       // (s_K, z_K, s_V, z_V) per key, token order
     alignas(16) uint8_t rec[kStageRecBytes];
@@ -309,7 +310,7 @@ __device__ __forceinline__ void process_key(KeyState &st, const QRegs &qr, float
 {
     constexpr int GROUP = D / 16;
     const bool valid = (ent & kValid) != 0;
-    const uint8_t *r = sg.rec + ((ent >> 9) & 0x7FFFu);
+    const uint8_t *r = sg.rec + (ent & 0x7FFFu);
     float part = 0.f;
     if (valid) {
         if (CLS == 0) part = dot_codes2(qr, reinterpret_cast<const uint32_t *>(r)[gl]);
@@ -321,7 +322,7 @@ __device__ __forceinline__ void process_key(KeyState &st, const QRegs &qr, float
 #pragma unroll
     for (int d = 1; d < GROUP; d <<= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
     if (!valid) return;
-    const float4 sd = sg.side[ent & 127u];
+    const float4 sd = sg.side[(ent >> 16) & 127u];
     const float dot = (CLS == 3) ? part * kDotNativeUnscale : fmaf(sd.x, part * kDotCodeUnscale, sd.y * qsum);
     const float lg = dot * qk_scale;
     if (lg > st.m) {                          // new running max of this key group
@@ -345,6 +346,17 @@ __device__ __forceinline__ void process_key(KeyState &st, const QRegs &qr, float
         else if (CLS == 1) acc_codes4(st.o, wv, reinterpret_cast<const uint2 *>(rv)[gl]);
         else acc_codes8(st.o, wv, reinterpret_cast<const uint4 *>(rv)[gl]);
     }
+}
+
+// This warp's chunks ch, ch + kConsumerWarps, ... below `end`, all of width class CLS.
+template <int D, int CLS>
+__device__ __forceinline__ int run_class(KeyState &st, const QRegs &qr, float qsum, float qk_scale,
+                                         const Stage<D> &sg, int ch, int end, int g, int gl)
+{
+    constexpr int KEYS_PER_STEP = 32 / (D / 16);
+    for (; ch < end; ch += kConsumerWarps)
+        process_key<D, CLS>(st, qr, qsum, qk_scale, sg, sg.perm[KEYS_PER_STEP * ch + g], gl);
+    return ch;
 }
 
 template <int D>
@@ -474,9 +486,10 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     cl_of[r] = (k >= w0 && k < w1) ? (int)(m[r] & 3u) : 4;
                     pos_of[r] = 0;
                 }
-                int pstart = 0, pad_cls = -1, pad_pos = 0;
+                int pstart = 0, pad_pos = -1, cls_chunk[4];
 #pragma unroll
                 for (int cl = 0; cl < 4; ++cl) {
+                    cls_chunk[cl] = pstart / KEYS_PER_STEP;
                     int before = 0;
 #pragma unroll
                     for (int r = 0; r < KPL; ++r) {
@@ -485,10 +498,8 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                         before += __popc(b);
                     }
                     const int padded = (before + PADL) / KEYS_PER_STEP * KEYS_PER_STEP;
-                    if (lane / PADL == cl && before + lane % PADL < padded) {   // PADL lanes per width
-                        pad_cls = cl;
+                    if (lane / PADL == cl && before + lane % PADL < padded)     // PADL lanes per width
                         pad_pos = pstart + before + lane % PADL;
-                    }
                     pstart += padded;
                 }
 
@@ -501,16 +512,18 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                         // keeps every shared-memory read of the consumers inside the stage
                         const uint32_t ro = min((m[r] & ~15u) - off0,
                                                 kStageRecBytes - (uint32_t)(D * (2 << cl_of[r])) / 4u);
-                        sg.perm[pos_of[r]] = kValid | (ro << 9) | ((uint32_t)cl_of[r] << 7) |
-                                             (uint32_t)(lane + 32 * r - w0);
+                        sg.perm[pos_of[r]] = kValid | ((uint32_t)(lane + 32 * r - w0) << 16) | ro;
                     }
                 }
-                if (pad_cls >= 0) sg.perm[pad_pos] = (uint32_t)pad_cls << 7;
+                if (pad_pos >= 0) sg.perm[pad_pos] = 0u;
                 if (lane == 0) {
                     sg.info[0] = it;
                     sg.info[1] = n;
                     sg.info[2] = (new_item ? kNewItem : 0) | (last ? kLastSub : 0);
                     sg.info[3] = pstart / KEYS_PER_STEP;
+#pragma unroll
+                    for (int cl = 0; cl < 4; ++cl) sg.cls_chunk[cl] = cls_chunk[cl];
+                    sg.cls_chunk[4] = pstart / KEYS_PER_STEP;
                 }
                 __syncwarp();
                 if (lane == 0) {
@@ -551,7 +564,6 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
             if (!mbar_wait(&sm.full[stage], phase, c.status)) return;
             Stage<D> &sg = sm.st[stage];
             const int flags = sg.info[2];
-            const int n_chunks = sg.info[3];
             last = (flags & kLastSub) != 0;
             if (flags & kNewItem) {
                 // query: this lane's 16 channels, scaled per width; sum(q) over all D
@@ -584,15 +596,13 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
 #pragma unroll
                 for (int d = 1; d < GROUP; d <<= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, d);
             }
-            // class-pure chunks, dealt to the warps round-robin (rotated every stage)
-            for (int ch = (warp + kConsumerWarps - rot) % kConsumerWarps; ch < n_chunks; ch += kConsumerWarps) {
-                const uint32_t ent = sg.perm[KEYS_PER_STEP * ch + g];
-                const int cls = (ent >> 7) & 3u;           // the same for the whole chunk
-                if (cls == 0) process_key<D, 0>(ks, qr, qsum, qk_scale, sg, ent, gl);
-                else if (cls == 1) process_key<D, 1>(ks, qr, qsum, qk_scale, sg, ent, gl);
-                else if (cls == 2) process_key<D, 2>(ks, qr, qsum, qk_scale, sg, ent, gl);
-                else process_key<D, 3>(ks, qr, qsum, qk_scale, sg, ent, gl);
-            }
+            // class-pure chunks, dealt to the warps round-robin (rotated every stage); the
+            // chunks are sorted by width, so the warp walks one run per width class
+            int ch = (warp + kConsumerWarps - rot) % kConsumerWarps;
+            ch = run_class<D, 0>(ks, qr, qsum, qk_scale, sg, ch, sg.cls_chunk[1], g, gl);
+            ch = run_class<D, 1>(ks, qr, qsum, qk_scale, sg, ch, sg.cls_chunk[2], g, gl);
+            ch = run_class<D, 2>(ks, qr, qsum, qk_scale, sg, ch, sg.cls_chunk[3], g, gl);
+            run_class<D, 3>(ks, qr, qsum, qk_scale, sg, ch, sg.cls_chunk[4], g, gl);
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);
             rot = (rot + 1) % kConsumerWarps;

@@ -123,8 +123,8 @@ write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *
 
 // Staging of the quantize kernel: each CTA copies the fp16 K and V rows of T tokens x HG
 // heads (at most kWqHalves values per tensor) into shared memory with two bulk copies.
-constexpr int kWqThreads = 256;
-constexpr int kWqHalves = 8192;          // 16 KB of K and 16 KB of V per CTA
+constexpr int kWqThreads = 128;
+constexpr int kWqHalves = 4096;          // 8 KB of K and 8 KB of V per CTA
 constexpr int kWqMaxPairs = kWqHalves / 64;
 
 struct WqPair {                          // one (token, head) of the CTA
