@@ -387,9 +387,12 @@ def run_ours(args):
             "pairs": pre["pairs"], "flops": pre["flops"],
             "roofline": {"kernel": "prefill attention", "bound": "tensor", "achieved": pre["tflops"],
                          "peak": bf16, "peak_kind": pk_kind + " bf16 dense (burst)", "unit": "TFLOP/s",
-                         "frac": pre["tflops"] / bf16, "traffic": None},
+                         "frac": pre["tflops"] / bf16,
+                         "traffic": _profiled_traffic("prefill_tc_ragged_prefill.md", "kvq_prefill_tc.cu")},
             "quantize": {"gbs": pre["write_gbs"], "bytes": pre["write_bytes"],
-                         "seconds": pre["write_s"], "frac_of_hbm": pre["write_gbs"] / hbm_peak}}
+                         "seconds": pre["write_s"], "frac_of_hbm": pre["write_gbs"] / hbm_peak,
+                         # DRAM bytes of the quantize kernel (the scan kernel's are not included)
+                         "traffic": _profiled_traffic("write_quant_ragged_prefill.md", "kvq_write.cu")}}
     if rank == 0 and not args.no_cpu_baseline:
         v_cpu, n_keys, secs, desc = oracle_decode_sample(wl, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": 1, "kind": "oracle",
