@@ -39,6 +39,8 @@ int cuda_fail(cudaError_t e, const char *what)
 
 __global__ void truncate_kernel(kvq::CacheView c, const int32_t *__restrict__ lengths)
 {
+    kvq::pdl_wait();
+    kvq::pdl_trigger();
     const int sh = blockIdx.x * blockDim.x + threadIdx.x;
     if (sh >= c.B * c.H) return;
     const int s = sh / c.H, h = sh % c.H;
@@ -284,7 +286,8 @@ int kvq_cache_truncate(kvq_cache *c, const int32_t *lengths, kvq_stream_t stream
     if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_cache_truncate: bad cache");
     if (!lengths) return fail(KVQ_ERR_ARG, "kvq_cache_truncate: lengths is NULL");
     const int BH = c->B * c->H;
-    truncate_kernel<<<(BH + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c->view, lengths);
+    kvq::launch_pdl(truncate_kernel, dim3((BH + 255) / 256), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream),
+                    c->view, lengths);
     cudaError_t e = cudaGetLastError();
     return e ? cuda_fail(e, "kvq_cache_truncate") : ok();
 }

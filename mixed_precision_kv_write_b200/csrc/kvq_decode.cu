@@ -100,6 +100,8 @@ __global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ mod
 {
     __shared__ int warp_tot[32];
     __shared__ int carry_sh;
+    pdl_wait();
+    pdl_trigger();
     const int BH = c.B * c.H;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (tid == 0) carry_sh = 0;
@@ -369,6 +371,8 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     extern __shared__ __align__(128) uint8_t smem_raw[];
     DecodeSmem<D> &sm = *reinterpret_cast<DecodeSmem<D> *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    pdl_trigger();
     const int n_items = *wk.count;
 
     if (tid == 0) {
@@ -662,6 +666,8 @@ __global__ void __launch_bounds__(D)
 decode_combine_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
 {
     __shared__ float red[D / 32];
+    pdl_wait();
+    pdl_trigger();
     const int sh = blockIdx.x, ch = threadIdx.x, lane = ch & 31, wid = ch >> 5;
     const int first = wk.head_first[sh], cnt = wk.head_cnt[sh];
     const float *P = wk.partials + (int64_t)first * (D + 4);
@@ -710,7 +716,8 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const __half *q, const uint8
                             float *out, cudaStream_t st)
 {
     const CacheView &c = cache->view;
-    decode_sched_kernel<<<1, 1024, 0, st>>>(c, modes, w, cache->work);
+    cudaError_t le = launch_pdl(decode_sched_kernel, dim3(1), dim3(1024), 0, st, c, modes, w, cache->work);
+    if (le != cudaSuccess) return le;
     const size_t smem = sizeof(DecodeSmem<D>);
     static bool attr_done = false;
     if (!attr_done) {
@@ -721,9 +728,11 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const __half *q, const uint8
     }
     const int grid = (int)std::min<int64_t>(cache->work.max_items, 3 * (int64_t)num_sms());
     profile_before(st);
-    decode_splitk_kernel<D><<<grid, kThreads, smem, st>>>(c, q, cache->work);
+    le = launch_pdl(decode_splitk_kernel<D>, dim3(grid), dim3(kThreads), smem, st, c, q, cache->work);
+    if (le != cudaSuccess) return le;
     profile_after(st);
-    decode_combine_kernel<D><<<c.B * c.H, D, 0, st>>>(c, cache->work, out);
+    le = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H), dim3(D), 0, st, c, cache->work, out);
+    if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
@@ -777,14 +786,16 @@ cudaError_t launch_decode_static(const kvq_cache *cache, const DecodeWork &wk, c
                                  const uint8_t *modes, int w, float *out, cudaStream_t st)
 {
     const CacheView &c = cache->view;
-    decode_sched_kernel<<<1, 1024, 0, st>>>(c, modes, w, wk);
-    const size_t smem = sizeof(DecodeSmem<D>);
-    cudaError_t e = cudaFuncSetAttribute(decode_splitk_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = launch_pdl(decode_sched_kernel, dim3(1), dim3(1024), 0, st, c, modes, w, wk);
     if (e != cudaSuccess) return e;
-    const int grid = (int)std::min<int64_t>(wk.max_items, 2 * (int64_t)num_sms());
-    decode_splitk_kernel<D><<<grid, kThreads, smem, st>>>(c, q, wk);
-    decode_combine_kernel<D><<<c.B * c.H, D, 0, st>>>(c, wk, out);
+    const size_t smem = sizeof(DecodeSmem<D>);
+    e = cudaFuncSetAttribute(decode_splitk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(wk.max_items, 3 * (int64_t)num_sms());
+    e = launch_pdl(decode_splitk_kernel<D>, dim3(grid), dim3(kThreads), smem, st, c, q, wk);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H), dim3(D), 0, st, c, wk, out);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

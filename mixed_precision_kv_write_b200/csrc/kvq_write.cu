@@ -32,6 +32,8 @@ write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *
     constexpr int PER = 8;                       // tokens per thread per pass
     constexpr int WARPS = TPS / 32;
     __shared__ uint32_t wsum[BS / 32];
+    pdl_wait();
+    pdl_trigger();
     const int tid = threadIdx.x % TPS, lane = threadIdx.x & 31;
     const int grp = threadIdx.x / TPS, wig = tid >> 5;     // group in block, warp in group
     const int64_t gsh = (int64_t)blockIdx.x * (BS / TPS) + grp;
@@ -228,6 +230,8 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
     __shared__ uint8_t order[kWqMaxPairs];   // written pairs sorted by width
     __shared__ int n_written;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    pdl_trigger();
     const int H = c.H;
     const int64_t t0 = (int64_t)blockIdx.x * T;
     const int h0 = blockIdx.y * HG;
@@ -365,16 +369,18 @@ cudaError_t launch_write(kvq_cache *cache, const __half *k, const __half *v,
 {
     const CacheView &c = cache->view;
     const uint32_t gen = ++cache->write_gen;
+    cudaError_t le = cudaSuccess;
     profile_before(st);
     {
         const int64_t groups = (int64_t)c.B * c.H;
         // a warp per (sequence, head) for short appends (decode steps), a block for long ones
         if (n_tok <= 64 * (int64_t)c.B) {
             const int64_t blocks = (groups + 7) / 8;
-            write_scan_kernel<32><<<(unsigned)blocks, 256, 0, st>>>(c, bits, cu, n_tok, gen);
+            le = launch_pdl(write_scan_kernel<32>, dim3((unsigned)blocks), dim3(256), 0, st, c, bits, cu, n_tok, gen);
         } else {
-            write_scan_kernel<1024><<<(unsigned)groups, 1024, 0, st>>>(c, bits, cu, n_tok, gen);
+            le = launch_pdl(write_scan_kernel<1024>, dim3((unsigned)groups), dim3(1024), 0, st, c, bits, cu, n_tok, gen);
         }
+        if (le != cudaSuccess) return le;
     }
     if (n_tok > 0) {
         // tiles of T tokens x HG heads, at most kWqHalves values per tensor; one token per
@@ -385,9 +391,10 @@ cudaError_t launch_write(kvq_cache *cache, const __half *k, const __half *v,
         const dim3 grid((unsigned)((n_tok + T - 1) / T), (unsigned)((c.H + HG - 1) / HG));
         const size_t smem = 2 * kWqHalves * sizeof(__half);
         if (c.D == 128)
-            write_quant_kernel<128><<<grid, kWqThreads, smem, st>>>(c, k, v, cu, n_tok, gen, T, HG);
+            le = launch_pdl(write_quant_kernel<128>, grid, dim3(kWqThreads), smem, st, c, k, v, cu, n_tok, gen, T, HG);
         else
-            write_quant_kernel<64><<<grid, kWqThreads, smem, st>>>(c, k, v, cu, n_tok, gen, T, HG);
+            le = launch_pdl(write_quant_kernel<64>, grid, dim3(kWqThreads), smem, st, c, k, v, cu, n_tok, gen, T, HG);
+        if (le != cudaSuccess) return le;
     }
     profile_after(st);
     return cudaGetLastError();
