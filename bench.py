@@ -165,7 +165,7 @@ def decode_step(st, w, events=None):
         kvq.kvq_set_profile_events(None, None)
 
 
-LAUNCHES_PER_DECODE_STEP = 6   # truncate, write scan, write quantize, sched, split-K, combine
+LAUNCHES_PER_DECODE_STEP = 5   # truncate, write (single-launch append), sched, split-K, combine
 
 
 def prefill_measure(dev, reps=5, warm=2):

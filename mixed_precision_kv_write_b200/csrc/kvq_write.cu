@@ -211,6 +211,52 @@ __device__ __forceinline__ void quant_store(const uint4 (&raw)[NC], float z, flo
     }
 }
 
+// min and max of a vector spread over VL adjacent lanes (NC 8-value chunks per lane), in
+// fp16 (exact); (min, -max) travel as one half2 through the shuffles. Every lane of the
+// warp takes part.
+template <int NC, int VL>
+__device__ __forceinline__ __half2 vec_minmax(const uint4 (&raw)[NC])
+{
+    const __half2 (&h2)[4 * NC] = *reinterpret_cast<const __half2 (*)[4 * NC]>(raw);
+    __half2 lo2 = h2[0], hi2 = h2[0];
+#pragma unroll
+    for (int e = 1; e < 4 * NC; ++e) {
+        lo2 = __hmin2(lo2, h2[e]);
+        hi2 = __hmax2(hi2, h2[e]);
+    }
+    __half2 mm = __halves2half2(__hmin(__low2half(lo2), __high2half(lo2)),
+                                __hneg(__hmax(__low2half(hi2), __high2half(hi2))));
+#pragma unroll
+    for (int d = VL / 2; d >= 1; d >>= 1) {
+        const uint32_t o = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t *>(&mm), d);
+        mm = __hmin2(mm, *reinterpret_cast<const __half2 *>(&o));
+    }
+    return mm;
+}
+
+// This lane's share of one vector's record part at `dst` (b-bit codes, or the fp16 values
+// for b = 16) and, from the vector's first lane, its (s, z) side entry.
+template <int NC, int VL>
+__device__ __forceinline__ void vec_store(const CacheView &c, const uint4 (&raw)[NC], __half2 mm, int b,
+                                          uint8_t *dst, int64_t slot, int part, int li)
+{
+    float sc = 1.0f, z = 0.0f;
+    if (b == 16) {
+#pragma unroll
+        for (int j = 0; j < NC; ++j) reinterpret_cast<uint4 *>(dst)[j * VL + li] = raw[j];
+    } else {
+        const float mn = __low2float(mm), mx = -__high2float(mm);
+        const float top = (float)((1u << b) - 1u);
+        // zeros are stored as +0 (the min scan may meet -0 or +0 first)
+        sc = __fadd_rn(__fdiv_rn(__fsub_rn(mx, mn), top), 0.0f);
+        z = __fadd_rn(mn, 0.0f);
+        if (b == 8) quant_store<8, NC, VL>(raw, z, sc, dst, li);
+        else if (b == 4) quant_store<4, NC, VL>(raw, z, sc, dst, li);
+        else quant_store<2, NC, VL>(raw, z, sc, dst, li);
+    }
+    if (li == 0) reinterpret_cast<float2 *>(&c.side[slot])[part] = make_float2(sc, z);
+}
+
 // One CTA per tile of T tokens x HG heads. Warp 0 starts two bulk copies (the tile's K and
 // V rows are contiguous when HG = H, else one copy per token and tensor); meanwhile every
 // thread resolves the destination of one (token, head): its sequence (binary search of
@@ -325,40 +371,113 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
 #pragma unroll
             for (int j = 0; j < NC; ++j) raw[j] = src[j * VL + li];
         }
-        const __half2 (&h2)[4 * NC] = *reinterpret_cast<const __half2 (*)[4 * NC]>(raw);
-        // min and max in fp16 (exact); (min, -max) travel as one half2 through the shuffles
-        __half2 lo2 = h2[0], hi2 = h2[0];
-#pragma unroll
-        for (int e = 1; e < 4 * NC; ++e) {
-            lo2 = __hmin2(lo2, h2[e]);
-            hi2 = __hmax2(hi2, h2[e]);
-        }
-        __half2 mm = __halves2half2(__hmin(__low2half(lo2), __high2half(lo2)),
-                                    __hneg(__hmax(__low2half(hi2), __high2half(hi2))));
-#pragma unroll
-        for (int d = VL / 2; d >= 1; d >>= 1) {
-            const uint32_t o = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t *>(&mm), d);
-            mm = __hmin2(mm, *reinterpret_cast<const __half2 *>(&o));
-        }
+        const __half2 mm = vec_minmax<NC, VL>(raw);
         if (!in_range) continue;
         const WqPair pr = pairs[pi];
         const int b = 2 << (pr.meta & 3u);
-        uint8_t *dst = c.rec + pr.rec + part * (b * D / 8);
-        float sc = 1.0f, z = 0.0f;
-        if (b == 16) {
-#pragma unroll
-            for (int j = 0; j < NC; ++j) reinterpret_cast<uint4 *>(dst)[j * VL + li] = raw[j];
-        } else {
-            const float mn = __low2float(mm), mx = -__high2float(mm);
-            const float top = (float)((1u << b) - 1u);
-            // zeros are stored as +0 (the min scan may meet -0 or +0 first)
-            sc = __fadd_rn(__fdiv_rn(__fsub_rn(mx, mn), top), 0.0f);
-            z = __fadd_rn(mn, 0.0f);
-            if (b == 8) quant_store<8, NC, VL>(raw, z, sc, dst, li);
-            else if (b == 4) quant_store<4, NC, VL>(raw, z, sc, dst, li);
-            else quant_store<2, NC, VL>(raw, z, sc, dst, li);
+        vec_store<NC, VL>(c, raw, mm, b, c.rec + pr.rec + part * (b * D / 8), pr.slot, part, li);
+    }
+}
+
+// Short appends (decode steps): one CTA of 256 threads per sequence does the scan and the
+// quantization of all the sequence's new (token, head) pairs in one launch. Phase 1, a
+// warp per head: capacity, widths and record offsets (warp prefix sum) of the sequence's
+// tokens. Phase 2, after the block has seen every head's verdict: D/8 lanes per vector
+// (one (token, head) pair per warp pass at head_dim 128), values straight from global
+// memory. Same results as the scan + quantize pair of kernels.
+template <int D>
+__global__ void __launch_bounds__(256)
+write_append_kernel(CacheView c, const __half *__restrict__ k, const __half *__restrict__ v,
+                    const uint8_t *__restrict__ bits, const int32_t *__restrict__ cu, int64_t n_tok,
+                    uint32_t gen)
+{
+    constexpr int VL = D / 8, VPW = 32 / VL;
+    __shared__ int bad_sh;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    pdl_trigger();
+    const int s = blockIdx.x, H = c.H;
+    const int64_t t0 = cu[s], t1 = cu[s + 1];
+    if (t0 < 0 || t1 < t0 || t1 > n_tok || (s == 0 && t0 != 0)) {
+        if (tid == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+        return;
+    }
+    const int n = (int)(t1 - t0);
+    if (n == 0) return;
+    if (tid == 0) bad_sh = 0;
+    __syncthreads();
+    for (int h = warp; h < H; h += 8) {
+        const int sh = s * H + h;
+        const int L0 = c.len[sh];
+        if ((int64_t)L0 + n > c.cap[s]) {
+            if (lane == 0) {
+                set_status(c.status, KVQ_ERR_CAPACITY);
+                c.wstart[sh] = -1;
+            }
+            continue;
         }
-        if (li == 0) reinterpret_cast<float2 *>(&c.side[pr.slot])[part] = make_float2(sc, z);
+        const int64_t slot0 = slot_of(c, s, h, L0);
+        uint32_t off = c.end[sh];
+        bool bad = false;
+        for (int base = 0; base < n; base += 32) {
+            const int i = base + lane;
+            uint32_t sz = 0, wc = 0;
+            if (i < n) {
+                const int b = bits[(t0 + i) * H + h];
+                const int w = width_code(b);
+                if (w < 0) bad = true;
+                else {
+                    wc = (uint32_t)w;
+                    sz = (uint32_t)(b * D / 4);
+                }
+            }
+            uint32_t incl = sz;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += y;
+            }
+            if (i < n) c.meta[slot0 + i] = (off + incl - sz) | wc;
+            off += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&bad_sh, 1);
+        if (lane == 0) {
+            c.wstart[sh] = L0;
+            c.wend[sh] = off;
+        }
+    }
+    __syncthreads();
+    if (bad_sh) {                                // the sequence's write is refused for every head
+        if (tid == 0) {
+            c.bad[s] = gen;
+            set_status(c.status, KVQ_ERR_BITS);
+        }
+        return;
+    }
+    const int n_vec = 2 * n * H;                 // vector vi: pair vi / 2 = i * H + h, K or V
+    const int li = lane % VL;
+    for (int vb = warp * VPW; vb < n_vec; vb += 8 * VPW) {
+        const int vi = vb + lane / VL;
+        const bool in_range = vi < n_vec;
+        const int p = vi >> 1, part = vi & 1;
+        const int i = p / H, h = p % H;
+        uint4 raw[1] = {make_uint4(0u, 0u, 0u, 0u)};
+        if (in_range) raw[0] = reinterpret_cast<const uint4 *>((part ? v : k) + ((t0 + i) * H + h) * D)[li];
+        const __half2 mm = vec_minmax<1, VL>(raw);
+        if (!in_range) continue;
+        const int st = c.wstart[s * H + h];
+        if (st < 0) continue;
+        const int64_t slot = slot_of(c, s, h, st + i);
+        const uint32_t meta = c.meta[slot];
+        const int b = 2 << (meta & 3u);
+        vec_store<1, VL>(c, raw, mm, b, stream_of(c, s, h) + (meta & ~15u) + part * (b * D / 8), slot, part, li);
+    }
+    for (int h = tid; h < H; h += 256) {         // commit the new lengths and stream ends
+        const int st = c.wstart[s * H + h];
+        if (st >= 0) {
+            c.len[s * H + h] = st + n;
+            c.end[s * H + h] = c.wend[s * H + h];
+        }
     }
 }
 
@@ -371,6 +490,15 @@ cudaError_t launch_write(kvq_cache *cache, const __half *k, const __half *v,
     const uint32_t gen = ++cache->write_gen;
     cudaError_t le = cudaSuccess;
     profile_before(st);
+    if (n_tok > 0 && n_tok <= 2 * (int64_t)c.B && n_tok <= 4096) {
+        // short append (decode steps): scan and quantize in one launch, a CTA per sequence
+        if (c.D == 128)
+            le = launch_pdl(write_append_kernel<128>, dim3(c.B), dim3(256), 0, st, c, k, v, bits, cu, n_tok, gen);
+        else
+            le = launch_pdl(write_append_kernel<64>, dim3(c.B), dim3(256), 0, st, c, k, v, bits, cu, n_tok, gen);
+        profile_after(st);
+        return le != cudaSuccess ? le : cudaGetLastError();
+    }
     {
         const int64_t groups = (int64_t)c.B * c.H;
         // a warp per (sequence, head) for short appends (decode steps), a block for long ones

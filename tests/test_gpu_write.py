@@ -123,3 +123,60 @@ def test_host_argument_errors():
     m = torch.zeros((1, 2), dtype=torch.uint8, device="cuda")
     with pytest.raises(kvq.KVQError):
         kvq.routed_attn_decode(q, cache, m, -1)
+
+
+def _append_rows(k, v, bits, cu, pos, counts):
+    """The call's tensors for appending counts[s] tokens after position pos[s] of each
+    sequence (rows of the packed full-sequence tensors, in sequence order)."""
+    rows = [cu[s] + pos[s] + i for s in range(len(counts)) for i in range(counts[s])]
+    idx = torch.tensor(rows, dtype=torch.long, device=k.device)
+    cus = torch.tensor([0] + np.cumsum(counts).tolist(), dtype=torch.int32, device=k.device)
+    return k[idx].contiguous(), v[idx].contiguous(), bits[idx].contiguous(), cus
+
+
+@pytest.mark.parametrize("name", ["decode_1p3b", "prefill_160m"])
+def test_short_appends_bit_exact(name):
+    # a long first write, then calls of at most 2 tokens per sequence (n_tok <= 2 * batch:
+    # the single-launch append path), ragged and with empty sequences
+    wl = synth.scaled(W[name], seqlens=(40, 7, 0, 33, 12))
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cu = synth.cu_seqlens(wl.seqlens).tolist()
+    cache = kvq.KVQCache(wl.batch, wl.heads, wl.head_dim, [max(1, L) for L in wl.seqlens])
+    pos = [0] * wl.batch
+    first = [min(5, L) for L in wl.seqlens]
+    kvq.kvq_write(*_append_rows(k, v, bits, cu, pos, first), cache)
+    pos = first[:]
+    rng = np.random.default_rng(1)
+    calls = 0
+    while any(pos[s] < wl.seqlens[s] for s in range(wl.batch)):
+        counts = [int(min(rng.integers(0, 3), wl.seqlens[s] - pos[s])) for s in range(wl.batch)]
+        kvq.kvq_write(*_append_rows(k, v, bits, cu, pos, counts), cache)
+        pos = [p + c for p, c in zip(pos, counts)]
+        calls += 1
+    assert calls > 10
+    cache.check()
+    assert cache.lengths().tolist() == list(wl.seqlens)
+    pairs = [(s, h) for s in range(wl.batch) for h in range(wl.heads)]
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), pairs)
+
+
+def test_short_append_errors():
+    # one token per sequence: a bad width in sequence 1 refuses its write for every head;
+    # sequence 2 is full; the others are written
+    wl = synth.scaled(W["decode_1p3b"], seqlens=(3, 3, 3, 3), heads=4)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cu = synth.cu_seqlens(wl.seqlens).tolist()
+    cache = kvq.KVQCache(4, wl.heads, wl.head_dim, [3, 3, 2, 3])
+    pos = [0, 0, 0, 0]
+    for _ in range(2):
+        kvq.kvq_write(*_append_rows(k, v, bits, cu, pos, [1, 1, 1, 1]), cache)
+        pos = [p + 1 for p in pos]
+    cache.check()
+    kk, vv, bb, cus = _append_rows(k, v, bits, cu, pos, [1, 1, 1, 1])
+    bb[1, 2] = 3
+    kvq.kvq_write(kk, vv, bb, cus, cache)
+    with pytest.raises(kvq.KVQError) as e:
+        cache.check()
+    assert e.value.code in (kvq.KVQ_ERR_BITS, kvq.KVQ_ERR_CAPACITY)
+    assert cache.lengths().tolist() == [3, 2, 2, 3]
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), [(s, h) for s in (0, 3) for h in range(4)])
