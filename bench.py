@@ -275,8 +275,19 @@ def max_over_ranks(x: float, pg: bool, dev) -> float:
 
 def barrier(pg, dev):
     if pg:
-        torch.distributed.barrier(device_ids=[dev.index])
-    torch.cuda.synchronize(dev)
+        if dev.type == "cuda":
+            torch.distributed.barrier(device_ids=[dev.index])
+        else:
+            torch.distributed.barrier()
+    if dev.type == "cuda":
+        torch.cuda.synchronize(dev)
+
+
+def weak_scaling_value(units_per_rank: float, elapsed: float, pg: bool, dev, world: int):
+    """Every rank processes the same units (one replica of the workload each): the job's
+    throughput is all ranks' units over the slowest rank's time. Returns (value, max time)."""
+    elapsed_max = max_over_ranks(elapsed, pg, dev)
+    return units_per_rank * world / elapsed_max, elapsed_max
 
 
 def run_ours(args):
@@ -317,14 +328,13 @@ def run_ours(args):
     sampler.stop()
     st["cache"].check()
     elapsed = e0.elapsed_time(e1) * 1e-3
-    elapsed_max = max_over_ranks(elapsed, pg, dev)
     k_times = [a.elapsed_time(b) * 1e-3 for a, b in ev_k]
     k_avg = statistics.mean(k_times)
     clocks = sampler.summary(t_begin, t_end)
 
     keys = st["keys"]
     routed = st["rec_bytes"] + st["side_bytes"]
-    value = keys * args.steps * world / elapsed_max
+    value, elapsed_max = weak_scaling_value(keys * args.steps, elapsed, pg, dev, world)
     ms_step = elapsed_max / args.steps * 1e3
     kernel_bytes = routed + st["q_bytes"]
     hbm_peak = float(pk["hbm_gbs"])
@@ -353,8 +363,7 @@ def run_ours(args):
         e2e_step()
     f1.record(stream)
     barrier(pg, dev)
-    e2e_s = max_over_ranks(f0.elapsed_time(f1) * 1e-3, pg, dev)
-    e2e_value = keys * args.steps * world / e2e_s
+    e2e_value, _ = weak_scaling_value(keys * args.steps, f0.elapsed_time(f1) * 1e-3, pg, dev, world)
 
     pre = prefill_measure(dev) if not args.no_prefill else None
     barrier(pg, dev)

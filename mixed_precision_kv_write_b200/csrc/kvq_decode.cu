@@ -109,9 +109,15 @@ __global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ mod
     for (int base = 0; base < BH; base += blockDim.x) {
         const int i = base + tid;
         int cnt = 0, lo = 0, hi = 0, L = 0;
+        int64_t sb = 0;
+        uint32_t end_i = 0;
         if (i < BH) {
+            // every load of this head up front: one round trip before the scan
+            const int s = i / c.H, h = i % c.H;
             const int m = modes[i];
             L = c.len[i];
+            end_i = c.end[i];
+            sb = slot_of(c, s, h, 0);
             if (m > KVQ_MODE_FULL) {
                 set_status(c.status, KVQ_ERR_MODE);
             } else if (m != KVQ_MODE_SKIP && L > 0) {
@@ -144,8 +150,6 @@ __global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ mod
             wk.head_first[i] = first;
             wk.head_cnt[i] = cnt;
             if (cnt > 0) {
-                const int s = i / c.H, h = i % c.H;
-                const int64_t sb = slot_of(c, s, h, 0);
                 const int n = hi - lo, per = n / cnt, rem = n % cnt;
                 int j0 = lo;
                 for (int k = 0; k < cnt; ++k) {               // near-equal, non-empty items
@@ -156,7 +160,7 @@ __global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ mod
                     j0 = it.j1;
                     // the stream end for the item ending at the last token; else the
                     // producer reads the offset of key j1 itself
-                    it.end_off = (it.j1 < L) ? kReadEndFromMeta : c.end[i];
+                    it.end_off = (it.j1 < L) ? kReadEndFromMeta : end_i;
                     it.sbase = sb;
                     wk.items[first + k] = it;
                 }
