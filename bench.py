@@ -341,28 +341,63 @@ def run_ours(args):
     achieved = kernel_bytes / k_avg / 1e9
     traffic = _profiled_traffic("decode_splitk_decode_1p3b.md", "kvq_decode.cu")
 
-    # end to end through host buffers: per step H2D of the step inputs (pinned), D2H of out
-    host = {n: st[n].cpu().pin_memory() for n in ("k_step", "v_step", "b_step", "q", "modes")}
-    out_h = torch.empty(st["out"].shape, dtype=torch.float32, pin_memory=True)
+    # End to end through host buffers: every step copies its inputs from pinned host memory
+    # (H2D) and reads its output back (D2H), inside the timed region. The copies run on a
+    # second stream with two buffer sets, so step i+1's inputs and step i's output move
+    # while the next step computes; the cache steps stay in order on the compute stream.
+    names = ("k_step", "v_step", "b_step", "q", "modes")
+    host = {n: st[n].cpu().pin_memory() for n in names}
+    out_h = [torch.empty(st["out"].shape, dtype=torch.float32, pin_memory=True) for _ in range(2)]
+    bufs = []
+    for _ in range(2):
+        b = {n: torch.empty_like(st[n]) for n in names}
+        b["out"] = torch.empty_like(st["out"])
+        bufs.append(b)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * 4
-    from mixed_precision_kv_write_b200 import kvq as _k
+    d2h = out_h[0].numel() * 4
+    copy = torch.cuda.Stream(dev)
 
-    def e2e_step():
-        for n, t in host.items():
-            st[n].copy_(t, non_blocking=True)
-        decode_step(st, wl.w)
-        out_h.copy_(st["out"], non_blocking=True)
+    def e2e_run(n_steps, f0=None, f1=None):
+        landed = [torch.cuda.Event() for _ in range(2)]     # inputs of the buffer set copied
+        done = [torch.cuda.Event() for _ in range(2)]       # step that used the set finished
+        readback = [torch.cuda.Event() for _ in range(2)]   # its output copied to the host
 
-    for _ in range(max(3, args.warmup)):
-        e2e_step()
+        def h2d_copy(i):
+            b = bufs[i % 2]
+            with torch.cuda.stream(copy):
+                if i >= 2:
+                    copy.wait_event(done[i % 2])
+                for n in names:
+                    b[n].copy_(host[n], non_blocking=True)
+                landed[i % 2].record(copy)
+
+        if f0 is not None:
+            f0.record(copy)
+        h2d_copy(0)
+        for i in range(n_steps):
+            if i + 1 < n_steps:
+                h2d_copy(i + 1)
+            b = bufs[i % 2]
+            stream.wait_event(landed[i % 2])
+            if i >= 2:
+                stream.wait_event(readback[i % 2])
+            sti = dict(st)
+            sti.update(b)
+            decode_step(sti, wl.w)
+            done[i % 2].record(stream)
+            with torch.cuda.stream(copy):
+                copy.wait_event(done[i % 2])
+                out_h[i % 2].copy_(b["out"], non_blocking=True)
+                readback[i % 2].record(copy)
+        if f1 is not None:
+            f1.record(copy)
+
+    e2e_run(max(3, args.warmup))
     barrier(pg, dev)
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    f1.record(stream)
+    e2e_run(args.steps, f0, f1)
     barrier(pg, dev)
+    copy.synchronize()
     e2e_value, _ = weak_scaling_value(keys * args.steps, f0.elapsed_time(f1) * 1e-3, pg, dev, world)
 
     pre = prefill_measure(dev) if not args.no_prefill else None
