@@ -59,6 +59,8 @@ def _load():
             lib.oracle_routed_attention_head.restype = ctypes.c_int
             lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
             lib.oracle_half_to_double.restype = ctypes.c_double
+            lib.oracle_route_argmax.argtypes = [p, ctypes.c_int64, ctypes.c_int, p]
+            lib.oracle_route_argmax.restype = None
             _lib = lib
     return _lib
 
@@ -140,3 +142,22 @@ def routed_attention_head(q, pos, modes, w: int, k, v, bits) -> np.ndarray:
 
 def half_to_double(h: int) -> float:
     return _load().oracle_half_to_double(int(h))
+
+
+WIDTHS = (2, 4, 8, 16)
+
+
+def route_argmax(z_attn=None, z_bits=None):
+    """Inference-time router (Eq. 5 heads, hard argmax): modes uint8 [...] from z_attn
+    [..., 3] (0 skip, 1 local, 2 full) and widths uint8 [...] in {2, 4, 8, 16} from
+    z_bits [..., 4]. Either input may be None."""
+    def amax(z, k):
+        z = np.ascontiguousarray(np.asarray(z, dtype=np.float32))
+        if z.shape[-1] != k:
+            raise ValueError(f"last dimension must be {k}")
+        out = np.empty(z.shape[:-1], dtype=np.uint8)
+        _load().oracle_route_argmax(_ptr(z), int(out.size), k, _ptr(out))
+        return out
+    modes = None if z_attn is None else amax(z_attn, 3)
+    bits = None if z_bits is None else np.asarray(WIDTHS, dtype=np.uint8)[amax(z_bits, 4)]
+    return modes, bits

@@ -16,6 +16,10 @@
  *                        skip -> 0, local -> Attn(q_t, K[t-w, t], V[t-w, t]),
  *                        full -> Attn(q_t, K[<=t], V[<=t]), over the dequantized cache,
  *                        softmax in fp64.
+ *   - oracle_route_argmax: the inference-time router (section 3 item 5, Eq. 5, and the
+ *                        "inference" paragraph of the training procedure): the hard argmax
+ *                        of each row of controller logits, z^a over {skip, local, full} and
+ *                        z^b over the widths {2, 4, 8, 16}.
  *
  * Readings taken where the pages leave a step open (each is also listed in the design notes):
  *   - the quantization group is one (token, head) vector of head_dim values;
@@ -23,7 +27,9 @@
  *     division and rint (the precision the kernels use), s = 0 gives code 0;
  *   - b = 16 keeps the raw fp16 bits, with side entry (s, z) = (1, 0);
  *   - local window is inclusive, keys max(0, t - w) .. t (w + 1 keys once t >= w);
- *   - the softmax scale is 1/sqrt(head_dim); the output is stored as fp32.
+ *   - the softmax scale is 1/sqrt(head_dim); the output is stored as fp32;
+ *   - the router's argmax compares the fp32 logits as given; a tie goes to the first
+ *     (lowest) index, and a NaN logit never wins (all-NaN rows give index 0).
  *
  * Build: gcc -O2 -std=c99 -ffp-contract=off -fno-fast-math -shared -fPIC
  * (no FMA contraction, so every fp32 operation rounds exactly once as written).
@@ -213,4 +219,23 @@ done:
     free(qd);
     free(codes);
     return rc;
+}
+
+/*
+ * Hard argmax of n rows of k fp32 logits (row-major), first index on ties: the router at
+ * inference picks the mode (k = 3: skip, local, full) and the width index (k = 4:
+ * b = 2, 4, 8, 16) of each (token, head). NaN entries are passed over; a row of NaNs
+ * gives index 0.
+ */
+void oracle_route_argmax(const float *z, int64_t n, int k, uint8_t *out)
+{
+    for (int64_t r = 0; r < n; ++r) {
+        const float *row = z + r * k;
+        int best = -1;
+        for (int i = 0; i < k; ++i) {
+            if (isnan(row[i])) continue;
+            if (best < 0 || row[i] > row[best]) best = i;
+        }
+        out[r] = (uint8_t)(best < 0 ? 0 : best);
+    }
 }
