@@ -211,12 +211,28 @@ def prefill_measure(dev, reps=5, warm=2):
             tw.append(e[0].elapsed_time(e[1]) * 1e-3)
             tp.append(e[2].elapsed_time(e[3]) * 1e-3)
     cache.check()
+    # router hard argmax on the same (token, head) rows: 3 + 4 fp32 logits in, 2 bytes out
+    za, zb = synth.router_logits(wl, dev)
+    route_bytes = wl.n_tok * H * (7 * 4 + 2)
+    tr = []
+    for r in range(warm + reps):
+        flush.fill_(r & 255)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        kvq.route_argmax(za, zb)
+        e[1].record(stream)
+        stream.synchronize()
+        if r >= warm:
+            tr.append(e[0].elapsed_time(e[1]) * 1e-3)
     flops = 4.0 * D * pairs
     t_p, t_w = statistics.median(tp), statistics.median(tw)
+    t_r = statistics.median(tr)
     return dict(workload="ragged_prefill: lengths {1024,3000,8192,5555}, H=16, head_dim 128, w=512, "
                 "bits p=.3/.4/.2/.1, modes p=.2/.4/.4, 1% outlier channels x8",
                 pairs=pairs, flops=flops, prefill_s=t_p, tflops=flops / t_p / 1e12,
-                write_s=t_w, write_bytes=write_bytes, write_gbs=write_bytes / t_w / 1e9)
+                write_s=t_w, write_bytes=write_bytes, write_gbs=write_bytes / t_w / 1e9,
+                route_s=t_r, route_rows=wl.n_tok * H, route_bytes=route_bytes,
+                route_gbs=route_bytes / t_r / 1e9)
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -443,7 +459,10 @@ def run_ours(args):
             "quantize": {"gbs": pre["write_gbs"], "bytes": pre["write_bytes"],
                          "seconds": pre["write_s"], "frac_of_hbm": pre["write_gbs"] / hbm_peak,
                          # DRAM bytes of the quantize kernel (the scan kernel's are not included)
-                         "traffic": _profiled_traffic("write_quant_ragged_prefill.md", "kvq_write.cu")}}
+                         "traffic": _profiled_traffic("write_quant_ragged_prefill.md", "kvq_write.cu")},
+            "route": {"rows": pre["route_rows"], "bytes": pre["route_bytes"], "seconds": pre["route_s"],
+                      "gbs": pre["route_gbs"], "frac_of_hbm": pre["route_gbs"] / hbm_peak,
+                      "note": "router hard argmax (kvq_route_argmax), L2 flushed before each rep"}}
     if rank == 0 and not args.no_cpu_baseline:
         v_cpu, n_keys, secs, desc = oracle_decode_sample(wl, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": 1, "kind": "oracle",

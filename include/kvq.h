@@ -184,6 +184,22 @@ int kvq_check(kvq_cache *cache, kvq_stream_t stream);
  */
 int kvq_set_profile_events(void *before, void *after);
 
+/*
+ * Router hard argmax at inference (section 3 item 5, Eq. 5: the controller's attention head
+ * z^a and bit head z^b; the inference paragraph: the router takes the hard argmax and each
+ * token's KV is stored at its chosen width). For n rows, one per (token, head):
+ *   z_attn: fp32 [n][3] logits over (skip, local, full) -> modes: uint8 [n] in {0, 1, 2};
+ *   z_bits: fp32 [n][4] logits over the widths (2, 4, 8, 16) -> bits: uint8 [n] in
+ *           {2, 4, 8, 16}.
+ * The first index wins a tie; NaN entries are passed over, and an all-NaN row gives
+ * index 0. Either pair (z_attn, modes) or (z_bits, bits) may be NULL, not both. All four
+ * are DEVICE pointers: z_attn and z_bits 16-byte aligned, modes and bits 4-byte aligned.
+ * The outputs are the `bits` of kvq_write and the `modes` of routed_attn_prefill /
+ * routed_attn_decode (laid out [n_tok][heads] or [batch][heads]).
+ */
+int kvq_route_argmax(const float *z_attn, const float *z_bits, int64_t n, uint8_t *modes,
+                     uint8_t *bits, kvq_stream_t stream);
+
 /* Text of the last host-side error on this thread ("" if none). */
 const char *kvq_last_error(void);
 

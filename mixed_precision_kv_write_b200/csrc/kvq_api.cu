@@ -141,6 +141,20 @@ int num_sms()
 
 extern "C" {
 
+int kvq_route_argmax(const float *z_attn, const float *z_bits, int64_t n, uint8_t *modes,
+                     uint8_t *bits, kvq_stream_t stream)
+{
+    if (n < 0) return fail(KVQ_ERR_ARG, "kvq_route_argmax: n = %lld < 0", (long long)n);
+    if ((!z_attn) != (!modes)) return fail(KVQ_ERR_ARG, "kvq_route_argmax: z_attn and modes go together");
+    if ((!z_bits) != (!bits)) return fail(KVQ_ERR_ARG, "kvq_route_argmax: z_bits and bits go together");
+    if (!z_attn && !z_bits) return fail(KVQ_ERR_ARG, "kvq_route_argmax: nothing to do");
+    if (((reinterpret_cast<uintptr_t>(z_attn) | reinterpret_cast<uintptr_t>(z_bits)) & 15u) ||
+        ((reinterpret_cast<uintptr_t>(modes) | reinterpret_cast<uintptr_t>(bits)) & 3u))
+        return fail(KVQ_ERR_ARG, "kvq_route_argmax: logits must be 16-byte aligned, outputs 4-byte aligned");
+    cudaError_t e = kvq::launch_route_argmax(z_attn, z_bits, n, modes, bits, reinterpret_cast<cudaStream_t>(stream));
+    return e ? cuda_fail(e, "kvq_route_argmax") : ok();
+}
+
 const char *kvq_last_error(void) { return g_err.c_str(); }
 
 int kvq_set_profile_events(void *before, void *after)

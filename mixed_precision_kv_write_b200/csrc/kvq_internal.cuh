@@ -234,6 +234,8 @@ struct kvq_cache {
 };
 
 namespace kvq {
+cudaError_t launch_route_argmax(const float *za, const float *zb, int64_t n, uint8_t *modes,
+                                uint8_t *bits, cudaStream_t st);
 cudaError_t launch_write(kvq_cache *c, const __half *k, const __half *v, const uint8_t *bits,
                          const int32_t *cu, int64_t n_tok, cudaStream_t st);
 cudaError_t launch_decode(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,

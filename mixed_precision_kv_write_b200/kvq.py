@@ -23,7 +23,7 @@ MODE_SKIP, MODE_LOCAL, MODE_FULL = 0, 1, 2
 EXPORTS = ("kvq_cache_create", "kvq_cache_destroy", "kvq_cache_reset", "kvq_cache_truncate",
            "kvq_cache_lengths", "kvq_write", "routed_attn_prefill", "routed_attn_decode",
            "routed_attn_decode_noalloc", "kvq_cache_export", "kvq_check", "kvq_set_profile_events",
-           "kvq_last_error")
+           "kvq_route_argmax", "kvq_last_error")
 
 _lib = None
 
@@ -57,6 +57,7 @@ def load_library(path: str = LIB_PATH):
         "kvq_cache_export": ([vp, i32, i32, i64, i64, vp, vp, vp, vp, vp], i32),
         "kvq_check": ([vp, vp], i32),
         "kvq_set_profile_events": ([vp, vp], i32),
+        "kvq_route_argmax": ([vp, vp, i64, vp, vp, vp], i32),
         "kvq_last_error": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -227,3 +228,32 @@ def routed_attn_decode_noalloc(q, cache: KVQCache, modes, w: int, out=None, stre
     _raise(load_library().routed_attn_decode_noalloc(_ptr(q), cache.handle, _ptr(modes), int(w),
                                                      _ptr(out), _stream(stream, dev)))
     return out
+
+
+def route_argmax(z_attn=None, z_bits=None, stream=None):
+    """Router hard argmax (Eq. 5 heads): modes uint8 [...] from z_attn fp32 [..., 3] and
+    bits uint8 [...] in {2, 4, 8, 16} from z_bits fp32 [..., 4]; either may be None."""
+    ref = z_attn if z_attn is not None else z_bits
+    if ref is None:
+        raise ValueError("route_argmax: pass z_attn, z_bits or both")
+    dev = ref.device
+    if dev.type != "cuda":
+        raise ValueError(f"route_argmax: logits must be on a CUDA device (got {dev})")
+    outs, n = [], None
+    for z, k in ((z_attn, 3), (z_bits, 4)):
+        if z is None:
+            outs.append(None)
+            continue
+        if z.dtype != torch.float32 or not z.is_contiguous() or z.shape[-1] != k or z.device != dev:
+            raise ValueError(f"route_argmax: expected contiguous fp32 [..., {k}] on {dev}")
+        rows = z.numel() // k
+        if n is not None and rows != n:
+            raise ValueError("route_argmax: z_attn and z_bits have different row counts")
+        n = rows
+        outs.append(torch.empty(z.shape[:-1], dtype=torch.uint8, device=dev))
+    _raise(load_library().kvq_route_argmax(_ptr(z_attn) if z_attn is not None else None,
+                                           _ptr(z_bits) if z_bits is not None else None, n,
+                                           _ptr(outs[0]) if outs[0] is not None else None,
+                                           _ptr(outs[1]) if outs[1] is not None else None,
+                                           _stream(stream, dev)))
+    return outs[0], outs[1]

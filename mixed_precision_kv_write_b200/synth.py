@@ -29,6 +29,7 @@ MODE_SKIP, MODE_LOCAL, MODE_FULL = 0, 1, 2
 
 # stream ids
 _S_Q, _S_K, _S_V, _S_OQ, _S_OK, _S_OV, _S_BITS, _S_MODES, _S_DQ, _S_DMODES = range(1, 11)
+_S_ZA, _S_ZB = 11, 12
 
 
 @dataclass(frozen=True)
@@ -164,6 +165,21 @@ def decode_queries(wl: Workload, device):
     modes = categorical((wl.batch, H), wl.modes_p, (MODE_SKIP, MODE_LOCAL, MODE_FULL),
                         wl.seed, _S_DMODES, 0, device)
     return q, modes
+
+
+def router_logits(wl: Workload, device, ties: bool = True):
+    """Synthetic controller logits per (token, head): z_attn fp32 [n_tok, H, 3] and z_bits
+    fp32 [n_tok, H, 4], N(0, 1). With ties=True every 8th row is rounded to multiples of
+    0.5, so tied maxima occur. (Trained controller weights are not available; these only
+    exercise the argmax.)"""
+    out = []
+    for stream, k in ((_S_ZA, 3), (_S_ZB, 4)):
+        g = _gen(wl.seed, stream, 0, device)
+        z = torch.randn((wl.n_tok, wl.heads, k), generator=g, device=device, dtype=torch.float32)
+        if ties:
+            z[::8] = torch.round(z[::8] * 2) / 2
+        out.append(z)
+    return out[0], out[1]
 
 
 def scaled(wl: Workload, seqlens=None, heads=None, name=None) -> Workload:
