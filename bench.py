@@ -235,6 +235,55 @@ def prefill_measure(dev, reps=5, warm=2):
                 route_gbs=route_bytes / t_r / 1e9)
 
 
+def gqa_decode_measure(dev, reps=20, warm=3, group=4):
+    """decode_1p3b with grouped-query attention: 16 query heads sharing 4 KV heads (groups
+    of 4, the pages' H_kv = H/4), batch 64, context 8192, w = 512. Times the whole
+    routed_attn_decode call (scheduler, split-K, combine)."""
+    from mixed_precision_kv_write_b200 import kvq, synth
+    base = synth.WORKLOADS["decode_1p3b"]
+    wl = synth.scaled(base, heads=base.heads // group)          # the KV heads
+    B, Hk, D, L, w = wl.batch, wl.heads, wl.head_dim, wl.seqlens[0], wl.w
+    HQ = Hk * group
+    cache = kvq.KVQCache(B, Hk, D, [L] * B, device=dev, query_group=group)
+    q, modes = synth.decode_queries(base, dev)                  # [B, HQ, D], [B, HQ]
+    idx = torch.arange(L, device=dev)
+    kv_of = torch.arange(HQ, device=dev) // group
+    keys = routed = unique = 0
+    for s in range(B):
+        ks, vs, bs = synth.kv_sequence(wl, s, dev)
+        one = synth.cu_seqlens([L if i == s else 0 for i in range(B)], dev)
+        kvq.kvq_write(ks, vs, bs, one, cache)
+        m = modes[s].to(torch.int64)                                   # [HQ]
+        lo = torch.where(m == 1, torch.clamp(torch.tensor(L - 1 - w, device=dev), min=0),
+                         torch.zeros_like(m))
+        read = (idx[:, None] >= lo[None, :]) & (m[None, :] != 0)       # [L, HQ]
+        bk = bs.to(torch.int64)                                        # [L, Hk]
+        per_tok = bk * D // 4 + 16 * (bk < 16)                         # record + side bytes
+        keys += int(read.sum())
+        routed += int((per_tok[:, kv_of] * read).sum())
+        unique += int((per_tok * read.view(L, Hk, group).any(-1)).sum())
+        del ks, vs, bs
+    cache.check()
+    out = torch.empty((B, HQ, D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ts = []
+    for r in range(warm + reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kvq.routed_attn_decode(q, cache, modes, w, out=out)
+        e1.record(stream)
+        stream.synchronize()
+        if r >= warm:
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+    cache.check()
+    t = statistics.median(ts)
+    return dict(workload=f"decode_1p3b with GQA: {HQ} query heads in groups of {group} over {Hk} KV heads, "
+                         f"batch {B}, context {L}, w={w}",
+                keys=keys, seconds=t, tokens_per_s=keys / t,
+                routed_bytes=routed, routed_gbs=routed / t / 1e9,
+                unique_kv_bytes=unique, unique_gbs=unique / t / 1e9)
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 def oracle_decode_sample(wl, budget_s=12.0, max_pairs=None):
     """Time the CPU oracle on decode queries of the workload (skip heads excluded from the
@@ -417,6 +466,7 @@ def run_ours(args):
     e2e_value, _ = weak_scaling_value(keys * args.steps, f0.elapsed_time(f1) * 1e-3, pg, dev, world)
 
     pre = prefill_measure(dev) if not args.no_prefill else None
+    gq = gqa_decode_measure(dev) if not args.no_prefill else None
     barrier(pg, dev)
 
     line = {
@@ -463,6 +513,14 @@ def run_ours(args):
             "route": {"rows": pre["route_rows"], "bytes": pre["route_bytes"], "seconds": pre["route_s"],
                       "gbs": pre["route_gbs"], "frac_of_hbm": pre["route_gbs"] / hbm_peak,
                       "note": "router hard argmax (kvq_route_argmax), L2 flushed before each rep"}}
+    if gq:
+        line["gqa_decode"] = {
+            "workload": gq["workload"], "value": gq["tokens_per_s"], "unit": UNIT,
+            "ms_per_call": gq["seconds"] * 1e3, "attended_keys": gq["keys"],
+            "routed_bytes_per_query_head_sum": gq["routed_bytes"], "routed_gbs": gq["routed_gbs"],
+            "unique_kv_bytes": gq["unique_kv_bytes"], "unique_kv_gbs": gq["unique_gbs"],
+            "note": "each query head reads its own key range of the shared KV stream; time of the whole "
+                    "routed_attn_decode call (scheduler, split-K, combine)"}
     if rank == 0 and not args.no_cpu_baseline:
         v_cpu, n_keys, secs, desc = oracle_decode_sample(wl, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": 1, "kind": "oracle",

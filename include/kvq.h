@@ -69,6 +69,17 @@ enum { KVQ_MODE_SKIP = 0, KVQ_MODE_LOCAL = 1, KVQ_MODE_FULL = 2 };
 int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
                      const int64_t *capacity_tokens, kvq_stream_t stream);
 
+/*
+ * Grouped-query attention variant of kvq_cache_create (the pages' models share each KV
+ * head among a group of query heads; model table, H_kv = H/4). `heads` is the number of KV
+ * heads, which is what kvq_write stores (k, v, bits are [n_tok][heads]...). The attention
+ * calls on this cache take heads * query_group query heads: q, modes and out are
+ * [..][heads * query_group][..], and query head hq reads KV head hq / query_group with its
+ * own mode. query_group = 1 is kvq_cache_create. 1 <= query_group <= 64.
+ */
+int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group, int head_dim,
+                         const int64_t *capacity_tokens, kvq_stream_t stream);
+
 /* Free every device buffer of the cache (synchronizes the device first). NULL is a no-op. */
 int kvq_cache_destroy(kvq_cache *cache);
 

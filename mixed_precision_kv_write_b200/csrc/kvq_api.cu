@@ -169,9 +169,19 @@ int kvq_set_profile_events(void *before, void *after)
 int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
                      const int64_t *capacity_tokens, kvq_stream_t stream)
 {
+    return kvq_cache_create_gqa(out, batch, heads, 1, head_dim, capacity_tokens, stream);
+}
+
+int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group, int head_dim,
+                         const int64_t *capacity_tokens, kvq_stream_t stream)
+{
     if (!out) return fail(KVQ_ERR_ARG, "kvq_cache_create: out is NULL");
     *out = nullptr;
     if (batch <= 0 || heads <= 0) return fail(KVQ_ERR_ARG, "kvq_cache_create: batch and heads must be > 0");
+    if (query_group < 1 || query_group > 64)
+        return fail(KVQ_ERR_ARG, "kvq_cache_create: query_group = %d outside [1, 64]", query_group);
+    if ((int64_t)batch * heads * query_group > (1 << 24))
+        return fail(KVQ_ERR_ARG, "kvq_cache_create: batch*heads*query_group too large");
     if ((int64_t)batch * heads > (1 << 24)) return fail(KVQ_ERR_ARG, "kvq_cache_create: batch*heads too large");
     if (head_dim != 64 && head_dim != 128)
         return fail(KVQ_ERR_ARG, "kvq_cache_create: head_dim must be 64 or 128 (got %d)", head_dim);
@@ -189,7 +199,7 @@ int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
         cap_pad[s] = (int32_t)((cp + 4) & ~int64_t(3));    // >= cp + 1, multiple of 4
         slot_base[s] = slots;
         slots += (int64_t)heads * cap_pad[s];
-        max_items += (int64_t)heads * ((cp + kvq::kDecodeItemKeys - 1) / kvq::kDecodeItemKeys);
+        max_items += (int64_t)heads * query_group * ((cp + kvq::kDecodeItemKeys - 1) / kvq::kDecodeItemKeys);
         max_cap = std::max(max_cap, cap[s]);
     }
     if (max_items > INT32_MAX / 2) return fail(KVQ_ERR_ARG, "kvq_cache_create: too many decode items");
@@ -211,10 +221,12 @@ int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
         return p;
     };
     const int BH = batch * heads;
+    const int BHQ = BH * query_group;      // query heads
     kvq::CacheView &v = c->view;
     v.B = batch;
     v.H = heads;
     v.D = head_dim;
+    v.G = query_group;
     bool okk = true;
     int32_t *cap_d = (int32_t *)alloc(sizeof(int32_t) * batch);
     int32_t *cap_pad_d = (int32_t *)alloc(sizeof(int32_t) * batch);
@@ -232,13 +244,13 @@ int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
     wk.max_items = max_items;
     wk.items = (kvq::DecodeItem *)alloc(sizeof(kvq::DecodeItem) * (size_t)max_items);
     wk.count = (int32_t *)alloc(sizeof(int32_t));
-    wk.head_first = (int32_t *)alloc(sizeof(int32_t) * BH);
-    wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * BH);
+    wk.head_first = (int32_t *)alloc(sizeof(int32_t) * BHQ);
+    wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * BHQ);
     wk.partials = (float *)alloc(sizeof(float) * (size_t)max_items * (head_dim + 4));
-    c->pf_max_tiles = slots / 128 + 2LL * BH;
+    c->pf_max_tiles = slots * query_group / 128 + 2LL * BHQ;
     c->pf_tiles = alloc(sizeof(int32_t) * 4 * (size_t)c->pf_max_tiles);
     c->pf_count = (int32_t *)alloc(sizeof(int32_t));
-    c->pf_qidx = (int32_t *)alloc(sizeof(int32_t) * (size_t)slots);
+    c->pf_qidx = (int32_t *)alloc(sizeof(int32_t) * (size_t)slots * query_group);
     for (int i = 0; i < c->n_allocs; ++i) okk = okk && c->allocs[i];
     if (!okk || c->n_allocs != 20) {
         kvq_cache_destroy(c);
@@ -335,7 +347,7 @@ int routed_attn_prefill(const void *q, const kvq_cache *c, const uint8_t *modes,
 {
     if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "routed_attn_prefill: bad cache");
     if (w < 0) return fail(KVQ_ERR_ARG, "routed_attn_prefill: w = %d < 0", w);
-    if (n_tok < 0 || n_tok > (int64_t)INT32_MAX / c->H)
+    if (n_tok < 0 || n_tok > (int64_t)INT32_MAX / ((int64_t)c->H * c->view.G))
         return fail(KVQ_ERR_ARG, "routed_attn_prefill: n_tok = %lld out of range", (long long)n_tok);
     if (!cu_seqlens) return fail(KVQ_ERR_ARG, "routed_attn_prefill: cu_seqlens is NULL");
     if (n_tok > 0 && (!q || !modes || !out))

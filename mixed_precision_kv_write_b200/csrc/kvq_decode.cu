@@ -102,7 +102,8 @@ __global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ mod
     __shared__ int carry_sh;
     pdl_wait();
     pdl_trigger();
-    const int BH = c.B * c.H;
+    const int HQ = c.H * c.G;                 // query heads; query head hq reads KV head hq / G
+    const int BH = c.B * HQ;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (tid == 0) carry_sh = 0;
     __syncthreads();
@@ -113,10 +114,10 @@ __global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ mod
         uint32_t end_i = 0;
         if (i < BH) {
             // every load of this head up front: one round trip before the scan
-            const int s = i / c.H, h = i % c.H;
+            const int s = i / HQ, h = (i % HQ) / c.G, shk = s * c.H + h;
             const int m = modes[i];
-            L = c.len[i];
-            end_i = c.end[i];
+            L = c.len[shk];
+            end_i = c.end[shk];
             sb = slot_of(c, s, h, 0);
             if (m > KVQ_MODE_FULL) {
                 set_status(c.status, KVQ_ERR_MODE);
@@ -735,7 +736,7 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const __half *q, const uint8
     le = launch_pdl(decode_splitk_kernel<D>, dim3(grid), dim3(kThreads), smem, st, c, q, cache->work);
     if (le != cudaSuccess) return le;
     profile_after(st);
-    le = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H), dim3(D), 0, st, c, cache->work, out);
+    le = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H * c.G), dim3(D), 0, st, c, cache->work, out);
     if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
@@ -798,7 +799,7 @@ cudaError_t launch_decode_static(const kvq_cache *cache, const DecodeWork &wk, c
     const int grid = (int)std::min<int64_t>(wk.max_items, 3 * (int64_t)num_sms());
     e = launch_pdl(decode_splitk_kernel<D>, dim3(grid), dim3(kThreads), smem, st, c, q, wk);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H), dim3(D), 0, st, c, wk, out);
+    e = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H * c.G), dim3(D), 0, st, c, wk, out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -824,7 +825,7 @@ extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache,
 
     // scratch layout: count | head_first | head_cnt | items | partials, each 256-byte aligned,
     // sized for the cache's worst case (every head full at capacity)
-    const int BH = cache->B * cache->H;
+    const int BH = cache->B * cache->H * cache->view.G;     // query heads
     const int64_t items = cache->work.max_items;
     const size_t o_first = 256;
     const size_t o_cnt = o_first + align256(sizeof(int32_t) * (size_t)BH);

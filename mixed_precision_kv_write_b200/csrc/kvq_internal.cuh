@@ -26,6 +26,7 @@ namespace kvq {
 
 struct CacheView {
     int B, H, D;
+    int G;                    // query heads per KV head (grouped-query attention); 1 = MHA
     const int32_t *cap;       // [B] capacity in tokens
     const int32_t *cap_pad;   // [B] slots per (s, h)
     const int64_t *slot_base; // [B] first slot of sequence s

@@ -198,11 +198,12 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const PfTile tile = tiles[blockIdx.x];
-    const int H = c.H, sh = tile.sh, s = sh / H, h = sh % H;
+    // tile.sh = (sequence, query head); query head hq reads KV head hq / G
+    const int H = c.H * c.G, sh = tile.sh, s = sh / H, h = sh % H, hk = h / c.G;
     const int n_s = cu[s + 1] - cu[s];
-    const int pos0 = c.len[sh] - n_s;
-    const int64_t sbase = slot_of(c, s, h, 0);
-    const uint8_t *stream = stream_of(c, s, h);
+    const int pos0 = c.len[s * c.H + hk] - n_s;
+    const int64_t sbase = slot_of(c, s, hk, 0);
+    const uint8_t *stream = stream_of(c, s, hk);
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -557,12 +558,13 @@ prefill_sched_kernel(CacheView c, const uint8_t *__restrict__ modes, const int32
     __shared__ int wsum[kSchedThreads / 32];
     __shared__ int carry_l, carry_f;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int H = c.H, sh = blockIdx.x, s = sh / H, h = sh % H;
+    // one CTA per (sequence, query head); query head h reads KV head h / G
+    const int H = c.H * c.G, sh = blockIdx.x, s = sh / H, h = sh % H;
     const int64_t t0 = cu[s], t1 = cu[s + 1];
     if (t0 < 0 || t1 < t0 || t1 > n_tok) return;      // flagged by the write's checks
     const int n = (int)(t1 - t0);
     if (n == 0) return;
-    if (c.len[sh] - n < 0) {
+    if (c.len[s * c.H + h / c.G] - n < 0) {
         if (tid == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
         return;
     }
@@ -655,9 +657,9 @@ cudaError_t run_tc(const kvq_cache *cache, const __half *q, const uint8_t *modes
     PfTile *tiles = reinterpret_cast<PfTile *>(cache->pf_tiles);
     cudaError_t e = cudaMemsetAsync(cache->pf_count, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return e;
-    prefill_sched_kernel<<<c.B * c.H, kSchedThreads, 0, st>>>(c, modes, cu, n_tok, D, out, tiles, cache->pf_count,
+    prefill_sched_kernel<<<c.B * c.H * c.G, kSchedThreads, 0, st>>>(c, modes, cu, n_tok, D, out, tiles, cache->pf_count,
                                                      cache->pf_qidx);
-    const int64_t max_tiles = n_tok * c.H / kQRows + 2LL * c.B * c.H;
+    const int64_t max_tiles = n_tok * c.H * c.G / kQRows + 2LL * c.B * c.H * c.G;
     const size_t smem = sizeof(PfSmem<D>) + 1024;
     static bool attr_done = false;
     if (!attr_done) {

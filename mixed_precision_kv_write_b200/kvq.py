@@ -20,7 +20,7 @@ KVQ_OK, KVQ_ERR_ARG, KVQ_ERR_BITS, KVQ_ERR_MODE, KVQ_ERR_CAPACITY, KVQ_ERR_CUDA,
 MODE_SKIP, MODE_LOCAL, MODE_FULL = 0, 1, 2
 
 # every symbol include/kvq.h declares
-EXPORTS = ("kvq_cache_create", "kvq_cache_destroy", "kvq_cache_reset", "kvq_cache_truncate",
+EXPORTS = ("kvq_cache_create", "kvq_cache_create_gqa", "kvq_cache_destroy", "kvq_cache_reset", "kvq_cache_truncate",
            "kvq_cache_lengths", "kvq_write", "routed_attn_prefill", "routed_attn_decode",
            "routed_attn_decode_noalloc", "kvq_cache_export", "kvq_check", "kvq_set_profile_events",
            "kvq_route_argmax", "kvq_last_error")
@@ -46,6 +46,7 @@ def load_library(path: str = LIB_PATH):
     vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
     sig = {
         "kvq_cache_create": ([ctypes.POINTER(vp), i32, i32, i32, vp, vp], i32),
+        "kvq_cache_create_gqa": ([ctypes.POINTER(vp), i32, i32, i32, i32, vp, vp], i32),
         "kvq_cache_destroy": ([vp], i32),
         "kvq_cache_reset": ([vp, vp], i32),
         "kvq_cache_truncate": ([vp, vp, vp], i32),
@@ -99,7 +100,8 @@ def _check(t, name, dtype, device, shape=None):
 class KVQCache:
     """Owning handle of a routed mixed-precision KV cache (kvq_cache_create/destroy)."""
 
-    def __init__(self, batch: int, heads: int, head_dim: int, capacity, device=None, stream=None):
+    def __init__(self, batch: int, heads: int, head_dim: int, capacity, device=None, stream=None,
+                 query_group: int = 1):
         lib = load_library()
         dev = torch.device("cuda") if device is None else torch.device(device)
         if dev.type != "cuda":
@@ -110,12 +112,14 @@ class KVQCache:
         if len(cap) != batch:
             raise ValueError("capacity must be an int or have one entry per sequence")
         self.batch, self.heads, self.head_dim, self.capacity = batch, heads, head_dim, cap
+        self.query_group = int(query_group)
+        self.query_heads = heads * self.query_group      # heads of q / modes / out
         arr = (ctypes.c_int64 * batch)(*cap)
         h = ctypes.c_void_p()
         with torch.cuda.device(self.device):
-            _raise(lib.kvq_cache_create(ctypes.byref(h), batch, heads, head_dim,
-                                        ctypes.cast(arr, ctypes.c_void_p),
-                                        _stream(stream, self.device)))
+            _raise(lib.kvq_cache_create_gqa(ctypes.byref(h), batch, heads, self.query_group, head_dim,
+                                            ctypes.cast(arr, ctypes.c_void_p),
+                                            _stream(stream, self.device)))
         self._h = h
 
     @property
@@ -188,12 +192,12 @@ def routed_attn_prefill(q, cache: KVQCache, modes, w: int, cu_seqlens, out=None,
     """Routed causal attention (Eq. 2) of q [n_tok, H, D] over the cache; returns fp32 out."""
     dev = cache.device
     n = q.shape[0]
-    _check(q, "q", torch.float16, dev, (n, cache.heads, cache.head_dim))
-    _check(modes, "modes", torch.uint8, dev, (n, cache.heads))
+    _check(q, "q", torch.float16, dev, (n, cache.query_heads, cache.head_dim))
+    _check(modes, "modes", torch.uint8, dev, (n, cache.query_heads))
     _check(cu_seqlens, "cu_seqlens", torch.int32, dev, (cache.batch + 1,))
     if out is None:
-        out = torch.empty((n, cache.heads, cache.head_dim), dtype=torch.float32, device=dev)
-    _check(out, "out", torch.float32, dev, (n, cache.heads, cache.head_dim))
+        out = torch.empty((n, cache.query_heads, cache.head_dim), dtype=torch.float32, device=dev)
+    _check(out, "out", torch.float32, dev, (n, cache.query_heads, cache.head_dim))
     _raise(load_library().routed_attn_prefill(_ptr(q), cache.handle, _ptr(modes), int(w),
                                               _ptr(cu_seqlens), n, _ptr(out), _stream(stream, dev)))
     return out
@@ -202,7 +206,7 @@ def routed_attn_prefill(q, cache: KVQCache, modes, w: int, cu_seqlens, out=None,
 def routed_attn_decode(q, cache: KVQCache, modes, w: int, out=None, stream=None):
     """Routed decode attention (Eq. 2), q [B, H, D] at t = len - 1; returns fp32 out."""
     dev = cache.device
-    shape = (cache.batch, cache.heads, cache.head_dim)
+    shape = (cache.batch, cache.query_heads, cache.head_dim)
     _check(q, "q", torch.float16, dev, shape)
     _check(modes, "modes", torch.uint8, dev, shape[:2])
     if out is None:
@@ -219,7 +223,7 @@ def routed_attn_decode_noalloc(q, cache: KVQCache, modes, w: int, out=None, stre
     the whole call allocation-free; the first call on a device should precede any stream
     capture, and calls that overlap on the GPU race on the shared scratch."""
     dev = cache.device
-    shape = (cache.batch, cache.heads, cache.head_dim)
+    shape = (cache.batch, cache.query_heads, cache.head_dim)
     _check(q, "q", torch.float16, dev, shape)
     _check(modes, "modes", torch.uint8, dev, shape[:2])
     if out is None:
