@@ -564,9 +564,16 @@ def run_reference(args):
 
 
 def _src_hash(name):
+    """Hash of a kernel source with its comments and blank lines removed, so that an edit
+    of comments alone does not orphan the profile of an unchanged kernel."""
     import hashlib
-    with open(os.path.join(ROOT, "mixed_precision_kv_write_b200", "csrc", name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    import re
+    with open(os.path.join(ROOT, "mixed_precision_kv_write_b200", "csrc", name)) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def _profiled_traffic(summary, source):

@@ -10,8 +10,11 @@
  *     covers a token's K and V (the equation quantizes the pair (k_t, v_t) together).
  *   - Eq. 2 (attention resolution): each (token, head) query has a mode
  *     skip -> 0, local-w -> attention over keys [t - w, t], full -> keys [0, t].
- *   - Inference paragraph after Algorithm 1: skipped attention is never materialised
- *     and each token's KV is stored at its chosen width.
+ *   - Inference paragraph after Algorithm 1: the router takes the hard argmax of its
+ *     logits (Eq. 5's attention and bit heads: kvq_route_argmax), skipped attention is
+ *     never materialised, and each token's KV is stored at its chosen width.
+ *   - Experimental setup, model table: KV heads shared by groups of query heads
+ *     (kvq_cache_create_gqa).
  *
  * Conventions shared by every entry point:
  *   - All tensor arguments are DEVICE pointers owned by the caller, except where marked

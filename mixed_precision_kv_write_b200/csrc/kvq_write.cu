@@ -1,6 +1,8 @@
 // Quantize-on-write (TriRoute paper review page, section 3, Eq. 4).
 //
-// Two launches per kvq_write call:
+// A call with at most 2 * batch tokens (decode steps) is one launch of
+//   write_append_kernel a CTA per sequence doing both steps below for its tokens;
+// longer calls take two launches:
 //   write_scan_kernel   a warp (short appends) or a block (long ones) per (sequence, head):
 //                       validates capacity and widths (a bad width rejects the sequence's
 //                       write for every head) and assigns each new token's record offset
