@@ -6,9 +6,12 @@ head_dim 128, 8192 cached tokens, w = 512): roll each sequence back to 8191 toke
 quantize-on-write the step's new token of every (sequence, head) (Eq. 4), then routed
 decode attention (Eq. 2: scheduler, split-K kernel, log-sum-exp combine) for the query at
 t = 8191. `value` = attended KV tokens per second (keys actually read; skip heads read
-none, local heads w + 1). The same line carries the HBM rate of the routed bytes, the
-roofline of the split-K kernel, the prefill workload (ragged prefill + write: TFLOP/s), an
-end-to-end figure through host buffers and the CPU oracle as a baseline.
+none, local heads w + 1), timed over K back-to-back steps with nothing recorded between
+launches. A separate pass records CUDA events around the split-K kernel of each step for
+the kernel's roofline. The same line carries the HBM rate of the routed bytes, the other
+workloads (long-context decode; ragged and 160M-like prefill + write: TFLOP/s and GB/s;
+grouped-query decode), an end-to-end figure through host buffers and the CPU oracle as a
+baseline (one thread and all host cores).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -113,66 +116,126 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workload setup
-def decode_setup(wl, dev):
+def decode_setup(wl, dev, group=1):
     """Cache holding L - 1 tokens per sequence; the step's token, query and modes; the
-    exact keys and routed bytes one step reads."""
+    exact keys and routed bytes one step reads. With group > 1 the cache holds wl.heads KV
+    heads shared by groups of `group` query heads (grouped-query attention)."""
     from mixed_precision_kv_write_b200 import kvq, synth
     B, H, D, L, w = wl.batch, wl.heads, wl.head_dim, wl.seqlens[0], wl.w
-    cache = kvq.KVQCache(B, H, D, [L + 4] * B, device=dev)
-    q, modes = synth.decode_queries(wl, dev)
+    HQ = H * group
+    cache = kvq.KVQCache(B, H, D, [L + 4] * B, device=dev, query_group=group)
+    q, modes = synth.decode_queries(synth.scaled(wl, heads=HQ) if group > 1 else wl, dev)
     k_step = torch.empty((B, H, D), dtype=torch.float16, device=dev)
     v_step = torch.empty_like(k_step)
     b_step = torch.empty((B, H), dtype=torch.uint8, device=dev)
-    keys = 0
-    rec_bytes = 0
-    side_bytes = 0
+    keys = rec_bytes = side_bytes = unique_bytes = 0
     idx = torch.arange(L, device=dev)
+    kv_of = torch.arange(HQ, device=dev) // group
     for s in range(B):
         ks, vs, bs = synth.kv_sequence(wl, s, dev)
         one = synth.cu_seqlens([L - 1 if i == s else 0 for i in range(B)], dev)
         kvq.kvq_write(ks[:-1].contiguous(), vs[:-1].contiguous(), bs[:-1].contiguous(), one, cache)
         k_step[s], v_step[s], b_step[s] = ks[-1], vs[-1], bs[-1]
-        m = modes[s].to(torch.int64)                                   # [H]
+        m = modes[s].to(torch.int64)                                   # [HQ]
         lo = torch.where(m == 1, torch.clamp(torch.tensor(L - 1 - w, device=dev), min=0),
                          torch.zeros_like(m))
-        read = (idx[:, None] >= lo[None, :]) & (m[None, :] != 0)       # [L, H]
-        bf = bs.to(torch.int64)
+        read = (idx[:, None] >= lo[None, :]) & (m[None, :] != 0)       # [L, HQ]
+        bf = bs.to(torch.int64)[:, kv_of]                              # [L, HQ]
         keys += int(read.sum())
         rec_bytes += int(((bf * D // 4) * read).sum())
         side_bytes += int((16 * (bf < 16) * read).sum())
+        bk = bs.to(torch.int64)
+        unique_bytes += int(((bk * D // 4 + 16 * (bk < 16)) * read.view(L, H, group).any(-1)).sum())
         del ks, vs, bs
     torch.cuda.synchronize(dev)
     cache.check()
     return dict(cache=cache, q=q, modes=modes, k_step=k_step, v_step=v_step, b_step=b_step,
                 cu_one=synth.cu_seqlens([1] * B, dev),
                 roll=torch.full((B,), L - 1, dtype=torch.int32, device=dev),
-                out=torch.empty((B, H, D), dtype=torch.float32, device=dev),
-                keys=keys, rec_bytes=rec_bytes, side_bytes=side_bytes,
-                q_bytes=B * H * D * 2, out_bytes=B * H * D * 4)
+                out=torch.empty((B, HQ, D), dtype=torch.float32, device=dev),
+                keys=keys, rec_bytes=rec_bytes, side_bytes=side_bytes, unique_bytes=unique_bytes,
+                q_bytes=B * HQ * D * 2, out_bytes=B * HQ * D * 4)
 
 
 def decode_step(st, w, events=None):
-    """One step; `events` (before, after) are recorded around the split-K kernel only, so
-    the other kernels of the step stay back to back in the stream."""
+    """One step through kvq_decode_step: roll each sequence back to L - 1 tokens, append the
+    step's token at its width, decode. `events` (before, after) are recorded around the
+    split-K kernel only, so the other kernels of the step stay back to back in the stream."""
     from mixed_precision_kv_write_b200 import kvq
-    c = st["cache"]
-    c.truncate(st["roll"])
-    kvq.kvq_write(st["k_step"], st["v_step"], st["b_step"], st["cu_one"], c)
     if events is not None:
         kvq.kvq_set_profile_events(*events)
-    kvq.routed_attn_decode(st["q"], c, st["modes"], w, out=st["out"])
+    kvq.decode_step(st["q"], st["k_step"], st["v_step"], st["b_step"], st["cu_one"], st["cache"],
+                    st["modes"], w, positions=st["roll"], out=st["out"])
     if events is not None:
         kvq.kvq_set_profile_events(None, None)
 
 
-LAUNCHES_PER_DECODE_STEP = 5   # truncate, write (single-launch append), sched, split-K, combine
+LAUNCHES_PER_DECODE_STEP = 3   # plan (roll-back + append + schedule), split-K, combine
 
 
-def prefill_measure(dev, reps=5, warm=2):
-    """Ragged prefill + quantize-on-write workload: lengths {1024, 3000, 8192, 5555},
-    16 heads, head_dim 128, w = 512."""
+def decode_kernel_times(st, w, steps, stream):
+    """Mean duration of the split-K kernel over `steps` decode steps (events recorded
+    around that kernel by the library's profiling hook). A pass of its own: the events
+    between launches stop the programmatic overlap of neighbouring kernels, so the
+    headline loop records none."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        decode_step(st, w, ev[i])
+    stream.synchronize()
+    return statistics.mean(a.elapsed_time(b) * 1e-3 for a, b in ev)
+
+
+def decode_roofline(st, k_avg, pk, pk_kind, profile_summary):
+    kernel_bytes = st["rec_bytes"] + st["side_bytes"] + st["q_bytes"]
+    achieved = kernel_bytes / k_avg / 1e9
+    hbm_peak = float(pk["hbm_gbs"])
+    return {"kernel": "decode_splitk_kernel<128>", "bound": "hbm", "achieved": achieved,
+            "peak": hbm_peak, "peak_kind": pk_kind, "unit": "GB/s", "frac": achieved / hbm_peak,
+            "traffic": _profiled_traffic(profile_summary, "kvq_decode.cu") if profile_summary else None,
+            "algorithmic_bytes_per_launch": kernel_bytes, "avg_launch_s": k_avg}
+
+
+def decode_workload_measure(name, dev, pk, pk_kind, steps=20, warm=5, group=1, profile_summary=None):
+    """A decode workload other than the headline: its steps timed back to back (no events
+    between launches), then a pass with events around the split-K kernel."""
+    from mixed_precision_kv_write_b200 import synth
+    wl = synth.WORKLOADS[name]
+    if group > 1:
+        wl = synth.scaled(wl, heads=wl.heads // group)
+    st = decode_setup(wl, dev, group)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warm):
+        decode_step(st, wl.w)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        decode_step(st, wl.w)
+    e1.record(stream)
+    stream.synchronize()
+    t_step = e0.elapsed_time(e1) * 1e-3 / steps
+    k_avg = decode_kernel_times(st, wl.w, steps, stream)
+    st["cache"].check()
+    routed = st["rec_bytes"] + st["side_bytes"]
+    res = {"value": st["keys"] / t_step, "unit": UNIT, "ms_per_step": t_step * 1e3,
+           "attended_keys_per_step": st["keys"], "routed_bytes_per_step": routed,
+           "hbm_gbs": routed / t_step / 1e9, "hbm_frac_of_8tbs": routed / t_step / 1e9 / NOMINAL_HBM_GBS,
+           "roofline": decode_roofline(st, k_avg, pk, pk_kind, profile_summary)}
+    if group > 1:
+        res["unique_kv_bytes_per_step"] = st["unique_bytes"]
+        res["unique_kv_gbs"] = st["unique_bytes"] / t_step / 1e9
+    del st
+    torch.cuda.empty_cache()
+    return res
+
+
+def prefill_measure(name, dev, pk, pk_kind, reps=5, warm=2, route=False, profiles=(None, None)):
+    """A prefill + quantize-on-write workload: kvq_write of every token, then routed
+    causal attention of every query. L2 is flushed (256 MB memset) before each rep; the
+    write (scan + quantize kernels) and the attention kernel are timed with events the
+    library records around them."""
     from mixed_precision_kv_write_b200 import kvq, synth
-    wl = synth.WORKLOADS["ragged_prefill"]
+    wl = synth.WORKLOADS[name]
     H, D = wl.heads, wl.head_dim
     k, v, bits = synth.kv_tokens(wl, dev)
     q, modes = synth.prefill_queries(wl, dev)
@@ -211,106 +274,102 @@ def prefill_measure(dev, reps=5, warm=2):
             tw.append(e[0].elapsed_time(e[1]) * 1e-3)
             tp.append(e[2].elapsed_time(e[3]) * 1e-3)
     cache.check()
-    # router hard argmax on the same (token, head) rows: 3 + 4 fp32 logits in, 2 bytes out
-    za, zb = synth.router_logits(wl, dev)
-    route_bytes = wl.n_tok * H * (7 * 4 + 2)
-    tr = []
-    for r in range(warm + reps):
-        flush.fill_(r & 255)
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        e[0].record(stream)
-        kvq.route_argmax(za, zb)
-        e[1].record(stream)
-        stream.synchronize()
-        if r >= warm:
-            tr.append(e[0].elapsed_time(e[1]) * 1e-3)
     flops = 4.0 * D * pairs
     t_p, t_w = statistics.median(tp), statistics.median(tw)
-    t_r = statistics.median(tr)
-    return dict(workload="ragged_prefill: lengths {1024,3000,8192,5555}, H=16, head_dim 128, w=512, "
-                "bits p=.3/.4/.2/.1, modes p=.2/.4/.4, 1% outlier channels x8",
-                pairs=pairs, flops=flops, prefill_s=t_p, tflops=flops / t_p / 1e12,
-                write_s=t_w, write_bytes=write_bytes, write_gbs=write_bytes / t_w / 1e9,
-                route_s=t_r, route_rows=wl.n_tok * H, route_bytes=route_bytes,
-                route_gbs=route_bytes / t_r / 1e9)
-
-
-def gqa_decode_measure(dev, reps=20, warm=3, group=4):
-    """decode_1p3b with grouped-query attention: 16 query heads sharing 4 KV heads (groups
-    of 4, the pages' H_kv = H/4), batch 64, context 8192, w = 512. Times the whole
-    routed_attn_decode call (scheduler, split-K, combine)."""
-    from mixed_precision_kv_write_b200 import kvq, synth
-    base = synth.WORKLOADS["decode_1p3b"]
-    wl = synth.scaled(base, heads=base.heads // group)          # the KV heads
-    B, Hk, D, L, w = wl.batch, wl.heads, wl.head_dim, wl.seqlens[0], wl.w
-    HQ = Hk * group
-    cache = kvq.KVQCache(B, Hk, D, [L] * B, device=dev, query_group=group)
-    q, modes = synth.decode_queries(base, dev)                  # [B, HQ, D], [B, HQ]
-    idx = torch.arange(L, device=dev)
-    kv_of = torch.arange(HQ, device=dev) // group
-    keys = routed = unique = 0
-    for s in range(B):
-        ks, vs, bs = synth.kv_sequence(wl, s, dev)
-        one = synth.cu_seqlens([L if i == s else 0 for i in range(B)], dev)
-        kvq.kvq_write(ks, vs, bs, one, cache)
-        m = modes[s].to(torch.int64)                                   # [HQ]
-        lo = torch.where(m == 1, torch.clamp(torch.tensor(L - 1 - w, device=dev), min=0),
-                         torch.zeros_like(m))
-        read = (idx[:, None] >= lo[None, :]) & (m[None, :] != 0)       # [L, HQ]
-        bk = bs.to(torch.int64)                                        # [L, Hk]
-        per_tok = bk * D // 4 + 16 * (bk < 16)                         # record + side bytes
-        keys += int(read.sum())
-        routed += int((per_tok[:, kv_of] * read).sum())
-        unique += int((per_tok * read.view(L, Hk, group).any(-1)).sum())
-        del ks, vs, bs
-    cache.check()
-    out = torch.empty((B, HQ, D), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    ts = []
-    for r in range(warm + reps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        kvq.routed_attn_decode(q, cache, modes, w, out=out)
-        e1.record(stream)
-        stream.synchronize()
-        if r >= warm:
-            ts.append(e0.elapsed_time(e1) * 1e-3)
-    cache.check()
-    t = statistics.median(ts)
-    return dict(workload=f"decode_1p3b with GQA: {HQ} query heads in groups of {group} over {Hk} KV heads, "
-                         f"batch {B}, context {L}, w={w}",
-                keys=keys, seconds=t, tokens_per_s=keys / t,
-                routed_bytes=routed, routed_gbs=routed / t / 1e9,
-                unique_kv_bytes=unique, unique_gbs=unique / t / 1e9)
+    bf16 = float(pk["bf16_tflops"])
+    hbm_peak = float(pk["hbm_gbs"])
+    res = {"workload": wl.note + f"; bits p={wl.bits_p}, modes p={wl.modes_p}",
+           "tflops": flops / t_p / 1e12, "seconds": t_p, "pairs": pairs, "flops": flops,
+           "roofline": {"kernel": f"prefill_tc_kernel<{D}>", "bound": "tensor", "achieved": flops / t_p / 1e12,
+                        "peak": bf16, "peak_kind": pk_kind + " bf16 dense (burst)", "unit": "TFLOP/s",
+                        "frac": flops / t_p / 1e12 / bf16,
+                        "traffic": _profiled_traffic(profiles[0], "kvq_prefill_tc.cu") if profiles[0] else None},
+           "quantize": {"gbs": write_bytes / t_w / 1e9, "bytes": write_bytes, "seconds": t_w,
+                        "frac_of_hbm": write_bytes / t_w / 1e9 / hbm_peak,
+                        # DRAM bytes of the quantize kernel (the scan kernel's are not included)
+                        "traffic": _profiled_traffic(profiles[1], "kvq_write.cu") if profiles[1] else None}}
+    if route:
+        # router hard argmax on the same (token, head) rows: 3 + 4 fp32 logits in, 2 bytes out
+        za, zb = synth.router_logits(wl, dev)
+        route_bytes = wl.n_tok * H * (7 * 4 + 2)
+        tr = []
+        for r in range(warm + reps):
+            flush.fill_(r & 255)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            e[0].record(stream)
+            kvq.route_argmax(za, zb)
+            e[1].record(stream)
+            stream.synchronize()
+            if r >= warm:
+                tr.append(e[0].elapsed_time(e[1]) * 1e-3)
+        t_r = statistics.median(tr)
+        res["route"] = {"rows": wl.n_tok * H, "bytes": route_bytes, "seconds": t_r,
+                        "gbs": route_bytes / t_r / 1e9, "frac_of_hbm": route_bytes / t_r / 1e9 / hbm_peak,
+                        "note": "router hard argmax (kvq_route_argmax), L2 flushed before each rep"}
+    del cache, k, v, q, out, flush
+    torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_decode_sample(wl, budget_s=12.0, max_pairs=None):
-    """Time the CPU oracle on decode queries of the workload (skip heads excluded from the
-    sample: they do no work). Returns (keys/s, keys, seconds, description)."""
-    import oracle
+def _oracle_decode_jobs(wl, n_seq):
+    """Host copies of the non-skip decode queries of the first n_seq sequences: one job
+    per (sequence, head) with its query, mode, position and the head's fp16 K/V/widths."""
     from mixed_precision_kv_write_b200 import synth
     q, modes = synth.decode_queries(wl, "cpu")
-    L, done_keys, t_total, n = wl.seqlens[0], 0, 0.0, 0
-    for s in range(wl.batch):
-        ks, vs, bs = synth.kv_sequence(wl, s, "cuda" if torch.cuda.is_available() else "cpu")
+    L = wl.seqlens[0]
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    jobs = []
+    for s in range(min(n_seq, wl.batch)):
+        ks, vs, bs = synth.kv_sequence(wl, s, gen_dev)
         ks, vs, bs = ks.cpu(), vs.cpu(), bs.cpu()
         for h in range(wl.heads):
             m = int(modes[s, h])
             if m == 0:
                 continue
-            kh, vh, bh = ks[:, h].contiguous().numpy(), vs[:, h].contiguous().numpy(), bs[:, h].numpy()
-            t0 = time.perf_counter()
-            oracle.routed_attention_head(q[s, h][None].numpy(), [L - 1], [m], wl.w, kh, vh, bh)
-            t_total += time.perf_counter() - t0
-            done_keys += L if m == 2 else min(L, wl.w + 1)
-            n += 1
-            if t_total >= budget_s or (max_pairs and n >= max_pairs):
-                desc = (f"oracle decode of {n} non-skip (sequence, head) queries of "
-                        f"{wl.name} in order, single-threaded C")
-                return done_keys / t_total, done_keys, t_total, desc
-    desc = f"oracle decode of all {n} non-skip queries of {wl.name}, single-threaded C"
-    return done_keys / t_total, done_keys, t_total, desc
+            jobs.append((q[s, h][None].numpy(), m, L, ks[:, h].contiguous().numpy(),
+                         vs[:, h].contiguous().numpy(), bs[:, h].contiguous().numpy()))
+    return jobs
+
+
+def _oracle_run(jobs, w, threads):
+    """Run the oracle on `jobs` with `threads` host threads (the oracle is C behind ctypes,
+    which releases the GIL during the call). Returns (keys, seconds)."""
+    import concurrent.futures as cf
+    import oracle
+
+    def one(j):
+        qv, m, L, kh, vh, bh = j
+        oracle.routed_attention_head(qv, [L - 1], [m], w, kh, vh, bh)
+        return L if m == 2 else min(L, w + 1)
+
+    t0 = time.perf_counter()
+    if threads == 1:
+        keys = sum(one(j) for j in jobs)
+    else:
+        with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+            keys = sum(ex.map(one, jobs))
+    return keys, time.perf_counter() - t0
+
+
+def oracle_baseline(wl, budget_s=12.0, max_seq=32):
+    """The CPU oracle on decode queries of the workload, on one host thread and on all
+    host cores. The one-thread sample is the first n1 non-skip queries, sized to about
+    half the budget; the all-core sample is every non-skip query of the first sequences
+    (at most max_seq, to bound the host memory the K/V copies take)."""
+    cores = os.cpu_count() or 1
+    probe = _oracle_decode_jobs(wl, 1)
+    _, tp = _oracle_run(probe[:3], wl.w, 1)
+    per_job = tp / 3
+    n1 = max(1, int(0.5 * budget_s / per_job))
+    per_seq = max(1, len(probe))
+    n_seq = min(wl.batch, max_seq, max(2, -(-max(n1, cores * n1) // per_seq)))
+    jobs = _oracle_decode_jobs(wl, n_seq)
+    n1 = min(n1, len(jobs))
+    k1, t1 = _oracle_run(jobs[:n1], wl.w, 1)
+    kn, tn = _oracle_run(jobs, wl.w, cores)
+    return {"single": (k1 / t1, k1, t1, n1), "all": (kn / tn, kn, tn, len(jobs)), "cores": cores,
+            "n_seq": n_seq}
 
 
 # ------------------------------------------------------------------ arms
@@ -356,7 +415,7 @@ def weak_scaling_value(units_per_rank: float, elapsed: float, pg: bool, dev, wor
 
 
 def run_ours(args):
-    from mixed_precision_kv_write_b200 import build as kbuild, kvq, synth
+    from mixed_precision_kv_write_b200 import build as kbuild, synth
     kbuild.build()
     import oracle
     oracle.build()
@@ -373,19 +432,14 @@ def run_ours(args):
     sampler.start()
     for _ in range(args.warmup):
         decode_step(st, wl.w)
-    # per-step events around the split-K kernel (profiling hook of the C ABI)
-    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    for a, b in ev_k:       # create the CUDA events now, outside the timed region
-        a.record(stream)
-        b.record(stream)
+    # headline: K steps back to back, nothing recorded between their launches
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(pg, dev)
     t_begin = time.time()
     torch.cuda.nvtx.range_push("decode_timed")
     e0.record(stream)
-    for i in range(args.steps):
-        decode_step(st, wl.w, ev_k[i])
+    for _ in range(args.steps):
+        decode_step(st, wl.w)
     e1.record(stream)
     torch.cuda.nvtx.range_pop()
     barrier(pg, dev)
@@ -393,18 +447,14 @@ def run_ours(args):
     sampler.stop()
     st["cache"].check()
     elapsed = e0.elapsed_time(e1) * 1e-3
-    k_times = [a.elapsed_time(b) * 1e-3 for a, b in ev_k]
-    k_avg = statistics.mean(k_times)
     clocks = sampler.summary(t_begin, t_end)
+    # the split-K kernel alone, in a pass of its own (events around it in every step)
+    k_avg = decode_kernel_times(st, wl.w, args.steps, stream)
 
     keys = st["keys"]
     routed = st["rec_bytes"] + st["side_bytes"]
     value, elapsed_max = weak_scaling_value(keys * args.steps, elapsed, pg, dev, world)
     ms_step = elapsed_max / args.steps * 1e3
-    kernel_bytes = routed + st["q_bytes"]
-    hbm_peak = float(pk["hbm_gbs"])
-    achieved = kernel_bytes / k_avg / 1e9
-    traffic = _profiled_traffic("decode_splitk_decode_1p3b.md", "kvq_decode.cu")
 
     # End to end through host buffers: every step copies its inputs from pinned host memory
     # (H2D) and reads its output back (D2H), inside the timed region. The copies run on a
@@ -464,9 +514,22 @@ def run_ours(args):
     barrier(pg, dev)
     copy.synchronize()
     e2e_value, _ = weak_scaling_value(keys * args.steps, f0.elapsed_time(f1) * 1e-3, pg, dev, world)
+    full = args.decode_batch == synth.WORKLOADS["decode_1p3b"].batch
+    roof = decode_roofline(st, k_avg, pk, pk_kind, "decode_splitk_decode_1p3b.md" if full else None)
+    del st, bufs, host
+    torch.cuda.empty_cache()
 
-    pre = prefill_measure(dev) if not args.no_prefill else None
-    gq = gqa_decode_measure(dev) if not args.no_prefill else None
+    extra = {}
+    if not args.no_prefill:
+        extra["prefill"] = prefill_measure("ragged_prefill", dev, pk, pk_kind, route=True,
+                                           profiles=("prefill_tc_ragged_prefill.md", "write_quant_ragged_prefill.md"))
+        extra["prefill_160m"] = prefill_measure("prefill_160m", dev, pk, pk_kind)
+        extra["decode_long"] = decode_workload_measure("decode_long", dev, pk, pk_kind)
+        gq = decode_workload_measure("decode_1p3b", dev, pk, pk_kind, group=4)
+        gq["workload"] = ("decode_1p3b with grouped-query attention: 16 query heads in groups of 4 over "
+                          "4 KV heads, batch 64, context 8192, w=512")
+        extra["gqa_decode"] = gq
+        extra["decode_long"]["workload"] = synth.WORKLOADS["decode_long"].note
     barrier(pg, dev)
 
     line = {
@@ -479,7 +542,7 @@ def run_ours(args):
                         "bits p(2/4/8/16)=.25/.45/.2/.1, modes p(skip/local/full)=.15/.45/.4",
             "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
             "context": wl.seqlens[0], "w": wl.w,
-            "step": "truncate to 8191, kvq_write of the step token, routed_attn_decode",
+            "step": "kvq_decode_step: roll back to 8191 tokens, append the step token (Eq. 4), routed decode",
             "l2": "no flush: each step reads %.0f MB of routed cache bytes > 126 MB L2" % (routed / 1e6),
             "parallelism": f"{world} independent replica(s), no data-path collective",
             "storage": "packed u2/u4/u8 codes + fp16, fp32 side table"},
@@ -487,44 +550,25 @@ def run_ours(args):
         "routed_bytes_per_step": routed,
         "hbm_gbs": routed / (elapsed_max / args.steps) / 1e9,
         "hbm_frac_of_8tbs": routed / (elapsed_max / args.steps) / 1e9 / NOMINAL_HBM_GBS,
-        "roofline": {"kernel": "decode_splitk_kernel<128>", "bound": "hbm", "achieved": achieved,
-                     "peak": hbm_peak, "peak_kind": pk_kind, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": kernel_bytes,
-                     "avg_launch_s": k_avg},
+        "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": clocks,
         "gpu_launches": LAUNCHES_PER_DECODE_STEP * args.steps,
     }
-    if pre:
-        bf16 = float(pk["bf16_tflops"])
-        line["prefill"] = {
-            "workload": pre["workload"], "tflops": pre["tflops"], "seconds": pre["prefill_s"],
-            "pairs": pre["pairs"], "flops": pre["flops"],
-            "roofline": {"kernel": "prefill attention", "bound": "tensor", "achieved": pre["tflops"],
-                         "peak": bf16, "peak_kind": pk_kind + " bf16 dense (burst)", "unit": "TFLOP/s",
-                         "frac": pre["tflops"] / bf16,
-                         "traffic": _profiled_traffic("prefill_tc_ragged_prefill.md", "kvq_prefill_tc.cu")},
-            "quantize": {"gbs": pre["write_gbs"], "bytes": pre["write_bytes"],
-                         "seconds": pre["write_s"], "frac_of_hbm": pre["write_gbs"] / hbm_peak,
-                         # DRAM bytes of the quantize kernel (the scan kernel's are not included)
-                         "traffic": _profiled_traffic("write_quant_ragged_prefill.md", "kvq_write.cu")},
-            "route": {"rows": pre["route_rows"], "bytes": pre["route_bytes"], "seconds": pre["route_s"],
-                      "gbs": pre["route_gbs"], "frac_of_hbm": pre["route_gbs"] / hbm_peak,
-                      "note": "router hard argmax (kvq_route_argmax), L2 flushed before each rep"}}
-    if gq:
-        line["gqa_decode"] = {
-            "workload": gq["workload"], "value": gq["tokens_per_s"], "unit": UNIT,
-            "ms_per_call": gq["seconds"] * 1e3, "attended_keys": gq["keys"],
-            "routed_bytes_per_query_head_sum": gq["routed_bytes"], "routed_gbs": gq["routed_gbs"],
-            "unique_kv_bytes": gq["unique_kv_bytes"], "unique_kv_gbs": gq["unique_gbs"],
-            "note": "each query head reads its own key range of the shared KV stream; time of the whole "
-                    "routed_attn_decode call (scheduler, split-K, combine)"}
+    line.update(extra)
     if rank == 0 and not args.no_cpu_baseline:
-        v_cpu, n_keys, secs, desc = oracle_decode_sample(wl, budget_s=args.cpu_budget)
-        line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                "sample": f"{desc}: {n_keys} keys in {secs:.1f} s"}
+        ob = oracle_baseline(wl, budget_s=args.cpu_budget)
+        v1, k1, t1, n1 = ob["single"]
+        vn, kn, tn, nn = ob["all"]
+        line["cpu_baseline"] = {
+            "value": vn, "unit": UNIT, "cores": ob["cores"], "kind": "oracle",
+            "sample": (f"oracle decode (C, fp64 softmax) of all {nn} non-skip (sequence, head) queries of "
+                       f"the first {ob['n_seq']} sequences of {wl.name} on {ob['cores']} host threads: "
+                       f"{kn} keys in {tn:.2f} s"),
+            "single_thread": {"value": v1, "unit": UNIT, "cores": 1,
+                              "sample": f"first {n1} non-skip queries: {k1} keys in {t1:.2f} s"},
+            "host_cores": os.cpu_count()}
     if pg:
         torch.distributed.destroy_process_group()
     if rank == 0:
@@ -533,7 +577,8 @@ def run_ours(args):
 
 def run_reference(args):
     """The reference arm is the CPU oracle (no other implementation of this path exists):
-    each step decodes a bounded sample of the same workload on the host cores."""
+    each step decodes a bounded sample of the same workload's queries, one query per host
+    core in parallel."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -542,22 +587,29 @@ def run_reference(args):
     from mixed_precision_kv_write_b200 import synth
     oracle.build()
     wl = synth.WORKLOADS["decode_1p3b"]
-    per_step = 4   # non-skip (sequence, head) queries per step
-    for _ in range(args.warmup):
-        oracle_decode_sample(wl, budget_s=1e9, max_pairs=1)
-    keys = 0
-    secs = 0.0
-    for _ in range(args.steps):
-        _, k, s, desc = oracle_decode_sample(wl, budget_s=1e9, max_pairs=per_step)
+    cores = os.cpu_count() or 1
+    jobs = _oracle_decode_jobs(wl, 4)
+    per_step = max(1, min(cores, len(jobs)))
+
+    def step(i):
+        sel = [jobs[(i * per_step + j) % len(jobs)] for j in range(per_step)]
+        return _oracle_run(sel, wl.w, per_step)
+
+    for i in range(args.warmup):
+        step(i)
+    keys, secs = 0, 0.0
+    for i in range(args.steps):
+        k, s = step(args.warmup + i)
         keys += k
         secs += s
     v = keys / secs
+    desc = (f"oracle decode (C, fp64 softmax) of {per_step} non-skip (sequence, head) queries per step, "
+            f"one per host thread, cycling through the first 4 sequences of decode_1p3b")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": "decode_1p3b (sampled: the first "
-                                            f"{per_step} non-skip queries per step)"},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "data": "synthetic", "config": {"workload": "decode_1p3b (sampled: " + desc + ")"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": per_step, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -597,7 +649,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--decode-batch", type=int, default=64,
                     help="sequences of the decode workload (64; smaller only for profiler captures)")
     args = ap.parse_args()

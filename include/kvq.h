@@ -149,6 +149,24 @@ int routed_attn_decode(const void *q, const kvq_cache *cache, const uint8_t *mod
                        float *out, kvq_stream_t stream);
 
 /*
+ * One decode step in three launches: the step's tokens are written (Eq. 4) and then every
+ * query attends over the cache that holds them (Eq. 2), the per-layer order of the
+ * inference procedure after Algorithm 1 (attention in the routed mode, KV stored at the
+ * routed width). Same results as kvq_cache_truncate (when positions is given), kvq_write
+ * and routed_attn_decode called in turn.
+ *   q, modes, w, out:           as routed_attn_decode.
+ *   k, v, bits, cu_seqlens, n_tok: as kvq_write (one token per sequence in a decode step;
+ *                               any n_tok is accepted, appended by one CTA per sequence).
+ *   positions:                  DEVICE int32 [batch] or NULL. When given, sequence s first
+ *                               keeps only its first min(len, positions[s]) tokens (a
+ *                               negative entry keeps it whole), then its tokens are appended:
+ *                               re-decoding a position, as after a rejected speculation.
+ */
+int kvq_decode_step(const void *q, const void *k, const void *v, const uint8_t *bits,
+                    const int32_t *cu_seqlens, int64_t n_tok, const int32_t *positions,
+                    const uint8_t *modes, int w, kvq_cache *cache, float *out, kvq_stream_t stream);
+
+/*
  * Allocation-free variant of routed_attn_decode (no counterpart in the paper).
  * Same arguments, same arithmetic and the same kernels, but the per-call scratch (the
  * scheduler's work list and the split-K partials) lives in a 16 MiB array in the library's
@@ -213,6 +231,27 @@ int kvq_set_profile_events(void *before, void *after);
  */
 int kvq_route_argmax(const float *z_attn, const float *z_bits, int64_t n, uint8_t *modes,
                      uint8_t *bits, kvq_stream_t stream);
+
+/*
+ * Testing hooks for the failure paths (no counterpart in the paper). Neither faults,
+ * traps or hangs the GPU; both exist so that tests can drive an error path on demand.
+ *
+ * kvq_test_fail_alloc: the nth device allocation (1-based) made by the next
+ * kvq_cache_create / kvq_cache_create_gqa call is reported as failed, as if cudaMalloc had
+ * returned an error. That create then frees what it had allocated, leaves *out NULL and
+ * returns KVQ_ERR_NOMEM. nth = 0 turns a pending injection off. Process-wide; consumed
+ * by the next create call whether or not it reaches the nth allocation.
+ */
+int kvq_test_fail_alloc(int nth);
+
+/*
+ * kvq_test_bounded_wait: launch on `stream` a one-thread kernel that waits, with the same
+ * bounded mbarrier wait the kernels of this library use, on a barrier that no thread ever
+ * completes. After limit_ns nanoseconds (1e3 <= limit_ns <= 1e8) the wait gives up,
+ * records KVQ_ERR_DEVICE_CHECK in the cache's device status word and the kernel returns;
+ * kvq_check() then reports it. The CUDA context stays usable.
+ */
+int kvq_test_bounded_wait(kvq_cache *cache, int64_t limit_ns, kvq_stream_t stream);
 
 /* Text of the last host-side error on this thread ("" if none). */
 const char *kvq_last_error(void);

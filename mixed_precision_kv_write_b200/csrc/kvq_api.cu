@@ -4,7 +4,9 @@
 #include <algorithm>
 #include <cstdarg>
 #include <cstdio>
+#include <atomic>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -126,16 +128,58 @@ int report_error(int code, const char *msg)
     return fail(code, "%s", msg);
 }
 
+namespace {
+// Launch state that depends on the device: the SM count, and which kernels already had
+// their dynamic shared-memory limit raised on which device. One process may drive several
+// GPUs (a thread per device), so both are kept per device ordinal under a mutex.
+constexpr int kMaxDevices = 256;
+std::mutex g_dev_mu;
+int g_sms[kMaxDevices] = {};
+std::vector<std::pair<const void *, int>> g_attr_done;   // (kernel, device)
+
+int current_device()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+    return dev;
+}
+} // namespace
+
 int num_sms()
 {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (g_sms[dev] <= 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        g_sms[dev] = n;
     }
-    return n;
+    return g_sms[dev];
+}
+
+cudaError_t ensure_smem_attr(const void *func, size_t bytes)
+{
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    for (const auto &e : g_attr_done)
+        if (e.first == func && e.second == dev) return cudaSuccess;
+    const cudaError_t err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (err == cudaSuccess) g_attr_done.emplace_back(func, dev);
+    return err;
+}
+
+// Testing hook state: the n-th device allocation of the next cache creation fails.
+std::atomic<int> g_fail_alloc_nth{0};
+
+// One thread waits, with the library's bounded wait, on a barrier that no thread ever
+// completes; after `limit_ns` it records KVQ_ERR_DEVICE_CHECK and returns.
+__global__ void bounded_wait_kernel(int32_t *status, uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0, status, limit_ns);
 }
 } // namespace kvq
 
@@ -199,7 +243,7 @@ int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group,
         cap_pad[s] = (int32_t)((cp + 4) & ~int64_t(3));    // >= cp + 1, multiple of 4
         slot_base[s] = slots;
         slots += (int64_t)heads * cap_pad[s];
-        max_items += (int64_t)heads * query_group * ((cp + kvq::kDecodeItemKeys - 1) / kvq::kDecodeItemKeys);
+        max_items += (int64_t)heads * kvq::decode_max_items(cp, query_group);
         max_cap = std::max(max_cap, cap[s]);
     }
     if (max_items > INT32_MAX / 2) return fail(KVQ_ERR_ARG, "kvq_cache_create: too many decode items");
@@ -214,8 +258,11 @@ int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group,
     cudaGetDevice(&c->device);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
+    const int fail_nth = kvq::g_fail_alloc_nth.exchange(0);   // testing hook, normally 0
+    int n_tried = 0;
     auto alloc = [&](size_t bytes) -> void * {
         void *p = nullptr;
+        if (++n_tried == fail_nth) return nullptr;
         if (cudaMalloc(&p, std::max<size_t>(bytes, 16)) != cudaSuccess) return nullptr;
         c->allocs[c->n_allocs++] = p;
         return p;
@@ -242,17 +289,18 @@ int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group,
     v.status = (int32_t *)alloc(sizeof(int32_t));
     kvq::DecodeWork &wk = c->work;
     wk.max_items = max_items;
+    wk.qslots = std::min(query_group, kvq::kDecodeMaxQ);
     wk.items = (kvq::DecodeItem *)alloc(sizeof(kvq::DecodeItem) * (size_t)max_items);
-    wk.count = (int32_t *)alloc(sizeof(int32_t));
-    wk.head_first = (int32_t *)alloc(sizeof(int32_t) * BHQ);
-    wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * BHQ);
-    wk.partials = (float *)alloc(sizeof(float) * (size_t)max_items * (head_dim + 4));
+    wk.count = (unsigned long long *)alloc(sizeof(unsigned long long));
+    wk.head_first = (int32_t *)alloc(sizeof(int32_t) * BH);
+    wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * BH);
+    wk.partials = (float *)alloc(sizeof(float) * (size_t)max_items * wk.qslots * (head_dim + 4));
     c->pf_max_tiles = slots * query_group / 128 + 2LL * BHQ;
     c->pf_tiles = alloc(sizeof(int32_t) * 4 * (size_t)c->pf_max_tiles);
     c->pf_count = (int32_t *)alloc(sizeof(int32_t));
     c->pf_qidx = (int32_t *)alloc(sizeof(int32_t) * (size_t)slots * query_group);
     for (int i = 0; i < c->n_allocs; ++i) okk = okk && c->allocs[i];
-    if (!okk || c->n_allocs != 20) {
+    if (!okk || c->n_allocs != n_tried) {
         kvq_cache_destroy(c);
         return fail(KVQ_ERR_NOMEM, "kvq_cache_create: cudaMalloc failed (%lld slots, %.2f GB of records)",
                     (long long)slots, (double)slots * 4 * head_dim / 1e9);
@@ -271,7 +319,7 @@ int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group,
     e = e ? e : cudaMemsetAsync(v.bad, 0, sizeof(uint32_t) * batch, st);
     e = e ? e : cudaMemsetAsync(v.status, 0, sizeof(int32_t), st);
     e = e ? e : cudaMemsetAsync(v.meta, 0, sizeof(uint32_t) * (size_t)slots, st);
-    e = e ? e : cudaMemsetAsync(wk.count, 0, sizeof(int32_t), st);
+    e = e ? e : cudaMemsetAsync(wk.count, 0, sizeof(unsigned long long), st);
     if (!e) {
         init_side_kernel<<<1024, 256, 0, st>>>(v.side, slots);
         e = cudaGetLastError();
@@ -374,6 +422,25 @@ int routed_attn_decode(const void *q, const kvq_cache *c, const uint8_t *modes, 
     return e ? cuda_fail(e, "routed_attn_decode") : ok();
 }
 
+int kvq_decode_step(const void *q, const void *k, const void *v, const uint8_t *bits, const int32_t *cu_seqlens,
+                    int64_t n_tok, const int32_t *positions, const uint8_t *modes, int w, kvq_cache *c,
+                    float *out, kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_decode_step: bad cache");
+    if (w < 0) return fail(KVQ_ERR_ARG, "kvq_decode_step: w = %d < 0", w);
+    if (n_tok < 0 || n_tok > (int64_t)INT32_MAX / c->H)
+        return fail(KVQ_ERR_ARG, "kvq_decode_step: n_tok = %lld out of range", (long long)n_tok);
+    if (!q || !modes || !out || !cu_seqlens) return fail(KVQ_ERR_ARG, "kvq_decode_step: q, modes, out or cu_seqlens is NULL");
+    if (n_tok > 0 && (!k || !v || !bits)) return fail(KVQ_ERR_ARG, "kvq_decode_step: k, v or bits is NULL");
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(k) |
+         reinterpret_cast<uintptr_t>(v)) & 15u)
+        return fail(KVQ_ERR_ARG, "kvq_decode_step: q, k, v and out must be 16-byte aligned");
+    cudaError_t e = kvq::launch_decode_step(c, static_cast<const __half *>(q), static_cast<const __half *>(k),
+                                            static_cast<const __half *>(v), bits, cu_seqlens, n_tok, positions,
+                                            modes, w, out, reinterpret_cast<cudaStream_t>(stream));
+    return e ? cuda_fail(e, "kvq_decode_step") : ok();
+}
+
 int kvq_cache_export(const kvq_cache *c, int seq, int head, int64_t first, int64_t count,
                      uint16_t *k_codes, uint16_t *v_codes, float *side, uint8_t *bits, kvq_stream_t stream)
 {
@@ -388,6 +455,24 @@ int kvq_cache_export(const kvq_cache *c, int seq, int head, int64_t first, int64
         c->view, seq, head, first, count, k_codes, v_codes, side, bits);
     cudaError_t e = cudaGetLastError();
     return e ? cuda_fail(e, "kvq_cache_export") : ok();
+}
+
+int kvq_test_fail_alloc(int nth)
+{
+    if (nth < 0) return fail(KVQ_ERR_ARG, "kvq_test_fail_alloc: nth = %d < 0", nth);
+    kvq::g_fail_alloc_nth.store(nth);
+    return ok();
+}
+
+int kvq_test_bounded_wait(kvq_cache *c, int64_t limit_ns, kvq_stream_t stream)
+{
+    if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_test_bounded_wait: bad cache");
+    if (limit_ns < 1000 || limit_ns > 100000000)
+        return fail(KVQ_ERR_ARG, "kvq_test_bounded_wait: limit_ns = %lld outside [1e3, 1e8]", (long long)limit_ns);
+    kvq::bounded_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c->view.status,
+                                                                               (uint64_t)limit_ns);
+    cudaError_t e = cudaGetLastError();
+    return e ? cuda_fail(e, "kvq_test_bounded_wait") : ok();
 }
 
 int kvq_check(kvq_cache *c, kvq_stream_t stream)

@@ -1,24 +1,32 @@
 // Routed decode attention (TriRoute paper review page, section 3, Eq. 2) over the
-// mixed-precision cache of Eq. 4: one query per (sequence, head) at t = len - 1.
+// mixed-precision cache of Eq. 4: one query per (sequence, query head) at t = len - 1.
 //
-// Three launches:
-//   decode_sched_kernel   mode-aware scheduler: skip heads and empty sequences get no
-//                         work, local heads are clamped to keys [max(0, t - w), t], full
-//                         heads read [0, t]; each range is cut into near-equal items of at
-//                         most 512 keys, listed on the device (no host round trip).
-//   decode_splitk_kernel  three CTAs per SM. A producer warp walks the CTA's items in
-//                         stages of at most 128 keys and 24 KB of records: it keeps a ring
-//                         of record-offset windows fetched ahead, cuts each stage at the
-//                         byte budget, sorts the stage's keys by width once (so the
-//                         consumers' 4-key steps rarely mix widths), and streams the stage's
-//                         contiguous record bytes, side entries and (for a new item) the
-//                         query into shared memory with 1-D bulk copies (2-stage mbarrier
-//                         pipeline). Five consumer warps split each stage's keys: 8 lanes
-//                         per key, 16 channels per lane, K dot product -> logit -> online
-//                         softmax kept per 8-lane group -> V accumulation, all in registers;
-//                         the groups' states are merged once per item into a partial
-//                         (m, l, o[D]).
-//   decode_combine_kernel log-sum-exp merge of the item partials of each (sequence, head),
+// Three launches (programmatic dependent launch between them):
+//   decode_plan_kernel    one CTA per sequence. Optionally first appends the step's tokens
+//                         (Eq. 4 quantize-on-write, after an optional roll-back), so one
+//                         decode step is three launches. Then the mode-aware schedule: skip
+//                         queries get no work, local queries read keys [max(0, t - w), t],
+//                         full queries [0, t]. A KV head's query group (grouped-query
+//                         attention) is served in subgroups of up to 4 queries that share
+//                         every record read: the key range is the union of the subgroup's
+//                         ranges, cut where the local window starts, so within an item
+//                         every active query reads every key. Ranges are cut into
+//                         near-equal items of at most 576 keys. Each CTA reserves its items
+//                         with one atomic on a (call generation, count) word.
+//   decode_splitk_kernel  three CTAs per SM, one producer and four consumer warps each. The
+//                         producer walks the CTA's items in stages of at most 128 keys and
+//                         24 KB of records: a ring of record-offset windows is bulk-copied
+//                         ahead, each stage's keys are sorted by width into chunks of one
+//                         width (8 keys at head_dim 128), and the stage's contiguous record
+//                         bytes, side entries and (for a new item) queries are bulk-copied
+//                         into a 2-stage mbarrier pipeline. Consumer lanes: head_dim/32
+//                         lanes per key, 32 channels per lane; K dot product on raw codes ->
+//                         logit -> online softmax per key group (the running max moves only
+//                         when a logit exceeds it by more than 8 in log2 units, a
+//                         warp-uniform branch) -> V accumulation. Each warp serves one query
+//                         of the item; the warps' states are merged into a partial per
+//                         (item, query).
+//   decode_combine_kernel log-sum-exp merge of the partials of each (sequence, query head),
 //                         one thread per channel; zeros for skip heads and empty sequences.
 //
 // Arithmetic. With codes c, scale s and zero z (Eq. 4):
@@ -26,49 +34,70 @@
 //   sum_j p_j deq(v_j) = sum_j (p_j s_j) c_j + (sum_j p_j z_j) * 1
 // Codes are never converted with an int->float instruction: a b-bit field masked in place
 // inside a 32-bit word (bits below 23) IS the fp32 subnormal c * 2^(pos - 149), and FFMA
-// multiplies subnormal operands exactly at full rate. The position scale 2^(pos - 149) is
-// folded into the other operand (q for K, the softmax weight for V), which keeps the
-// unpack at one LOP3 per code. fp32 subnormals must not be flushed: build without
-// -ftz / fast-math.
+// multiplies subnormal operands exactly at full rate. For K the products at each bit
+// position accumulate separately and the position scales 2^-pos are applied once per key;
+// for V the softmax weight is scaled by 2^-pos once per position. Channels c and c + 16 of
+// a lane travel as one float2, so the FMAs are packed FFMA2 instructions (two fp32 FMAs,
+// each rounded as fmaf, subnormal operands kept). fp32 subnormals must not be flushed:
+// build without -ftz / fast-math.
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 
-#include "kvq_internal.cuh"
+#include "kvq_quant.cuh"
 
 namespace kvq {
 namespace {
 
-constexpr int kConsumerWarps = 5;
+constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kCtasPerSm = 3;
 constexpr int kStages = 2;                        // record stages in flight per CTA
 constexpr int kWin = kDecodeWindowKeys;           // keys per window of record offsets
 constexpr uint32_t kStageRecBytes = 24576;        // record bytes per stage, at most
-constexpr int kPermSlots = kWin + 32;             // width-sorted keys padded to whole chunks
+constexpr int kPermSlots = kWin + 64;             // width-sorted keys padded to whole chunks
 constexpr int kMetaSlots = 6;                     // windows of record offsets fetched ahead
 constexpr int kMetaWords = kWin + 8;
 constexpr int kNewItem = 1, kLastSub = 2;         // stage flags
 constexpr uint32_t kReadEndFromMeta = 0xFFFFFFFFu;
 constexpr uint32_t kValid = 0x80000000u;
+constexpr float kLazy = 8.f;                      // running-max slack, log2 units
+constexpr float kMInit = -1e30f;                  // running max before the first key
+constexpr int kPlanThreads = 256;
 
-// q'_b[k] = q[k] * 2^(60 - pos_b(k)); the code field of channel k sits at pos_b(k) after
-// unpack: b = 2 -> 2*(k % 8), b = 4 -> 4*(k % 4), b = 8 -> 0. Dot products over codes
-// come out scaled by 2^(60 - 149) = 2^-89; over native fp16 values by 2^60.
-constexpr float kQScale = 1152921504606846976.0f;      // 2^60
-constexpr float kDotCodeUnscale = 618970019642690137449562112.0f;  // 2^89
-constexpr float kDotNativeUnscale = 8.673617379884035e-19f;        // 2^-60
+// q' = q * 2^60. A code field at bit position pos is c * 2^(pos - 149), so q' * field =
+// q * c * 2^(pos - 89): per-position sums are unscaled by 2^(89 - pos). Native fp16 values
+// give q * x * 2^60.
+constexpr float kQScale = 1152921504606846976.0f;                   // 2^60
+constexpr float kDotCodeUnscale = 618970019642690137449562112.0f;   // 2^89
+constexpr float kDotNativeUnscale = 8.673617379884035e-19f;         // 2^-60
 // V weights: w' = p * s * 2^(100 - pos); accumulators hold o * 2^-49.
-constexpr float kWScale = 1267650600228229401496703205376.0f;      // 2^100
-constexpr float kONativeScale = 1.7763568394002505e-15f;           // 2^-49
-constexpr float kOUnscale = 562949953421312.0f;                    // 2^49
+constexpr float kWScale = 1267650600228229401496703205376.0f;       // 2^100
+constexpr float kONativeScale = 1.7763568394002505e-15f;            // 2^-49
+constexpr float kOUnscale = 562949953421312.0f;                     // 2^49
+
+template <int D>
+struct Geo {
+    static constexpr int LPK = D / 32;             // lanes per key, 32 channels per lane
+    static constexpr int KPS = 32 / LPK;           // keys per warp step (chunk)
+};
+
+struct AppendArgs {
+    const __half *k, *v;
+    const uint8_t *bits;
+    const int32_t *cu, *positions;
+    int64_t n_tok;
+    uint32_t gen;
+};
 
 template <int D>
 struct Stage {
-    // width-sorted keys in class-pure chunks: kValid | (key << 16) | offset in rec;
+    // width-sorted keys in chunks of one width: kValid | (key << 16) | offset in rec;
     // padding entries are 0
     uint32_t perm[kPermSlots];
-    int32_t info[4];         // item index, keys in the stage, flags, chunks
+    int32_t info[8];         // item index, keys in the stage, flags, chunks, qinfo
     int32_t cls_chunk[8];    // first chunk of each width class (b = 2, 4, 8, 16), [4] = chunks
-    __half q[D];             // the item's query (copied with the item's first stage)
+    __half q[kDecodeMaxQ][D];  // the item's queries (copied with the item's first stage)
     float4 side[kWin];       // (s_K, z_K, s_V, z_V) per key, token order
     alignas(16) uint8_t rec[kStageRecBytes];
 };
@@ -79,7 +108,7 @@ struct alignas(16) MetaSlot {
     int32_t it, j, j1, ja;
     uint32_t end_off, first;
     int64_t sbase;
-    int32_t sh, pad;
+    int32_t sh, qinfo;
 };
 
 template <int D>
@@ -91,294 +120,374 @@ struct DecodeSmem {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t mfull[kMetaSlots];
+    int32_t abort_flag;
 };
 
 __device__ __forceinline__ float fld(uint32_t bits) { return __uint_as_float(bits); }
+__device__ __forceinline__ float2 fpair(uint32_t a, uint32_t b) { return make_float2(fld(a), fld(b)); }
+__device__ __forceinline__ float2 bcast(float a) { return make_float2(a, a); }
 
-__global__ void decode_sched_kernel(CacheView c, const uint8_t *__restrict__ modes, int w,
-                                    DecodeWork wk)
+// 2^x with the hardware's approximate exp2 (relative error of a few ulp; 2^-inf = 0,
+// results below 2^-126 flush to 0): the softmax weights.
+__device__ __forceinline__ float ex2(float x)
 {
-    __shared__ int warp_tot[32];
-    __shared__ int carry_sh;
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float h2f_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu))); }
+__device__ __forceinline__ float h2f_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
+
+// ------------------------------------------------------------------ planning
+// Appends the step's tokens of sequence blockIdx.x (APPEND), then lists the decode items of
+// its (KV head, subgroup) units.
+template <int D, bool APPEND>
+__global__ void __launch_bounds__(kPlanThreads)
+decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, DecodeWork wk, uint32_t gen,
+                   AppendArgs ap)
+{
+    __shared__ int bad_sh;
+    __shared__ int warp_tot[kPlanThreads / 32];
+    __shared__ int cnt_sh[kPlanThreads];
+    __shared__ uint32_t base_sh;
     pdl_wait();
     pdl_trigger();
-    const int HQ = c.H * c.G;                 // query heads; query head hq reads KV head hq / G
-    const int BH = c.B * HQ;
+    const int s = blockIdx.x;
+    if (APPEND) append_seq<D>(c, ap.k, ap.v, ap.bits, ap.cu, ap.n_tok, ap.gen, ap.positions, s, bad_sh);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    if (tid == 0) carry_sh = 0;
-    __syncthreads();
-    for (int base = 0; base < BH; base += blockDim.x) {
-        const int i = base + tid;
-        int cnt = 0, lo = 0, hi = 0, L = 0;
-        int64_t sb = 0;
-        uint32_t end_i = 0;
-        if (i < BH) {
-            // every load of this head up front: one round trip before the scan
-            const int s = i / HQ, h = (i % HQ) / c.G, shk = s * c.H + h;
-            const int m = modes[i];
-            L = c.len[shk];
-            end_i = c.end[shk];
-            sb = slot_of(c, s, h, 0);
-            if (m > KVQ_MODE_FULL) {
-                set_status(c.status, KVQ_ERR_MODE);
-            } else if (m != KVQ_MODE_SKIP && L > 0) {
-                hi = L;
-                lo = (m == KVQ_MODE_LOCAL) ? max(0, L - 1 - w) : 0;
-                cnt = (hi - lo + kDecodeItemKeys - 1) / kDecodeItemKeys;
+    const int H = c.H, G = c.G, HQ = H * G;
+    const int nsub = (G + kDecodeMaxQ - 1) / kDecodeMaxQ;
+    const int units = H * nsub;
+    const int per_pass = (kPlanThreads / nsub) * nsub;      // whole KV heads per pass
+    for (int u0 = 0; u0 < units; u0 += per_pass) {
+        const int u = u0 + tid;
+        const bool mine = tid < per_pass && u < units;
+        int L = 0, lo_loc = 0, nA = 0, nB = 0, mA = 0, mB = 0, g0 = 0, hk = 0;
+        if (mine) {
+            hk = u / nsub;
+            g0 = (u % nsub) * kDecodeMaxQ;
+            L = c.len[s * H + hk];
+            lo_loc = max(0, L - 1 - w);
+            int full = 0, local = 0;
+            for (int i = 0; i < kDecodeMaxQ && g0 + i < G; ++i) {
+                const int m = modes[(int64_t)s * HQ + hk * G + g0 + i];
+                if (m > KVQ_MODE_FULL) set_status(c.status, KVQ_ERR_MODE);
+                else if (m == KVQ_MODE_FULL) full |= 1 << i;
+                else if (m == KVQ_MODE_LOCAL) local |= 1 << i;
+            }
+            if (L > 0) {
+                if (local == 0 || full == 0) {       // one region: the mode set is the same throughout
+                    mB = full | local;
+                    nB = mB ? (local ? L - lo_loc : L) : 0;
+                } else {                             // full queries alone before the window
+                    mA = full;
+                    nA = lo_loc;
+                    mB = full | local;
+                    nB = L - lo_loc;
+                }
             }
         }
+        const int cA = (nA + kDecodeItemKeys - 1) / kDecodeItemKeys;
+        const int cB = (nB + kDecodeItemKeys - 1) / kDecodeItemKeys;
+        const int cnt = cA + cB;
+        cnt_sh[tid] = cnt;
         int incl = cnt;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            int y = __shfl_up_sync(0xffffffffu, incl, d);
+            const int y = __shfl_up_sync(0xffffffffu, incl, d);
             if (lane >= d) incl += y;
         }
         if (lane == 31) warp_tot[wid] = incl;
         __syncthreads();
-        if (wid == 0) {
-            int t = (lane < (int)(blockDim.x >> 5)) ? warp_tot[lane] : 0;
+        int wpre = 0, tot = 0;
 #pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                int y = __shfl_up_sync(0xffffffffu, t, d);
-                if (lane >= d) t += y;
+        for (int qq = 0; qq < kPlanThreads / 32; ++qq) {
+            const int t = warp_tot[qq];
+            if (qq < wid) wpre += t;
+            tot += t;
+        }
+        if (tid == 0) {
+            // reserve [base, base + tot) in this call's list; the first CTA of a call to
+            // arrive resets the count left by the previous call
+            unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(wk.count), nw;
+            uint32_t base;
+            while (true) {
+                if ((uint32_t)(old >> 32) != gen) {
+                    base = 0;
+                    nw = ((unsigned long long)gen << 32) | (unsigned long long)tot;
+                } else {
+                    base = (uint32_t)old;
+                    nw = old + (unsigned long long)tot;
+                }
+                const unsigned long long prev = atomicCAS(wk.count, old, nw);
+                if (prev == old) break;
+                old = prev;
             }
-            warp_tot[lane] = t;   // inclusive over warps
+            base_sh = base;
         }
         __syncthreads();
-        const int carry = carry_sh;
-        const int first = carry + (wid > 0 ? warp_tot[wid - 1] : 0) + incl - cnt;
-        if (i < BH) {
-            wk.head_first[i] = first;
-            wk.head_cnt[i] = cnt;
-            if (cnt > 0) {
-                const int n = hi - lo, per = n / cnt, rem = n % cnt;
-                int j0 = lo;
-                for (int k = 0; k < cnt; ++k) {               // near-equal, non-empty items
-                    DecodeItem it;
-                    it.sh = i;
-                    it.j0 = j0;
-                    it.j1 = j0 + per + (k < rem ? 1 : 0);
-                    j0 = it.j1;
-                    // the stream end for the item ending at the last token; else the
-                    // producer reads the offset of key j1 itself
-                    it.end_off = (it.j1 < L) ? kReadEndFromMeta : end_i;
-                    it.sbase = sb;
-                    wk.items[first + k] = it;
+        const int64_t first = (int64_t)base_sh + wpre + incl - cnt;
+        if (mine) {
+            if (u % nsub == 0) {                     // the KV head's items: its subgroups' runs
+                int n_all = 0;
+                for (int k = 0; k < nsub; ++k) n_all += cnt_sh[tid + k];
+                wk.head_first[s * H + hk] = (int32_t)first;
+                wk.head_cnt[s * H + hk] = n_all;
+            }
+            if (first + cnt > wk.max_items) {
+                set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+            } else if (cnt > 0) {
+                const int64_t sbase = slot_of(c, s, hk, 0);
+                const uint32_t end_s = c.end[s * H + hk];
+                int64_t it = first;
+                for (int r = 0; r < 2; ++r) {
+                    const int n = r ? nB : nA, ci = r ? cB : cA;
+                    const int lo = r ? L - nB : 0;
+                    const int msk = r ? mB : mA;
+                    if (ci == 0) continue;
+                    const int per = n / ci, rem = n % ci;
+                    int j0 = lo;
+                    for (int k = 0; k < ci; ++k) {       // near-equal, non-empty items
+                        DecodeItem d;
+                        d.sh = s * H + hk;
+                        d.j0 = j0;
+                        d.j1 = j0 + per + (k < rem ? 1 : 0);
+                        j0 = d.j1;
+                        // the stream end for the item ending at the last token; else the
+                        // producer reads the offset of key j1 itself
+                        d.end_off = (d.j1 < L) ? kReadEndFromMeta : end_s;
+                        d.sbase = sbase;
+                        d.qinfo = g0 | (msk << 8);
+                        d.pad = 0;
+                        wk.items[it++] = d;
+                    }
                 }
             }
         }
-        __syncthreads();
-        if (tid == 0) carry_sh = carry + warp_tot[(blockDim.x >> 5) - 1];
-        __syncthreads();
+        __syncthreads();                             // cnt_sh / warp_tot reused by the next pass
     }
-    if (tid == 0) *wk.count = carry_sh;
 }
 
-// ---- per-width dot products and accumulations for one lane's 16 channels ----------
-// Channels c and c + 8 of the lane travel as one float2, so every FMA is a packed FFMA2
-// (two fp32 FMAs, each with the rounding of fmaf, subnormal operands kept).
+// ------------------------------------------------------------------ per-width lane math
+// A lane holds 32 channels (c0 .. c0 + 31) of one key; its share of a record part is 4*b
+// bytes starting at byte 4*b*li. Pairs (k, k + 16) of the lane's channels share a float2.
 struct QRegs {
-    float2 q2[8], q4[8], q8[8];   // (q[j], q[j + 8]) * 2^(60 - pos_b)
+    float2 q[16];            // (q[k], q[k + 16]) * 2^60
 };
 
-__device__ __forceinline__ float2 fpair(uint32_t a, uint32_t b) { return make_float2(fld(a), fld(b)); }
-__device__ __forceinline__ float2 bcast(float a) { return make_float2(a, a); }
-
-__device__ __forceinline__ float dot_codes2(const QRegs &q, uint32_t x)
+// Lane partial of q . c (scaled as described above), by width class.
+template <int CLS>
+__device__ __forceinline__ float lane_dot(const QRegs &Q, const uint8_t *p)
 {
-    const uint32_t y = x >> 16;                 // channels 8..15
-    float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    if (CLS == 0) {                                   // 2-bit: 2 words, 8 positions per half
+        const uint2 x = *reinterpret_cast<const uint2 *>(p);
+        const uint32_t y0 = x.x >> 16, y1 = x.y >> 16;
+        float2 a[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const uint32_t m = 3u << (2 * k);
-        a[k & 1] = __ffma2_rn(q.q2[k], fpair(x & m, y & m), a[k & 1]);
-    }
-    return (a[0].x + a[1].x) + (a[0].y + a[1].y);
-}
-
-__device__ __forceinline__ float dot_codes4(const QRegs &q, uint2 x)
-{
-    const uint32_t lo0 = x.x, hi0 = x.x >> 16, lo1 = x.y, hi1 = x.y >> 16;
-    float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t m = 3u << (2 * j);
+            a[j] = __fmul2_rn(Q.q[j], fpair(x.x & m, x.y & m));
+            a[j] = __ffma2_rn(Q.q[8 + j], fpair(y0 & m, y1 & m), a[j]);
+        }
+        float r = a[7].x + a[7].y;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint32_t m = 15u << (4 * k);
-        a[0] = __ffma2_rn(q.q4[k], fpair(lo0 & m, lo1 & m), a[0]);          // channels k, 8 + k
-        a[1] = __ffma2_rn(q.q4[4 + k], fpair(hi0 & m, hi1 & m), a[1]);      // 4 + k, 12 + k
-    }
-    return (a[0].x + a[1].x) + (a[0].y + a[1].y);
-}
-
-__device__ __forceinline__ float dot_codes8(const QRegs &q, uint4 x)
-{
-    float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        for (int j = 6; j >= 0; --j) r = fmaf(r, 0.25f, a[j].x + a[j].y);   // sum_j 2^(-2j) a_j
+        return r;
+    } else if (CLS == 1) {                            // 4-bit: 4 words, 4 positions per half
+        const uint4 x = *reinterpret_cast<const uint4 *>(p);
+        const uint32_t h0 = x.x >> 16, h1 = x.y >> 16, h2 = x.z >> 16, h3 = x.w >> 16;
+        float2 a[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const uint32_t sel = 0x4440 + e;
-        a[0] = __ffma2_rn(q.q8[e], fpair(__byte_perm(x.x, 0u, sel), __byte_perm(x.z, 0u, sel)), a[0]);
-        a[1] = __ffma2_rn(q.q8[4 + e], fpair(__byte_perm(x.y, 0u, sel), __byte_perm(x.w, 0u, sel)), a[1]);
-    }
-    return (a[0].x + a[1].x) + (a[0].y + a[1].y);
-}
-
-__device__ __forceinline__ float dot_native(const QRegs &q, uint4 x0, uint4 x1)
-{
-    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t m = 15u << (4 * j);
+            a[j] = __fmul2_rn(Q.q[j], fpair(x.x & m, x.z & m));
+            a[j] = __ffma2_rn(Q.q[4 + j], fpair(h0 & m, h2 & m), a[j]);
+            a[j] = __ffma2_rn(Q.q[8 + j], fpair(x.y & m, x.w & m), a[j]);
+            a[j] = __ffma2_rn(Q.q[12 + j], fpair(h1 & m, h3 & m), a[j]);
+        }
+        float r = a[3].x + a[3].y;
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {               // word h: channels 2h, 2h + 1; word h + 4: + 8
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
-        const float2 g = __half22float2(*reinterpret_cast<const __half2 *>(&w[h + 4]));
-        a[0] = __ffma2_rn(q.q8[2 * h], make_float2(f.x, g.x), a[0]);
-        a[1] = __ffma2_rn(q.q8[2 * h + 1], make_float2(f.y, g.y), a[1]);
-    }
-    return (a[0].x + a[1].x) + (a[0].y + a[1].y);
-}
-
-__device__ __forceinline__ void acc_codes2(float2 (&o)[8], float wv, uint32_t x)
-{
-    const uint32_t y = x >> 16;
+        for (int j = 2; j >= 0; --j) r = fmaf(r, 0.0625f, a[j].x + a[j].y);
+        return r;
+    } else if (CLS == 2) {                            // 8-bit: 8 words, bytes moved to position 0
+        const uint4 x0 = reinterpret_cast<const uint4 *>(p)[0];
+        const uint4 x1 = reinterpret_cast<const uint4 *>(p)[1];
+        const uint32_t wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float wk = wv * __uint_as_float((127u - 2u * k) << 23);   // wv * 2^-2k
-        const uint32_t m = 3u << (2 * k);
-        o[k] = __ffma2_rn(bcast(wk), fpair(x & m, y & m), o[k]);
-    }
-}
-
-__device__ __forceinline__ void acc_codes4(float2 (&o)[8], float wv, uint2 x)
-{
-    const uint32_t hi0 = x.x >> 16, hi1 = x.y >> 16;
+        for (int i = 0; i < 4; ++i) {                 // word i: channels 4i..4i+3; word i+4: +16
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float2 wk = bcast(wv * __uint_as_float((127u - 4u * k) << 23));   // wv * 2^-4k
-        const uint32_t m = 15u << (4 * k);
-        o[k] = __ffma2_rn(wk, fpair(x.x & m, x.y & m), o[k]);
-        o[4 + k] = __ffma2_rn(wk, fpair(hi0 & m, hi1 & m), o[4 + k]);
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t sel = 0x4440 + e;
+                a[e & 1] = __ffma2_rn(Q.q[4 * i + e], fpair(__byte_perm(wv[i], 0u, sel), __byte_perm(wv[i + 4], 0u, sel)),
+                                      a[e & 1]);
+            }
+        }
+        return (a[0].x + a[1].x) + (a[0].y + a[1].y);
+    } else {                                          // 16-bit: 16 words of fp16 pairs
+        uint32_t wv[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 x = reinterpret_cast<const uint4 *>(p)[i];
+            wv[4 * i] = x.x;
+            wv[4 * i + 1] = x.y;
+            wv[4 * i + 2] = x.z;
+            wv[4 * i + 3] = x.w;
+        }
+        float2 a[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {                 // word i: channels 2i, 2i+1; word i+8: +16
+            a[0] = __ffma2_rn(Q.q[2 * i], make_float2(h2f_lo(wv[i]), h2f_lo(wv[i + 8])), a[0]);
+            a[1] = __ffma2_rn(Q.q[2 * i + 1], make_float2(h2f_hi(wv[i]), h2f_hi(wv[i + 8])), a[1]);
+        }
+        return (a[0].x + a[1].x) + (a[0].y + a[1].y);
     }
 }
 
-__device__ __forceinline__ void acc_codes8(float2 (&o)[8], float wv, uint4 x)
+// o[k] += weight * (c_k, c_{k+16}) for the lane's 32 V values of width class CLS.
+template <int CLS>
+__device__ __forceinline__ void lane_acc(float2 (&o)[16], float wv, const uint8_t *p)
 {
-    const float2 w2 = bcast(wv);
+    if (CLS == 0) {
+        const uint2 x = *reinterpret_cast<const uint2 *>(p);
+        const uint32_t y0 = x.x >> 16, y1 = x.y >> 16;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const uint32_t sel = 0x4440 + e;
-        o[e] = __ffma2_rn(w2, fpair(__byte_perm(x.x, 0u, sel), __byte_perm(x.z, 0u, sel)), o[e]);
-        o[4 + e] = __ffma2_rn(w2, fpair(__byte_perm(x.y, 0u, sel), __byte_perm(x.w, 0u, sel)), o[4 + e]);
-    }
-}
-
-__device__ __forceinline__ void acc_native(float2 (&o)[8], float wv, uint4 x0, uint4 x1)
-{
-    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    const float2 w2 = bcast(wv);
+        for (int j = 0; j < 8; ++j) {
+            const float2 wj = bcast(wv * __uint_as_float((127u - 2u * j) << 23));   // wv * 2^-2j
+            const uint32_t m = 3u << (2 * j);
+            o[j] = __ffma2_rn(wj, fpair(x.x & m, x.y & m), o[j]);
+            o[8 + j] = __ffma2_rn(wj, fpair(y0 & m, y1 & m), o[8 + j]);
+        }
+    } else if (CLS == 1) {
+        const uint4 x = *reinterpret_cast<const uint4 *>(p);
+        const uint32_t h0 = x.x >> 16, h1 = x.y >> 16, h2 = x.z >> 16, h3 = x.w >> 16;
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
-        const float2 g = __half22float2(*reinterpret_cast<const __half2 *>(&w[h + 4]));
-        o[2 * h] = __ffma2_rn(w2, make_float2(f.x, g.x), o[2 * h]);
-        o[2 * h + 1] = __ffma2_rn(w2, make_float2(f.y, g.y), o[2 * h + 1]);
-    }
-}
-
-// merge the online-softmax state (m, l, pz, o) of this lane with the lane `mask` away
-__device__ __forceinline__ void merge_state(float &m, float &l, float &pz, float2 (&o)[8], int mask)
-{
-    const float mp = __shfl_xor_sync(0xffffffffu, m, mask);
-    const float lp = __shfl_xor_sync(0xffffffffu, l, mask);
-    const float zp = __shfl_xor_sync(0xffffffffu, pz, mask);
-    const float M = fmaxf(m, mp);
-    const float fa = (m == -INFINITY) ? 0.f : exp2f(m - M);
-    const float fb = (mp == -INFINITY) ? 0.f : exp2f(mp - M);
+        for (int j = 0; j < 4; ++j) {
+            const float2 wj = bcast(wv * __uint_as_float((127u - 4u * j) << 23));   // wv * 2^-4j
+            const uint32_t m = 15u << (4 * j);
+            o[j] = __ffma2_rn(wj, fpair(x.x & m, x.z & m), o[j]);
+            o[4 + j] = __ffma2_rn(wj, fpair(h0 & m, h2 & m), o[4 + j]);
+            o[8 + j] = __ffma2_rn(wj, fpair(x.y & m, x.w & m), o[8 + j]);
+            o[12 + j] = __ffma2_rn(wj, fpair(h1 & m, h3 & m), o[12 + j]);
+        }
+    } else if (CLS == 2) {
+        const uint4 x0 = reinterpret_cast<const uint4 *>(p)[0];
+        const uint4 x1 = reinterpret_cast<const uint4 *>(p)[1];
+        const uint32_t wd[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        const float2 w2 = bcast(wv);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float2 op = make_float2(__shfl_xor_sync(0xffffffffu, o[k].x, mask),
-                                      __shfl_xor_sync(0xffffffffu, o[k].y, mask));
-        o[k] = __ffma2_rn(op, bcast(fb), __fmul2_rn(o[k], bcast(fa)));
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t sel = 0x4440 + e;
+                o[4 * i + e] = __ffma2_rn(w2, fpair(__byte_perm(wd[i], 0u, sel), __byte_perm(wd[i + 4], 0u, sel)),
+                                          o[4 * i + e]);
+            }
+        }
+    } else {
+        uint32_t wd[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 x = reinterpret_cast<const uint4 *>(p)[i];
+            wd[4 * i] = x.x;
+            wd[4 * i + 1] = x.y;
+            wd[4 * i + 2] = x.z;
+            wd[4 * i + 3] = x.w;
+        }
+        const float2 w2 = bcast(wv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            o[2 * i] = __ffma2_rn(w2, make_float2(h2f_lo(wd[i]), h2f_lo(wd[i + 8])), o[2 * i]);
+            o[2 * i + 1] = __ffma2_rn(w2, make_float2(h2f_hi(wd[i]), h2f_hi(wd[i + 8])), o[2 * i + 1]);
+        }
     }
-    l = l * fa + lp * fb;
-    pz = pz * fa + zp * fb;
-    m = M;
 }
 
 struct KeyState {
     float m, l, pz;
-    float2 o[8];      // (o[j], o[j + 8]) of the lane's 16 channels
+    float2 o[16];      // (o[c0 + k], o[c0 + k + 16]) of the lane's 32 channels
 };
 
-// One key per 8-lane group (16 lanes x 4 groups for head_dim 64: 4 lanes x 8 groups), all
-// of width class CLS (warp-uniform): K dot product on the codes, logit, online-softmax
-// update of the group's state, V accumulation. Lanes of invalid entries only take part in
-// the shuffles.
-template <int D, int CLS>
-__device__ __forceinline__ void process_key(KeyState &st, const QRegs &qr, float qsum, float qk_scale,
-                                            const Stage<D> &sg, uint32_t ent, int gl)
+// merge the online-softmax state of this lane with the lane `mask` away
+__device__ __forceinline__ void merge_state(KeyState &st, int mask)
 {
-    constexpr int GROUP = D / 16;
-    const bool valid = (ent & kValid) != 0;
-    const uint8_t *r = sg.rec + (ent & 0x7FFFu);
-    float part = 0.f;
-    if (valid) {
-        if (CLS == 0) part = dot_codes2(qr, reinterpret_cast<const uint32_t *>(r)[gl]);
-        else if (CLS == 1) part = dot_codes4(qr, reinterpret_cast<const uint2 *>(r)[gl]);
-        else if (CLS == 2) part = dot_codes8(qr, reinterpret_cast<const uint4 *>(r)[gl]);
-        else part = dot_native(qr, reinterpret_cast<const uint4 *>(r)[2 * gl],
-                               reinterpret_cast<const uint4 *>(r)[2 * gl + 1]);
-    }
+    const float mp = __shfl_xor_sync(0xffffffffu, st.m, mask);
+    const float lp = __shfl_xor_sync(0xffffffffu, st.l, mask);
+    const float zp = __shfl_xor_sync(0xffffffffu, st.pz, mask);
+    const float M = fmaxf(st.m, mp);
+    const float fa = ex2(st.m - M), fb = ex2(mp - M);
 #pragma unroll
-    for (int d = 1; d < GROUP; d <<= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
-    if (!valid) return;
+    for (int k = 0; k < 16; ++k) {
+        const float2 op = make_float2(__shfl_xor_sync(0xffffffffu, st.o[k].x, mask),
+                                      __shfl_xor_sync(0xffffffffu, st.o[k].y, mask));
+        st.o[k] = __ffma2_rn(op, bcast(fb), __fmul2_rn(st.o[k], bcast(fa)));
+    }
+    st.l = st.l * fa + lp * fb;
+    st.pz = st.pz * fa + zp * fb;
+    st.m = M;
+}
+
+// One chunk: a key per LPK-lane group, all of width class CLS (warp-uniform): K dot product
+// on the codes, logit, online-softmax update of the group's state, V accumulation.
+// Padding entries (no valid bit) read the stage's first bytes and get weight 0.
+template <int D, int CLS>
+__device__ __forceinline__ void process_chunk(KeyState &st, const QRegs &Q, float qsum_l, float cdot,
+                                              const Stage<D> &sg, uint32_t ent, int li)
+{
+    constexpr int LPK = Geo<D>::LPK;
+    constexpr int BITS = 2 << CLS;
+    const uint8_t *r = sg.rec + (ent & 0x7FFFu);
+    float part = lane_dot<CLS>(Q, r + 4 * BITS * li);
+#pragma unroll
+    for (int d = 1; d < LPK; d <<= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
     const float4 sd = sg.side[(ent >> 16) & 127u];
-    const float dot = (CLS == 3) ? part * kDotNativeUnscale : fmaf(sd.x, part * kDotCodeUnscale, sd.y * qsum);
-    const float lg = dot * qk_scale;
-    if (lg > st.m) {                          // new running max of this key group
-        const float corr = exp2f(st.m - lg);
+    float lg = (CLS == 3) ? part * cdot : fmaf(sd.x * cdot, part, sd.y * qsum_l);
+    lg = (ent & kValid) ? lg : -INFINITY;
+    if (__any_sync(0xffffffffu, lg > st.m + kLazy)) {      // rare after an item's first keys
+        const float m_new = (lg > st.m + kLazy) ? lg : st.m;
+        const float corr = ex2(st.m - m_new);
         st.l *= corr;
         st.pz *= corr;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) st.o[k] = __fmul2_rn(st.o[k], bcast(corr));
-        st.m = lg;
+        for (int k = 0; k < 16; ++k) st.o[k] = __fmul2_rn(st.o[k], bcast(corr));
+        st.m = m_new;
     }
-    const float p = exp2f(lg - st.m);
+    const float p = ex2(lg - st.m);
     st.l += p;
-    const uint8_t *rv = r + (D * (2 << CLS)) / 8;
+    const uint8_t *rv = r + (D * BITS) / 8 + 4 * BITS * li;
     if (CLS == 3) {
-        acc_native(st.o, p * kONativeScale, reinterpret_cast<const uint4 *>(rv)[2 * gl],
-                   reinterpret_cast<const uint4 *>(rv)[2 * gl + 1]);
+        lane_acc<3>(st.o, p * kONativeScale, rv);
     } else {
         st.pz = fmaf(p, sd.w, st.pz);
-        const float wv = p * sd.z * kWScale;
-        if (CLS == 0) acc_codes2(st.o, wv, reinterpret_cast<const uint32_t *>(rv)[gl]);
-        else if (CLS == 1) acc_codes4(st.o, wv, reinterpret_cast<const uint2 *>(rv)[gl]);
-        else acc_codes8(st.o, wv, reinterpret_cast<const uint4 *>(rv)[gl]);
+        lane_acc<CLS>(st.o, p * (sd.z * kWScale), rv);
     }
 }
 
-// This warp's chunks ch, ch + kConsumerWarps, ... below `end`, all of width class CLS.
+// This warp's chunks ch, ch + step, ... below `end`, all of width class CLS.
 template <int D, int CLS>
-__device__ __forceinline__ int run_class(KeyState &st, const QRegs &qr, float qsum, float qk_scale,
-                                         const Stage<D> &sg, int ch, int end, int g, int gl)
+__device__ __forceinline__ int run_class(KeyState &st, const QRegs &Q, float qsum_l, float cdot,
+                                         const Stage<D> &sg, int ch, int end, int step, int g, int li)
 {
-    constexpr int KEYS_PER_STEP = 32 / (D / 16);
-    for (; ch < end; ch += kConsumerWarps)
-        process_key<D, CLS>(st, qr, qsum, qk_scale, sg, sg.perm[KEYS_PER_STEP * ch + g], gl);
+    constexpr int KPS = Geo<D>::KPS;
+    for (; ch < end; ch += step) process_chunk<D, CLS>(st, Q, qsum_l, cdot, sg, sg.perm[KPS * ch + g], li);
     return ch;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
 {
-    constexpr int GROUP = D / 16;                 // lanes per key (16 channels per lane)
-    constexpr int KEYS_PER_STEP = 32 / GROUP;     // keys per chunk step of a warp
+    constexpr int LPK = Geo<D>::LPK;
+    constexpr int KPS = Geo<D>::KPS;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     DecodeSmem<D> &sm = *reinterpret_cast<DecodeSmem<D> *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait();
     pdl_trigger();
-    const int n_items = *wk.count;
+    const int n_items = (int)min((int64_t)(uint32_t)(*wk.count), wk.max_items);
+    const int HQ = c.H * c.G;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -386,6 +495,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
             mbar_init(&sm.empty[i], kConsumerWarps);
         }
         for (int i = 0; i < kMetaSlots; ++i) mbar_init(&sm.mfull[i], 1);
+        sm.abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
@@ -395,17 +505,17 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         // A filler cursor runs up to kMetaSlots windows ahead and bulk-copies each window of
         // 128 record offsets into a shared ring; the record cursor reads a window from shared
         // memory, cuts it into stages of at most kStageRecBytes, sorts each stage's keys by
-        // width and issues the stage's copies.
+        // width and issues the stage's copies. On a timed-out wait it stops issuing, waits
+        // (bounded) for the copies already in flight and returns.
         constexpr int KPL = kWin / 32;                // window keys per lane: lane + 32 r
         int f_it = blockIdx.x;
         if (f_it >= n_items) return;
         DecodeItem f_d = wk.items[f_it];
         int f_j = f_d.j0;
-        bool f_valid = true;
-        int filled = 0, consumed = 0, stage = 0;
-        uint32_t phase = 0;
+        bool f_valid = true, aborted = false;
+        int filled = 0, consumed = 0, issued = 0;
         const uint32_t lt = (1u << lane) - 1u;
-        while (true) {
+        while (!aborted) {
             while (f_valid && filled < consumed + kMetaSlots) {
                 const int slot = filled % kMetaSlots;
                 MetaSlot &ms = sm.ms[slot];
@@ -420,6 +530,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     ms.first = (f_j == f_d.j0);
                     ms.sbase = f_d.sbase;
                     ms.sh = f_d.sh;
+                    ms.qinfo = f_d.qinfo;
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     mbar_arrive_expect_tx(&sm.mfull[slot], 4u * (uint32_t)(jb - ja));
                     bulk_g2s(ms.meta, c.meta + f_d.sbase + ja, 4u * (uint32_t)(jb - ja), &sm.mfull[slot]);
@@ -438,9 +549,12 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
             }
             if (consumed == filled) break;
             const int slot = consumed % kMetaSlots;
-            if (!mbar_wait(&sm.mfull[slot], (uint32_t)(consumed / kMetaSlots) & 1u, c.status)) return;
+            if (!mbar_wait(&sm.mfull[slot], (uint32_t)(consumed / kMetaSlots) & 1u, c.status)) {
+                aborted = true;
+                break;
+            }
             const MetaSlot &ms = sm.ms[slot];
-            const int j = ms.j, it = ms.it;
+            const int j = ms.j, it = ms.it, qinfo = ms.qinfo;
             const int nwin = min(kWin, ms.j1 - j);
             const bool lastwin = (j + nwin == ms.j1), first = ms.first != 0;
             const uint32_t *mw = ms.meta + (j - ms.ja);
@@ -486,8 +600,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
                     rec_bytes = 0;
                 }
-                // counting sort by width, each width's run padded to whole chunks of KEYS_PER_STEP
-                constexpr int PADL = KEYS_PER_STEP - 1;       // pad entries per width, at most
+                // counting sort by width, each width's run padded to whole chunks of KPS keys
                 int cl_of[KPL], pos_of[KPL];
 #pragma unroll
                 for (int r = 0; r < KPL; ++r) {
@@ -495,10 +608,10 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     cl_of[r] = (k >= w0 && k < w1) ? (int)(m[r] & 3u) : 4;
                     pos_of[r] = 0;
                 }
-                int pstart = 0, pad_pos = -1, cls_chunk[4];
+                int pstart = 0, cls_chunk[4], pad_at[4], pad_n[4];
 #pragma unroll
                 for (int cl = 0; cl < 4; ++cl) {
-                    cls_chunk[cl] = pstart / KEYS_PER_STEP;
+                    cls_chunk[cl] = pstart / KPS;
                     int before = 0;
 #pragma unroll
                     for (int r = 0; r < KPL; ++r) {
@@ -506,13 +619,18 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                         if (cl_of[r] == cl) pos_of[r] = pstart + before + __popc(b & lt);
                         before += __popc(b);
                     }
-                    const int padded = (before + PADL) / KEYS_PER_STEP * KEYS_PER_STEP;
-                    if (lane / PADL == cl && before + lane % PADL < padded)     // PADL lanes per width
-                        pad_pos = pstart + before + lane % PADL;
+                    const int padded = (before + KPS - 1) / KPS * KPS;
+                    pad_at[cl] = pstart + before;
+                    pad_n[cl] = padded - before;
                     pstart += padded;
                 }
 
-                if (!mbar_wait(&sm.empty[stage], phase ^ 1u, c.status)) return;
+                const int stage = issued % kStages;
+                const uint32_t phase = (uint32_t)(issued / kStages) & 1u;
+                if (!mbar_wait(&sm.empty[stage], phase ^ 1u, c.status)) {
+                    aborted = true;
+                    break;
+                }
                 Stage<D> &sg = sm.st[stage];
 #pragma unroll
                 for (int r = 0; r < KPL; ++r) {
@@ -524,94 +642,126 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                         sg.perm[pos_of[r]] = kValid | ((uint32_t)(lane + 32 * r - w0) << 16) | ro;
                     }
                 }
-                if (pad_pos >= 0) sg.perm[pad_pos] = 0u;
+#pragma unroll
+                for (int cl = 0; cl < 4; ++cl)
+                    if (lane < pad_n[cl]) sg.perm[pad_at[cl] + lane] = 0u;
                 if (lane == 0) {
                     sg.info[0] = it;
                     sg.info[1] = n;
                     sg.info[2] = (new_item ? kNewItem : 0) | (last ? kLastSub : 0);
-                    sg.info[3] = pstart / KEYS_PER_STEP;
+                    sg.info[3] = pstart / KPS;
+                    sg.info[4] = qinfo;
 #pragma unroll
                     for (int cl = 0; cl < 4; ++cl) sg.cls_chunk[cl] = cls_chunk[cl];
-                    sg.cls_chunk[4] = pstart / KEYS_PER_STEP;
+                    sg.cls_chunk[4] = pstart / KPS;
                 }
                 __syncwarp();
                 if (lane == 0) {
-                    const uint32_t q_bytes = new_item ? 2u * D : 0u;
+                    // the item's subgroup of queries: rows (s, hk * G + g0 ..) of q, contiguous
+                    const int g0 = qinfo & 0xFF;
+                    const int nq = min(kDecodeMaxQ, c.G - g0);
+                    const uint32_t q_bytes = new_item ? (uint32_t)(2 * D * nq) : 0u;
+                    const int s_of = sh / c.H, hk = sh % c.H;
                     mbar_arrive_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
                     bulk_g2s(sg.side, c.side + sbase + j + w0, 16u * n, &sm.full[stage]);
                     if (rec_bytes)
                         bulk_g2s(sg.rec, c.rec + sbase * (int64_t)(4 * D) + off0, rec_bytes, &sm.full[stage]);
-                    if (q_bytes) bulk_g2s(sg.q, q + (int64_t)sh * D, q_bytes, &sm.full[stage]);
+                    if (q_bytes)
+                        bulk_g2s(sg.q, q + ((int64_t)s_of * HQ + hk * c.G + g0) * D, q_bytes, &sm.full[stage]);
                 }
-                if (++stage == kStages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                ++issued;
                 w0 = w1;
             }
+        }
+        if (aborted) {
+            // no copy may still be writing this CTA's shared memory when it exits: wait
+            // (bounded) for the last copy issued into each stage and each offset window
+            sm.abort_flag = 1;
+            for (int b = 0; b < kStages; ++b)
+                if (issued > b) {
+                    const int i_last = b + kStages * ((issued - 1 - b) / kStages);
+                    mbar_wait(&sm.full[b], (uint32_t)(i_last / kStages) & 1u, c.status, 100000000ull);
+                }
+            for (int b = 0; b < kMetaSlots; ++b)
+                if (filled > b) {
+                    const int i_last = b + kMetaSlots * ((filled - 1 - b) / kMetaSlots);
+                    mbar_wait(&sm.mfull[b], (uint32_t)(i_last / kMetaSlots) & 1u, c.status, 100000000ull);
+                }
         }
         return;
     }
 
     // -------------------------------- consumers -------------------------------------
-    const int g = lane / GROUP;          // key slot within a chunk step
-    const int gl = lane % GROUP;         // channel block: channels [16 gl, 16 gl + 16)
+    // Every consumer warp takes part in every item's merge (two named barriers per item),
+    // also after a timed-out wait: a warp that gave up only skips the waits and the work.
+    const int g = lane / LPK;            // key slot within a chunk
+    const int li = lane % LPK;           // channel block: channels [32 li, 32 li + 32)
     const float qk_scale = kLog2e * rsqrtf((float)D);   // logits in log2 units
     int stage = 0, rot = 0;
     uint32_t phase = 0;
-    QRegs qr;
-    float qsum = 0.f;
+    bool dead = false;
+    QRegs Q;
+    float qsum_l = 0.f;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
         KeyState ks;
-        ks.m = -INFINITY;
+        ks.m = kMInit;
         ks.l = 0.f;
         ks.pz = 0.f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) ks.o[k] = make_float2(0.f, 0.f);
+        for (int k = 0; k < 16; ++k) ks.o[k] = make_float2(0.f, 0.f);
+        int nq = 1, slot = 0, rank = warp, nws = kConsumerWarps;
         bool last = false;
-        while (!last) {
-            if (!mbar_wait(&sm.full[stage], phase, c.status)) return;
+        while (!last && !dead) {
+            if (*reinterpret_cast<volatile int32_t *>(&sm.abort_flag) ||
+                !mbar_wait(&sm.full[stage], phase, c.status)) {
+                dead = true;
+                sm.abort_flag = 1;
+                break;
+            }
             Stage<D> &sg = sm.st[stage];
             const int flags = sg.info[2];
             last = (flags & kLastSub) != 0;
             if (flags & kNewItem) {
-                // query: this lane's 16 channels, scaled per width; sum(q) over all D
-                const uint4 a = reinterpret_cast<const uint4 *>(sg.q + 16 * gl)[0];
-                const uint4 bq = reinterpret_cast<const uint4 *>(sg.q + 16 * gl)[1];
-                const uint32_t hw[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
-                qsum = 0.f;
+                const int qmask = sg.info[4] >> 8;
+                nq = __popc(qmask);
+                const int sidx = warp % nq;        // the sidx-th active query of the item
+                rank = warp / nq;
+                nws = (kConsumerWarps - sidx + nq - 1) / nq;
+                int qi = 0;
+                for (int b = 0, seen = 0; b < kDecodeMaxQ; ++b)
+                    if ((qmask >> b) & 1) {
+                        if (seen == sidx) qi = b;
+                        ++seen;
+                    }
+                slot = qi;                         // the query's slot in the item's partials
+                // this lane's 32 channels of query g0 + qi, scaled; sum(q) over all D
+                const uint4 *src = reinterpret_cast<const uint4 *>(sg.q[qi] + 32 * li);
+                float qs = 0.f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hw[e]));
-                    const float fv[2] = {f.x, f.y};
+                for (int u = 0; u < 2; ++u) {
+                    const uint4 a = src[u], b = src[2 + u];     // channels 8u.., 16 + 8u..
+                    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int k = 2 * e + u;        // channel 16 gl + k -> pair k % 8, half k / 8
-                        qsum += fv[u];
-                        const float v8 = fv[u] * kQScale;
-                        const float v4 = v8 * __uint_as_float((127u - 4u * (k % 4)) << 23);
-                        const float v2 = v8 * __uint_as_float((127u - 2u * (k % 8)) << 23);
-                        if (k < 8) {
-                            qr.q8[k].x = v8;
-                            qr.q4[k].x = v4;
-                            qr.q2[k].x = v2;
-                        } else {
-                            qr.q8[k - 8].y = v8;
-                            qr.q4[k - 8].y = v4;
-                            qr.q2[k - 8].y = v2;
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 fa = __half22float2(*reinterpret_cast<const __half2 *>(&wa[e]));
+                        const float2 fb = __half22float2(*reinterpret_cast<const __half2 *>(&wb[e]));
+                        qs += (fa.x + fa.y) + (fb.x + fb.y);
+                        Q.q[8 * u + 2 * e] = make_float2(fa.x * kQScale, fb.x * kQScale);
+                        Q.q[8 * u + 2 * e + 1] = make_float2(fa.y * kQScale, fb.y * kQScale);
                     }
                 }
 #pragma unroll
-                for (int d = 1; d < GROUP; d <<= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, d);
+                for (int d = 1; d < LPK; d <<= 1) qs += __shfl_xor_sync(0xffffffffu, qs, d);
+                qsum_l = qs * qk_scale;
             }
-            // class-pure chunks, dealt to the warps round-robin (rotated every stage); the
-            // chunks are sorted by width, so the warp walks one run per width class
-            int ch = (warp + kConsumerWarps - rot) % kConsumerWarps;
-            ch = run_class<D, 0>(ks, qr, qsum, qk_scale, sg, ch, sg.cls_chunk[1], g, gl);
-            ch = run_class<D, 1>(ks, qr, qsum, qk_scale, sg, ch, sg.cls_chunk[2], g, gl);
-            ch = run_class<D, 2>(ks, qr, qsum, qk_scale, sg, ch, sg.cls_chunk[3], g, gl);
-            run_class<D, 3>(ks, qr, qsum, qk_scale, sg, ch, sg.cls_chunk[4], g, gl);
+            const float cdot = qk_scale * kDotCodeUnscale;
+            // chunks sorted by width: the warps of this query deal them round-robin
+            // (rotated every stage) and walk one run per width class
+            int ch = (rank + rot) % nws;
+            ch = run_class<D, 0>(ks, Q, qsum_l, cdot, sg, ch, sg.cls_chunk[1], nws, g, li);
+            ch = run_class<D, 1>(ks, Q, qsum_l, cdot, sg, ch, sg.cls_chunk[2], nws, g, li);
+            ch = run_class<D, 2>(ks, Q, qsum_l, cdot, sg, ch, sg.cls_chunk[3], nws, g, li);
+            run_class<D, 3>(ks, Q, qsum_l, qk_scale * kDotNativeUnscale, sg, ch, sg.cls_chunk[4], nws, g, li);
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);
             rot = (rot + 1) % kConsumerWarps;
@@ -621,39 +771,36 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
             }
         }
 
-        // merge the key groups of the warp, then the warps, into the item's partial
+        // merge the key groups of the warp, then the warps of each query, into the
+        // item's partials
 #pragma unroll
-        for (int mask = GROUP; mask < 32; mask <<= 1) merge_state(ks.m, ks.l, ks.pz, ks.o, mask);
+        for (int mask = LPK; mask < 32; mask <<= 1) merge_state(ks, mask);
         if (g == 0) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                sm.red_o[warp][16 * gl + k] = ks.o[k].x;
-                sm.red_o[warp][16 * gl + 8 + k] = ks.o[k].y;
+            for (int k = 0; k < 16; ++k) {
+                sm.red_o[warp][32 * li + k] = ks.o[k].x;
+                sm.red_o[warp][32 * li + 16 + k] = ks.o[k].y;
             }
-            if (gl == 0) {
+            if (li == 0) {
                 sm.red_m[warp] = ks.m;
                 sm.red_l[warp] = ks.l;
                 sm.red_pz[warp] = ks.pz;
             }
         }
         named_bar_sync(1, 32 * kConsumerWarps);
-        if (warp == 0) {
-            float M = -INFINITY;
-#pragma unroll
-            for (int wv = 0; wv < kConsumerWarps; ++wv) M = fmaxf(M, sm.red_m[wv]);
-            float f[kConsumerWarps];
+        if (!dead && rank == 0) {                 // the first warp of each query
+            float M = kMInit;
+            for (int wv = warp; wv < kConsumerWarps; wv += nq) M = fmaxf(M, sm.red_m[wv]);
             float L = 0.f, PZ = 0.f;
-#pragma unroll
-            for (int wv = 0; wv < kConsumerWarps; ++wv) {
-                f[wv] = (sm.red_m[wv] == -INFINITY) ? 0.f : exp2f(sm.red_m[wv] - M);
-                L = fmaf(sm.red_l[wv], f[wv], L);
-                PZ = fmaf(sm.red_pz[wv], f[wv], PZ);
+            for (int wv = warp; wv < kConsumerWarps; wv += nq) {
+                const float f = ex2(sm.red_m[wv] - M);
+                L = fmaf(sm.red_l[wv], f, L);
+                PZ = fmaf(sm.red_pz[wv], f, PZ);
             }
-            float *part = wk.partials + (int64_t)it * (D + 4);
+            float *part = wk.partials + ((int64_t)it * wk.qslots + slot) * (D + 4);
             for (int chn = lane; chn < D; chn += 32) {
                 float acc = 0.f;
-#pragma unroll
-                for (int wv = 0; wv < kConsumerWarps; ++wv) acc = fmaf(sm.red_o[wv][chn], f[wv], acc);
+                for (int wv = warp; wv < kConsumerWarps; wv += nq) acc = fmaf(sm.red_o[wv][chn], ex2(sm.red_m[wv] - M), acc);
                 part[4 + chn] = fmaf(acc, kOUnscale, PZ);
             }
             if (lane == 0) {
@@ -665,80 +812,76 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     }
 }
 
-// One CTA of D threads per (sequence, head): thread = channel.
+// One CTA of D threads per (sequence, query head): thread = channel. The query's partials
+// are those of its KV head's items whose subgroup holds it as an active query.
 template <int D>
 __global__ void __launch_bounds__(D)
 decode_combine_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
 {
-    __shared__ float red[D / 32];
     pdl_wait();
     pdl_trigger();
-    const int sh = blockIdx.x, ch = threadIdx.x, lane = ch & 31, wid = ch >> 5;
-    const int first = wk.head_first[sh], cnt = wk.head_cnt[sh];
-    const float *P = wk.partials + (int64_t)first * (D + 4);
+    const int HQ = c.H * c.G;
+    const int shq = blockIdx.x, ch = threadIdx.x;
+    const int s = shq / HQ, hq = shq % HQ, hk = hq / c.G, gq = hq % c.G;
+    const int unit = s * c.H + hk;
+    const int first = wk.head_first[unit], cnt = wk.head_cnt[unit];
+    const int QS = wk.qslots;
+    float M = kMInit;
+    bool any = false;
+    for (int i = 0; i < cnt; ++i) {
+        const int qinfo = wk.items[first + i].qinfo;
+        const int d = gq - (qinfo & 0xFF);
+        if (d < 0 || d >= kDecodeMaxQ || !((qinfo >> (8 + d)) & 1)) continue;
+        M = fmaxf(M, wk.partials[((int64_t)(first + i) * QS + d) * (D + 4)]);
+        any = true;
+    }
     float res = 0.f;
-    if (cnt > 0) {
-        float M = -INFINITY;
-        for (int i = ch; i < cnt; i += D) M = fmaxf(M, P[(int64_t)i * (D + 4)]);
-#pragma unroll
-        for (int d = 16; d >= 1; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
-        if (lane == 0) red[wid] = M;
-        __syncthreads();
-        M = red[0];
-#pragma unroll
-        for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
+    if (any) {
         float L = 0.f, acc = 0.f;
-        int i = 0;
-        for (; i + 4 <= cnt; i += 4) {
-            float mm[4], ll[4], oo[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float *p = P + (int64_t)(i + u) * (D + 4);
-                mm[u] = p[0];
-                ll[u] = p[1];
-                oo[u] = p[4 + ch];
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float f = exp2f(mm[u] - M);
-                L = fmaf(ll[u], f, L);
-                acc = fmaf(oo[u], f, acc);
-            }
-        }
-        for (; i < cnt; ++i) {
-            const float *p = P + (int64_t)i * (D + 4);
-            const float f = exp2f(p[0] - M);
+        for (int i = 0; i < cnt; ++i) {
+            const int qinfo = wk.items[first + i].qinfo;
+            const int d = gq - (qinfo & 0xFF);
+            if (d < 0 || d >= kDecodeMaxQ || !((qinfo >> (8 + d)) & 1)) continue;
+            const float *p = wk.partials + ((int64_t)(first + i) * QS + d) * (D + 4);
+            const float f = ex2(p[0] - M);
             L = fmaf(p[1], f, L);
             acc = fmaf(p[4 + ch], f, acc);
         }
         res = acc / L;
     }
-    out[(int64_t)sh * D + ch] = res;
+    out[(int64_t)shq * D + ch] = res;
 }
 
 template <int D>
-cudaError_t launch_decode_t(const kvq_cache *cache, const __half *q, const uint8_t *modes, int w,
-                            float *out, cudaStream_t st)
+cudaError_t launch_decode_t(const kvq_cache *cache, const DecodeWork &wk, uint32_t gen, const __half *q,
+                            const uint8_t *modes, int w, float *out, cudaStream_t st, const AppendArgs *ap)
 {
     const CacheView &c = cache->view;
-    cudaError_t le = launch_pdl(decode_sched_kernel, dim3(1), dim3(1024), 0, st, c, modes, w, cache->work);
-    if (le != cudaSuccess) return le;
+    cudaError_t e;
+    if (ap)
+        e = launch_pdl(decode_plan_kernel<D, true>, dim3(c.B), dim3(kPlanThreads), 0, st, c, modes, w, wk, gen, *ap);
+    else
+        e = launch_pdl(decode_plan_kernel<D, false>, dim3(c.B), dim3(kPlanThreads), 0, st, c, modes, w, wk, gen,
+                       AppendArgs{});
+    if (e != cudaSuccess) return e;
     const size_t smem = sizeof(DecodeSmem<D>);
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(decode_splitk_kernel<D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
-    const int grid = (int)std::min<int64_t>(cache->work.max_items, 3 * (int64_t)num_sms());
+    e = ensure_smem_attr((const void *)decode_splitk_kernel<D>, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(wk.max_items, kCtasPerSm * (int64_t)num_sms());
     profile_before(st);
-    le = launch_pdl(decode_splitk_kernel<D>, dim3(grid), dim3(kThreads), smem, st, c, q, cache->work);
-    if (le != cudaSuccess) return le;
+    e = launch_pdl(decode_splitk_kernel<D>, dim3(grid), dim3(kThreads), smem, st, c, q, wk);
+    if (e != cudaSuccess) return e;
     profile_after(st);
-    le = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H * c.G), dim3(D), 0, st, c, cache->work, out);
-    if (le != cudaSuccess) return le;
+    e = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H * c.G), dim3(D), 0, st, c, wk, out);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+cudaError_t launch_any(const kvq_cache *cache, const DecodeWork &wk, uint32_t gen, const __half *q,
+                       const uint8_t *modes, int w, float *out, cudaStream_t st, const AppendArgs *ap)
+{
+    if (cache->D == 128) return launch_decode_t<128>(cache, wk, gen, q, modes, w, out, st, ap);
+    return launch_decode_t<64>(cache, wk, gen, q, modes, w, out, st, ap);
 }
 
 } // namespace
@@ -746,8 +889,21 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const __half *q, const uint8
 cudaError_t launch_decode(const kvq_cache *cache, const __half *q, const uint8_t *modes, int w,
                           float *out, cudaStream_t st)
 {
-    if (cache->D == 128) return launch_decode_t<128>(cache, q, modes, w, out, st);
-    return launch_decode_t<64>(cache, q, modes, w, out, st);
+    kvq_cache *mc = const_cast<kvq_cache *>(cache);   // the call's generation id only
+    uint32_t gen = ++mc->decode_gen;
+    if (gen == 0) gen = ++mc->decode_gen;             // 0 is the count word's initial generation
+    return launch_any(cache, cache->work, gen, q, modes, w, out, st, nullptr);
+}
+
+cudaError_t launch_decode_step(kvq_cache *cache, const __half *q, const __half *k, const __half *v,
+                               const uint8_t *bits, const int32_t *cu, int64_t n_tok,
+                               const int32_t *positions, const uint8_t *modes, int w, float *out,
+                               cudaStream_t st)
+{
+    AppendArgs ap{k, v, bits, cu, positions, n_tok, ++cache->write_gen};
+    uint32_t gen = ++cache->decode_gen;
+    if (gen == 0) gen = ++cache->decode_gen;
+    return launch_any(cache, cache->work, gen, q, modes, w, out, st, &ap);
 }
 
 } // namespace kvq
@@ -769,6 +925,7 @@ namespace {
 
 std::mutex g_scratch_mu;
 void *g_scratch_addr[256] = {};   // device address of g_decode_scratch, per device ordinal
+std::atomic<uint32_t> g_static_gen{0};
 
 cudaError_t static_scratch(int dev, unsigned char **out)
 {
@@ -785,24 +942,6 @@ cudaError_t static_scratch(int dev, unsigned char **out)
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
-template <int D>
-cudaError_t launch_decode_static(const kvq_cache *cache, const DecodeWork &wk, const __half *q,
-                                 const uint8_t *modes, int w, float *out, cudaStream_t st)
-{
-    const CacheView &c = cache->view;
-    cudaError_t e = launch_pdl(decode_sched_kernel, dim3(1), dim3(1024), 0, st, c, modes, w, wk);
-    if (e != cudaSuccess) return e;
-    const size_t smem = sizeof(DecodeSmem<D>);
-    e = cudaFuncSetAttribute(decode_splitk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int grid = (int)std::min<int64_t>(wk.max_items, 3 * (int64_t)num_sms());
-    e = launch_pdl(decode_splitk_kernel<D>, dim3(grid), dim3(kThreads), smem, st, c, q, wk);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H * c.G), dim3(D), 0, st, c, wk, out);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-}
 
 } // namespace
 } // namespace kvq
@@ -825,13 +964,14 @@ extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache,
 
     // scratch layout: count | head_first | head_cnt | items | partials, each 256-byte aligned,
     // sized for the cache's worst case (every head full at capacity)
-    const int BH = cache->B * cache->H * cache->view.G;     // query heads
+    const int BH = cache->B * cache->H;                     // (sequence, KV head) units
     const int64_t items = cache->work.max_items;
+    const int qslots = cache->work.qslots;
     const size_t o_first = 256;
     const size_t o_cnt = o_first + align256(sizeof(int32_t) * (size_t)BH);
     const size_t o_items = o_cnt + align256(sizeof(int32_t) * (size_t)BH);
     const size_t o_part = o_items + align256(sizeof(DecodeItem) * (size_t)items);
-    const size_t need = o_part + sizeof(float) * (size_t)items * (cache->D + 4);
+    const size_t need = o_part + sizeof(float) * (size_t)items * qslots * (cache->D + 4);
     if (need > kStaticScratchBytes) {
         char msg[256];
         snprintf(msg, sizeof(msg),
@@ -844,15 +984,19 @@ extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache,
     e = static_scratch(dev, &base);
     if (e != cudaSuccess) return report_error(KVQ_ERR_CUDA, "routed_attn_decode_noalloc: cudaGetSymbolAddress failed");
     DecodeWork wk;
-    wk.count = reinterpret_cast<int32_t *>(base);
+    wk.count = reinterpret_cast<unsigned long long *>(base);
     wk.head_first = reinterpret_cast<int32_t *>(base + o_first);
     wk.head_cnt = reinterpret_cast<int32_t *>(base + o_cnt);
     wk.items = reinterpret_cast<DecodeItem *>(base + o_items);
     wk.partials = reinterpret_cast<float *>(base + o_part);
     wk.max_items = items;
+    wk.qslots = qslots;
+    // a generation id no earlier call on the shared array used (never 0: the array starts
+    // zeroed, and the first planning CTA of this call resets the count it finds)
+    uint32_t gen = ++g_static_gen;
+    if (gen == 0) gen = ++g_static_gen;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    e = (cache->D == 128) ? launch_decode_static<128>(cache, wk, static_cast<const __half *>(q), modes, w, out, st)
-                          : launch_decode_static<64>(cache, wk, static_cast<const __half *>(q), modes, w, out, st);
+    e = launch_any(cache, wk, gen, static_cast<const __half *>(q), modes, w, out, st, nullptr);
     if (e != cudaSuccess) return report_error(KVQ_ERR_CUDA, "routed_attn_decode_noalloc: kernel launch failed");
     return report_error(KVQ_OK, "");
 }

@@ -64,24 +64,35 @@ __device__ __forceinline__ void set_status(int32_t *status, int code)
 }
 
 // ---- scheduler work list (decode) ----------------------------------------------------
-constexpr int kDecodeItemKeys = 512;   // keys per split-K work item
+constexpr int kDecodeItemKeys = 576;   // keys per split-K work item, at most (w + 1 = 513 fits one)
 constexpr int kDecodeWindowKeys = 128; // keys per window of record offsets inside an item
+constexpr int kDecodeMaxQ = 4;         // query heads served by one item (a subgroup of a GQA group)
 
 struct __align__(16) DecodeItem {
-    int32_t sh, j0, j1;  // (sequence, head) and key range [j0, j1)
+    int32_t sh, j0, j1;  // (sequence, KV head) = s * H + hk, and key range [j0, j1)
     uint32_t end_off;    // byte offset of key j1 in the stream (the stream end if j1 = len)
-    int64_t sbase;       // slot of key 0 of (sequence, head)
-    int64_t pad;
+    int64_t sbase;       // slot of key 0 of (sequence, KV head)
+    int32_t qinfo;       // first query g0 of the subgroup | active-query mask << 8 (bit i: g0 + i)
+    int32_t pad;
 };
 
 struct DecodeWork {
     DecodeItem *items;   // [max_items]
-    int32_t *count;      // [1]
-    int32_t *head_first; // [B*H]
-    int32_t *head_cnt;   // [B*H]
-    float *partials;     // [max_items][D + 4]: (m, l, -, -, o[D])
+    unsigned long long *count; // [1]: call generation << 32 | items listed by the call
+    int32_t *head_first; // [B*H] first item of (sequence, KV head)
+    int32_t *head_cnt;   // [B*H] its items (all subgroups)
+    float *partials;     // [max_items][qslots][D + 4]: (m, l, -, -, o[D])
     int64_t max_items;
+    int qslots;          // min(G, kDecodeMaxQ)
 };
+
+// Upper bound of the items a decode call lists for a cache: per (sequence, KV head) and
+// subgroup of at most kDecodeMaxQ query heads, ceil(cap / kDecodeItemKeys) + 1 (the key
+// range may be cut once where the local window starts).
+inline int64_t decode_max_items(int64_t cap, int G)
+{
+    return (int64_t)((G + kDecodeMaxQ - 1) / kDecodeMaxQ) * ((cap + kDecodeItemKeys - 1) / kDecodeItemKeys + 1);
+}
 
 // ---- PTX helpers -----------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -120,10 +131,13 @@ __device__ __forceinline__ uint64_t global_ns()
 
 // Wait until the barrier's phase `parity` has completed. The waiting thread may be
 // suspended by the hardware for up to ~0.1 ms per try (woken when the phase completes),
-// so waiting warps do not spin on issue slots. Bounded: gives up after about two seconds,
-// records KVQ_ERR_DEVICE_CHECK and returns false, so a logic error ends the kernel with a
-// status instead of hanging the GPU.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status)
+// so waiting warps do not spin on issue slots. Bounded: gives up after `limit_ns` (about
+// two seconds by default), records KVQ_ERR_DEVICE_CHECK and returns false, so a logic
+// error ends the kernel with a status instead of hanging the GPU.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
+                                          uint64_t limit_ns = kWaitLimitNs)
 {
     const uint32_t addr = smem_u32(bar);
     const uint32_t suspend_ns = 100000;
@@ -140,7 +154,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_
         if ((it & 15u) == 0) {
             const uint64_t t = global_ns();
             if (t0 == 0) t0 = t;
-            else if (t - t0 > 2000000000ull) {
+            else if (t - t0 > limit_ns) {
                 set_status(status, KVQ_ERR_DEVICE_CHECK);
                 return false;
             }
@@ -212,6 +226,7 @@ struct kvq_cache {
     kvq::CacheView view;
     kvq::DecodeWork work;
     uint32_t write_gen;       // id of the last kvq_write call
+    uint32_t decode_gen;      // id of the last decode call on the cache's own work list
     void *pf_tiles;           // prefill tile list (PfTile = 4 x int32), pf_max_tiles entries
     int32_t *pf_count;        // [1]
     int32_t *pf_qidx;         // [total_slots] per-(sequence, head) query lists
@@ -227,9 +242,19 @@ cudaError_t launch_write(kvq_cache *c, const __half *k, const __half *v, const u
                          const int32_t *cu, int64_t n_tok, cudaStream_t st);
 cudaError_t launch_decode(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,
                           float *out, cudaStream_t st);
+// one decode step: append the step's tokens (optionally after rolling sequences back to
+// `positions`), then decode, in three launches
+cudaError_t launch_decode_step(kvq_cache *c, const __half *q, const __half *k, const __half *v,
+                               const uint8_t *bits, const int32_t *cu, int64_t n_tok,
+                               const int32_t *positions, const uint8_t *modes, int w, float *out,
+                               cudaStream_t st);
 cudaError_t launch_prefill_tc(const kvq_cache *c, const __half *q, const uint8_t *modes, int w,
                               const int32_t *cu, int64_t n_tok, float *out, cudaStream_t st);
+// SM count of the current device (cached per device ordinal)
 int num_sms();
+// Raise `func`'s dynamic shared-memory limit to `bytes` on the current device; done once
+// per (kernel, device), thread-safe.
+cudaError_t ensure_smem_attr(const void *func, size_t bytes);
 // records a host-side status for kvq_last_error() and returns `code`
 int report_error(int code, const char *msg);
 // profiling hook (kvq_set_profile_events): record the caller's events around a main kernel

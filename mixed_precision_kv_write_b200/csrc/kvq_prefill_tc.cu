@@ -661,12 +661,8 @@ cudaError_t run_tc(const kvq_cache *cache, const __half *q, const uint8_t *modes
                                                      cache->pf_qidx);
     const int64_t max_tiles = n_tok * c.H * c.G / kQRows + 2LL * c.B * c.H * c.G;
     const size_t smem = sizeof(PfSmem<D>) + 1024;
-    static bool attr_done = false;
-    if (!attr_done) {
-        e = cudaFuncSetAttribute(prefill_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    e = ensure_smem_attr((const void *)prefill_tc_kernel<D>, smem);
+    if (e != cudaSuccess) return e;
     profile_before(st);
     prefill_tc_kernel<D><<<(unsigned)max_tiles, kTcThreads, smem, st>>>(c, q, w, cu, tiles, cache->pf_count,
                                                                         cache->pf_qidx, out);

@@ -16,7 +16,7 @@
 // HBM traffic per (token, head): reads 2*D*2 bytes, writes b*D/4 + 16 + 4 bytes.
 #include <algorithm>
 
-#include "kvq_internal.cuh"
+#include "kvq_quant.cuh"
 
 namespace kvq {
 namespace {
@@ -137,127 +137,6 @@ struct WqPair {                          // one (token, head) of the CTA
     uint32_t meta;                       // width code in bits 0-1
     int32_t ok;                          // 0: not written (rejected write or bad call)
 };
-
-// Codes are rint(fl(u / s)) with u = fl(x - z), clamped to [0, 2^b - 1].
-// The correctly rounded quotient fl(u / s) is formed with Markstein's correction
-// (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Dev. 34(1), 1990): with y = RN(1/s) and the faithful q0 = RN(u y),
-// the remainder r = u - s q0 is exact in one FMA, and RN(q0 + r y) = RN(u / s). Because
-// 0 <= u <= fl(max - min) the quotient lies in [0, 2^b - 1 + 2^-14], so rint never leaves the
-// code range. rint is taken by adding 1.5 * 2^23: for 0 <= q < 2^22 the sum is
-// 1.5 * 2^23 + rint(q) exactly (round-to-nearest-even), the integer in the low mantissa bits.
-// A NaN quotient (NaN or infinite inputs) is caught by a running sum and the lane falls
-// back to the plain clamped formula, which maps it to code 0.
-constexpr float kRoundMagic = 12582912.0f;          // 1.5 * 2^23
-constexpr uint32_t kRoundMagicBits = 0x4B400000u;
-
-// Quantizes a lane's NC chunks of 8 fp16 values to BITS-bit codes. Chunk j holds channels
-// 8 * (j * VL + li) .. + 7 of the vector, so its 8 codes fill BITS bytes of the part at byte
-// BITS * (j * VL + li), and the VL lanes of a vector store adjacent chunks.
-template <int BITS, int NC, int VL>
-__device__ __forceinline__ void quant_store(const uint4 (&raw)[NC], float z, float sc,
-                                            uint8_t *dst, int li)
-{
-    uint32_t w[NC][2];
-#pragma unroll
-    for (int j = 0; j < NC; ++j) w[j][0] = w[j][1] = 0u;
-    if (sc != 0.0f) {
-        const float y = __frcp_rn(sc);
-        float nan_probe = 0.0f;
-#pragma unroll
-        for (int j = 0; j < NC; ++j) {
-            const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[j]);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float x = (e & 1) ? __high2float(h2[e >> 1]) : __low2float(h2[e >> 1]);
-                const float u = __fsub_rn(x, z);
-                const float q0 = __fmul_rn(u, y);
-                const float r = __fmaf_rn(-sc, q0, u);
-                const float q = __fmaf_rn(r, y, q0);
-                const float t = __fadd_rn(q, kRoundMagic);
-                nan_probe = __fadd_rn(nan_probe, q);
-                // code << shift; the 1.5 * 2^23 bits are taken off below
-                w[j][(e * BITS) >> 5] += __float_as_uint(t) << ((e * BITS) & 31);
-            }
-        }
-        constexpr int kWordBits = BITS * 8 < 32 ? BITS * 8 : 32;   // code bits per word
-        uint32_t magic = 0u;
-#pragma unroll
-        for (int sh = 0; sh < kWordBits; sh += BITS) magic += kRoundMagicBits << sh;
-#pragma unroll
-        for (int j = 0; j < NC; ++j) {
-            w[j][0] -= magic;
-            if (BITS == 8) w[j][1] -= magic;
-        }
-        if (nan_probe != nan_probe) {
-            const float top = (float)((1u << BITS) - 1u);
-#pragma unroll
-            for (int j = 0; j < NC; ++j) {
-                const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[j]);
-                w[j][0] = w[j][1] = 0u;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float x = (e & 1) ? __high2float(h2[e >> 1]) : __low2float(h2[e >> 1]);
-                    const float c = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x, z), sc)), 0.0f), top);
-                    w[j][(e * BITS) >> 5] |= __float2uint_rz(c) << ((e * BITS) & 31);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < NC; ++j) {
-        const int chunk = j * VL + li;
-        if (BITS == 8) reinterpret_cast<uint2 *>(dst)[chunk] = make_uint2(w[j][0], w[j][1]);
-        else if (BITS == 4) reinterpret_cast<uint32_t *>(dst)[chunk] = w[j][0];
-        else reinterpret_cast<uint16_t *>(dst)[chunk] = (uint16_t)w[j][0];
-    }
-}
-
-// min and max of a vector spread over VL adjacent lanes (NC 8-value chunks per lane), in
-// fp16 (exact); (min, -max) travel as one half2 through the shuffles. Every lane of the
-// warp takes part.
-template <int NC, int VL>
-__device__ __forceinline__ __half2 vec_minmax(const uint4 (&raw)[NC])
-{
-    const __half2 (&h2)[4 * NC] = *reinterpret_cast<const __half2 (*)[4 * NC]>(raw);
-    __half2 lo2 = h2[0], hi2 = h2[0];
-#pragma unroll
-    for (int e = 1; e < 4 * NC; ++e) {
-        lo2 = __hmin2(lo2, h2[e]);
-        hi2 = __hmax2(hi2, h2[e]);
-    }
-    __half2 mm = __halves2half2(__hmin(__low2half(lo2), __high2half(lo2)),
-                                __hneg(__hmax(__low2half(hi2), __high2half(hi2))));
-#pragma unroll
-    for (int d = VL / 2; d >= 1; d >>= 1) {
-        const uint32_t o = __shfl_xor_sync(0xffffffffu, *reinterpret_cast<uint32_t *>(&mm), d);
-        mm = __hmin2(mm, *reinterpret_cast<const __half2 *>(&o));
-    }
-    return mm;
-}
-
-// This lane's share of one vector's record part at `dst` (b-bit codes, or the fp16 values
-// for b = 16) and, from the vector's first lane, its (s, z) side entry.
-template <int NC, int VL>
-__device__ __forceinline__ void vec_store(const CacheView &c, const uint4 (&raw)[NC], __half2 mm, int b,
-                                          uint8_t *dst, int64_t slot, int part, int li)
-{
-    float sc = 1.0f, z = 0.0f;
-    if (b == 16) {
-#pragma unroll
-        for (int j = 0; j < NC; ++j) reinterpret_cast<uint4 *>(dst)[j * VL + li] = raw[j];
-    } else {
-        const float mn = __low2float(mm), mx = -__high2float(mm);
-        const float top = (float)((1u << b) - 1u);
-        // zeros are stored as +0 (the min scan may meet -0 or +0 first)
-        sc = __fadd_rn(__fdiv_rn(__fsub_rn(mx, mn), top), 0.0f);
-        z = __fadd_rn(mn, 0.0f);
-        if (b == 8) quant_store<8, NC, VL>(raw, z, sc, dst, li);
-        else if (b == 4) quant_store<4, NC, VL>(raw, z, sc, dst, li);
-        else quant_store<2, NC, VL>(raw, z, sc, dst, li);
-    }
-    if (li == 0) reinterpret_cast<float2 *>(&c.side[slot])[part] = make_float2(sc, z);
-}
 
 // One CTA per tile of T tokens x HG heads. Warp 0 starts two bulk copies (the tile's K and
 // V rows are contiguous when HG = H, else one copy per token and tensor); meanwhile every
@@ -382,105 +261,18 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
 }
 
 // Short appends (decode steps): one CTA of 256 threads per sequence does the scan and the
-// quantization of all the sequence's new (token, head) pairs in one launch. Phase 1, a
-// warp per head: capacity, widths and record offsets (warp prefix sum) of the sequence's
-// tokens. Phase 2, after the block has seen every head's verdict: D/8 lanes per vector
-// (one (token, head) pair per warp pass at head_dim 128), values straight from global
-// memory. Same results as the scan + quantize pair of kernels.
+// quantization of all the sequence's new (token, head) pairs in one launch (append_seq).
+// Same results as the scan + quantize pair of kernels.
 template <int D>
 __global__ void __launch_bounds__(256)
 write_append_kernel(CacheView c, const __half *__restrict__ k, const __half *__restrict__ v,
                     const uint8_t *__restrict__ bits, const int32_t *__restrict__ cu, int64_t n_tok,
                     uint32_t gen)
 {
-    constexpr int VL = D / 8, VPW = 32 / VL;
     __shared__ int bad_sh;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait();
     pdl_trigger();
-    const int s = blockIdx.x, H = c.H;
-    const int64_t t0 = cu[s], t1 = cu[s + 1];
-    if (t0 < 0 || t1 < t0 || t1 > n_tok || (s == 0 && t0 != 0)) {
-        if (tid == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
-        return;
-    }
-    const int n = (int)(t1 - t0);
-    if (n == 0) return;
-    if (tid == 0) bad_sh = 0;
-    __syncthreads();
-    for (int h = warp; h < H; h += 8) {
-        const int sh = s * H + h;
-        const int L0 = c.len[sh];
-        if ((int64_t)L0 + n > c.cap[s]) {
-            if (lane == 0) {
-                set_status(c.status, KVQ_ERR_CAPACITY);
-                c.wstart[sh] = -1;
-            }
-            continue;
-        }
-        const int64_t slot0 = slot_of(c, s, h, L0);
-        uint32_t off = c.end[sh];
-        bool bad = false;
-        for (int base = 0; base < n; base += 32) {
-            const int i = base + lane;
-            uint32_t sz = 0, wc = 0;
-            if (i < n) {
-                const int b = bits[(t0 + i) * H + h];
-                const int w = width_code(b);
-                if (w < 0) bad = true;
-                else {
-                    wc = (uint32_t)w;
-                    sz = (uint32_t)(b * D / 4);
-                }
-            }
-            uint32_t incl = sz;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
-                if (lane >= d) incl += y;
-            }
-            if (i < n) c.meta[slot0 + i] = (off + incl - sz) | wc;
-            off += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&bad_sh, 1);
-        if (lane == 0) {
-            c.wstart[sh] = L0;
-            c.wend[sh] = off;
-        }
-    }
-    __syncthreads();
-    if (bad_sh) {                                // the sequence's write is refused for every head
-        if (tid == 0) {
-            c.bad[s] = gen;
-            set_status(c.status, KVQ_ERR_BITS);
-        }
-        return;
-    }
-    const int n_vec = 2 * n * H;                 // vector vi: pair vi / 2 = i * H + h, K or V
-    const int li = lane % VL;
-    for (int vb = warp * VPW; vb < n_vec; vb += 8 * VPW) {
-        const int vi = vb + lane / VL;
-        const bool in_range = vi < n_vec;
-        const int p = vi >> 1, part = vi & 1;
-        const int i = p / H, h = p % H;
-        uint4 raw[1] = {make_uint4(0u, 0u, 0u, 0u)};
-        if (in_range) raw[0] = reinterpret_cast<const uint4 *>((part ? v : k) + ((t0 + i) * H + h) * D)[li];
-        const __half2 mm = vec_minmax<1, VL>(raw);
-        if (!in_range) continue;
-        const int st = c.wstart[s * H + h];
-        if (st < 0) continue;
-        const int64_t slot = slot_of(c, s, h, st + i);
-        const uint32_t meta = c.meta[slot];
-        const int b = 2 << (meta & 3u);
-        vec_store<1, VL>(c, raw, mm, b, stream_of(c, s, h) + (meta & ~15u) + part * (b * D / 8), slot, part, li);
-    }
-    for (int h = tid; h < H; h += 256) {         // commit the new lengths and stream ends
-        const int st = c.wstart[s * H + h];
-        if (st >= 0) {
-            c.len[s * H + h] = st + n;
-            c.end[s * H + h] = c.wend[s * H + h];
-        }
-    }
+    append_seq<D>(c, k, v, bits, cu, n_tok, gen, nullptr, blockIdx.x, bad_sh);
 }
 
 } // namespace

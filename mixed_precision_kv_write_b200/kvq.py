@@ -22,8 +22,8 @@ MODE_SKIP, MODE_LOCAL, MODE_FULL = 0, 1, 2
 # every symbol include/kvq.h declares
 EXPORTS = ("kvq_cache_create", "kvq_cache_create_gqa", "kvq_cache_destroy", "kvq_cache_reset", "kvq_cache_truncate",
            "kvq_cache_lengths", "kvq_write", "routed_attn_prefill", "routed_attn_decode",
-           "routed_attn_decode_noalloc", "kvq_cache_export", "kvq_check", "kvq_set_profile_events",
-           "kvq_route_argmax", "kvq_last_error")
+           "routed_attn_decode_noalloc", "kvq_decode_step", "kvq_cache_export", "kvq_check", "kvq_set_profile_events",
+           "kvq_route_argmax", "kvq_test_fail_alloc", "kvq_test_bounded_wait", "kvq_last_error")
 
 _lib = None
 
@@ -55,10 +55,13 @@ def load_library(path: str = LIB_PATH):
         "routed_attn_prefill": ([vp, vp, vp, i32, vp, i64, vp, vp], i32),
         "routed_attn_decode": ([vp, vp, vp, i32, vp, vp], i32),
         "routed_attn_decode_noalloc": ([vp, vp, vp, i32, vp, vp], i32),
+        "kvq_decode_step": ([vp, vp, vp, vp, vp, i64, vp, vp, i32, vp, vp, vp], i32),
         "kvq_cache_export": ([vp, i32, i32, i64, i64, vp, vp, vp, vp, vp], i32),
         "kvq_check": ([vp, vp], i32),
         "kvq_set_profile_events": ([vp, vp], i32),
         "kvq_route_argmax": ([vp, vp, i64, vp, vp, vp], i32),
+        "kvq_test_fail_alloc": ([i32], i32),
+        "kvq_test_bounded_wait": ([vp, i64, vp], i32),
         "kvq_last_error": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -214,6 +217,31 @@ def routed_attn_decode(q, cache: KVQCache, modes, w: int, out=None, stream=None)
     _check(out, "out", torch.float32, dev, shape)
     _raise(load_library().routed_attn_decode(_ptr(q), cache.handle, _ptr(modes), int(w), _ptr(out),
                                              _stream(stream, dev)))
+    return out
+
+
+def decode_step(q, k, v, bits, cu_seqlens, cache: KVQCache, modes, w: int, positions=None, out=None,
+                stream=None):
+    """One decode step (kvq_decode_step): append k, v [n_tok, H, D] at widths bits (Eq. 4),
+    optionally after rolling each sequence back to `positions` [B] (int32), then routed
+    decode attention (Eq. 2) of q [B, HQ, D]; returns fp32 out [B, HQ, D]."""
+    dev = cache.device
+    n = k.shape[0]
+    shape = (cache.batch, cache.query_heads, cache.head_dim)
+    _check(q, "q", torch.float16, dev, shape)
+    _check(modes, "modes", torch.uint8, dev, shape[:2])
+    _check(k, "k", torch.float16, dev, (n, cache.heads, cache.head_dim))
+    _check(v, "v", torch.float16, dev, (n, cache.heads, cache.head_dim))
+    _check(bits, "bits", torch.uint8, dev, (n, cache.heads))
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev, (cache.batch + 1,))
+    if positions is not None:
+        _check(positions, "positions", torch.int32, dev, (cache.batch,))
+    if out is None:
+        out = torch.empty(shape, dtype=torch.float32, device=dev)
+    _check(out, "out", torch.float32, dev, shape)
+    _raise(load_library().kvq_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(bits), _ptr(cu_seqlens), n,
+                                          _ptr(positions), _ptr(modes), int(w), cache.handle, _ptr(out),
+                                          _stream(stream, dev)))
     return out
 
 

@@ -63,6 +63,28 @@ def check_records(cache, wl, k_cpu, v_cpu, bits_cpu, pairs, tok_ranges=None):
                 f"side column {col} differs at (s={s}, h={h})"
 
 
+def check_records_seq(cache, s, heads, ks, vs, bs, what=""):
+    """Bit-exact check of every stored record of sequence s for the listed heads, given the
+    sequence's own fp16 K/V [L, H, D] and widths [L, H] on the CPU (all L tokens, including
+    any written by later short appends)."""
+    L = ks.shape[0]
+    for h in heads:
+        kc, vc, sd, bt = cache.export(s, h, 0, L)
+        torch.cuda.synchronize()
+        kc = kc.cpu().numpy().view(np.uint16)
+        vc = vc.cpu().numpy().view(np.uint16)
+        sd = sd.cpu().numpy()
+        bb = bs[:, h].numpy()
+        assert np.array_equal(bt.cpu().numpy(), bb), f"{what} widths differ at (s={s}, h={h})"
+        ck, sk, zk = oracle.quantize_many(ks[:, h].contiguous().numpy().view(np.uint16), bb)
+        cv, sv, zv = oracle.quantize_many(vs[:, h].contiguous().numpy().view(np.uint16), bb)
+        assert np.array_equal(kc, ck), f"{what} K codes differ at (s={s}, h={h})"
+        assert np.array_equal(vc, cv), f"{what} V codes differ at (s={s}, h={h})"
+        for col, ref in ((0, sk), (1, zk), (2, sv), (3, zv)):
+            assert np.array_equal(sd[:, col].view(np.uint32), ref.view(np.uint32)), \
+                f"{what} side column {col} differs at (s={s}, h={h})"
+
+
 def oracle_decode(wl, k_cpu, v_cpu, bits_cpu, q_cpu, modes_cpu, w, s, h, L=None):
     """Oracle output of the decode query of (s, h) at t = L - 1."""
     cu = synth.cu_seqlens(wl.seqlens).tolist()

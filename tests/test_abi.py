@@ -53,3 +53,9 @@ def test_calls_reject_null_cache(lib):
     assert lib.kvq_cache_export(None, 0, 0, 0, 1, None, None, None, None, None) == kvq.KVQ_ERR_ARG
     assert lib.kvq_cache_destroy(None) == kvq.KVQ_OK
     assert lib.kvq_last_error() == b""
+
+
+def test_test_hooks_check_arguments_on_host(lib):
+    assert lib.kvq_test_fail_alloc(-1) == kvq.KVQ_ERR_ARG
+    assert lib.kvq_test_fail_alloc(0) == kvq.KVQ_OK
+    assert lib.kvq_test_bounded_wait(None, 1000000, None) == kvq.KVQ_ERR_ARG

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 from mixed_precision_kv_write_b200 import kvq, synth
-from kvq_testlib import assert_close_attn, build_cache, oracle_decode
+from kvq_testlib import assert_close_attn, build_cache, check_records_seq, oracle_decode
 
 pytestmark = pytest.mark.gpu
 W = synth.WORKLOADS
@@ -104,24 +104,34 @@ def _decode_step_like_bench(wl):
     return out.cpu().numpy(), q.cpu(), modes.cpu(), cache
 
 
-@pytest.mark.parametrize("name,n_check", [("decode_1p3b", 96), ("decode_long", 48)])
-def test_decode_full_size_sampled(name, n_check):
+@pytest.mark.parametrize("name,n_check,n_rec", [("decode_1p3b", 96, 64), ("decode_long", 48, 40)])
+def test_decode_full_size_sampled(name, n_check, n_rec):
+    # Full-size cache built as the benchmark builds it (long write of L - 1 tokens, then the
+    # step token through the single-launch append). Attention is checked on n_check sampled
+    # (sequence, head) queries; the stored records (codes, scales, zeros, widths of all L
+    # tokens, the appended one included) bit-exactly on n_rec sampled (sequence, head) pairs.
     wl = W[name]
     out, qc, mc, cache = _decode_step_like_bench(wl)
     assert cache.lengths().tolist() == list(wl.seqlens)
     rng = np.random.default_rng(1)
     pairs = [(int(s), int(h)) for s, h in zip(rng.integers(0, wl.batch, n_check),
                                               rng.integers(0, wl.heads, n_check))]
+    rec_pairs = {(s, int(rng.integers(wl.heads))) for s in range(wl.batch)}
+    while len(rec_pairs) < n_rec:
+        rec_pairs.add((int(rng.integers(wl.batch)), int(rng.integers(wl.heads))))
     by_seq = {}
     for s, h in pairs:
-        by_seq.setdefault(s, set()).add(h)
-    for s, hs in by_seq.items():
+        by_seq.setdefault(s, [set(), set()])[0].add(h)
+    for s, h in rec_pairs:
+        by_seq.setdefault(s, [set(), set()])[1].add(h)
+    for s, (hs, hr) in sorted(by_seq.items()):
         ks, vs, bs = synth.kv_sequence(wl, s, "cuda")
         ks, vs, bs = ks.cpu(), vs.cpu(), bs.cpu()
         one = synth.scaled(wl, seqlens=(wl.seqlens[s],))
-        for h in hs:
+        for h in sorted(hs):
             ref = oracle_decode(one, ks, vs, bs, qc[s:s + 1], mc[s:s + 1], wl.w, 0, h)
             assert_close_attn(out[s, h], ref, f"{name} s={s} h={h} mode={int(mc[s, h])}")
+        check_records_seq(cache, s, sorted(hr), ks, vs, bs, name)
     # skip heads are exact zeros everywhere
     skip = (mc.numpy() == 0)
     assert np.all(out[skip] == 0)

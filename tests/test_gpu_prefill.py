@@ -7,20 +7,21 @@ import pytest
 import torch
 
 from mixed_precision_kv_write_b200 import kvq, synth
-from kvq_testlib import assert_close_attn, build_cache, oracle_prefill
+from kvq_testlib import assert_close_attn, build_cache, check_records, oracle_prefill
 
 pytestmark = pytest.mark.gpu
 W = synth.WORKLOADS
 
 
-def _prefill(wl, w=None):
+def _prefill(wl, w=None, with_cache=False):
     k, v, bits = synth.kv_tokens(wl, "cuda")
     q, modes = synth.prefill_queries(wl, "cuda")
     cache = build_cache(wl, k, v, bits)
     out = kvq.routed_attn_prefill(q, cache, modes, wl.w if w is None else w,
                                   synth.cu_seqlens(wl.seqlens, "cuda"))
     cache.check()
-    return out.cpu().numpy(), (k.cpu(), v.cpu(), bits.cpu(), q.cpu(), modes.cpu())
+    res = (out.cpu().numpy(), (k.cpu(), v.cpu(), bits.cpu(), q.cpu(), modes.cpu()))
+    return res + (cache,) if with_cache else res
 
 
 def _check_all(wl, out, cpu, w, heads=None, queries=None):
@@ -94,13 +95,20 @@ def test_prefill_all_skip_is_zero():
 
 @pytest.mark.parametrize("name,per_seq", [("prefill_160m", 24), ("ragged_prefill", 24)])
 def test_prefill_full_size_sampled(name, per_seq):
+    # The full workload in one write + one prefill call, as the benchmark runs it: the
+    # stored records of every (sequence, head) are checked bit-exactly, and the attention
+    # of every head on a sample of each sequence's queries (first, last and per_seq random).
     wl = W[name]
-    out, cpu = _prefill(wl)
+    out, cpu, cache = _prefill(wl, with_cache=True)
+    kc, vc, bc = cpu[:3]
+    check_records(cache, wl, kc, vc, bc, [(s, h) for s in range(wl.batch) for h in range(wl.heads)])
     rng = np.random.default_rng(3)
+    qs = {}
 
     def queries(s):
-        L = wl.seqlens[s]
-        return np.unique(np.concatenate([[0, L - 1], rng.integers(0, L, per_seq)]))
+        if s not in qs:
+            L = wl.seqlens[s]
+            qs[s] = np.unique(np.concatenate([[0, L - 1], rng.integers(0, L, per_seq)]))
+        return qs[s]
 
-    heads = [int(x) for x in rng.choice(wl.heads, 2, replace=False)]
-    _check_all(wl, out, cpu, wl.w, heads=heads, queries=queries)
+    _check_all(wl, out, cpu, wl.w, queries=queries)

@@ -45,6 +45,31 @@ def test_noalloc_matches_decode_on_two_calls_in_a_row():
     assert np.all(got2[modes2.cpu().numpy() == 0] == 0)
 
 
+@pytest.mark.parametrize("D,group", [(64, 1), (128, 4), (64, 4)])
+def test_noalloc_other_shapes_larger_then_smaller(D, group):
+    # The scratch layout depends on the number of query heads (work-list head tables) and
+    # on head_dim (partials stride). A call on a larger cache, then one on a smaller cache
+    # of another shape, each matches routed_attn_decode on its own cache.
+    base = synth.WORKLOADS["decode_1p3b"] if D == 128 else synth.WORKLOADS["prefill_160m"]
+    results = []
+    for seqlens, hk in (((1500, 700, 64, 2000, 9, 513), 4), ((300, 1), 2)):
+        wl = synth.scaled(base, seqlens=seqlens, heads=hk)
+        k, v, bits = synth.kv_tokens(wl, "cuda")
+        cache = kvq.KVQCache(wl.batch, hk, D, list(wl.seqlens), query_group=group)
+        kvq.kvq_write(k, v, bits, synth.cu_seqlens(wl.seqlens, "cuda"), cache)
+        g = torch.Generator(device="cuda").manual_seed(D + group + hk)
+        hq = hk * group
+        q = torch.randn((wl.batch, hq, D), generator=g, device="cuda").half()
+        modes = torch.randint(0, 3, (wl.batch, hq), generator=g, device="cuda").to(torch.uint8)
+        ref = kvq.routed_attn_decode(q, cache, modes, 77).cpu().numpy()
+        got = kvq.routed_attn_decode_noalloc(q, cache, modes, 77).cpu().numpy()
+        cache.check()
+        assert_close_attn(got, ref, f"noalloc D={D} G={group} heads={hk}")
+        assert np.all(got[modes.cpu().numpy() == 0] == 0)
+        results.append(got.shape)
+    assert results[0] != results[1]
+
+
 def test_noalloc_rejects_caches_beyond_the_static_scratch():
     # 64 x 1024 heads: its worst-case work list needs more than the 16 MiB of static scratch
     cache = kvq.KVQCache(64, 1024, 64, [1] * 64)
