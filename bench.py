@@ -116,14 +116,28 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workload setup
-def decode_setup(wl, dev, group=1):
+def paged_pool_pages(wl, page_bytes, dev):
+    """Pages a paged cache of the workload needs: each (sequence, head) stream's record
+    bytes (widths from the seeded draws) rounded up to whole pages."""
+    from mixed_precision_kv_write_b200 import synth
+    n = 0
+    for s in range(wl.batch):
+        per = (synth.widths(wl, s, dev).to(torch.int64) * wl.head_dim // 4).sum(0)
+        n += int(((per + page_bytes - 1) // page_bytes).sum())
+    return n
+
+
+def decode_setup(wl, dev, group=1, page_bytes=0):
     """Cache holding L - 1 tokens per sequence; the step's token, query and modes; the
     exact keys and routed bytes one step reads. With group > 1 the cache holds wl.heads KV
-    heads shared by groups of `group` query heads (grouped-query attention)."""
+    heads shared by groups of `group` query heads (grouped-query attention); with
+    page_bytes > 0 the records live in a page pool sized for the workload's widths."""
     from mixed_precision_kv_write_b200 import kvq, synth
     B, H, D, L, w = wl.batch, wl.heads, wl.head_dim, wl.seqlens[0], wl.w
     HQ = H * group
-    cache = kvq.KVQCache(B, H, D, [L + 4] * B, device=dev, query_group=group)
+    pool = paged_pool_pages(wl, page_bytes, dev) + B * H if page_bytes else 0
+    cache = kvq.KVQCache(B, H, D, [L + 4] * B, device=dev, query_group=group, page_bytes=page_bytes,
+                         pool_pages=pool)
     q, modes = synth.decode_queries(synth.scaled(wl, heads=HQ) if group > 1 else wl, dev)
     k_step = torch.empty((B, H, D), dtype=torch.float16, device=dev)
     v_step = torch.empty_like(k_step)
@@ -196,14 +210,15 @@ def decode_roofline(st, k_avg, pk, pk_kind, profile_summary):
             "algorithmic_bytes_per_launch": kernel_bytes, "avg_launch_s": k_avg}
 
 
-def decode_workload_measure(name, dev, pk, pk_kind, steps=20, warm=5, group=1, profile_summary=None):
+def decode_workload_measure(name, dev, pk, pk_kind, steps=20, warm=5, group=1, profile_summary=None,
+                            page_bytes=0):
     """A decode workload other than the headline: its steps timed back to back (no events
     between launches), then a pass with events around the split-K kernel."""
     from mixed_precision_kv_write_b200 import synth
     wl = synth.WORKLOADS[name]
     if group > 1:
         wl = synth.scaled(wl, heads=wl.heads // group)
-    st = decode_setup(wl, dev, group)
+    st = decode_setup(wl, dev, group, page_bytes)
     stream = torch.cuda.current_stream(dev)
     for _ in range(warm):
         decode_step(st, wl.w)
@@ -224,6 +239,11 @@ def decode_workload_measure(name, dev, pk, pk_kind, steps=20, warm=5, group=1, p
     if group > 1:
         res["unique_kv_bytes_per_step"] = st["unique_bytes"]
         res["unique_kv_gbs"] = st["unique_bytes"] / t_step / 1e9
+    if page_bytes:
+        c = st["cache"]
+        res["pages"] = {"page_bytes": page_bytes, "pool_pages": c.pool_pages,
+                        "pool_bytes": c.pool_pages * page_bytes,
+                        "contiguous_worst_case_bytes": wl.batch * wl.heads * (wl.seqlens[0] + 4) * 4 * wl.head_dim}
     del st
     torch.cuda.empty_cache()
     return res
@@ -530,6 +550,10 @@ def run_ours(args):
                           "4 KV heads, batch 64, context 8192, w=512")
         extra["gqa_decode"] = gq
         extra["decode_long"]["workload"] = synth.WORKLOADS["decode_long"].note
+        pg_line = decode_workload_measure("decode_1p3b", dev, pk, pk_kind, page_bytes=65536)
+        pg_line["workload"] = ("decode_1p3b on a paged cache: 64 KiB pages from a pool sized for the seeded "
+                               "widths, pages handed out in a scrambled order")
+        extra["paged_decode"] = pg_line
     barrier(pg, dev)
 
     line = {

@@ -83,10 +83,32 @@ int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
 int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group, int head_dim,
                          const int64_t *capacity_tokens, kvq_stream_t stream);
 
+/*
+ * Paged variant of kvq_cache_create_gqa (the pages' inference procedure says the routed
+ * cache works with KV paging; their limitations section notes that variable-width records
+ * complicate it). The record bytes live in a pool of pool_pages pages of page_bytes bytes
+ * each (a power of two in [4 KiB, 2 MiB]) instead of a worst-case stream per (sequence,
+ * head): pool memory can be sized for the expected average width. Each (sequence, KV head)
+ * stream is a list of logical pages; a write takes physical pages from the pool when its
+ * records first reach a logical page (in a scrambled pool order, so pages of different
+ * streams interleave), and a stream keeps its pages until kvq_cache_reset returns all of
+ * them. Records are packed back to back in the logical stream as in a contiguous cache
+ * and may straddle two pages; every call reads and writes through the page table.
+ * Offsets, side entries and capacities are as in kvq_cache_create_gqa (capacity_tokens
+ * bounds each sequence's tokens; the record offsets and side table stay per token).
+ * A write that would need more pages than the pool has left is refused for that head with
+ * KVQ_ERR_CAPACITY (device check), like a capacity overflow. page_bytes = 0 creates a
+ * contiguous cache (pool_pages ignored).
+ */
+int kvq_cache_create_paged(kvq_cache **out, int batch, int heads, int query_group, int head_dim,
+                           const int64_t *capacity_tokens, int64_t page_bytes, int64_t pool_pages,
+                           kvq_stream_t stream);
+
 /* Free every device buffer of the cache (synchronizes the device first). NULL is a no-op. */
 int kvq_cache_destroy(kvq_cache *cache);
 
-/* Set every sequence's length to 0 and clear the device status word. */
+/* Set every sequence's length to 0 and clear the device status word; a paged cache's
+   pages all go back to its pool. */
 int kvq_cache_reset(kvq_cache *cache, kvq_stream_t stream);
 
 /*

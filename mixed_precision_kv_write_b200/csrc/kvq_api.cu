@@ -75,18 +75,17 @@ __global__ void export_kernel(kvq::CacheView c, int s, int h, int64_t first, int
     const int64_t slot = kvq::slot_of(c, s, h, j);
     const uint32_t mt = c.meta[slot];
     const int b = 2 << (mt & 3u);
-    const uint8_t *rec = kvq::stream_of(c, s, h) + (mt & ~15u);
     for (int part = 0; part < 2; ++part) {
         uint16_t *dst = part == 0 ? k_codes : v_codes;
         if (!dst) continue;
-        const uint8_t *p = rec + part * (b * D / 8);
+        const kvq::RecLoc p = kvq::rec_loc(c, s, h, (mt & ~15u) + part * (b * D / 8));
         for (int ch = lane; ch < D; ch += 32) {
             uint16_t val;
             if (b == 16) {
-                val = reinterpret_cast<const uint16_t *>(p)[ch];
+                val = *reinterpret_cast<const uint16_t *>(p.at(2u * ch));
             } else {
                 const int bit = b * ch;
-                val = (uint16_t)((reinterpret_cast<const uint32_t *>(p)[bit >> 5] >> (bit & 31)) &
+                val = (uint16_t)((*reinterpret_cast<const uint32_t *>(p.at(4u * (bit >> 5))) >> (bit & 31)) &
                                  ((1u << b) - 1u));
             }
             dst[i * D + ch] = val;
@@ -219,6 +218,13 @@ int kvq_cache_create(kvq_cache **out, int batch, int heads, int head_dim,
 int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group, int head_dim,
                          const int64_t *capacity_tokens, kvq_stream_t stream)
 {
+    return kvq_cache_create_paged(out, batch, heads, query_group, head_dim, capacity_tokens, 0, 0, stream);
+}
+
+int kvq_cache_create_paged(kvq_cache **out, int batch, int heads, int query_group, int head_dim,
+                           const int64_t *capacity_tokens, int64_t page_bytes, int64_t pool_pages,
+                           kvq_stream_t stream)
+{
     if (!out) return fail(KVQ_ERR_ARG, "kvq_cache_create: out is NULL");
     *out = nullptr;
     if (batch <= 0 || heads <= 0) return fail(KVQ_ERR_ARG, "kvq_cache_create: batch and heads must be > 0");
@@ -230,6 +236,17 @@ int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group,
     if (head_dim != 64 && head_dim != 128)
         return fail(KVQ_ERR_ARG, "kvq_cache_create: head_dim must be 64 or 128 (got %d)", head_dim);
     if (!capacity_tokens) return fail(KVQ_ERR_ARG, "kvq_cache_create: capacity_tokens is NULL");
+    const bool paged = page_bytes != 0;
+    int page_shift = 31;
+    if (paged) {
+        if (page_bytes < 4096 || page_bytes > (1 << 21) || (page_bytes & (page_bytes - 1)))
+            return fail(KVQ_ERR_ARG, "kvq_cache_create_paged: page_bytes = %lld is not a power of two in [4 KiB, 2 MiB]",
+                        (long long)page_bytes);
+        if (pool_pages < 1 || pool_pages > (int64_t)INT32_MAX / 2)
+            return fail(KVQ_ERR_ARG, "kvq_cache_create_paged: pool_pages = %lld out of range", (long long)pool_pages);
+        page_shift = 0;
+        while ((int64_t(1) << page_shift) < page_bytes) ++page_shift;
+    }
     std::vector<int32_t> cap(batch), cap_pad(batch);
     std::vector<int64_t> slot_base(batch);
     int64_t slots = 0, max_items = 0;
@@ -278,7 +295,19 @@ int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group,
     int32_t *cap_d = (int32_t *)alloc(sizeof(int32_t) * batch);
     int32_t *cap_pad_d = (int32_t *)alloc(sizeof(int32_t) * batch);
     int64_t *slot_base_d = (int64_t *)alloc(sizeof(int64_t) * batch);
-    v.rec = (uint8_t *)alloc((size_t)slots * 4 * head_dim);
+    // paged: logical pages per stream, enough for the worst case (b = 16) at capacity
+    const int64_t max_lpages = paged ? ((int64_t)max_cap * 4 * head_dim + page_bytes - 1) / page_bytes + 1 : 0;
+    v.rec = (uint8_t *)alloc(paged ? (size_t)pool_pages * page_bytes : (size_t)slots * 4 * head_dim);
+    if (paged) {
+        v.ptab = (uint32_t *)alloc(sizeof(uint32_t) * (size_t)BH * max_lpages);
+        v.npages = (int32_t *)alloc(sizeof(int32_t) * BH);
+        v.pool_next = (int32_t *)alloc(sizeof(int32_t));
+        v.pool_list = (const uint32_t *)alloc(sizeof(uint32_t) * (size_t)pool_pages);
+    }
+    v.max_lpages = (int32_t)max_lpages;
+    v.pool_pages = (int32_t)pool_pages;
+    v.page_shift = (uint32_t)page_shift;
+    c->page_bytes = paged ? page_bytes : 0;
     v.meta = (uint32_t *)alloc(sizeof(uint32_t) * (size_t)slots);
     v.side = (float4 *)alloc(sizeof(float4) * (size_t)slots);
     v.len = (int32_t *)alloc(sizeof(int32_t) * BH);
@@ -296,14 +325,26 @@ int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group,
     wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * BH);
     wk.partials = (float *)alloc(sizeof(float) * (size_t)max_items * wk.qslots * (head_dim + 4));
     c->pf_max_tiles = slots * query_group / 128 + 2LL * BHQ;
-    c->pf_tiles = alloc(sizeof(int32_t) * 4 * (size_t)c->pf_max_tiles);
+    c->pf_tiles = alloc(sizeof(int32_t) * 16 * (size_t)c->pf_max_tiles);    // two lists of 32-byte tiles
     c->pf_count = (int32_t *)alloc(sizeof(int32_t));
     c->pf_qidx = (int32_t *)alloc(sizeof(int32_t) * (size_t)slots * query_group);
     for (int i = 0; i < c->n_allocs; ++i) okk = okk && c->allocs[i];
     if (!okk || c->n_allocs != n_tried) {
         kvq_cache_destroy(c);
         return fail(KVQ_ERR_NOMEM, "kvq_cache_create: cudaMalloc failed (%lld slots, %.2f GB of records)",
-                    (long long)slots, (double)slots * 4 * head_dim / 1e9);
+                    (long long)slots,
+                    (paged ? (double)pool_pages * page_bytes : (double)slots * 4 * head_dim) / 1e9);
+    }
+    // the pool hands out its pages in a scrambled order (xorshift-driven Fisher-Yates), so
+    // neighbouring logical pages are not neighbours in memory; nothing depends on the order
+    std::vector<uint32_t> plist(paged ? (size_t)pool_pages : 0);
+    for (size_t i = 0; i < plist.size(); ++i) plist[i] = (uint32_t)i;
+    uint64_t xs = 0x9E3779B97F4A7C15ull ^ (uint64_t)pool_pages;
+    for (size_t i = plist.size(); i > 1; --i) {
+        xs ^= xs << 13;
+        xs ^= xs >> 7;
+        xs ^= xs << 17;
+        std::swap(plist[i - 1], plist[xs % i]);
     }
     v.cap = cap_d;
     v.cap_pad = cap_pad_d;
@@ -320,6 +361,12 @@ int kvq_cache_create_gqa(kvq_cache **out, int batch, int heads, int query_group,
     e = e ? e : cudaMemsetAsync(v.status, 0, sizeof(int32_t), st);
     e = e ? e : cudaMemsetAsync(v.meta, 0, sizeof(uint32_t) * (size_t)slots, st);
     e = e ? e : cudaMemsetAsync(wk.count, 0, sizeof(unsigned long long), st);
+    if (paged) {
+        e = e ? e : cudaMemsetAsync(v.npages, 0, sizeof(int32_t) * BH, st);
+        e = e ? e : cudaMemsetAsync(v.pool_next, 0, sizeof(int32_t), st);
+        e = e ? e : cudaMemcpyAsync(const_cast<uint32_t *>(v.pool_list), plist.data(), sizeof(uint32_t) * plist.size(),
+                                    cudaMemcpyHostToDevice, st);
+    }
     if (!e) {
         init_side_kernel<<<1024, 256, 0, st>>>(v.side, slots);
         e = cudaGetLastError();
@@ -352,6 +399,10 @@ int kvq_cache_reset(kvq_cache *c, kvq_stream_t stream)
     cudaError_t e = cudaMemsetAsync(c->view.len, 0, sizeof(int32_t) * BH, st);
     e = e ? e : cudaMemsetAsync(c->view.end, 0, sizeof(uint32_t) * BH, st);
     e = e ? e : cudaMemsetAsync(c->view.status, 0, sizeof(int32_t), st);
+    if (c->view.ptab) {                          // every page goes back to the pool
+        e = e ? e : cudaMemsetAsync(c->view.npages, 0, sizeof(int32_t) * BH, st);
+        e = e ? e : cudaMemsetAsync(c->view.pool_next, 0, sizeof(int32_t), st);
+    }
     return e ? cuda_fail(e, "kvq_cache_reset") : ok();
 }
 

@@ -49,14 +49,32 @@
 namespace kvq {
 namespace {
 
-constexpr int kConsumerWarps = 4;
+// Launch shape of the split-K kernel (build-time tunables; the defaults are the measured
+// best on B200).
+#ifndef KVQ_DECODE_CONSUMERS
+#define KVQ_DECODE_CONSUMERS 4
+#endif
+#ifndef KVQ_DECODE_CTAS_PER_SM
+#define KVQ_DECODE_CTAS_PER_SM 3
+#endif
+#ifndef KVQ_DECODE_STAGES
+#define KVQ_DECODE_STAGES 2
+#endif
+#ifndef KVQ_DECODE_STAGE_BYTES
+#define KVQ_DECODE_STAGE_BYTES 24576
+#endif
+#ifndef KVQ_DECODE_META_SLOTS
+#define KVQ_DECODE_META_SLOTS 6
+#endif
+constexpr int kConsumerWarps = KVQ_DECODE_CONSUMERS;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kCtasPerSm = 3;
-constexpr int kStages = 2;                        // record stages in flight per CTA
+constexpr int kCtasPerSm = KVQ_DECODE_CTAS_PER_SM;
+constexpr int kStages = KVQ_DECODE_STAGES;        // record stages in flight per CTA
 constexpr int kWin = kDecodeWindowKeys;           // keys per window of record offsets
-constexpr uint32_t kStageRecBytes = 24576;        // record bytes per stage, at most
+constexpr uint32_t kStageRecBytes = KVQ_DECODE_STAGE_BYTES;   // record bytes per stage, at most
 constexpr int kPermSlots = kWin + 64;             // width-sorted keys padded to whole chunks
-constexpr int kMetaSlots = 6;                     // windows of record offsets fetched ahead
+constexpr int kMetaSlots = KVQ_DECODE_META_SLOTS; // windows of record offsets fetched ahead
+static_assert(kStageRecBytes <= 32768, "stage offsets are 15 bits");
 constexpr int kMetaWords = kWin + 8;
 constexpr int kNewItem = 1, kLastSub = 2;         // stage flags
 constexpr uint32_t kReadEndFromMeta = 0xFFFFFFFFu;
@@ -93,7 +111,7 @@ struct AppendArgs {
 template <int D>
 struct Stage {
     // width-sorted keys in chunks of one width: kValid | (key << 16) | offset in rec;
-    // padding entries are 0
+    // padding entries are a key of the same width without kValid
     uint32_t perm[kPermSlots];
     int32_t info[8];         // item index, keys in the stage, flags, chunks, qinfo
     int32_t cls_chunk[8];    // first chunk of each width class (b = 2, 4, 8, 16), [4] = chunks
@@ -430,7 +448,7 @@ __device__ __forceinline__ void merge_state(KeyState &st, int mask)
 
 // One chunk: a key per LPK-lane group, all of width class CLS (warp-uniform): K dot product
 // on the codes, logit, online-softmax update of the group's state, V accumulation.
-// Padding entries (no valid bit) read the stage's first bytes and get weight 0.
+// Padding entries (no valid bit) read a real record of the same width and get weight 0.
 template <int D, int CLS>
 __device__ __forceinline__ void process_chunk(KeyState &st, const QRegs &Q, float qsum_l, float cdot,
                                               const Stage<D> &sg, uint32_t ent, int li)
@@ -507,27 +525,30 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         // memory, cuts it into stages of at most kStageRecBytes, sorts each stage's keys by
         // width and issues the stage's copies. On a timed-out wait it stops issuing, waits
         // (bounded) for the copies already in flight and returns.
-        constexpr int KPL = kWin / 32;                // window keys per lane: lane + 32 r
+        // A window's record offsets sit in slots 0..131 of its ring entry, key ja + i in slot
+        // i (ja = the window's first key rounded down to a multiple of 4); lane l holds
+        // slots 4l .. 4l + 3 (one 16-byte shared load). Windows after an item's first end
+        // on 4-aligned keys, so a window's keys fit slots [d, d + nwin) with d + nwin <= 128.
         int f_it = blockIdx.x;
         if (f_it >= n_items) return;
         DecodeItem f_d = wk.items[f_it];
         int f_j = f_d.j0;
         bool f_valid = true, aborted = false;
         int filled = 0, consumed = 0, issued = 0;
-        const uint32_t lt = (1u << lane) - 1u;
         while (!aborted) {
             while (f_valid && filled < consumed + kMetaSlots) {
                 const int slot = filled % kMetaSlots;
                 MetaSlot &ms = sm.ms[slot];
                 const int ja = f_j & ~3;
-                const int jb = (min(f_j + kWin + 1, f_d.j1 + 1) + 3) & ~3;
+                const int nwin = min(kWin - (f_j - ja), f_d.j1 - f_j);
+                const int jb = (f_j + nwin + 1 + 3) & ~3;    // includes the key after the window
                 if (lane == 0) {
                     ms.it = f_it;
                     ms.j = f_j;
-                    ms.j1 = f_d.j1;
+                    ms.j1 = f_j + nwin;
                     ms.ja = ja;
-                    ms.end_off = f_d.end_off;
-                    ms.first = (f_j == f_d.j0);
+                    ms.end_off = (f_j + nwin == f_d.j1) ? f_d.end_off : kReadEndFromMeta;
+                    ms.first = (f_j == f_d.j0) | ((f_j + nwin == f_d.j1) ? 2 : 0);
                     ms.sbase = f_d.sbase;
                     ms.sh = f_d.sh;
                     ms.qinfo = f_d.qinfo;
@@ -536,7 +557,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     bulk_g2s(ms.meta, c.meta + f_d.sbase + ja, 4u * (uint32_t)(jb - ja), &sm.mfull[slot]);
                 }
                 ++filled;
-                f_j += kWin;
+                f_j += nwin;
                 if (f_j >= f_d.j1) {
                     f_it += gridDim.x;
                     if (f_it < n_items) {
@@ -554,74 +575,80 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 break;
             }
             const MetaSlot &ms = sm.ms[slot];
-            const int j = ms.j, it = ms.it, qinfo = ms.qinfo;
-            const int nwin = min(kWin, ms.j1 - j);
-            const bool lastwin = (j + nwin == ms.j1), first = ms.first != 0;
-            const uint32_t *mw = ms.meta + (j - ms.ja);
-            uint32_t m[KPL], nx[KPL];
-#pragma unroll
-            for (int r = 0; r < KPL; ++r) m[r] = (lane + 32 * r < nwin) ? mw[lane + 32 * r] : 0u;
-            const uint32_t bnd = ((!lastwin || ms.end_off == kReadEndFromMeta) ? mw[nwin] : ms.end_off) & ~15u;
+            const int it = ms.it, qinfo = ms.qinfo, ja = ms.ja;
+            const int d = ms.j - ja, dend = ms.j1 - ja;       // the window's keys: slots [d, dend)
+            const bool first = (ms.first & 1) != 0, lastwin = (ms.first & 2) != 0;
+            const uint4 mv = reinterpret_cast<const uint4 *>(ms.meta)[lane];
+            const uint32_t m[4] = {mv.x, mv.y, mv.z, mv.w};
+            const uint32_t bnd = (ms.end_off == kReadEndFromMeta ? ms.meta[dend] : ms.end_off) & ~15u;
             const int64_t sbase = ms.sbase;
             const int sh = ms.sh;
-            // nx[r]: offset right after key lane + 32 r (the next key's offset, or the bound)
+            // nx[r]: the offset right after the key in slot 4 lane + r (the next key's offset,
+            // or the bound after the window's last key)
+            uint32_t nx[4];
+            const uint32_t next_lane = __shfl_down_sync(0xffffffffu, m[0], 1);
 #pragma unroll
-            for (int r = 0; r < KPL; ++r) {
-                const uint32_t dn = __shfl_down_sync(0xffffffffu, m[r], 1) & ~15u;
-                const uint32_t wrap = (r + 1 < KPL) ? (__shfl_sync(0xffffffffu, m[(r + 1) % KPL], 0) & ~15u) : bnd;
-                nx[r] = (lane == 31) ? wrap : dn;
-                if (lane + 32 * r + 1 >= nwin) nx[r] = bnd;
+            for (int r = 0; r < 4; ++r) {
+                const int sl = 4 * lane + r;
+                nx[r] = (sl + 1 == dend) ? bnd : ((r < 3 ? m[(r + 1) & 3] : next_lane) & ~15u);
             }
             ++consumed;
 
-            for (int w0 = 0; w0 < nwin;) {
-                // the stage: keys [w0, w1) of the window, at most kStageRecBytes of records
-                const uint32_t mstart = __shfl_sync(0xffffffffu, (w0 / 32 == 0) ? m[0] : (w0 / 32 == 1) ? m[1 % KPL]
-                                                                   : (w0 / 32 == 2) ? m[2 % KPL] : m[3 % KPL], w0 & 31);
-                const uint32_t off0 = mstart & ~15u;
-                int n = 0;
+            for (int s0 = d; s0 < dend;) {
+                // the stage: slots [s0, s1), at most kStageRecBytes of records and (paged
+                // caches) bytes in at most two pages
+                const int r0 = s0 & 3;
+                const uint32_t off0 = __shfl_sync(0xffffffffu, r0 == 0 ? m[0] : r0 == 1 ? m[1] : r0 == 2 ? m[2] : m[3],
+                                                  s0 >> 2) & ~15u;
+                const uint32_t plast = (off0 >> c.page_shift) + 1u;
+                uint32_t cnt = 0;
 #pragma unroll
-                for (int r = 0; r < KPL; ++r) {
-                    const int k = lane + 32 * r;
-                    n += __popc(__ballot_sync(0xffffffffu, k >= w0 && k < nwin && nx[r] - off0 <= kStageRecBytes));
+                for (int r = 0; r < 4; ++r) {
+                    const int sl = 4 * lane + r;
+                    cnt += (sl >= s0 && sl < dend && nx[r] - off0 <= kStageRecBytes &&
+                            ((nx[r] - 1u) >> c.page_shift) <= plast) ? 1u : 0u;
                 }
+                int n = (int)__reduce_add_sync(0xffffffffu, cnt);
                 if (n < 1) {          // only with corrupt offsets: flag it, keep making progress
                     if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
                     n = 1;
                 }
-                const int w1 = w0 + n;
-                const int kl = w1 - 1;
-                const uint32_t nxl = __shfl_sync(0xffffffffu, (kl / 32 == 0) ? nx[0] : (kl / 32 == 1) ? nx[1 % KPL]
-                                                             : (kl / 32 == 2) ? nx[2 % KPL] : nx[3 % KPL], kl & 31);
-                const bool last = lastwin && w1 == nwin;
-                const bool new_item = first && w0 == 0;
+                const int s1 = s0 + n;
+                const int kl = s1 - 1, rl = kl & 3;
+                const uint32_t nxl = __shfl_sync(0xffffffffu, rl == 0 ? nx[0] : rl == 1 ? nx[1] : rl == 2 ? nx[2] : nx[3],
+                                                 kl >> 2);
+                const bool last = lastwin && s1 == dend;
+                const bool new_item = first && s0 == d;
                 uint32_t rec_bytes = nxl - off0;
                 if (nxl < off0 || rec_bytes > kStageRecBytes) {   // corrupt offsets
                     if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
                     rec_bytes = 0;
                 }
-                // counting sort by width, each width's run padded to whole chunks of KPS keys
-                int cl_of[KPL], pos_of[KPL];
+                // counting sort by width: per-lane counts of the four classes packed in one
+                // word (8 bits each), one warp prefix sum; each class's run padded to whole
+                // chunks of KPS keys
+                uint32_t lc = 0;
 #pragma unroll
-                for (int r = 0; r < KPL; ++r) {
-                    const int k = lane + 32 * r;
-                    cl_of[r] = (k >= w0 && k < w1) ? (int)(m[r] & 3u) : 4;
-                    pos_of[r] = 0;
+                for (int r = 0; r < 4; ++r) {
+                    const int sl = 4 * lane + r;
+                    if (sl >= s0 && sl < s1) lc += 1u << (8 * (m[r] & 3u));
                 }
-                int pstart = 0, cls_chunk[4], pad_at[4], pad_n[4];
+                uint32_t incl = lc;
+#pragma unroll
+                for (int dd = 1; dd < 32; dd <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, dd);
+                    if (lane >= dd) incl += y;
+                }
+                const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+                uint32_t run = incl - lc;               // this lane's first rank in each class
+                int cstart[4], pad_at[4], pad_n[4], pstart = 0;
 #pragma unroll
                 for (int cl = 0; cl < 4; ++cl) {
-                    cls_chunk[cl] = pstart / KPS;
-                    int before = 0;
-#pragma unroll
-                    for (int r = 0; r < KPL; ++r) {
-                        const uint32_t b = __ballot_sync(0xffffffffu, cl_of[r] == cl);
-                        if (cl_of[r] == cl) pos_of[r] = pstart + before + __popc(b & lt);
-                        before += __popc(b);
-                    }
-                    const int padded = (before + KPS - 1) / KPS * KPS;
-                    pad_at[cl] = pstart + before;
-                    pad_n[cl] = padded - before;
+                    const int tc = (int)((tot >> (8 * cl)) & 0xFFu);
+                    const int padded = (tc + KPS - 1) / KPS * KPS;
+                    cstart[cl] = pstart;
+                    pad_at[cl] = pstart + tc;
+                    pad_n[cl] = padded - tc;
                     pstart += padded;
                 }
 
@@ -633,18 +660,25 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 }
                 Stage<D> &sg = sm.st[stage];
 #pragma unroll
-                for (int r = 0; r < KPL; ++r) {
-                    if (cl_of[r] < 4) {
+                for (int r = 0; r < 4; ++r) {
+                    const int sl = 4 * lane + r;
+                    if (sl >= s0 && sl < s1) {
+                        const uint32_t cl = m[r] & 3u;
+                        const int start = cl == 0 ? cstart[0] : cl == 1 ? cstart[1] : cl == 2 ? cstart[2] : cstart[3];
+                        const int pos = start + (int)((run >> (8 * cl)) & 0xFFu);
+                        run += 1u << (8 * cl);
                         // offset inside the stage; the clamp only bites on corrupt offsets and
                         // keeps every shared-memory read of the consumers inside the stage
-                        const uint32_t ro = min((m[r] & ~15u) - off0,
-                                                kStageRecBytes - (uint32_t)(D * (2 << cl_of[r])) / 4u);
-                        sg.perm[pos_of[r]] = kValid | ((uint32_t)(lane + 32 * r - w0) << 16) | ro;
+                        const uint32_t ro = min((m[r] & ~15u) - off0, kStageRecBytes - (uint32_t)(D * (2 << cl)) / 4u);
+                        sg.perm[pos] = kValid | ((uint32_t)(sl - s0) << 16) | ro;
                     }
                 }
+                // padding entries repeat the first key of their class without the valid bit:
+                // the consumers read finite data of the right width there and weight it 0
+                __syncwarp();
 #pragma unroll
                 for (int cl = 0; cl < 4; ++cl)
-                    if (lane < pad_n[cl]) sg.perm[pad_at[cl] + lane] = 0u;
+                    if (lane < pad_n[cl]) sg.perm[pad_at[cl] + lane] = sg.perm[cstart[cl]] & ~kValid;
                 if (lane == 0) {
                     sg.info[0] = it;
                     sg.info[1] = n;
@@ -652,7 +686,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     sg.info[3] = pstart / KPS;
                     sg.info[4] = qinfo;
 #pragma unroll
-                    for (int cl = 0; cl < 4; ++cl) sg.cls_chunk[cl] = cls_chunk[cl];
+                    for (int cl = 0; cl < 4; ++cl) sg.cls_chunk[cl] = cstart[cl] / KPS;
                     sg.cls_chunk[4] = pstart / KPS;
                 }
                 __syncwarp();
@@ -663,14 +697,20 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     const uint32_t q_bytes = new_item ? (uint32_t)(2 * D * nq) : 0u;
                     const int s_of = sh / c.H, hk = sh % c.H;
                     mbar_arrive_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
-                    bulk_g2s(sg.side, c.side + sbase + j + w0, 16u * n, &sm.full[stage]);
-                    if (rec_bytes)
-                        bulk_g2s(sg.rec, c.rec + sbase * (int64_t)(4 * D) + off0, rec_bytes, &sm.full[stage]);
+                    bulk_g2s(sg.side, c.side + sbase + ja + s0, 16u * n, &sm.full[stage]);
+                    if (rec_bytes) {
+                        const RecLoc L = rec_loc(c, s_of, hk, 0);
+                        // a paged stream: one copy per page the stage's bytes touch
+                        const uint32_t n0 = L.pt ? min(rec_bytes, (((off0 >> c.page_shift) + 1u) << c.page_shift) - off0)
+                                                 : rec_bytes;
+                        bulk_g2s(sg.rec, L.at(off0), n0, &sm.full[stage]);
+                        if (rec_bytes > n0) bulk_g2s(sg.rec + n0, L.at(off0 + n0), rec_bytes - n0, &sm.full[stage]);
+                    }
                     if (q_bytes)
                         bulk_g2s(sg.q, q + ((int64_t)s_of * HQ + hk * c.G + g0) * D, q_bytes, &sm.full[stage]);
                 }
                 ++issued;
-                w0 = w1;
+                s0 = s1;
             }
         }
         if (aborted) {

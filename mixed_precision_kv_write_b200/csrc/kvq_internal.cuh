@@ -12,6 +12,13 @@
 //   len/end  per (s, h): tokens held and the stream's end offset in bytes.
 // Slots: slot(s, h, j) = slot_base[s] + h * cap_pad[s] + j, cap_pad a multiple of 4 that
 // leaves at least one spare slot, so 16-byte bulk copies of meta may round to 4 slots.
+// Record bytes, contiguous cache: stream (s, h) starts at byte slot(s, h, 0) * 4 * D of
+// `rec`, with room for the worst case. Paged cache: `rec` is a pool of fixed-size pages
+// (2^page_shift bytes); stream (s, h) is a sequence of logical pages, logical page lp at
+// physical page ptab[(s * H + h) * max_lpages + lp]. Pages are taken from the pool when a
+// write first reaches them (pool_list[pool_next ..], in the order the pool hands them
+// out) and stay with (s, h) until kvq_cache_reset. Offsets inside a stream are the same in
+// both layouts; a record may straddle two pages (every 16-byte chunk lies in one page).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -39,6 +46,13 @@ struct CacheView {
     uint32_t *wend;           // [B*H] stream end after the current write
     uint32_t *bad;            // [B] id of the last write call that saw a bad width
     int32_t *status;          // [1] first device-side error (kvq_status), 0 = none
+    // paged record storage (ptab == nullptr: contiguous streams)
+    uint32_t *ptab;           // [B*H][max_lpages] physical page of each logical page
+    int32_t *npages;          // [B*H] logical pages mapped
+    int32_t *pool_next;       // [1] pages handed out since the last reset
+    const uint32_t *pool_list;// [pool_pages] the order in which the pool hands out pages
+    int32_t max_lpages, pool_pages;
+    uint32_t page_shift;      // log2 of the page size (31 for contiguous caches)
 };
 
 __device__ __forceinline__ int64_t slot_of(const CacheView &c, int s, int h, int64_t j)
@@ -49,6 +63,62 @@ __device__ __forceinline__ int64_t slot_of(const CacheView &c, int s, int h, int
 __device__ __forceinline__ uint8_t *stream_of(const CacheView &c, int s, int h)
 {
     return c.rec + slot_of(c, s, h, 0) * (int64_t)(4 * c.D);
+}
+
+// Locator of record bytes of one stream: at(rel) is the address of logical byte off + rel.
+// A chunk of up to 16 bytes at a 16-byte aligned logical offset never straddles a page.
+struct RecLoc {
+    uint8_t *base;            // contiguous: stream + off; paged: the pool
+    const uint32_t *pt;       // paged: the stream's page table row; contiguous: nullptr
+    uint32_t off, shift;
+    __device__ __forceinline__ uint8_t *at(uint32_t rel) const
+    {
+        if (!pt) return base + rel;
+        const uint32_t o = off + rel;
+        return base + ((size_t)pt[o >> shift] << shift) + (o & ((1u << shift) - 1u));
+    }
+};
+
+__device__ __forceinline__ RecLoc rec_loc(const CacheView &c, int s, int h, uint32_t off)
+{
+    RecLoc r;
+    if (c.ptab) {
+        r.base = c.rec;
+        r.pt = c.ptab + (size_t)(s * c.H + h) * c.max_lpages;
+        r.off = off;
+        r.shift = c.page_shift;
+    } else {
+        r.base = stream_of(c, s, h) + off;
+        r.pt = nullptr;
+        r.off = 0;
+        r.shift = 0;
+    }
+    return r;
+}
+
+// Paged caches: give (s, h) physical pages for every logical page that a stream end of
+// end_bytes reaches (one thread per (s, h)). Returns false, mapping nothing, when the
+// pool has too few pages left. Contiguous caches: always true.
+__device__ __forceinline__ bool map_pages(const CacheView &c, int s, int h, uint32_t end_bytes)
+{
+    if (!c.ptab) return true;
+    const int sh = s * c.H + h;
+    const int need = (int)(((uint64_t)end_bytes + (1u << c.page_shift) - 1u) >> c.page_shift);
+    const int have = c.npages[sh];
+    if (need <= have) return true;
+    if (need > c.max_lpages) return false;
+    const int k = need - have;
+    int old = *reinterpret_cast<volatile int32_t *>(c.pool_next);
+    while (true) {
+        if (old + k > c.pool_pages) return false;
+        const int prev = atomicCAS(c.pool_next, old, old + k);
+        if (prev == old) break;
+        old = prev;
+    }
+    uint32_t *pt = c.ptab + (size_t)sh * c.max_lpages;
+    for (int i = 0; i < k; ++i) pt[have + i] = c.pool_list[old + i];
+    c.npages[sh] = need;
+    return true;
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -64,7 +134,10 @@ __device__ __forceinline__ void set_status(int32_t *status, int code)
 }
 
 // ---- scheduler work list (decode) ----------------------------------------------------
-constexpr int kDecodeItemKeys = 576;   // keys per split-K work item, at most (w + 1 = 513 fits one)
+#ifndef KVQ_DECODE_ITEM_KEYS
+#define KVQ_DECODE_ITEM_KEYS 576
+#endif
+constexpr int kDecodeItemKeys = KVQ_DECODE_ITEM_KEYS;   // keys per split-K work item, at most (w + 1 = 513 fits one)
 constexpr int kDecodeWindowKeys = 128; // keys per window of record offsets inside an item
 constexpr int kDecodeMaxQ = 4;         // query heads served by one item (a subgroup of a GQA group)
 
@@ -227,11 +300,12 @@ struct kvq_cache {
     kvq::DecodeWork work;
     uint32_t write_gen;       // id of the last kvq_write call
     uint32_t decode_gen;      // id of the last decode call on the cache's own work list
-    void *pf_tiles;           // prefill tile list (PfTile = 4 x int32), pf_max_tiles entries
+    void *pf_tiles;           // prefill tile lists (PfTile = 8 x int32): as listed, then ordered
     int32_t *pf_count;        // [1]
     int32_t *pf_qidx;         // [total_slots] per-(sequence, head) query lists
     int64_t pf_max_tiles;
-    void *allocs[24];
+    int64_t page_bytes;       // 0: contiguous streams
+    void *allocs[32];
     int n_allocs;
 };
 

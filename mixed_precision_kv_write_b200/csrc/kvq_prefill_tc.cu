@@ -168,6 +168,7 @@ __device__ __forceinline__ float ex2(float x)
 
 struct PfTile {
     int32_t sh, mode, start, count;   // (sequence, head), mode, first list entry, queries
+    int32_t nkeys, pad[3];            // keys the tile's range spans (its work, for ordering)
 };
 
 template <int D>
@@ -203,7 +204,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     const int n_s = cu[s + 1] - cu[s];
     const int pos0 = c.len[s * c.H + hk] - n_s;
     const int64_t sbase = slot_of(c, s, hk, 0);
-    const uint8_t *stream = stream_of(c, s, hk);
+    const RecLoc stream = rec_loc(c, s, hk, 0);
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -359,17 +360,17 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             if (t < n_kt && mt != kNone) {
                 const int bits = 2 << (mt & 3u);
                 const uint32_t part = (uint32_t)(CH * bits / 8);          // bytes of this half
-                const uint8_t *rk = stream + (mt & ~15u) + half * part;
-                const uint8_t *rv = stream + (mt & ~15u) + (uint32_t)(bits * D / 8) + half * part;
+                const uint32_t ok = (mt & ~15u) + half * part;               // stream offsets
+                const uint32_t ov = (mt & ~15u) + (uint32_t)(bits * D / 8) + half * part;
                 uint8_t *dst = sm.raw[t & 1][u];
                 if (part >= 16) {
                     for (uint32_t o = 0; o < part; o += 16) {
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + o)), "l"(rk + o) : "memory");
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + D + o)), "l"(rv + o) : "memory");
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + o)), "l"(stream.at(ok + o)) : "memory");
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + D + o)), "l"(stream.at(ov + o)) : "memory");
                     }
                 } else {                                                   // 8 bytes (head_dim 64, b = 2)
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(rk) : "memory");
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst + D)), "l"(rv) : "memory");
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(stream.at(ok)) : "memory");
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst + D)), "l"(stream.at(ov)) : "memory");
                 }
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
@@ -551,7 +552,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
 constexpr int kSchedThreads = 1024, kSchedPer = 4;
 
 __global__ void __launch_bounds__(kSchedThreads)
-prefill_sched_kernel(CacheView c, const uint8_t *__restrict__ modes, const int32_t *__restrict__ cu,
+prefill_sched_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, const int32_t *__restrict__ cu,
                      int64_t n_tok, int D, float *__restrict__ out, PfTile *__restrict__ tiles,
                      int32_t *__restrict__ tile_count, int32_t *__restrict__ qidx)
 {
@@ -641,12 +642,52 @@ prefill_sched_kernel(CacheView c, const uint8_t *__restrict__ modes, const int32
         const int ntl = (tot_l + kQRows - 1) / kQRows, ntf = (tot_f + kQRows - 1) / kQRows;
         const int first = atomicAdd(tile_count, ntl + ntf);
         const int32_t off = (int32_t)(t0 * H + (int64_t)h * n);
-        for (int k = 0; k < ntl; ++k)
-            tiles[first + k] = PfTile{sh, KVQ_MODE_LOCAL, off + k * kQRows, min(kQRows, tot_l - k * kQRows)};
-        for (int k = 0; k < ntf; ++k)
-            tiles[first + ntl + k] = PfTile{sh, KVQ_MODE_FULL, off + n - tot_f + k * kQRows,
-                                            min(kQRows, tot_f - k * kQRows)};
+        const int pos0 = c.len[s * c.H + h / c.G] - n;
+        // local list: query indices ascending; full list (from the back): descending
+        for (int k = 0; k < ntl; ++k) {
+            const int cnt = min(kQRows, tot_l - k * kQRows);
+            const int t_lo = pos0 + region[k * kQRows], t_hi = pos0 + region[k * kQRows + cnt - 1];
+            tiles[first + k] = PfTile{sh, KVQ_MODE_LOCAL, off + k * kQRows, cnt, t_hi - max(0, t_lo - w) + 1, {0, 0, 0}};
+        }
+        for (int k = 0; k < ntf; ++k) {
+            const int st = n - tot_f + k * kQRows;
+            tiles[first + ntl + k] = PfTile{sh, KVQ_MODE_FULL, off + st, min(kQRows, tot_f - k * kQRows),
+                                            pos0 + region[st] + 1, {0, 0, 0}};
+        }
     }
+}
+
+// Longest tile first: one CTA orders the tile list by the keys each tile spans
+// (descending, in buckets of 64 keys), so the long full-range tiles start in the first
+// wave and the short ones fill in behind them.
+constexpr int kSortBuckets = 1024;
+
+__global__ void __launch_bounds__(1024)
+prefill_order_kernel(const PfTile *__restrict__ in, const int32_t *__restrict__ tile_count, PfTile *__restrict__ out)
+{
+    __shared__ int hist[kSortBuckets];
+    const int n = *tile_count, tid = threadIdx.x;
+    for (int b = tid; b < kSortBuckets; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    auto bucket = [](int nkeys) { return kSortBuckets - 1 - min(kSortBuckets - 1, (nkeys + 63) / 64); };
+    for (int i = tid; i < n; i += blockDim.x) atomicAdd(&hist[bucket(in[i].nkeys)], 1);
+    __syncthreads();
+    if (tid < 32) {                              // exclusive prefix over the buckets, one warp
+        int carry = 0;
+        for (int b0 = 0; b0 < kSortBuckets; b0 += 32) {
+            const int x = hist[b0 + tid];
+            int incl = x;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, d);
+                if (tid >= d) incl += y;
+            }
+            hist[b0 + tid] = carry + incl - x;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += blockDim.x) out[atomicAdd(&hist[bucket(in[i].nkeys)], 1)] = in[i];
 }
 
 template <int D>
@@ -655,16 +696,18 @@ cudaError_t run_tc(const kvq_cache *cache, const __half *q, const uint8_t *modes
 {
     const CacheView &c = cache->view;
     PfTile *tiles = reinterpret_cast<PfTile *>(cache->pf_tiles);
+    PfTile *ordered = tiles + cache->pf_max_tiles;
     cudaError_t e = cudaMemsetAsync(cache->pf_count, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return e;
-    prefill_sched_kernel<<<c.B * c.H * c.G, kSchedThreads, 0, st>>>(c, modes, cu, n_tok, D, out, tiles, cache->pf_count,
-                                                     cache->pf_qidx);
+    prefill_sched_kernel<<<c.B * c.H * c.G, kSchedThreads, 0, st>>>(c, modes, w, cu, n_tok, D, out, tiles,
+                                                                    cache->pf_count, cache->pf_qidx);
+    prefill_order_kernel<<<1, 1024, 0, st>>>(tiles, cache->pf_count, ordered);
     const int64_t max_tiles = n_tok * c.H * c.G / kQRows + 2LL * c.B * c.H * c.G;
     const size_t smem = sizeof(PfSmem<D>) + 1024;
     e = ensure_smem_attr((const void *)prefill_tc_kernel<D>, smem);
     if (e != cudaSuccess) return e;
     profile_before(st);
-    prefill_tc_kernel<D><<<(unsigned)max_tiles, kTcThreads, smem, st>>>(c, q, w, cu, tiles, cache->pf_count,
+    prefill_tc_kernel<D><<<(unsigned)max_tiles, kTcThreads, smem, st>>>(c, q, w, cu, ordered, cache->pf_count,
                                                                         cache->pf_qidx, out);
     profile_after(st);
     return cudaGetLastError();

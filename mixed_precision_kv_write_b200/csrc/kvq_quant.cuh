@@ -26,7 +26,7 @@ constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 // BITS * (j * VL + li), and the VL lanes of a vector store adjacent chunks.
 template <int BITS, int NC, int VL>
 __device__ __forceinline__ void quant_store(const uint4 (&raw)[NC], float z, float sc,
-                                            uint8_t *dst, int li)
+                                            const RecLoc &dst, int li)
 {
     uint32_t w[NC][2];
 #pragma unroll
@@ -77,9 +77,10 @@ __device__ __forceinline__ void quant_store(const uint4 (&raw)[NC], float z, flo
 #pragma unroll
     for (int j = 0; j < NC; ++j) {
         const int chunk = j * VL + li;
-        if (BITS == 8) reinterpret_cast<uint2 *>(dst)[chunk] = make_uint2(w[j][0], w[j][1]);
-        else if (BITS == 4) reinterpret_cast<uint32_t *>(dst)[chunk] = w[j][0];
-        else reinterpret_cast<uint16_t *>(dst)[chunk] = (uint16_t)w[j][0];
+        uint8_t *d = dst.at((uint32_t)(BITS * chunk));
+        if (BITS == 8) *reinterpret_cast<uint2 *>(d) = make_uint2(w[j][0], w[j][1]);
+        else if (BITS == 4) *reinterpret_cast<uint32_t *>(d) = w[j][0];
+        else *reinterpret_cast<uint16_t *>(d) = (uint16_t)w[j][0];
     }
 }
 
@@ -110,12 +111,12 @@ __device__ __forceinline__ __half2 vec_minmax(const uint4 (&raw)[NC])
 // for b = 16) and, from the vector's first lane, its (s, z) side entry.
 template <int NC, int VL>
 __device__ __forceinline__ void vec_store(const CacheView &c, const uint4 (&raw)[NC], __half2 mm, int b,
-                                          uint8_t *dst, int64_t slot, int part, int li)
+                                          const RecLoc &dst, int64_t slot, int part, int li)
 {
     float sc = 1.0f, z = 0.0f;
     if (b == 16) {
 #pragma unroll
-        for (int j = 0; j < NC; ++j) reinterpret_cast<uint4 *>(dst)[j * VL + li] = raw[j];
+        for (int j = 0; j < NC; ++j) *reinterpret_cast<uint4 *>(dst.at(16u * (j * VL + li))) = raw[j];
     } else {
         const float mn = __low2float(mm), mx = -__high2float(mm);
         const float top = (float)((1u << b) - 1u);
@@ -200,8 +201,12 @@ __device__ __forceinline__ void append_seq(const CacheView &c, const __half *__r
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&bad_sh, 1);
         if (lane == 0) {
-            c.wstart[sh] = L0;
-            c.wend[sh] = off;
+            if (map_pages(c, s, h, off)) {       // paged caches: pages for the new bytes
+                c.wstart[sh] = L0;
+                c.wend[sh] = off;
+            } else {
+                set_status(c.status, KVQ_ERR_CAPACITY);
+            }
         }
     }
     __syncthreads();
@@ -230,7 +235,7 @@ __device__ __forceinline__ void append_seq(const CacheView &c, const __half *__r
         const int64_t slot = slot_of(c, s, h, st + i);
         const uint32_t meta = c.meta[slot];
         const int b = 2 << (meta & 3u);
-        vec_store<1, VL>(c, raw, mm, b, stream_of(c, s, h) + (meta & ~15u) + part * (b * D / 8), slot, part, li);
+        vec_store<1, VL>(c, raw, mm, b, rec_loc(c, s, h, (meta & ~15u) + part * (b * D / 8)), slot, part, li);
     }
     __syncthreads();
     for (int h = tid; h < H; h += blockDim.x) {  // commit the new lengths and stream ends

@@ -120,8 +120,13 @@ write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *
         set_status(c.status, KVQ_ERR_BITS);
     }
     if (tid == 0) {
-        c.wstart[sh] = L0;
-        c.wend[sh] = off;
+        if (map_pages(c, s, h, off)) {           // paged caches: pages for the new bytes
+            c.wstart[sh] = L0;
+            c.wend[sh] = off;
+        } else {
+            set_status(c.status, KVQ_ERR_CAPACITY);
+            c.wstart[sh] = -1;
+        }
     }
 }
 
@@ -133,9 +138,10 @@ constexpr int kWqMaxPairs = kWqHalves / 64;
 
 struct WqPair {                          // one (token, head) of the CTA
     int64_t slot;                        // side-table slot
-    int64_t rec;                         // byte offset of the record in the record array
-    uint32_t meta;                       // width code in bits 0-1
-    int32_t ok;                          // 0: not written (rejected write or bad call)
+    uint32_t meta;                       // record offset in the stream | width code
+    int32_t s;                           // sequence; -1: not written (rejected write or bad call)
+    int32_t h;
+    int32_t pad;
 };
 
 // One CTA per tile of T tokens x HG heads. Warp 0 starts two bulk copies (the tile's K and
@@ -193,9 +199,10 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
         const int h = h0 + i % HGc;
         WqPair pr;
         pr.slot = 0;
-        pr.rec = 0;
         pr.meta = 0;
-        pr.ok = 0;
+        pr.s = -1;
+        pr.h = h;
+        pr.pad = 0;
         int lo = 0, hi = c.B;                // cu[lo] <= tk < cu[hi]
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
@@ -209,8 +216,7 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
                 const int64_t t_in_seq = tk - cu[s];
                 pr.slot = slot_of(c, s, h, st + t_in_seq);
                 pr.meta = c.meta[pr.slot];
-                pr.rec = slot_of(c, s, h, 0) * (int64_t)(4 * D) + (pr.meta & ~15u);
-                pr.ok = 1;
+                pr.s = s;
                 if (t_in_seq == 0) {          // commit the new length and stream end
                     c.len[s * H + h] = st + (cu[s + 1] - cu[s]);
                     c.end[s * H + h] = c.wend[s * H + h];
@@ -227,7 +233,7 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
         for (int cls = 0; cls < 4; ++cls) {
             for (int i0 = 0; i0 < n_pairs; i0 += 32) {
                 const int i = i0 + lane;
-                const bool in = i < n_pairs && pairs[i].ok && (int)(pairs[i].meta & 3u) == cls;
+                const bool in = i < n_pairs && pairs[i].s >= 0 && (int)(pairs[i].meta & 3u) == cls;
                 const uint32_t m = __ballot_sync(0xffffffffu, in);
                 if (in) order[base + __popc(m & ((1u << lane) - 1u))] = (uint8_t)i;
                 base += __popc(m);
@@ -256,7 +262,8 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
         if (!in_range) continue;
         const WqPair pr = pairs[pi];
         const int b = 2 << (pr.meta & 3u);
-        vec_store<NC, VL>(c, raw, mm, b, c.rec + pr.rec + part * (b * D / 8), pr.slot, part, li);
+        vec_store<NC, VL>(c, raw, mm, b, rec_loc(c, pr.s, pr.h, (pr.meta & ~15u) + part * (b * D / 8)), pr.slot,
+                          part, li);
     }
 }
 

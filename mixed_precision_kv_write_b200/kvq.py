@@ -20,7 +20,7 @@ KVQ_OK, KVQ_ERR_ARG, KVQ_ERR_BITS, KVQ_ERR_MODE, KVQ_ERR_CAPACITY, KVQ_ERR_CUDA,
 MODE_SKIP, MODE_LOCAL, MODE_FULL = 0, 1, 2
 
 # every symbol include/kvq.h declares
-EXPORTS = ("kvq_cache_create", "kvq_cache_create_gqa", "kvq_cache_destroy", "kvq_cache_reset", "kvq_cache_truncate",
+EXPORTS = ("kvq_cache_create", "kvq_cache_create_gqa", "kvq_cache_create_paged", "kvq_cache_destroy", "kvq_cache_reset", "kvq_cache_truncate",
            "kvq_cache_lengths", "kvq_write", "routed_attn_prefill", "routed_attn_decode",
            "routed_attn_decode_noalloc", "kvq_decode_step", "kvq_cache_export", "kvq_check", "kvq_set_profile_events",
            "kvq_route_argmax", "kvq_test_fail_alloc", "kvq_test_bounded_wait", "kvq_last_error")
@@ -47,6 +47,7 @@ def load_library(path: str = LIB_PATH):
     sig = {
         "kvq_cache_create": ([ctypes.POINTER(vp), i32, i32, i32, vp, vp], i32),
         "kvq_cache_create_gqa": ([ctypes.POINTER(vp), i32, i32, i32, i32, vp, vp], i32),
+        "kvq_cache_create_paged": ([ctypes.POINTER(vp), i32, i32, i32, i32, vp, i64, i64, vp], i32),
         "kvq_cache_destroy": ([vp], i32),
         "kvq_cache_reset": ([vp, vp], i32),
         "kvq_cache_truncate": ([vp, vp, vp], i32),
@@ -104,7 +105,7 @@ class KVQCache:
     """Owning handle of a routed mixed-precision KV cache (kvq_cache_create/destroy)."""
 
     def __init__(self, batch: int, heads: int, head_dim: int, capacity, device=None, stream=None,
-                 query_group: int = 1):
+                 query_group: int = 1, page_bytes: int = 0, pool_pages: int = 0):
         lib = load_library()
         dev = torch.device("cuda") if device is None else torch.device(device)
         if dev.type != "cuda":
@@ -119,10 +120,11 @@ class KVQCache:
         self.query_heads = heads * self.query_group      # heads of q / modes / out
         arr = (ctypes.c_int64 * batch)(*cap)
         h = ctypes.c_void_p()
+        self.page_bytes, self.pool_pages = int(page_bytes), int(pool_pages)
         with torch.cuda.device(self.device):
-            _raise(lib.kvq_cache_create_gqa(ctypes.byref(h), batch, heads, self.query_group, head_dim,
-                                            ctypes.cast(arr, ctypes.c_void_p),
-                                            _stream(stream, self.device)))
+            _raise(lib.kvq_cache_create_paged(ctypes.byref(h), batch, heads, self.query_group, head_dim,
+                                              ctypes.cast(arr, ctypes.c_void_p), self.page_bytes,
+                                              self.pool_pages, _stream(stream, self.device)))
         self._h = h
 
     @property

@@ -139,6 +139,11 @@ def kv_tokens(wl: Workload, device, seq_range=None):
     return torch.cat(ks), torch.cat(vs), torch.cat(bs)
 
 
+def widths(wl: Workload, s: int, device):
+    """bits uint8 [L_s, H] of sequence s alone (the same draws as kv_tokens on `device`)."""
+    return categorical((wl.seqlens[s], wl.heads), wl.bits_p, BIT_VALUES, wl.seed, _S_BITS, s, device)
+
+
 def kv_sequence(wl: Workload, s: int, device):
     """K, V [L_s, H, D] and bits [L_s, H] of sequence s alone (same values as kv_tokens)."""
     return kv_tokens(wl, device, seq_range=[s])

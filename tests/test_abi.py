@@ -59,3 +59,14 @@ def test_test_hooks_check_arguments_on_host(lib):
     assert lib.kvq_test_fail_alloc(-1) == kvq.KVQ_ERR_ARG
     assert lib.kvq_test_fail_alloc(0) == kvq.KVQ_OK
     assert lib.kvq_test_bounded_wait(None, 1000000, None) == kvq.KVQ_ERR_ARG
+
+
+def test_paged_create_checks_pages_on_host(lib):
+    h = ctypes.c_void_p()
+    cap = (ctypes.c_int64 * 2)(16, 16)
+    capp = ctypes.cast(cap, ctypes.c_void_p)
+    assert lib.kvq_cache_create_paged(ctypes.byref(h), 2, 4, 1, 128, capp, 3000, 8, None) == kvq.KVQ_ERR_ARG
+    assert b"page_bytes" in lib.kvq_last_error()
+    assert lib.kvq_cache_create_paged(ctypes.byref(h), 2, 4, 1, 128, capp, 8192, 0, None) == kvq.KVQ_ERR_ARG
+    assert lib.kvq_cache_create_paged(ctypes.byref(h), 2, 4, 1, 128, capp, 1 << 22, 8, None) == kvq.KVQ_ERR_ARG
+    assert h.value is None
