@@ -169,6 +169,12 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
     __shared__ int warp_tot[kPlanThreads / 32];
     __shared__ int cnt_sh[kPlanThreads];
     __shared__ uint32_t base_sh;
+    // per unit of the pass: first item (relative to the pass), items of regions A and B,
+    // region sizes, query masks and subgroup, KV head, length, stream end, first slot
+    __shared__ int u_start[kPlanThreads + 1], u_cA[kPlanThreads], u_nA[kPlanThreads], u_nB[kPlanThreads];
+    __shared__ int u_cB[kPlanThreads], u_q[kPlanThreads], u_L[kPlanThreads];
+    __shared__ uint32_t u_end[kPlanThreads];
+    __shared__ int64_t u_sbase[kPlanThreads];
     pdl_wait();
     pdl_trigger();
     const int s = blockIdx.x;
@@ -243,47 +249,65 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
                 old = prev;
             }
             base_sh = base;
+            u_start[kPlanThreads] = tot;
+        }
+        const int rel = wpre + incl - cnt;            // the unit's first item within the pass
+        u_start[tid] = rel;
+        u_cA[tid] = cA;
+        u_cB[tid] = cB;
+        u_nA[tid] = nA;
+        u_nB[tid] = nB;
+        u_q[tid] = g0 | (mA << 8) | (mB << 12);
+        u_L[tid] = L;
+        if (mine && cnt > 0) {
+            u_end[tid] = c.end[s * H + hk];
+            u_sbase[tid] = slot_of(c, s, hk, 0);
         }
         __syncthreads();
-        const int64_t first = (int64_t)base_sh + wpre + incl - cnt;
-        if (mine) {
-            if (u % nsub == 0) {                     // the KV head's items: its subgroups' runs
-                int n_all = 0;
-                for (int k = 0; k < nsub; ++k) n_all += cnt_sh[tid + k];
-                wk.head_first[s * H + hk] = (int32_t)first;
-                wk.head_cnt[s * H + hk] = n_all;
-            }
-            if (first + cnt > wk.max_items) {
-                set_status(c.status, KVQ_ERR_DEVICE_CHECK);
-            } else if (cnt > 0) {
-                const int64_t sbase = slot_of(c, s, hk, 0);
-                const uint32_t end_s = c.end[s * H + hk];
-                int64_t it = first;
-                for (int r = 0; r < 2; ++r) {
-                    const int n = r ? nB : nA, ci = r ? cB : cA;
-                    const int lo = r ? L - nB : 0;
-                    const int msk = r ? mB : mA;
-                    if (ci == 0) continue;
-                    const int per = n / ci, rem = n % ci;
-                    int j0 = lo;
-                    for (int k = 0; k < ci; ++k) {       // near-equal, non-empty items
-                        DecodeItem d;
-                        d.sh = s * H + hk;
-                        d.j0 = j0;
-                        d.j1 = j0 + per + (k < rem ? 1 : 0);
-                        j0 = d.j1;
-                        // the stream end for the item ending at the last token; else the
-                        // producer reads the offset of key j1 itself
-                        d.end_off = (d.j1 < L) ? kReadEndFromMeta : end_s;
-                        d.sbase = sbase;
-                        d.qinfo = g0 | (msk << 8);
-                        d.pad = 0;
-                        wk.items[it++] = d;
-                    }
+        const int64_t base = base_sh;
+        if (mine && u % nsub == 0) {                  // the KV head's items: its subgroups' runs
+            int n_all = 0;
+            for (int k = 0; k < nsub; ++k) n_all += cnt_sh[tid + k];
+            wk.head_first[s * H + hk] = (int32_t)(base + rel);
+            wk.head_cnt[s * H + hk] = n_all;
+        }
+        if (base + tot > wk.max_items) {
+            if (tid == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+        } else {
+            // every thread writes items: item i of the pass belongs to the last unit whose
+            // first item is <= i (binary search over the pass's units)
+            const int n_units = min(per_pass, units - u0);
+            for (int i = tid; i < tot; i += kPlanThreads) {
+                int lo = 0, hi = n_units;                  // u_start[lo] <= i < u_start[hi]
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (u_start[mid] <= i) lo = mid;
+                    else hi = mid;
                 }
+                while (lo + 1 < n_units && u_start[lo + 1] <= i) ++lo;   // skip units with no items
+                const int k0 = i - u_start[lo];
+                const bool inA = k0 < u_cA[lo];
+                const int k = inA ? k0 : k0 - u_cA[lo];
+                const int n = inA ? u_nA[lo] : u_nB[lo], ci = inA ? u_cA[lo] : u_cB[lo];
+                const int Lu = u_L[lo];
+                const int first_key = inA ? 0 : Lu - u_nB[lo];
+                const int per = n / ci, rem = n % ci;     // near-equal, non-empty items
+                const int qv = u_q[lo];
+                const int uu = u0 + lo;
+                DecodeItem d;
+                d.sh = s * H + uu / nsub;
+                d.j0 = first_key + k * per + min(k, rem);
+                d.j1 = d.j0 + per + (k < rem ? 1 : 0);
+                // the stream end for the item ending at the last token; else the producer
+                // reads the offset of key j1 itself
+                d.end_off = (d.j1 < Lu) ? kReadEndFromMeta : u_end[lo];
+                d.sbase = u_sbase[lo];
+                d.qinfo = (qv & 0xFF) | ((inA ? (qv >> 8) & 0xF : (qv >> 12) & 0xF) << 8);
+                d.pad = 0;
+                wk.items[base + i] = d;
             }
         }
-        __syncthreads();                             // cnt_sh / warp_tot reused by the next pass
+        __syncthreads();                             // the per-unit arrays are reused by the next pass
     }
 }
 
@@ -624,6 +648,33 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
                     rec_bytes = 0;
                 }
+                // the stage's copies go out first; the width sort below overlaps their flight
+                const int stage = issued % kStages;
+                const uint32_t phase = (uint32_t)(issued / kStages) & 1u;
+                if (!mbar_wait(&sm.empty[stage], phase ^ 1u, c.status)) {
+                    aborted = true;
+                    break;
+                }
+                Stage<D> &sg = sm.st[stage];
+                if (lane == 0) {
+                    // the item's subgroup of queries: rows (s, hk * G + g0 ..) of q, contiguous
+                    const int g0 = qinfo & 0xFF;
+                    const int nq = min(kDecodeMaxQ, c.G - g0);
+                    const uint32_t q_bytes = new_item ? (uint32_t)(2 * D * nq) : 0u;
+                    const int s_of = sh / c.H, hk = sh % c.H;
+                    mbar_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
+                    bulk_g2s(sg.side, c.side + sbase + ja + s0, 16u * n, &sm.full[stage]);
+                    if (rec_bytes) {
+                        const RecLoc L = rec_loc(c, s_of, hk, 0);
+                        // a paged stream: one copy per page the stage's bytes touch
+                        const uint32_t n0 = L.pt ? min(rec_bytes, (((off0 >> c.page_shift) + 1u) << c.page_shift) - off0)
+                                                 : rec_bytes;
+                        bulk_g2s(sg.rec, L.at(off0), n0, &sm.full[stage]);
+                        if (rec_bytes > n0) bulk_g2s(sg.rec + n0, L.at(off0 + n0), rec_bytes - n0, &sm.full[stage]);
+                    }
+                    if (q_bytes)
+                        bulk_g2s(sg.q, q + ((int64_t)s_of * HQ + hk * c.G + g0) * D, q_bytes, &sm.full[stage]);
+                }
                 // counting sort by width: per-lane counts of the four classes packed in one
                 // word (8 bits each), one warp prefix sum; each class's run padded to whole
                 // chunks of KPS keys
@@ -652,13 +703,6 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     pstart += padded;
                 }
 
-                const int stage = issued % kStages;
-                const uint32_t phase = (uint32_t)(issued / kStages) & 1u;
-                if (!mbar_wait(&sm.empty[stage], phase ^ 1u, c.status)) {
-                    aborted = true;
-                    break;
-                }
-                Stage<D> &sg = sm.st[stage];
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
                     const int sl = 4 * lane + r;
@@ -690,25 +734,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     sg.cls_chunk[4] = pstart / KPS;
                 }
                 __syncwarp();
-                if (lane == 0) {
-                    // the item's subgroup of queries: rows (s, hk * G + g0 ..) of q, contiguous
-                    const int g0 = qinfo & 0xFF;
-                    const int nq = min(kDecodeMaxQ, c.G - g0);
-                    const uint32_t q_bytes = new_item ? (uint32_t)(2 * D * nq) : 0u;
-                    const int s_of = sh / c.H, hk = sh % c.H;
-                    mbar_arrive_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
-                    bulk_g2s(sg.side, c.side + sbase + ja + s0, 16u * n, &sm.full[stage]);
-                    if (rec_bytes) {
-                        const RecLoc L = rec_loc(c, s_of, hk, 0);
-                        // a paged stream: one copy per page the stage's bytes touch
-                        const uint32_t n0 = L.pt ? min(rec_bytes, (((off0 >> c.page_shift) + 1u) << c.page_shift) - off0)
-                                                 : rec_bytes;
-                        bulk_g2s(sg.rec, L.at(off0), n0, &sm.full[stage]);
-                        if (rec_bytes > n0) bulk_g2s(sg.rec + n0, L.at(off0 + n0), rec_bytes - n0, &sm.full[stage]);
-                    }
-                    if (q_bytes)
-                        bulk_g2s(sg.q, q + ((int64_t)s_of * HQ + hk * c.G + g0) * D, q_bytes, &sm.full[stage]);
-                }
+                if (lane == 0) mbar_arrive(&sm.full[stage]);   // the stage's key list is written
                 ++issued;
                 s0 = s1;
             }
@@ -852,44 +878,88 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     }
 }
 
-// One CTA of D threads per (sequence, query head): thread = channel. The query's partials
-// are those of its KV head's items whose subgroup holds it as an active query.
+// One CTA of D threads per (sequence, query head). The query's partials are those of its
+// KV head's items whose subgroup holds it as an active query. The threads first share the
+// per-item work (the maximum, then each item's weight 2^(m_i - M) and the sum of l_i
+// weights, kept in shared memory for a chunk of items), then thread = channel sums the
+// weighted o_i of the chunk with independent loads.
+constexpr int kCombineChunk = 256;
+
 template <int D>
 __global__ void __launch_bounds__(D)
 decode_combine_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
 {
+    __shared__ float f_sh[kCombineChunk];
+    __shared__ int32_t idx_sh[kCombineChunk];
+    __shared__ float red[D / 32];
     pdl_wait();
     pdl_trigger();
     const int HQ = c.H * c.G;
-    const int shq = blockIdx.x, ch = threadIdx.x;
+    const int shq = blockIdx.x, ch = threadIdx.x, lane = ch & 31, wid = ch >> 5;
     const int s = shq / HQ, hq = shq % HQ, hk = hq / c.G, gq = hq % c.G;
     const int unit = s * c.H + hk;
     const int first = wk.head_first[unit], cnt = wk.head_cnt[unit];
     const int QS = wk.qslots;
-    float M = kMInit;
-    bool any = false;
-    for (int i = 0; i < cnt; ++i) {
+    auto part_of = [&](int i) -> int64_t {      // this query's partial of item first + i, or -1
         const int qinfo = wk.items[first + i].qinfo;
         const int d = gq - (qinfo & 0xFF);
-        if (d < 0 || d >= kDecodeMaxQ || !((qinfo >> (8 + d)) & 1)) continue;
-        M = fmaxf(M, wk.partials[((int64_t)(first + i) * QS + d) * (D + 4)]);
-        any = true;
+        if (d < 0 || d >= kDecodeMaxQ || !((qinfo >> (8 + d)) & 1)) return -1;
+        return ((int64_t)(first + i) * QS + d) * (D + 4);
+    };
+    float M = kMInit;
+    for (int i = ch; i < cnt; i += D) {
+        const int64_t p = part_of(i);
+        if (p >= 0) M = fmaxf(M, wk.partials[p]);
     }
-    float res = 0.f;
-    if (any) {
-        float L = 0.f, acc = 0.f;
-        for (int i = 0; i < cnt; ++i) {
-            const int qinfo = wk.items[first + i].qinfo;
-            const int d = gq - (qinfo & 0xFF);
-            if (d < 0 || d >= kDecodeMaxQ || !((qinfo >> (8 + d)) & 1)) continue;
-            const float *p = wk.partials + ((int64_t)(first + i) * QS + d) * (D + 4);
-            const float f = ex2(p[0] - M);
-            L = fmaf(p[1], f, L);
-            acc = fmaf(p[4 + ch], f, acc);
+#pragma unroll
+    for (int dd = 16; dd >= 1; dd >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, dd));
+    if (lane == 0) red[wid] = M;
+    __syncthreads();
+    M = red[0];
+#pragma unroll
+    for (int w2 = 1; w2 < D / 32; ++w2) M = fmaxf(M, red[w2]);
+    __syncthreads();
+    // (the summation order is fixed: results do not depend on thread timing)
+    float L = 0.f, acc = 0.f;
+    for (int i0 = 0; i0 < cnt; i0 += kCombineChunk) {
+        const int n = min(cnt - i0, kCombineChunk);
+        for (int k = ch; k < n; k += D) {
+            const int64_t p = part_of(i0 + k);
+            float f = 0.f;
+            if (p >= 0) {
+                f = ex2(wk.partials[p] - M);
+                L = fmaf(wk.partials[p + 1], f, L);
+            }
+            f_sh[k] = f;
+            idx_sh[k] = (p >= 0) ? (int32_t)(p / (D + 4)) : -1;
         }
-        res = acc / L;
+        __syncthreads();
+        int k = 0;
+        for (; k + 4 <= n; k += 4) {
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int32_t ix = idx_sh[k + u];
+                v[u] = (ix >= 0) ? wk.partials[(int64_t)ix * (D + 4) + 4 + ch] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc = fmaf(v[u], f_sh[k + u], acc);
+        }
+        for (; k < n; ++k) {
+            const int32_t ix = idx_sh[k];
+            if (ix >= 0) acc = fmaf(wk.partials[(int64_t)ix * (D + 4) + 4 + ch], f_sh[k], acc);
+        }
+        __syncthreads();
     }
-    out[(int64_t)shq * D + ch] = res;
+    // L: every thread summed the l of its own items; the block sum is the denominator
+#pragma unroll
+    for (int dd = 16; dd >= 1; dd >>= 1) L += __shfl_xor_sync(0xffffffffu, L, dd);
+    if (lane == 0) red[wid] = L;
+    __syncthreads();
+    L = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < D / 32; ++w2) L += red[w2];
+    out[(int64_t)shq * D + ch] = (L > 0.f) ? acc / L : 0.f;
 }
 
 template <int D>

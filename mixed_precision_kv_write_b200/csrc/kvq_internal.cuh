@@ -190,6 +190,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -209,20 +215,31 @@ __device__ __forceinline__ uint64_t global_ns()
 // error ends the kernel with a status instead of hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+#ifndef KVQ_WAIT_HINT_NS
+#define KVQ_WAIT_HINT_NS 100000
+#endif
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
                                           uint64_t limit_ns = kWaitLimitNs)
 {
     const uint32_t addr = smem_u32(bar);
-    const uint32_t suspend_ns = 100000;
     uint32_t done = 0;
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
+#if KVQ_WAIT_HINT_NS > 0
         asm volatile("{\n\t.reg .pred p;\n\t"
                      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
                      "selp.u32 %0, 1, 0, p;\n\t}"
                      : "=r"(done)
-                     : "r"(addr), "r"(parity), "r"(suspend_ns)
+                     : "r"(addr), "r"(parity), "r"((uint32_t)KVQ_WAIT_HINT_NS)
                      : "memory");
+#else
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(done)
+                     : "r"(addr), "r"(parity)
+                     : "memory");
+#endif
         if (done) return true;
         if ((it & 15u) == 0) {
             const uint64_t t = global_ns();

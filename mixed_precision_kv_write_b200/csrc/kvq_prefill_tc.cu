@@ -1,26 +1,29 @@
 // Routed causal prefill attention (TriRoute paper review page, section 3, Eq. 2) over the
 // mixed-precision cache of Eq. 4, on the sm_100a tensor cores (tcgen05 + TMEM).
 //
-// Two launches per call:
+// Three launches per call:
 //   prefill_sched_kernel  one CTA per (sequence, head): compacts the call's queries by
 //                         mode (stable) into a local list and a full list, cuts each into tiles of
 //                         at most 128 queries, and writes zeros for skip queries. A local
 //                         tile reads keys [min(t) - w, max(t)], a full tile [0, max(t)],
 //                         so local rows do not pay for a full tile's range.
+//   prefill_order_kernel  orders the tiles longest first (keys spanned, descending).
 //   prefill_tc_kernel     one CTA per tile:
 //     - warps 0-3 (one thread per query row): Q row -> shared (fp16, 128B-swizzled
 //       K-major); per key tile, S row from TMEM -> logits (s_K * (q.c) + z_K * sum(q)) /
 //       sqrt(D) with the row's causal/window mask -> online softmax -> P' = p * s_V split
 //       into fp16 hi + lo (fp16 rounding of P alone would cost ~1e-2 on outlier channels)
-//       -> shared; rescale the O row in TMEM when the row max grows; final O / l.
+//       -> TMEM (double buffered, the A operand of the PV MMA); rescale the O row in TMEM
+//       when the row max grows by more than 2^8; final O / l.
 //     - warps 4-7: unpack each 64-key tile's K and V codes into exact fp16 operands (codes
 //       are integers <= 255; b = 16 keys are the fp16 values) in shared memory, double
 //       buffered; K 128B-swizzled K-major, V 128B-swizzled MN-major. The packed bytes are
 //       fetched one tile ahead with cp.async and the record offsets three tiles ahead.
-//     - warp 8: owns 256 TMEM columns (S double buffer: 2 x 64, O: D) and issues the MMAs
-//       from one lane: S = Q C_K^T (M128 N64 K16 steps) as soon as a K tile is unpacked
-//       (up to one tile ahead), O += P'_hi V and O += P'_lo V (M128 ND K16) as soon as P' of
-//       the tile is in shared memory, whichever is ready first.
+//     - warp 8: owns 512 TMEM columns (S double buffer: 2 x 64, O: D, P' double buffer:
+//       2 x 64) and issues the MMAs from one lane: S = Q C_K^T (M128 N64 K16 steps, A and B
+//       in shared memory) as soon as a K tile is unpacked (up to one tile ahead), O += P'_hi V
+//       and O += P'_lo V (M128 ND K16, A in TMEM) as soon as P' of the tile is in TMEM,
+//       whichever is ready first.
 //   All mbarrier waits are bounded; on a timeout the CTA records KVQ_ERR_DEVICE_CHECK,
 //   leaves its loops, waits (bounded) for its MMAs and frees its TMEM before returning.
 #include "kvq_internal.cuh"
@@ -31,8 +34,11 @@ namespace {
 constexpr int kQRows = 128;     // queries per tile (MMA M)
 constexpr int kKeys = 64;       // keys per key tile (QK MMA N, PV MMA K)
 constexpr int kTcThreads = 288; // 9 warps
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTmemS = 0, kTmemO = 128;   // S double buffer at columns 0 and 64
+constexpr uint32_t kTmemCols = 512;
+// TMEM columns: S double buffer at 0 and 64 (fp32), O at 128 (D columns), P' double buffer at
+// 256 and 320: each buffer holds P'_hi in 32 columns then P'_lo in 32 (fp16 pairs, the A
+// operand of the PV MMA)
+constexpr uint32_t kTmemS = 0, kTmemO = 128, kTmemP = 256;
 
 // ---- tcgen05 / UMMA helpers -------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), descriptor version 1.
@@ -54,6 +60,16 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b
                  "setp.ne.b32 p, %4, 0;\n\t"
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
                  ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)acc)
+                 : "memory");
+}
+
+// D (TMEM) [+]= A (TMEM, K-major: row = lane, 2 fp16 per 32-bit column) * B (shared)
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, bool acc)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"((uint32_t)acc)
                  : "memory");
 }
 
@@ -100,6 +116,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
                    "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
                    "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
                    "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                   "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+                   "r"(v[15])
                  : "memory");
 }
 
@@ -176,13 +202,11 @@ struct alignas(1024) PfSmem {
     __half q[kQRows * D];             // K-major SW128, D/64 blocks of 128 rows x 128 B
     __half k[2][kKeys * D];           // K-major SW128, D/64 blocks of 64 rows x 128 B
     __half v[2][kKeys * D];           // MN-major SW128: atom (8 keys x 64 ch) at (key/8)*(D/64)+ch/64
-    __half p_hi[kQRows * kKeys];      // K-major SW128, 128 rows x 128 B
-    __half p_lo[kQRows * kKeys];
     float2 side_k[2][kKeys];          // (s_K * c, z_K * c) per key, c = log2(e)/sqrt(D)
     float2 side_v[2][kKeys];          // (s_V, z_V) per key
     uint8_t raw[2][kKeys * 2][2 * D + 16]; // packed K and V bytes of each (key, half), by cp.async
                                            // (16 bytes of padding spread the slots over the banks)
-    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full, pv_done, drain;
+    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], drain;
     uint32_t tmem_base;
     int32_t klo, khi, abort_flag;
 };
@@ -213,8 +237,10 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         }
         mbar_init(&sm.s_full[0], 1);
         mbar_init(&sm.s_full[1], 1);
-        mbar_init(&sm.p_full, 128);
-        mbar_init(&sm.pv_done, 1);
+        mbar_init(&sm.p_full[0], 128);
+        mbar_init(&sm.p_full[1], 128);
+        mbar_init(&sm.pv_done[0], 1);
+        mbar_init(&sm.pv_done[1], 1);
         mbar_init(&sm.drain, 1);
         sm.klo = INT32_MAX;
         sm.khi = -1;
@@ -265,7 +291,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     if (warp == 8) {
         // ------------------------------- MMA issuer --------------------------------
         // order: QK(0), then per tile t: QK(t+1) into the other S buffer, wait P(t), PV(t)
-        const uint32_t q0 = smem_u32(sm.q), p_hi0 = smem_u32(sm.p_hi), p_lo0 = smem_u32(sm.p_lo);
+        const uint32_t q0 = smem_u32(sm.q);
         constexpr uint32_t idesc_qk = umma_idesc(kKeys, false);
         constexpr uint32_t idesc_pv = umma_idesc(D, true);
         constexpr uint32_t v_sbo = (D / 64) * 1024;       // next 8 keys
@@ -290,15 +316,15 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             if (lane == 0) {
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    const uint32_t pb = half ? p_lo0 : p_hi0;
+                    // P'_hi then P'_lo of buffer t & 1: 8 TMEM columns per 16 keys
+                    const uint32_t pa = tmem + kTmemP + 64 * (t & 1) + 32 * half;
 #pragma unroll
                     for (int kk = 0; kk < kKeys / 16; ++kk) {
-                        const uint64_t da = umma_desc(pb + kk * 32, 16, 1024);
                         const uint64_t db = umma_desc(v0 + 2 * kk * v_sbo, 1024, v_sbo);
-                        umma_f16(tmem + kTmemO, da, db, idesc_pv, half > 0 || t > 0 || kk > 0);
+                        umma_f16_ts(tmem + kTmemO, pa + 8 * kk, db, idesc_pv, half > 0 || t > 0 || kk > 0);
                     }
                 }
-                umma_commit(&sm.pv_done);
+                umma_commit(&sm.pv_done[t & 1]);
                 umma_commit(&sm.kv_empty[t & 1]);
             }
             __syncwarp();
@@ -315,7 +341,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 issue_qk(next_qk++);
                 progressed = true;
             }
-            if (next_pv < next_qk && __all_sync(0xffffffffu, mbar_test(&sm.p_full, next_pv & 1))) {
+            if (next_pv < next_qk &&
+                __all_sync(0xffffffffu, mbar_test(&sm.p_full[next_pv & 1], (next_pv >> 1) & 1))) {
                 issue_pv(next_pv++);
                 progressed = true;
             }
@@ -422,11 +449,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
         // ------------------------------ softmax rows ---------------------------------
-        const int r = tid;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         float m_run = -INFINITY, l_run = 0.f, pz_run = 0.f;
-        uint8_t *ph = reinterpret_cast<uint8_t *>(sm.p_hi);
-        uint8_t *pl = reinterpret_cast<uint8_t *>(sm.p_lo);
         bool ok = true;
         for (int t = 0; t < n_kt; ++t) {
             const int b = t & 1;
@@ -475,47 +499,52 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             l_run = fmaf(l_run, corr, psum);
             pz_run = fmaf(pz_run, corr, pz);
             m_run = m_new;
-            if (t > 0) {
-                // PV(t-1) must be done: it reads P and accumulates into O
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (t - 1) & 1, c.status))) {
+            // P' buffer b was last read by PV(t-2); a rescale of O also needs PV(t-1) done
+            // (the MMAs complete in issue order, so waiting for PV(t-1) covers PV(t-2))
+            const bool rescale = t > 0 && __any_sync(0xffffffffu, bump);
+            const int t_wait = rescale ? t - 1 : t - 2;
+            if (t_wait >= 0) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t_wait & 1], (t_wait >> 1) & 1, c.status))) {
                     sm.abort_flag = 1;
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, bump)) {        // rescale this warp's O rows
+            }
+            if (rescale) {                                  // rescale this warp's O rows
 #pragma unroll
-                    for (int cb = 0; cb < D / 32; ++cb) {
-                        float ov[32];
-                        tmem_ld32(tmem + lane_base + kTmemO + cb * 32, ov);
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    float ov[32];
+                    tmem_ld32(tmem + lane_base + kTmemO + cb * 32, ov);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) ov[e] *= corr;
-                        tmem_st32(tmem + lane_base + kTmemO + cb * 32, ov);
-                    }
-                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    for (int e = 0; e < 32; ++e) ov[e] *= corr;
+                    tmem_st32(tmem + lane_base + kTmemO + cb * 32, ov);
                 }
             }
-            // P' = hi + lo, both fp16, row r of the two K-major P tiles
+            // P' = hi + lo, both fp16, row r of the TMEM A operand of buffer b: column j
+            // holds keys (2j, 2j + 1); hi in columns 0..31, lo in 32..63
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                uint32_t hw[4], lw[4];
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t hw[16], lw[16];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a = lg[8 * cc + 2 * e], bq = lg[8 * cc + 2 * e + 1];
+                for (int e = 0; e < 16; ++e) {
+                    const float a = lg[32 * hf + 2 * e], bq = lg[32 * hf + 2 * e + 1];
                     const __half2 hv = __floats2half2_rn(a, bq);
-                    const float2 hf = __half22float2(hv);
-                    const __half2 lv = __floats2half2_rn(a - hf.x, bq - hf.y);
+                    const float2 hfv = __half22float2(hv);
+                    const __half2 lv = __floats2half2_rn(a - hfv.x, bq - hfv.y);
                     hw[e] = *reinterpret_cast<const uint32_t *>(&hv);
                     lw[e] = *reinterpret_cast<const uint32_t *>(&lv);
                 }
-                *reinterpret_cast<uint4 *>(ph + kmajor_off(r, cc)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4 *>(pl + kmajor_off(r, cc)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                tmem_st16u(tmem + lane_base + kTmemP + 64 * b + 16 * hf, hw);
+                tmem_st16u(tmem + lane_base + kTmemP + 64 * b + 32 + 16 * hf, lw);
             }
-            fence_async_smem();
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
-            mbar_arrive(&sm.p_full);
+            mbar_arrive(&sm.p_full[b]);
         }
-        if (ok && n_kt > 0 && __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (n_kt - 1) & 1, c.status))) {
+        const int t_last = n_kt - 1;
+        if (ok && n_kt > 0 &&
+            __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t_last & 1], (t_last >> 1) & 1, c.status))) {
             tc_fence_after();
             const bool write = row_t >= 0;
             const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;

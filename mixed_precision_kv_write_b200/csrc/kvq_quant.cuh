@@ -32,24 +32,30 @@ __device__ __forceinline__ void quant_store(const uint4 (&raw)[NC], float z, flo
 #pragma unroll
     for (int j = 0; j < NC; ++j) w[j][0] = w[j][1] = 0u;
     if (sc != 0.0f) {
+        // Two values per instruction: the packed fp32 operations (FADD2/FMUL2/FFMA2) round
+        // each half exactly as the scalar operation would, so the codes are unchanged.
         const float y = __frcp_rn(sc);
-        float nan_probe = 0.0f;
+        const float2 y2 = make_float2(y, y), nz2 = make_float2(-z, -z), ns2 = make_float2(-sc, -sc);
+        const float2 mg2 = make_float2(kRoundMagic, kRoundMagic);
+        float2 probe = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
             const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[j]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float x = (e & 1) ? __high2float(h2[e >> 1]) : __low2float(h2[e >> 1]);
-                const float u = __fsub_rn(x, z);
-                const float q0 = __fmul_rn(u, y);
-                const float r = __fmaf_rn(-sc, q0, u);
-                const float q = __fmaf_rn(r, y, q0);
-                const float t = __fadd_rn(q, kRoundMagic);
-                nan_probe = __fadd_rn(nan_probe, q);
+            for (int e = 0; e < 4; ++e) {                 // channels 2e, 2e + 1 of the chunk
+                const float2 x = __half22float2(h2[e]);
+                const float2 u = __fadd2_rn(x, nz2);         // x - z
+                const float2 q0 = __fmul2_rn(u, y2);
+                const float2 r = __ffma2_rn(ns2, q0, u);     // u - s * q0, exact
+                const float2 q = __ffma2_rn(r, y2, q0);      // RN(u / s)
+                const float2 t = __fadd2_rn(q, mg2);
+                probe = __fadd2_rn(probe, q);
                 // code << shift; the 1.5 * 2^23 bits are taken off below
-                w[j][(e * BITS) >> 5] += __float_as_uint(t) << ((e * BITS) & 31);
+                w[j][(2 * e * BITS) >> 5] += __float_as_uint(t.x) << ((2 * e * BITS) & 31);
+                w[j][((2 * e + 1) * BITS) >> 5] += __float_as_uint(t.y) << (((2 * e + 1) * BITS) & 31);
             }
         }
+        const float nan_probe = probe.x + probe.y;
         constexpr int kWordBits = BITS * 8 < 32 ? BITS * 8 : 32;   // code bits per word
         uint32_t magic = 0u;
 #pragma unroll
