@@ -11,7 +11,7 @@
 //                         every record read: the key range is the union of the subgroup's
 //                         ranges, cut where the local window starts, so within an item
 //                         every active query reads every key. Ranges are cut into
-//                         near-equal items of at most 576 keys. Each CTA reserves its items
+//                         near-equal items of at most 1152 keys. Each CTA reserves its items
 //                         with one atomic on a (call generation, count) word.
 //   decode_splitk_kernel  three CTAs per SM, one producer and four consumer warps each. The
 //                         producer walks the CTA's items in stages of at most 128 keys and
@@ -24,8 +24,9 @@
 //                         logit -> online softmax per key group (the running max moves only
 //                         when a logit exceeds it by more than 8 in log2 units, a
 //                         warp-uniform branch) -> V accumulation. Each warp serves one query
-//                         of the item; the warps' states are merged into a partial per
-//                         (item, query).
+//                         of the item; at the item's end each warp deposits its state and
+//                         the last warp to do so merges them into a partial per (item,
+//                         query), while the others go on with the next item.
 //   decode_combine_kernel log-sum-exp merge of the partials of each (sequence, query head),
 //                         one thread per channel; zeros for skip heads and empty sequences.
 //
@@ -70,12 +71,20 @@ constexpr int kConsumerWarps = KVQ_DECODE_CONSUMERS;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
 constexpr int kCtasPerSm = KVQ_DECODE_CTAS_PER_SM;
 constexpr int kStages = KVQ_DECODE_STAGES;        // record stages in flight per CTA
-constexpr int kWin = kDecodeWindowKeys;           // keys per window of record offsets
+#ifndef KVQ_DECODE_WINDOW
+#define KVQ_DECODE_WINDOW 128
+#endif
+constexpr int kWin = KVQ_DECODE_WINDOW;           // keys per window of record offsets (128 or 256)
+constexpr int KPL = kWin / 32;                    // window slots per producer lane
+static_assert(kWin == 128 || kWin == 256, "window of 128 or 256 keys");
 constexpr uint32_t kStageRecBytes = KVQ_DECODE_STAGE_BYTES;   // record bytes per stage, at most
 constexpr int kPermSlots = kWin + 64;             // width-sorted keys padded to whole chunks
 constexpr int kMetaSlots = KVQ_DECODE_META_SLOTS; // windows of record offsets fetched ahead
 static_assert(kStageRecBytes <= 32768, "stage offsets are 15 bits");
 constexpr int kMetaWords = kWin + 8;
+// A consumer warp can run at most kStages items ahead of the slowest one (the stages are
+// shared and every item has at least one), so kStages + 1 merge slots never collide.
+constexpr int kMergeRing = kStages + 1;
 constexpr int kNewItem = 1, kLastSub = 2;         // stage flags
 constexpr uint32_t kReadEndFromMeta = 0xFFFFFFFFu;
 constexpr uint32_t kValid = 0x80000000u;
@@ -133,8 +142,10 @@ template <int D>
 struct DecodeSmem {
     Stage<D> st[kStages];
     MetaSlot ms[kMetaSlots];
-    float red_o[kConsumerWarps][D];
-    float red_m[kConsumerWarps], red_l[kConsumerWarps], red_pz[kConsumerWarps];
+    // item merges: a ring of kMergeRing items (states deposited by each consumer warp)
+    float red_o[kMergeRing][kConsumerWarps][D];
+    float red_m[kMergeRing][kConsumerWarps], red_l[kMergeRing][kConsumerWarps], red_pz[kMergeRing][kConsumerWarps];
+    int32_t merge_cnt[kMergeRing];
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t mfull[kMetaSlots];
@@ -483,7 +494,7 @@ __device__ __forceinline__ void process_chunk(KeyState &st, const QRegs &Q, floa
     float part = lane_dot<CLS>(Q, r + 4 * BITS * li);
 #pragma unroll
     for (int d = 1; d < LPK; d <<= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
-    const float4 sd = sg.side[(ent >> 16) & 127u];
+    const float4 sd = sg.side[(ent >> 16) & 0xFFu];
     float lg = (CLS == 3) ? part * cdot : fmaf(sd.x * cdot, part, sd.y * qsum_l);
     lg = (ent & kValid) ? lg : -INFINITY;
     if (__any_sync(0xffffffffu, lg > st.m + kLazy)) {      // rare after an item's first keys
@@ -537,6 +548,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
             mbar_init(&sm.empty[i], kConsumerWarps);
         }
         for (int i = 0; i < kMetaSlots; ++i) mbar_init(&sm.mfull[i], 1);
+        for (int i = 0; i < kMergeRing; ++i) sm.merge_cnt[i] = 0;
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -549,16 +561,25 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         // memory, cuts it into stages of at most kStageRecBytes, sorts each stage's keys by
         // width and issues the stage's copies. On a timed-out wait it stops issuing, waits
         // (bounded) for the copies already in flight and returns.
-        // A window's record offsets sit in slots 0..131 of its ring entry, key ja + i in slot
-        // i (ja = the window's first key rounded down to a multiple of 4); lane l holds
-        // slots 4l .. 4l + 3 (one 16-byte shared load). Windows after an item's first end
-        // on 4-aligned keys, so a window's keys fit slots [d, d + nwin) with d + nwin <= 128.
+        // A window's record offsets sit in slots 0..kWin+3 of its ring entry, key ja + i in
+        // slot i (ja = the window's first key rounded down to a multiple of 4); lane l holds
+        // slots KPL*l .. KPL*l + KPL - 1 (16-byte shared loads). Windows after an item's first
+        // end on 4-aligned keys, so a window's keys fit slots [d, d + nwin) with
+        // d + nwin <= kWin. The next item's descriptor is loaded one item ahead.
         int f_it = blockIdx.x;
         if (f_it >= n_items) return;
         DecodeItem f_d = wk.items[f_it];
+        DecodeItem f_nx = f_d;
+        if (f_it + (int)gridDim.x < n_items) f_nx = wk.items[f_it + gridDim.x];
         int f_j = f_d.j0;
         bool f_valid = true, aborted = false;
         int filled = 0, consumed = 0, issued = 0;
+        auto pick = [](const uint32_t (&a)[KPL], int i) {       // a[i], i warp-uniform
+            uint32_t v = a[0];
+#pragma unroll
+            for (int r = 1; r < KPL; ++r) v = (i == r) ? a[r] : v;
+            return v;
+        };
         while (!aborted) {
             while (f_valid && filled < consumed + kMetaSlots) {
                 const int slot = filled % kMetaSlots;
@@ -585,8 +606,9 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 if (f_j >= f_d.j1) {
                     f_it += gridDim.x;
                     if (f_it < n_items) {
-                        f_d = wk.items[f_it];
+                        f_d = f_nx;
                         f_j = f_d.j0;
+                        if (f_it + (int)gridDim.x < n_items) f_nx = wk.items[f_it + gridDim.x];
                     } else {
                         f_valid = false;
                     }
@@ -602,34 +624,39 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
             const int it = ms.it, qinfo = ms.qinfo, ja = ms.ja;
             const int d = ms.j - ja, dend = ms.j1 - ja;       // the window's keys: slots [d, dend)
             const bool first = (ms.first & 1) != 0, lastwin = (ms.first & 2) != 0;
-            const uint4 mv = reinterpret_cast<const uint4 *>(ms.meta)[lane];
-            const uint32_t m[4] = {mv.x, mv.y, mv.z, mv.w};
+            uint32_t m[KPL];
+#pragma unroll
+            for (int v4 = 0; v4 < KPL / 4; ++v4) {
+                const uint4 mv = reinterpret_cast<const uint4 *>(ms.meta)[KPL / 4 * lane + v4];
+                m[4 * v4] = mv.x;
+                m[4 * v4 + 1] = mv.y;
+                m[4 * v4 + 2] = mv.z;
+                m[4 * v4 + 3] = mv.w;
+            }
             const uint32_t bnd = (ms.end_off == kReadEndFromMeta ? ms.meta[dend] : ms.end_off) & ~15u;
             const int64_t sbase = ms.sbase;
             const int sh = ms.sh;
-            // nx[r]: the offset right after the key in slot 4 lane + r (the next key's offset,
-            // or the bound after the window's last key)
-            uint32_t nx[4];
+            // nx[r]: the offset right after the key in slot KPL lane + r (the next key's
+            // offset, or the bound after the window's last key)
+            uint32_t nx[KPL];
             const uint32_t next_lane = __shfl_down_sync(0xffffffffu, m[0], 1);
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int sl = 4 * lane + r;
-                nx[r] = (sl + 1 == dend) ? bnd : ((r < 3 ? m[(r + 1) & 3] : next_lane) & ~15u);
+            for (int r = 0; r < KPL; ++r) {
+                const int sl = KPL * lane + r;
+                nx[r] = (sl + 1 == dend) ? bnd : ((r + 1 < KPL ? m[(r + 1) % KPL] : next_lane) & ~15u);
             }
             ++consumed;
 
             for (int s0 = d; s0 < dend;) {
-                // the stage: slots [s0, s1), at most kStageRecBytes of records and (paged
-                // caches) bytes in at most two pages
-                const int r0 = s0 & 3;
-                const uint32_t off0 = __shfl_sync(0xffffffffu, r0 == 0 ? m[0] : r0 == 1 ? m[1] : r0 == 2 ? m[2] : m[3],
-                                                  s0 >> 2) & ~15u;
+                // the stage: slots [s0, s1), at most kStageRecBytes of records, at most 255
+                // keys, and (paged caches) bytes in at most two pages
+                const uint32_t off0 = __shfl_sync(0xffffffffu, pick(m, s0 % KPL), s0 / KPL) & ~15u;
                 const uint32_t plast = (off0 >> c.page_shift) + 1u;
                 uint32_t cnt = 0;
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int sl = 4 * lane + r;
-                    cnt += (sl >= s0 && sl < dend && nx[r] - off0 <= kStageRecBytes &&
+                for (int r = 0; r < KPL; ++r) {
+                    const int sl = KPL * lane + r;
+                    cnt += (sl >= s0 && sl < dend && sl < s0 + 255 && nx[r] - off0 <= kStageRecBytes &&
                             ((nx[r] - 1u) >> c.page_shift) <= plast) ? 1u : 0u;
                 }
                 int n = (int)__reduce_add_sync(0xffffffffu, cnt);
@@ -638,9 +665,8 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     n = 1;
                 }
                 const int s1 = s0 + n;
-                const int kl = s1 - 1, rl = kl & 3;
-                const uint32_t nxl = __shfl_sync(0xffffffffu, rl == 0 ? nx[0] : rl == 1 ? nx[1] : rl == 2 ? nx[2] : nx[3],
-                                                 kl >> 2);
+                const int kl = s1 - 1;
+                const uint32_t nxl = __shfl_sync(0xffffffffu, pick(nx, kl % KPL), kl / KPL);
                 const bool last = lastwin && s1 == dend;
                 const bool new_item = first && s0 == d;
                 uint32_t rec_bytes = nxl - off0;
@@ -680,8 +706,8 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 // chunks of KPS keys
                 uint32_t lc = 0;
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int sl = 4 * lane + r;
+                for (int r = 0; r < KPL; ++r) {
+                    const int sl = KPL * lane + r;
                     if (sl >= s0 && sl < s1) lc += 1u << (8 * (m[r] & 3u));
                 }
                 uint32_t incl = lc;
@@ -704,8 +730,8 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 }
 
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int sl = 4 * lane + r;
+                for (int r = 0; r < KPL; ++r) {
+                    const int sl = KPL * lane + r;
                     if (sl >= s0 && sl < s1) {
                         const uint32_t cl = m[r] & 3u;
                         const int start = cl == 0 ? cstart[0] : cl == 1 ? cstart[1] : cl == 2 ? cstart[2] : cstart[3];
@@ -758,8 +784,8 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     }
 
     // -------------------------------- consumers -------------------------------------
-    // Every consumer warp takes part in every item's merge (two named barriers per item),
-    // also after a timed-out wait: a warp that gave up only skips the waits and the work.
+    // Every consumer warp deposits its state for every item, also after a timed-out wait: a
+    // warp that gave up only skips the waits and the work. Nothing waits on the deposits.
     const int g = lane / LPK;            // key slot within a chunk
     const int li = lane % LPK;           // channel block: channels [32 li, 32 li + 32)
     const float qk_scale = kLog2e * rsqrtf((float)D);   // logits in log2 units
@@ -768,14 +794,15 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     bool dead = false;
     QRegs Q;
     float qsum_l = 0.f;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    int ring = 0;                         // this item's merge slot
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ring = (ring + 1) % kMergeRing) {
         KeyState ks;
         ks.m = kMInit;
         ks.l = 0.f;
         ks.pz = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) ks.o[k] = make_float2(0.f, 0.f);
-        int nq = 1, slot = 0, rank = warp, nws = kConsumerWarps;
+        int nq = 1, rank = warp, nws = kConsumerWarps, qmask = 1;
         bool last = false;
         while (!last && !dead) {
             if (*reinterpret_cast<volatile int32_t *>(&sm.abort_flag) ||
@@ -788,7 +815,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
             const int flags = sg.info[2];
             last = (flags & kLastSub) != 0;
             if (flags & kNewItem) {
-                const int qmask = sg.info[4] >> 8;
+                qmask = sg.info[4] >> 8;
                 nq = __popc(qmask);
                 const int sidx = warp % nq;        // the sidx-th active query of the item
                 rank = warp / nq;
@@ -799,7 +826,6 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                         if (seen == sidx) qi = b;
                         ++seen;
                     }
-                slot = qi;                         // the query's slot in the item's partials
                 // this lane's 32 channels of query g0 + qi, scaled; sum(q) over all D
                 const uint4 *src = reinterpret_cast<const uint4 *>(sg.q[qi] + 32 * li);
                 float qs = 0.f;
@@ -837,44 +863,61 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
             }
         }
 
-        // merge the key groups of the warp, then the warps of each query, into the
-        // item's partials
+        // Merge the key groups of the warp, deposit the warp's state in the item's merge
+        // slot, and go on: the warp that deposits last merges the item's warps into the
+        // partials of each of its queries (no barrier across the consumer warps).
 #pragma unroll
         for (int mask = LPK; mask < 32; mask <<= 1) merge_state(ks, mask);
         if (g == 0) {
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                sm.red_o[warp][32 * li + k] = ks.o[k].x;
-                sm.red_o[warp][32 * li + 16 + k] = ks.o[k].y;
+                sm.red_o[ring][warp][32 * li + k] = ks.o[k].x;
+                sm.red_o[ring][warp][32 * li + 16 + k] = ks.o[k].y;
             }
             if (li == 0) {
-                sm.red_m[warp] = ks.m;
-                sm.red_l[warp] = ks.l;
-                sm.red_pz[warp] = ks.pz;
+                sm.red_m[ring][warp] = ks.m;
+                sm.red_l[ring][warp] = ks.l;
+                sm.red_pz[ring][warp] = ks.pz;
             }
         }
-        named_bar_sync(1, 32 * kConsumerWarps);
-        if (!dead && rank == 0) {                 // the first warp of each query
-            float M = kMInit;
-            for (int wv = warp; wv < kConsumerWarps; wv += nq) M = fmaxf(M, sm.red_m[wv]);
-            float L = 0.f, PZ = 0.f;
-            for (int wv = warp; wv < kConsumerWarps; wv += nq) {
-                const float f = ex2(sm.red_m[wv] - M);
-                L = fmaf(sm.red_l[wv], f, L);
-                PZ = fmaf(sm.red_pz[wv], f, PZ);
-            }
-            float *part = wk.partials + ((int64_t)it * wk.qslots + slot) * (D + 4);
-            for (int chn = lane; chn < D; chn += 32) {
-                float acc = 0.f;
-                for (int wv = warp; wv < kConsumerWarps; wv += nq) acc = fmaf(sm.red_o[wv][chn], ex2(sm.red_m[wv] - M), acc);
-                part[4 + chn] = fmaf(acc, kOUnscale, PZ);
-            }
-            if (lane == 0) {
-                part[0] = M;
-                part[1] = L;
-            }
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) {
+            __threadfence_block();
+            prev = atomicAdd(&sm.merge_cnt[ring], 1);
         }
-        named_bar_sync(1, 32 * kConsumerWarps);   // red_* are reused by the next item
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == kConsumerWarps - 1) {
+            __threadfence_block();
+            if (!dead) {
+                // query sidx of the item is served by warps sidx, sidx + nq, ...; its slot in
+                // the partials is the sidx-th set bit of the mask
+                for (int sidx = 0, qi = 0; sidx < nq; ++sidx, ++qi) {
+                    while (!((qmask >> qi) & 1)) ++qi;
+                    float M = kMInit;
+                    for (int wv = sidx; wv < kConsumerWarps; wv += nq) M = fmaxf(M, sm.red_m[ring][wv]);
+                    float L = 0.f, PZ = 0.f;
+                    for (int wv = sidx; wv < kConsumerWarps; wv += nq) {
+                        const float f = ex2(sm.red_m[ring][wv] - M);
+                        L = fmaf(sm.red_l[ring][wv], f, L);
+                        PZ = fmaf(sm.red_pz[ring][wv], f, PZ);
+                    }
+                    float *part = wk.partials + ((int64_t)it * wk.qslots + qi) * (D + 4);
+                    for (int chn = lane; chn < D; chn += 32) {
+                        float acc = 0.f;
+                        for (int wv = sidx; wv < kConsumerWarps; wv += nq)
+                            acc = fmaf(sm.red_o[ring][wv][chn], ex2(sm.red_m[ring][wv] - M), acc);
+                        part[4 + chn] = fmaf(acc, kOUnscale, PZ);
+                    }
+                    if (lane == 0) {
+                        part[0] = M;
+                        part[1] = L;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) atomicExch(&sm.merge_cnt[ring], 0);   // the slot is free again
+        }
     }
 }
 

@@ -135,7 +135,7 @@ __device__ __forceinline__ void set_status(int32_t *status, int code)
 
 // ---- scheduler work list (decode) ----------------------------------------------------
 #ifndef KVQ_DECODE_ITEM_KEYS
-#define KVQ_DECODE_ITEM_KEYS 576
+#define KVQ_DECODE_ITEM_KEYS 1152
 #endif
 constexpr int kDecodeItemKeys = KVQ_DECODE_ITEM_KEYS;   // keys per split-K work item, at most (w + 1 = 513 fits one)
 constexpr int kDecodeWindowKeys = 128; // keys per window of record offsets inside an item
@@ -277,6 +277,20 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
 __device__ __forceinline__ void named_bar_sync(int id, int threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Named barrier that also ORs a predicate over the participating threads.
+__device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.u32 p, %1, 0;\n\t"
+                 "bar.red.or.pred q, %2, %3, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"((uint32_t)pred), "r"(id), "r"(threads)
+                 : "memory");
+    return r != 0;
 }
 
 // Programmatic dependent launch. A kernel launched with launch_pdl may start while the

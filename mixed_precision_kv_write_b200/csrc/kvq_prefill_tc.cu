@@ -18,7 +18,7 @@
 //     - warps 4-7: unpack each 64-key tile's K and V codes into exact fp16 operands (codes
 //       are integers <= 255; b = 16 keys are the fp16 values) in shared memory, double
 //       buffered; K 128B-swizzled K-major, V 128B-swizzled MN-major. The packed bytes are
-//       fetched one tile ahead with cp.async and the record offsets three tiles ahead.
+//       fetched two tiles ahead with cp.async and the record offsets three tiles ahead.
 //     - warp 8: owns 512 TMEM columns (S double buffer: 2 x 64, O: D, P' double buffer:
 //       2 x 64) and issues the MMAs from one lane: S = Q C_K^T (M128 N64 K16 steps, A and B
 //       in shared memory) as soon as a K tile is unpacked (up to one tile ahead), O += P'_hi V
@@ -34,6 +34,7 @@ namespace {
 constexpr int kQRows = 128;     // queries per tile (MMA M)
 constexpr int kKeys = 64;       // keys per key tile (QK MMA N, PV MMA K)
 constexpr int kTcThreads = 288; // 9 warps
+constexpr int kRawBufs = 3;     // record staging buffers: records are fetched two tiles ahead
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S double buffer at 0 and 64 (fp32), O at 128 (D columns), P' double buffer at
 // 256 and 320: each buffer holds P'_hi in 32 columns then P'_lo in 32 (fp16 pairs, the A
@@ -204,8 +205,11 @@ struct alignas(1024) PfSmem {
     __half v[2][kKeys * D];           // MN-major SW128: atom (8 keys x 64 ch) at (key/8)*(D/64)+ch/64
     float2 side_k[2][kKeys];          // (s_K * c, z_K * c) per key, c = log2(e)/sqrt(D)
     float2 side_v[2][kKeys];          // (s_V, z_V) per key
-    uint8_t raw[2][kKeys * 2][2 * D + 16]; // packed K and V bytes of each (key, half), by cp.async
+    uint8_t raw[kRawBufs][kKeys * 2][2 * D + 16]; // packed K and V bytes of each (key, half), by cp.async
                                            // (16 bytes of padding spread the slots over the banks)
+    uint16_t task[kKeys * 2];               // unpack tasks of a tile, ordered by width class
+    uint32_t task_meta[kKeys * 2];          // each task's record offset | width code
+    int32_t cls_cnt[4][5];                  // per unpack warp: tasks of each class (4 = none)
     uint64_t kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], drain;
     uint32_t tmem_base;
     int32_t klo, khi, abort_flag;
@@ -366,9 +370,10 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         mbar_wait(&sm.drain, 0, c.status);
     } else if (warp >= 4) {
         // ------------------------------ K/V unpack -----------------------------------
-        // Thread = (key of the tile, half of the channels). Two-deep prefetch: record offset
-        // and side entry of tile t+2 in registers, packed record bytes of tile t+1 copied by
-        // cp.async into this thread's own staging slot, tile t converted to fp16 operands.
+        // Thread = (key of the tile, half of the channels). Record offsets and side entries
+        // of tiles t+1 .. t+3 in registers, packed record bytes of tiles t+1 and t+2 in
+        // flight by cp.async into this thread's own staging slots, tile t converted to fp16
+        // operands.
         const int u = tid - 128;
         const int kj = u >> 1, half = u & 1;
         constexpr int CH = D / 2;                    // channels per thread
@@ -389,7 +394,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 const uint32_t part = (uint32_t)(CH * bits / 8);          // bytes of this half
                 const uint32_t ok = (mt & ~15u) + half * part;               // stream offsets
                 const uint32_t ov = (mt & ~15u) + (uint32_t)(bits * D / 8) + half * part;
-                uint8_t *dst = sm.raw[t & 1][u];
+                uint8_t *dst = sm.raw[t % kRawBufs][u];
                 if (part >= 16) {
                     for (uint32_t o = 0; o < part; o += 16) {
                         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + o)), "l"(stream.at(ok + o)) : "memory");
@@ -408,15 +413,40 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         load_meta(1, m_n1, sd_n1);
         load_meta(2, m_n2, sd_n2);
         issue_records(0, m_cur);
+        issue_records(1, m_n1);
         for (int t = 0; t < n_kt; ++t) {
             const int b = t & 1;
-            issue_records(t + 1, m_n1);
+            issue_records(t + 2, m_n2);
             load_meta(t + 3, m_n3, sd_n3);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-            if (!mbar_wait(&sm.kv_empty[b], ((t >> 1) & 1) ^ 1, c.status) ||
-                *reinterpret_cast<volatile int *>(&sm.abort_flag)) {
-                sm.abort_flag = 1;
-                break;
+            asm volatile("cp.async.wait_group 2;" ::: "memory");   // tile t's group has landed
+            const bool waited = mbar_wait(&sm.kv_empty[b], ((t >> 1) & 1) ^ 1, c.status);
+            // Order the tile's 128 (key, half) tasks by width class, so that a warp's lanes
+            // run one width's conversion (the staged bytes of every task are visible to all
+            // unpack threads after the barrier). The barrier also makes the decision to stop
+            // (a timed-out wait, an abort) the same for all unpack threads.
+            {
+                const int cl = (m_cur == kNone) ? 4 : (int)(m_cur & 3u);
+                const int uw = u >> 5, ul = u & 31;
+                int rank = 0;
+#pragma unroll
+                for (int c2 = 0; c2 < 5; ++c2) {
+                    const uint32_t bal = __ballot_sync(0xffffffffu, cl == c2);
+                    if (cl == c2) rank = __popc(bal & ((1u << ul) - 1u));
+                    if (ul == 0) sm.cls_cnt[uw][c2] = __popc(bal);
+                }
+                if (named_bar_or(2, 128, !waited || *reinterpret_cast<volatile int *>(&sm.abort_flag))) {
+                    sm.abort_flag = 1;
+                    break;
+                }
+                int pos = rank;
+#pragma unroll
+                for (int c2 = 0; c2 < 5; ++c2)
+#pragma unroll
+                    for (int w2 = 0; w2 < 4; ++w2)
+                        pos += (c2 < cl || (c2 == cl && w2 < uw)) ? sm.cls_cnt[w2][c2] : 0;
+                sm.task[pos] = (uint16_t)u;
+                sm.task_meta[pos] = m_cur;
+                named_bar_sync(2, 128);
             }
             uint8_t *kb = reinterpret_cast<uint8_t *>(sm.k[b]);
             uint8_t *vb = reinterpret_cast<uint8_t *>(sm.v[b]);
@@ -425,17 +455,20 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 sm.side_k[b][kj] = make_float2(sd_cur.x * lsc, sd_cur.y * lsc);
                 sm.side_v[b][kj] = make_float2(sd_cur.z, sd_cur.w);
             }
-            const uint8_t *src = sm.raw[b][u];
-            const int bits = (m_cur == kNone) ? 0 : (2 << (m_cur & 3u));
+            const int tu = sm.task[u];                    // this thread's task
+            const uint32_t tmeta = sm.task_meta[u];
+            const int tkj = tu >> 1, thalf = tu & 1;
+            const uint8_t *src = sm.raw[t % kRawBufs][tu];
+            const int bits = (tmeta == kNone) ? 0 : (2 << (tmeta & 3u));
 #pragma unroll
             for (int cc = 0; cc < CH / 8; ++cc) {
-                const int chunk = half * (CH / 8) + cc;       // 8-channel chunk of the row
+                const int chunk = thalf * (CH / 8) + cc;      // 8-channel chunk of the row
                 const uint4 kx = bits ? unpack8(src, bits, cc) : make_uint4(0, 0, 0, 0);
                 const uint4 vx = bits ? unpack8(src + D, bits, cc) : make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(kj, chunk & 7)) = kx;
+                *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(tkj, chunk & 7)) = kx;
                 const int n = chunk * 8;
-                const int atom = (kj >> 3) * (D / 64) + (n >> 6);
-                *reinterpret_cast<uint4 *>(vb + atom * 1024 + (kj & 7) * 128 + ((((n & 63) >> 3) ^ (kj & 7)) << 4)) = vx;
+                const int atom = (tkj >> 3) * (D / 64) + (n >> 6);
+                *reinterpret_cast<uint4 *>(vb + atom * 1024 + (tkj & 7) * 128 + ((((n & 63) >> 3) ^ (tkj & 7)) << 4)) = vx;
             }
             fence_async_smem();
             mbar_arrive(&sm.kv_full[b]);

@@ -135,6 +135,7 @@ write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *
 constexpr int kWqThreads = 128;
 constexpr int kWqHalves = 4096;          // 8 KB of K and 8 KB of V per CTA
 constexpr int kWqMaxPairs = kWqHalves / 64;
+static_assert(kWqMaxPairs <= kWqThreads, "one (token, head) pair per thread");
 
 struct WqPair {                          // one (token, head) of the CTA
     int64_t slot;                        // side-table slot
@@ -163,7 +164,9 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
     __shared__ uint8_t order[kWqMaxPairs];   // written pairs sorted by width
     __shared__ int n_written;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    pdl_wait();
+    // Launched right after the scan kernel: the K/V copies and the sequence lookup read only
+    // the call's inputs and start before the scan has finished; pdl_wait() below comes
+    // before the first read of what the scan writes (widths verdict, write start, offsets).
     pdl_trigger();
     const int H = c.H;
     const int64_t t0 = (int64_t)blockIdx.x * T;
@@ -194,22 +197,29 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
         }
     }
 
-    for (int i = tid; i < Tc * HGc; i += kWqThreads) {
-        const int64_t tk = t0 + i / HGc;
-        const int h = h0 + i % HGc;
-        WqPair pr;
-        pr.slot = 0;
-        pr.meta = 0;
-        pr.s = -1;
-        pr.h = h;
-        pr.pad = 0;
+    // one (token, head) pair per thread (at most kWqMaxPairs <= kWqThreads pairs per tile)
+    const int i = tid;
+    const bool has_pair = i < Tc * HGc;
+    const int64_t tk = t0 + i / max(HGc, 1);
+    const int h = h0 + i % max(HGc, 1);
+    int s = 0;
+    if (has_pair) {
         int lo = 0, hi = c.B;                // cu[lo] <= tk < cu[hi]
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
             if (cu[mid] <= tk) lo = mid;
             else hi = mid;
         }
-        const int s = lo;
+        s = lo;
+    }
+    pdl_wait();
+    if (has_pair) {
+        WqPair pr;
+        pr.slot = 0;
+        pr.meta = 0;
+        pr.s = -1;
+        pr.h = h;
+        pr.pad = 0;
         if (tk < cu[s + 1] && c.bad[s] != gen) {
             const int st = c.wstart[s * H + h];
             if (st >= 0) {
