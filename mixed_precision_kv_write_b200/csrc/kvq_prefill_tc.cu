@@ -33,7 +33,16 @@ namespace {
 
 constexpr int kQRows = 128;     // queries per tile (MMA M)
 constexpr int kKeys = 64;       // keys per key tile (QK MMA N, PV MMA K)
-constexpr int kTcThreads = 288; // 9 warps
+// 16 warps: 0-3 softmax rows, 4-11 K/V unpack, 12 MMA issuer (13-15 idle, present so that
+// the MMA warp's warpgroup is whole for the register split below)
+constexpr int kTcThreads = 512;
+constexpr int kUnpackWarps = 8, kUnpackThreads = 32 * kUnpackWarps;
+constexpr int kMmaWarp = 4 + kUnpackWarps;
+constexpr int kQP = kUnpackThreads / 64;   // unpack threads per key (the tile's 64 keys)
+// Registers per thread after the split (launch: 128 x 512 threads = 65536): softmax 200,
+// unpack 96, MMA warpgroup 80: 128 x (200 + 2 x 96 + 80) = 60416 <= 65536.
+constexpr int kRegSoftmax = 200, kRegUnpack = 96, kRegMma = 80;
+static_assert(128 * (kRegSoftmax + 2 * kRegUnpack + kRegMma) <= 65536, "register split exceeds the launch");
 constexpr int kRawBufs = 3;     // record staging buffers: records are fetched two tiles ahead
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S double buffer at 0 and 64 (fp32), O at 128 (D columns), P' double buffer at
@@ -205,11 +214,11 @@ struct alignas(1024) PfSmem {
     __half v[2][kKeys * D];           // MN-major SW128: atom (8 keys x 64 ch) at (key/8)*(D/64)+ch/64
     float2 side_k[2][kKeys];          // (s_K * c, z_K * c) per key, c = log2(e)/sqrt(D)
     float2 side_v[2][kKeys];          // (s_V, z_V) per key
-    uint8_t raw[kRawBufs][kKeys * 2][2 * D + 16]; // packed K and V bytes of each (key, half), by cp.async
+    uint8_t raw[kRawBufs][kUnpackThreads][4 * (D / kQP) + 16]; // packed K and V bytes of each (key, part)
                                            // (16 bytes of padding spread the slots over the banks)
-    uint16_t task[kKeys * 2];               // unpack tasks of a tile, ordered by width class
-    uint32_t task_meta[kKeys * 2];          // each task's record offset | width code
-    int32_t cls_cnt[4][5];                  // per unpack warp: tasks of each class (4 = none)
+    uint16_t task[kUnpackThreads];          // unpack tasks of a tile, ordered by width class
+    uint32_t task_meta[kUnpackThreads];     // each task's record offset | width code
+    int32_t cls_cnt[kUnpackWarps][5];       // per unpack warp: tasks of each class (4 = none)
     uint64_t kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], drain;
     uint32_t tmem_base;
     int32_t klo, khi, abort_flag;
@@ -236,7 +245,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.kv_full[i], 128);
+            mbar_init(&sm.kv_full[i], kUnpackThreads);
             mbar_init(&sm.kv_empty[i], 1);
         }
         mbar_init(&sm.s_full[0], 1);
@@ -251,7 +260,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(&sm.tmem_base)), "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -291,8 +300,13 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     const int klo = sm.klo, khi = sm.khi;
     const int n_kt = (khi >= klo) ? (khi - klo + kKeys) / kKeys : 0;
     const uint32_t tmem = sm.tmem_base;
-
-    if (warp == 8) {
+    // Register split by warpgroup, at the head of each role: the softmax rows take what the
+    // unpack and MMA warpgroups give back (the sum stays within the launch's allocation,
+    // see kRegSoftmax).
+    if (warp >= kMmaWarp) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegMma));
+    }
+    if (warp == kMmaWarp) {
         // ------------------------------- MMA issuer --------------------------------
         // order: QK(0), then per tile t: QK(t+1) into the other S buffer, wait P(t), PV(t)
         const uint32_t q0 = smem_u32(sm.q);
@@ -368,15 +382,16 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         if (lane == 0) umma_commit(&sm.drain);
         __syncwarp();
         mbar_wait(&sm.drain, 0, c.status);
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < kMmaWarp) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegUnpack));
         // ------------------------------ K/V unpack -----------------------------------
-        // Thread = (key of the tile, half of the channels). Record offsets and side entries
-        // of tiles t+1 .. t+3 in registers, packed record bytes of tiles t+1 and t+2 in
-        // flight by cp.async into this thread's own staging slots, tile t converted to fp16
-        // operands.
+        // Thread = (key of the tile, a quarter of the channels). Record offsets and side
+        // entries of tiles t+1 .. t+3 in registers, packed record bytes of tiles t+1 and t+2
+        // in flight by cp.async into this thread's own staging slots, tile t converted to
+        // fp16 operands.
         const int u = tid - 128;
-        const int kj = u >> 1, half = u & 1;
-        constexpr int CH = D / 2;                    // channels per thread
+        const int kj = u / kQP, half = u % kQP;     // (key, channel part)
+        constexpr int CH = D / kQP;                  // channels per thread
         constexpr uint32_t kNone = 0xFFFFFFFFu;
         auto load_meta = [&](int t, uint32_t &mt, float4 &sd) {
             const int j = klo + t * kKeys + kj;
@@ -391,18 +406,22 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         auto issue_records = [&](int t, uint32_t mt) {
             if (t < n_kt && mt != kNone) {
                 const int bits = 2 << (mt & 3u);
-                const uint32_t part = (uint32_t)(CH * bits / 8);          // bytes of this half
+                const uint32_t part = (uint32_t)(CH * bits / 8);          // bytes of this part
                 const uint32_t ok = (mt & ~15u) + half * part;               // stream offsets
                 const uint32_t ov = (mt & ~15u) + (uint32_t)(bits * D / 8) + half * part;
                 uint8_t *dst = sm.raw[t % kRawBufs][u];
+                constexpr uint32_t kVo = 2 * CH;                             // V part in the slot
                 if (part >= 16) {
                     for (uint32_t o = 0; o < part; o += 16) {
                         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + o)), "l"(stream.at(ok + o)) : "memory");
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + D + o)), "l"(stream.at(ov + o)) : "memory");
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + kVo + o)), "l"(stream.at(ov + o)) : "memory");
                     }
-                } else {                                                   // 8 bytes (head_dim 64, b = 2)
+                } else if (part == 8) {
                     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(stream.at(ok)) : "memory");
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst + D)), "l"(stream.at(ov)) : "memory");
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst + kVo)), "l"(stream.at(ov)) : "memory");
+                } else {                                                   // 4 bytes (head_dim 64, b = 2)
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(stream.at(ok)) : "memory");
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst + kVo)), "l"(stream.at(ov)) : "memory");
                 }
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
@@ -416,11 +435,10 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         issue_records(1, m_n1);
         for (int t = 0; t < n_kt; ++t) {
             const int b = t & 1;
-            issue_records(t + 2, m_n2);
             load_meta(t + 3, m_n3, sd_n3);
-            asm volatile("cp.async.wait_group 2;" ::: "memory");   // tile t's group has landed
+            asm volatile("cp.async.wait_group 1;" ::: "memory");   // tile t's group has landed
             const bool waited = mbar_wait(&sm.kv_empty[b], ((t >> 1) & 1) ^ 1, c.status);
-            // Order the tile's 128 (key, half) tasks by width class, so that a warp's lanes
+            // Order the tile's 256 (key, part) tasks by width class, so that a warp's lanes
             // run one width's conversion (the staged bytes of every task are visible to all
             // unpack threads after the barrier). The barrier also makes the decision to stop
             // (a timed-out wait, an abort) the same for all unpack threads.
@@ -434,19 +452,22 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                     if (cl == c2) rank = __popc(bal & ((1u << ul) - 1u));
                     if (ul == 0) sm.cls_cnt[uw][c2] = __popc(bal);
                 }
-                if (named_bar_or(2, 128, !waited || *reinterpret_cast<volatile int *>(&sm.abort_flag))) {
+                if (named_bar_or(2, kUnpackThreads, !waited || *reinterpret_cast<volatile int *>(&sm.abort_flag))) {
                     sm.abort_flag = 1;
                     break;
                 }
+                // every unpack thread is past tile t-1's conversion, which read the staging
+                // buffer that tile t+2's records now go to
+                issue_records(t + 2, m_n2);
                 int pos = rank;
 #pragma unroll
                 for (int c2 = 0; c2 < 5; ++c2)
 #pragma unroll
-                    for (int w2 = 0; w2 < 4; ++w2)
+                    for (int w2 = 0; w2 < kUnpackWarps; ++w2)
                         pos += (c2 < cl || (c2 == cl && w2 < uw)) ? sm.cls_cnt[w2][c2] : 0;
                 sm.task[pos] = (uint16_t)u;
                 sm.task_meta[pos] = m_cur;
-                named_bar_sync(2, 128);
+                named_bar_sync(2, kUnpackThreads);
             }
             uint8_t *kb = reinterpret_cast<uint8_t *>(sm.k[b]);
             uint8_t *vb = reinterpret_cast<uint8_t *>(sm.v[b]);
@@ -457,14 +478,14 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             }
             const int tu = sm.task[u];                    // this thread's task
             const uint32_t tmeta = sm.task_meta[u];
-            const int tkj = tu >> 1, thalf = tu & 1;
+            const int tkj = tu / kQP, thalf = tu % kQP;
             const uint8_t *src = sm.raw[t % kRawBufs][tu];
             const int bits = (tmeta == kNone) ? 0 : (2 << (tmeta & 3u));
 #pragma unroll
             for (int cc = 0; cc < CH / 8; ++cc) {
                 const int chunk = thalf * (CH / 8) + cc;      // 8-channel chunk of the row
                 const uint4 kx = bits ? unpack8(src, bits, cc) : make_uint4(0, 0, 0, 0);
-                const uint4 vx = bits ? unpack8(src + D, bits, cc) : make_uint4(0, 0, 0, 0);
+                const uint4 vx = bits ? unpack8(src + 2 * CH, bits, cc) : make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(tkj, chunk & 7)) = kx;
                 const int n = chunk * 8;
                 const int atom = (tkj >> 3) * (D / 64) + (n >> 6);
@@ -480,7 +501,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             sd_n2 = sd_n3;
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-    } else {
+    } else if (warp < 4) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
         // ------------------------------ softmax rows ---------------------------------
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         float m_run = -INFINITY, l_run = 0.f, pz_run = 0.f;
@@ -602,7 +624,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     // ---- teardown: every role ends here; TMEM is freed even after an abort ----
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }

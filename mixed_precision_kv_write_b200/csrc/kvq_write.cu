@@ -132,8 +132,14 @@ write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *
 
 // Staging of the quantize kernel: each CTA copies the fp16 K and V rows of T tokens x HG
 // heads (at most kWqHalves values per tensor) into shared memory with two bulk copies.
-constexpr int kWqThreads = 128;
-constexpr int kWqHalves = 4096;          // 8 KB of K and 8 KB of V per CTA
+#ifndef KVQ_WQ_THREADS
+#define KVQ_WQ_THREADS 128
+#endif
+#ifndef KVQ_WQ_HALVES
+#define KVQ_WQ_HALVES 8192
+#endif
+constexpr int kWqThreads = KVQ_WQ_THREADS;
+constexpr int kWqHalves = KVQ_WQ_HALVES; // fp16 values of K (and of V) staged per CTA
 constexpr int kWqMaxPairs = kWqHalves / 64;
 static_assert(kWqMaxPairs <= kWqThreads, "one (token, head) pair per thread");
 
@@ -329,6 +335,9 @@ cudaError_t launch_write(kvq_cache *cache, const __half *k, const __half *v,
         if (n_tok < (int64_t)T * 2 * num_sms()) T = 1;
         const dim3 grid((unsigned)((n_tok + T - 1) / T), (unsigned)((c.H + HG - 1) / HG));
         const size_t smem = 2 * kWqHalves * sizeof(__half);
+        le = (c.D == 128) ? ensure_smem_attr((const void *)write_quant_kernel<128>, smem)
+                          : ensure_smem_attr((const void *)write_quant_kernel<64>, smem);
+        if (le != cudaSuccess) return le;
         if (c.D == 128)
             le = launch_pdl(write_quant_kernel<128>, grid, dim3(kWqThreads), smem, st, c, k, v, cu, n_tok, gen, T, HG);
         else
