@@ -232,8 +232,9 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
 {
     if ((int)blockIdx.x >= *tile_count) return;
     extern __shared__ uint8_t smem_raw[];
-    PfSmem<D> &sm = *reinterpret_cast<PfSmem<D> *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned (the 128B-swizzled operand tiles): offset the shared pointer itself,
+    // so that the compiler keeps every access in the shared address space
+    PfSmem<D> &sm = *reinterpret_cast<PfSmem<D> *>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const PfTile tile = tiles[blockIdx.x];
     // tile.sh = (sequence, query head); query head hq reads KV head hq / G

@@ -334,6 +334,7 @@ cudaError_t launch_write(kvq_cache *cache, const __half *k, const __half *v,
         int T = std::max(1, kWqHalves / (HG * c.D));
         if (n_tok < (int64_t)T * 2 * num_sms()) T = 1;
         const dim3 grid((unsigned)((n_tok + T - 1) / T), (unsigned)((c.H + HG - 1) / HG));
+
         const size_t smem = 2 * kWqHalves * sizeof(__half);
         le = (c.D == 128) ? ensure_smem_attr((const void *)write_quant_kernel<128>, smem)
                           : ensure_smem_attr((const void *)write_quant_kernel<64>, smem);
