@@ -33,17 +33,18 @@ namespace {
 
 constexpr int kQRows = 128;     // queries per tile (MMA M)
 constexpr int kKeys = 64;       // keys per key tile (QK MMA N, PV MMA K)
-// 16 warps: 0-3 softmax rows, 4-11 K/V unpack, 12 MMA issuer (13-15 idle, present so that
-// the MMA warp's warpgroup is whole for the register split below)
+// 16 warps: 0-3 softmax rows, 4-11 K/V unpack, 12 MMA issuer, 13 record stager (14-15 idle,
+// present so that the last warpgroup is whole for the register split below)
 constexpr int kTcThreads = 512;
 constexpr int kUnpackWarps = 8, kUnpackThreads = 32 * kUnpackWarps;
 constexpr int kMmaWarp = 4 + kUnpackWarps;
+constexpr int kStageWarp = kMmaWarp + 1;
 constexpr int kQP = kUnpackThreads / 64;   // unpack threads per key (the tile's 64 keys)
 // Registers per thread after the split (launch: 128 x 512 threads = 65536): softmax 200,
 // unpack 96, MMA warpgroup 80: 128 x (200 + 2 x 96 + 80) = 60416 <= 65536.
 constexpr int kRegSoftmax = 200, kRegUnpack = 96, kRegMma = 80;
 static_assert(128 * (kRegSoftmax + 2 * kRegUnpack + kRegMma) <= 65536, "register split exceeds the launch");
-constexpr int kRawBufs = 3;     // record staging buffers: records are fetched two tiles ahead
+constexpr int kRawBufs = 3;     // record staging buffers: a key tile's records land up to three tiles ahead
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S double buffer at 0 and 64 (fp32), O at 128 (D columns), P' double buffer at
 // 256 and 320: each buffer holds P'_hi in 32 columns then P'_lo in 32 (fp16 pairs, the A
@@ -108,6 +109,32 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 64 consecutive columns of this warp's 32 lanes, one load and one wait
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64])
+{
+    uint32_t r[64];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+                 "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+                 "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+                   "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+                   "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+                   "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+                   "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+                   "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+                   "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+                   "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+                   "=r"(r[62]), "=r"(r[63])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
@@ -194,11 +221,12 @@ __device__ __forceinline__ uint4 unpack8(const uint8_t *part, int bits, int chun
 }
 
 // 2^x with the hardware's approximate exp2 (relative error of a few ulp), used for the
-// softmax weights; 2^-inf = 0.
+// softmax weights; 2^-inf = 0. Results below 2^-126 flush to zero: a weight that small is
+// below 2^-118 of the row's sum (which holds a weight >= 2^-8), far under the tolerance.
 __device__ __forceinline__ float ex2(float x)
 {
     float y;
-    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 
@@ -212,13 +240,15 @@ struct alignas(1024) PfSmem {
     __half q[kQRows * D];             // K-major SW128, D/64 blocks of 128 rows x 128 B
     __half k[2][kKeys * D];           // K-major SW128, D/64 blocks of 64 rows x 128 B
     __half v[2][kKeys * D];           // MN-major SW128: atom (8 keys x 64 ch) at (key/8)*(D/64)+ch/64
-    float2 side_k[2][kKeys];          // (s_K * c, z_K * c) per key, c = log2(e)/sqrt(D)
-    float2 side_v[2][kKeys];          // (s_V, z_V) per key
-    uint8_t raw[kRawBufs][kUnpackThreads][4 * (D / kQP) + 16]; // packed K and V bytes of each (key, part)
-                                           // (16 bytes of padding spread the slots over the banks)
-    uint16_t task[kUnpackThreads];          // unpack tasks of a tile, ordered by width class
-    uint32_t task_meta[kUnpackThreads];     // each task's record offset | width code
-    int32_t cls_cnt[kUnpackWarps][5];       // per unpack warp: tasks of each class (4 = none)
+    // side entries of key pairs (2j, 2j + 1), laid out for packed fp32 arithmetic:
+    float4 side_k[2][kKeys / 2];      // (s_K c, s_K c, z_K c, z_K c), c = log2(e)/sqrt(D)
+    float4 side_v[2][kKeys / 2];      // (s_V, s_V, z_V, z_V)
+    uint8_t raw[kRawBufs][kKeys * 4 * D];   // a key tile's records as stored (one contiguous range
+                                            // of the stream; at most 64 keys x 2 x D fp16 values)
+    // the tile's 256 conversion tasks (key, part), ordered by width class:
+    // offset of the key's record in raw << 16 | class << 8 | key << 2 | part (class 4: no key)
+    uint32_t task[kRawBufs][kUnpackThreads];
+    uint64_t raw_full[kRawBufs], raw_empty[kRawBufs];
     uint64_t kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], drain;
     uint32_t tmem_base;
     int32_t klo, khi, abort_flag;
@@ -246,8 +276,12 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.kv_full[i], kUnpackThreads);
+            mbar_init(&sm.kv_full[i], kUnpackWarps);
             mbar_init(&sm.kv_empty[i], 1);
+        }
+        for (int i = 0; i < kRawBufs; ++i) {
+            mbar_init(&sm.raw_full[i], 1);
+            mbar_init(&sm.raw_empty[i], kUnpackWarps);
         }
         mbar_init(&sm.s_full[0], 1);
         mbar_init(&sm.s_full[1], 1);
@@ -383,130 +417,143 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         if (lane == 0) umma_commit(&sm.drain);
         __syncwarp();
         mbar_wait(&sm.drain, 0, c.status);
+    } else if (warp == kStageWarp) {
+        // ------------------------------ record stager ------------------------------------
+        // Per key tile: the 64 keys' record words, the tile's byte range in the stream (the
+        // records of consecutive keys are contiguous), one bulk copy of that range (cut at
+        // page ends) into a staging buffer, and the conversion tasks ordered by width class
+        // so that each unpack warp's lanes run one width's conversion.
+        constexpr uint32_t kNone = 0xFFFFFFFFu;
+        auto meta_of = [&](int t, int k) -> uint32_t {
+            const int j = klo + t * kKeys + k;
+            return (t < n_kt && j <= khi) ? c.meta[sbase + j] : kNone;
+        };
+        uint32_t ma = meta_of(0, lane), mb = meta_of(0, 32 + lane);
+        const uint32_t lt = (1u << lane) - 1u;
+        int issued = 0;
+        for (int t = 0; t < n_kt; ++t) {
+            const int st = t % kRawBufs;
+            const uint32_t na = meta_of(t + 1, lane), nb = meta_of(t + 1, 32 + lane);   // next tile, in flight
+            if (t >= kRawBufs &&
+                !__all_sync(0xffffffffu, mbar_wait(&sm.raw_empty[st], ((t / kRawBufs) - 1) & 1, c.status) &&
+                                             !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
+                sm.abort_flag = 1;
+                break;
+            }
+            const int ca = (ma == kNone) ? 4 : (int)(ma & 3u), cb = (mb == kNone) ? 4 : (int)(mb & 3u);
+            // byte range: from the first key's record (always present) to the end of the last
+            const uint32_t base = __shfl_sync(0xffffffffu, ma, 0) & ~15u;
+            const uint32_t va = __ballot_sync(0xffffffffu, ma != kNone), vb = __ballot_sync(0xffffffffu, mb != kNone);
+            const int last = vb ? 63 - __clz(vb) : 31 - __clz(va);
+            const uint32_t ml = __shfl_sync(0xffffffffu, last >= 32 ? mb : ma, last & 31);
+            const uint32_t end = (ml & ~15u) + (uint32_t)((2 << (ml & 3u)) * D / 4);    // K and V parts
+            if (end - base > (uint32_t)sizeof(sm.raw[0])) {      // records not contiguous: corrupt cache
+                if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+                sm.abort_flag = 1;
+                break;
+            }
+            // stable order by class (none last): key position among the tile's keys
+            int pa = 0, pb = 0, start = 0;
+#pragma unroll
+            for (int c2 = 0; c2 < 5; ++c2) {
+                const uint32_t ba = __ballot_sync(0xffffffffu, ca == c2), bb = __ballot_sync(0xffffffffu, cb == c2);
+                if (ca == c2) pa = start + __popc(ba & lt);
+                if (cb == c2) pb = start + __popc(ba) + __popc(bb & lt);
+                start += __popc(ba) + __popc(bb);
+            }
+            const uint32_t wa = ((ca < 4 ? (ma & ~15u) - base : 0u) << 16) | ((uint32_t)ca << 8) | ((uint32_t)lane << 2);
+            const uint32_t wb = ((cb < 4 ? (mb & ~15u) - base : 0u) << 16) | ((uint32_t)cb << 8) | ((uint32_t)(32 + lane) << 2);
+            *reinterpret_cast<uint4 *>(&sm.task[st][4 * pa]) = make_uint4(wa, wa | 1u, wa | 2u, wa | 3u);
+            *reinterpret_cast<uint4 *>(&sm.task[st][4 * pb]) = make_uint4(wb, wb | 1u, wb | 2u, wb | 3u);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.raw_full[st], end - base);
+                for (uint32_t o = base; o < end;) {
+                    uint32_t e2 = end;
+                    if (stream.pt) {                          // not past the page holding o
+                        const uint32_t pg_end = (((stream.off + o) >> stream.shift) + 1u) << stream.shift;
+                        e2 = min(end, pg_end - stream.off);
+                    }
+                    bulk_g2s(sm.raw[st] + (o - base), stream.at(o), e2 - o, &sm.raw_full[st]);
+                    o = e2;
+                }
+            }
+            __syncwarp();
+            ++issued;
+            ma = na;
+            mb = nb;
+        }
+        // the staging buffers must not receive bytes after the CTA ends: wait (bounded) for
+        // the copies of the last tiles (earlier ones were consumed before their buffer came back)
+        for (int t = max(0, issued - kRawBufs); t < issued; ++t)
+            mbar_wait(&sm.raw_full[t % kRawBufs], (t / kRawBufs) & 1, c.status);
     } else if (warp >= 4 && warp < kMmaWarp) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegUnpack));
         // ------------------------------ K/V unpack -----------------------------------
-        // Thread = (key of the tile, a quarter of the channels). Record offsets and side
-        // entries of tiles t+1 .. t+3 in registers, packed record bytes of tiles t+1 and t+2
-        // in flight by cp.async into this thread's own staging slots, tile t converted to
-        // fp16 operands.
+        // Thread = one conversion task of the tile (a key, a quarter of its channels), as
+        // ordered by the stager; the side entry of its own key kj = u / 4 is loaded three
+        // tiles ahead.
         const int u = tid - 128;
-        const int kj = u / kQP, half = u % kQP;     // (key, channel part)
-        constexpr int CH = D / kQP;                  // channels per thread
-        constexpr uint32_t kNone = 0xFFFFFFFFu;
-        auto load_meta = [&](int t, uint32_t &mt, float4 &sd) {
+        const int kj = u / kQP, half = u % kQP;
+        constexpr int CH = D / kQP;                  // channels per task
+        auto load_side = [&](int t) -> float4 {
             const int j = klo + t * kKeys + kj;
-            if (t < n_kt && j <= khi) {
-                mt = c.meta[sbase + j];
-                sd = c.side[sbase + j];
-            } else {
-                mt = kNone;
-                sd = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            return (half == 0 && t < n_kt && j <= khi) ? c.side[sbase + j] : make_float4(0.f, 0.f, 0.f, 0.f);
         };
-        auto issue_records = [&](int t, uint32_t mt) {
-            if (t < n_kt && mt != kNone) {
-                const int bits = 2 << (mt & 3u);
-                const uint32_t part = (uint32_t)(CH * bits / 8);          // bytes of this part
-                const uint32_t ok = (mt & ~15u) + half * part;               // stream offsets
-                const uint32_t ov = (mt & ~15u) + (uint32_t)(bits * D / 8) + half * part;
-                uint8_t *dst = sm.raw[t % kRawBufs][u];
-                constexpr uint32_t kVo = 2 * CH;                             // V part in the slot
-                if (part >= 16) {
-                    for (uint32_t o = 0; o < part; o += 16) {
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + o)), "l"(stream.at(ok + o)) : "memory");
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst + kVo + o)), "l"(stream.at(ov + o)) : "memory");
-                    }
-                } else if (part == 8) {
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(stream.at(ok)) : "memory");
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst + kVo)), "l"(stream.at(ov)) : "memory");
-                } else {                                                   // 4 bytes (head_dim 64, b = 2)
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(stream.at(ok)) : "memory");
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst + kVo)), "l"(stream.at(ov)) : "memory");
-                }
-            }
-            asm volatile("cp.async.commit_group;" ::: "memory");
-        };
-        uint32_t m_cur, m_n1, m_n2, m_n3;
-        float4 sd_cur, sd_n1, sd_n2, sd_n3;
-        load_meta(0, m_cur, sd_cur);
-        load_meta(1, m_n1, sd_n1);
-        load_meta(2, m_n2, sd_n2);
-        issue_records(0, m_cur);
-        issue_records(1, m_n1);
+        float4 sd_cur = load_side(0), sd_n1 = load_side(1), sd_n2 = load_side(2);
         for (int t = 0; t < n_kt; ++t) {
-            const int b = t & 1;
-            load_meta(t + 3, m_n3, sd_n3);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");   // tile t's group has landed
-            const bool waited = mbar_wait(&sm.kv_empty[b], ((t >> 1) & 1) ^ 1, c.status);
-            // Order the tile's 256 (key, part) tasks by width class, so that a warp's lanes
-            // run one width's conversion (the staged bytes of every task are visible to all
-            // unpack threads after the barrier). The barrier also makes the decision to stop
-            // (a timed-out wait, an abort) the same for all unpack threads.
-            {
-                const int cl = (m_cur == kNone) ? 4 : (int)(m_cur & 3u);
-                const int uw = u >> 5, ul = u & 31;
-                int rank = 0;
-#pragma unroll
-                for (int c2 = 0; c2 < 5; ++c2) {
-                    const uint32_t bal = __ballot_sync(0xffffffffu, cl == c2);
-                    if (cl == c2) rank = __popc(bal & ((1u << ul) - 1u));
-                    if (ul == 0) sm.cls_cnt[uw][c2] = __popc(bal);
-                }
-                if (named_bar_or(2, kUnpackThreads, !waited || *reinterpret_cast<volatile int *>(&sm.abort_flag))) {
-                    sm.abort_flag = 1;
-                    break;
-                }
-                // every unpack thread is past tile t-1's conversion, which read the staging
-                // buffer that tile t+2's records now go to
-                issue_records(t + 2, m_n2);
-                int pos = rank;
-#pragma unroll
-                for (int c2 = 0; c2 < 5; ++c2)
-#pragma unroll
-                    for (int w2 = 0; w2 < kUnpackWarps; ++w2)
-                        pos += (c2 < cl || (c2 == cl && w2 < uw)) ? sm.cls_cnt[w2][c2] : 0;
-                sm.task[pos] = (uint16_t)u;
-                sm.task_meta[pos] = m_cur;
-                named_bar_sync(2, kUnpackThreads);
+            const int b = t & 1, st = t % kRawBufs;
+            const float4 sd_n3 = load_side(t + 3);
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.raw_full[st], (t / kRawBufs) & 1, c.status) &&
+                                             mbar_wait(&sm.kv_empty[b], ((t >> 1) & 1) ^ 1, c.status) &&
+                                             !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
+                sm.abort_flag = 1;
+                break;
             }
             uint8_t *kb = reinterpret_cast<uint8_t *>(sm.k[b]);
             uint8_t *vb = reinterpret_cast<uint8_t *>(sm.v[b]);
             if (half == 0) {
                 const float lsc = kLog2e * rsqrtf((float)D);
-                sm.side_k[b][kj] = make_float2(sd_cur.x * lsc, sd_cur.y * lsc);
-                sm.side_v[b][kj] = make_float2(sd_cur.z, sd_cur.w);
+                float *sk = reinterpret_cast<float *>(&sm.side_k[b][kj >> 1]) + (kj & 1);
+                float *sv = reinterpret_cast<float *>(&sm.side_v[b][kj >> 1]) + (kj & 1);
+                sk[0] = sd_cur.x * lsc;
+                sk[2] = sd_cur.y * lsc;
+                sv[0] = sd_cur.z;
+                sv[2] = sd_cur.w;
             }
-            const int tu = sm.task[u];                    // this thread's task
-            const uint32_t tmeta = sm.task_meta[u];
-            const int tkj = tu / kQP, thalf = tu % kQP;
-            const uint8_t *src = sm.raw[t % kRawBufs][tu];
-            const int bits = (tmeta == kNone) ? 0 : (2 << (tmeta & 3u));
+            const uint32_t task = sm.task[st][u];
+            const int cls = (int)((task >> 8) & 7u), tkj = (int)((task >> 2) & 63u), thalf = (int)(task & 3u);
+            const int bits = (cls < 4) ? (2 << cls) : 0;
+            const uint8_t *rec = sm.raw[st] + (task >> 16);
+            const uint8_t *ksrc = rec + thalf * (CH * bits / 8);
+            const uint8_t *vsrc = ksrc + bits * D / 8;
 #pragma unroll
             for (int cc = 0; cc < CH / 8; ++cc) {
                 const int chunk = thalf * (CH / 8) + cc;      // 8-channel chunk of the row
-                const uint4 kx = bits ? unpack8(src, bits, cc) : make_uint4(0, 0, 0, 0);
-                const uint4 vx = bits ? unpack8(src + 2 * CH, bits, cc) : make_uint4(0, 0, 0, 0);
+                const uint4 kx = bits ? unpack8(ksrc, bits, cc) : make_uint4(0, 0, 0, 0);
+                const uint4 vx = bits ? unpack8(vsrc, bits, cc) : make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(tkj, chunk & 7)) = kx;
                 const int n = chunk * 8;
                 const int atom = (tkj >> 3) * (D / 64) + (n >> 6);
                 *reinterpret_cast<uint4 *>(vb + atom * 1024 + (tkj & 7) * 128 + ((((n & 63) >> 3) ^ (tkj & 7)) << 4)) = vx;
             }
             fence_async_smem();
-            mbar_arrive(&sm.kv_full[b]);
-            m_cur = m_n1;
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.kv_full[b]);
+                mbar_arrive(&sm.raw_empty[st]);
+            }
             sd_cur = sd_n1;
-            m_n1 = m_n2;
             sd_n1 = sd_n2;
-            m_n2 = m_n3;
             sd_n2 = sd_n3;
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < 4) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
         // ------------------------------ softmax rows ---------------------------------
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        float m_run = -INFINITY, l_run = 0.f, pz_run = 0.f;
+        float m_run = -INFINITY;
+        float2 l_run = make_float2(0.f, 0.f), pz_run = make_float2(0.f, 0.f);   // even / odd keys
+        const float2 qs2 = make_float2(qsum, qsum);
         bool ok = true;
         for (int t = 0; t < n_kt; ++t) {
             const int b = t & 1;
@@ -519,45 +566,73 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             }
             tc_fence_after();
             const int kt0 = klo + t * kKeys;
-            float lg[kKeys];
             // the row's keys in this tile: [max(row_lo, kt0), min(row_t, kt0 + 63)]
             const int c_lo = max(row_lo - kt0, 0), c_hi = min(row_t - kt0, kKeys - 1);
+            const bool interior = __all_sync(0xffffffffu, c_lo == 0 && c_hi == kKeys - 1);
+            // Logits in log2 units relative to the running max, in one pass over key pairs:
+            // e = s_K c (q.c) + (z_K c Sum(q) - m). A row with no key yet uses m = 0.
+            const float mref = (m_run == -INFINITY) ? 0.f : m_run;
+            const float2 nm2 = make_float2(-mref, -mref);
+            float2 e[kKeys / 2];
             float mx = -INFINITY;
+            {
+                float sv[kKeys];
+                tmem_ld64(tmem + lane_base + kTmemS + 64 * b, sv);
+                if (interior) {
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float sv[32];
-                tmem_ld32(tmem + lane_base + kTmemS + 64 * b + 32 * hf, sv);
+                    for (int j = 0; j < kKeys / 2; ++j) {
+                        const float4 sk = sm.side_k[b][j];
+                        e[j] = __ffma2_rn(make_float2(sk.x, sk.y), make_float2(sv[2 * j], sv[2 * j + 1]),
+                                          __ffma2_rn(make_float2(sk.z, sk.w), qs2, nm2));
+                        mx = fmaxf(mx, fmaxf(e[j].x, e[j].y));
+                    }
+                } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int cidx = 32 * hf + e;
-                    const float2 sd = sm.side_k[b][cidx];
-                    const float v = fmaf(sd.x, sv[e], sd.y * qsum);      // logit in log2 units
-                    lg[cidx] = (cidx >= c_lo && cidx <= c_hi) ? v : -INFINITY;
-                    mx = fmaxf(mx, lg[cidx]);
+                    for (int j = 0; j < kKeys / 2; ++j) {
+                        const float4 sk = sm.side_k[b][j];
+                        float2 x = __ffma2_rn(make_float2(sk.x, sk.y), make_float2(sv[2 * j], sv[2 * j + 1]),
+                                              __ffma2_rn(make_float2(sk.z, sk.w), qs2, nm2));
+                        x.x = (2 * j >= c_lo && 2 * j <= c_hi) ? x.x : -INFINITY;
+                        x.y = (2 * j + 1 >= c_lo && 2 * j + 1 <= c_hi) ? x.y : -INFINITY;
+                        e[j] = x;
+                        mx = fmaxf(mx, fmaxf(x.x, x.y));
+                    }
                 }
             }
-            // Lazy rescaling: the row keeps its running max until a new key exceeds it by
-            // more than 8 (so p <= 2^8 fits fp16 after the s_V scale); then O, l and pz are
-            // rescaled. The final O / l uses the same max, so the result is unchanged.
-            const bool bump = mx > m_run + 8.f;
-            const float m_new = bump ? mx : m_run;
-            const float corr = bump ? ((m_run == -INFINITY) ? 0.f : ex2(m_run - m_new)) : 1.f;
-            float psum = 0.f, pz = 0.f;
-            const float shift = (m_new == -INFINITY) ? 0.f : m_new;   // all keys masked so far
+            /*TRACE_MAX*/
+            // Lazy rescaling: the row keeps its running max until a key exceeds it by more
+            // than 8 (so p <= 2^8 fits fp16 after the s_V scale); then the logits, O, l and
+            // pz move to the new max. The final O / l uses the same max, so the result is
+            // unchanged.
+            const bool bump = (m_run == -INFINITY) ? (mx > -INFINITY) : (mx > 8.f);
+            float corr = 1.f;
+            if (__any_sync(0xffffffffu, bump)) {
+                const float d = bump ? mx : 0.f;
+                const float2 nd2 = make_float2(-d, -d);
 #pragma unroll
-            for (int cidx = 0; cidx < kKeys; ++cidx) {
-                const float2 sd = sm.side_v[b][cidx];
-                const float p = ex2(lg[cidx] - shift);                  // 2^-inf = 0 for masked keys
-                psum += p;
-                pz = fmaf(p, sd.y, pz);
-                lg[cidx] = p * sd.x;                                   // P' = p * s_V
+                for (int j = 0; j < kKeys / 2; ++j) e[j] = __fadd2_rn(e[j], nd2);
+                if (bump) {
+                    corr = (m_run == -INFINITY) ? 0.f : ex2(-mx);
+                    m_run = mref + mx;
+                }
             }
-            l_run = fmaf(l_run, corr, psum);
-            pz_run = fmaf(pz_run, corr, pz);
-            m_run = m_new;
+            float2 psum = make_float2(0.f, 0.f), pz = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < kKeys / 2; ++j) {
+                const float4 svz = sm.side_v[b][j];
+                const float2 p = make_float2(ex2(e[j].x), ex2(e[j].y));   // 2^-inf = 0: masked keys
+                psum = __fadd2_rn(psum, p);
+                pz = __ffma2_rn(p, make_float2(svz.z, svz.w), pz);
+                e[j] = __fmul2_rn(p, make_float2(svz.x, svz.y));           // P' = p * s_V
+            }
+            const float2 corr2 = make_float2(corr, corr);
+            l_run = __ffma2_rn(l_run, corr2, psum);
+            pz_run = __ffma2_rn(pz_run, corr2, pz);
+            /*TRACE_EXP*/
             // P' buffer b was last read by PV(t-2); a rescale of O also needs PV(t-1) done
             // (the MMAs complete in issue order, so waiting for PV(t-1) covers PV(t-2))
             const bool rescale = t > 0 && __any_sync(0xffffffffu, bump);
+            /*TRACE_RESC*/
             const int t_wait = rescale ? t - 1 : t - 2;
             if (t_wait >= 0) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t_wait & 1], (t_wait >> 1) & 1, c.status))) {
@@ -567,13 +642,14 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 }
                 tc_fence_after();
             }
+            /*TRACE_PVW*/
             if (rescale) {                                  // rescale this warp's O rows
 #pragma unroll
                 for (int cb = 0; cb < D / 32; ++cb) {
                     float ov[32];
                     tmem_ld32(tmem + lane_base + kTmemO + cb * 32, ov);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] *= corr;
+                    for (int i = 0; i < 32; ++i) ov[i] *= corr;
                     tmem_st32(tmem + lane_base + kTmemO + cb * 32, ov);
                 }
             }
@@ -583,13 +659,13 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             for (int hf = 0; hf < 2; ++hf) {
                 uint32_t hw[16], lw[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float a = lg[32 * hf + 2 * e], bq = lg[32 * hf + 2 * e + 1];
-                    const __half2 hv = __floats2half2_rn(a, bq);
+                for (int i = 0; i < 16; ++i) {
+                    const float2 a = e[16 * hf + i];
+                    const __half2 hv = __float22half2_rn(a);
                     const float2 hfv = __half22float2(hv);
-                    const __half2 lv = __floats2half2_rn(a - hfv.x, bq - hfv.y);
-                    hw[e] = *reinterpret_cast<const uint32_t *>(&hv);
-                    lw[e] = *reinterpret_cast<const uint32_t *>(&lv);
+                    const __half2 lv = __float22half2_rn(__fadd2_rn(a, make_float2(-hfv.x, -hfv.y)));
+                    hw[i] = *reinterpret_cast<const uint32_t *>(&hv);
+                    lw[i] = *reinterpret_cast<const uint32_t *>(&lv);
                 }
                 tmem_st16u(tmem + lane_base + kTmemP + 64 * b + 16 * hf, hw);
                 tmem_st16u(tmem + lane_base + kTmemP + 64 * b + 32 + 16 * hf, lw);
@@ -603,7 +679,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t_last & 1], (t_last >> 1) & 1, c.status))) {
             tc_fence_after();
             const bool write = row_t >= 0;
-            const float inv = (l_run > 0.f) ? 1.0f / l_run : 0.f;
+            const float l_sum = l_run.x + l_run.y, pz_sum = pz_run.x + pz_run.y;
+            const float inv = (l_sum > 0.f) ? 1.0f / l_sum : 0.f;
             float *dst = out + ((int64_t)(cu[s] + max(row_i, 0)) * H + h) * D;
 #pragma unroll
             for (int cb = 0; cb < D / 32; ++cb) {
@@ -613,8 +690,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
                         *reinterpret_cast<float4 *>(dst + cb * 32 + e) =
-                            make_float4((ov[e] + pz_run) * inv, (ov[e + 1] + pz_run) * inv,
-                                        (ov[e + 2] + pz_run) * inv, (ov[e + 3] + pz_run) * inv);
+                            make_float4((ov[e] + pz_sum) * inv, (ov[e + 1] + pz_sum) * inv,
+                                        (ov[e + 2] + pz_sum) * inv, (ov[e + 3] + pz_sum) * inv);
                 }
             }
         } else if (row_t >= 0) {
