@@ -8,22 +8,25 @@
 //                         tile reads keys [min(t) - w, max(t)], a full tile [0, max(t)],
 //                         so local rows do not pay for a full tile's range.
 //   prefill_order_kernel  orders the tiles longest first (keys spanned, descending).
-//   prefill_tc_kernel     one CTA per tile:
-//     - warps 0-3 (one thread per query row): Q row -> shared (fp16, 128B-swizzled
-//       K-major); per key tile, S row from TMEM -> logits (s_K * (q.c) + z_K * sum(q)) /
-//       sqrt(D) with the row's causal/window mask -> online softmax -> P' = p * s_V split
-//       into fp16 hi + lo (fp16 rounding of P alone would cost ~1e-2 on outlier channels)
-//       -> TMEM (double buffered, the A operand of the PV MMA); rescale the O row in TMEM
-//       when the row max grows by more than 2^8; final O / l.
-//     - warps 4-7: unpack each 64-key tile's K and V codes into exact fp16 operands (codes
-//       are integers <= 255; b = 16 keys are the fp16 values) in shared memory, double
-//       buffered; K 128B-swizzled K-major, V 128B-swizzled MN-major. The packed bytes are
-//       fetched two tiles ahead with cp.async and the record offsets three tiles ahead.
-//     - warp 8: owns 512 TMEM columns (S double buffer: 2 x 64, O: D, P' double buffer:
-//       2 x 64) and issues the MMAs from one lane: S = Q C_K^T (M128 N64 K16 steps, A and B
-//       in shared memory) as soon as a K tile is unpacked (up to one tile ahead), O += P'_hi V
-//       and O += P'_lo V (M128 ND K16, A in TMEM) as soon as P' of the tile is in TMEM,
-//       whichever is ready first.
+//   prefill_tc_kernel     one CTA per tile, 18 warps:
+//     - warps 0-7, softmax: thread = (query row 32 (w % 4) + lane, key half w / 4). Per 64-key
+//       tile the thread takes its 32 S values from TMEM, forms the logits
+//       s_K * (q.c) + z_K * sum(q) (log2 units, scaled by 1/sqrt(D)) with the row's causal/window
+//       mask, runs an online softmax with lazy rescaling over its half, and writes
+//       P' = p * s_V as fp16 hi + lo parts to TMEM (fp16 rounding of P alone would cost ~1e-2
+//       on outlier channels). Each key half has its own running max and its own O
+//       accumulator in TMEM, so the two warps of a row never wait for each other; the halves
+//       are merged once at the end.
+//     - warps 8-15: unpack each 64-key tile's K and V codes into exact fp16 operands (codes
+//       are integers <= 255; b = 16 keys are the fp16 values) in shared memory, three tiles
+//       in flight; K 128B-swizzled K-major, V 128B-swizzled MN-major.
+//     - warp 16: owns 512 TMEM columns (S, P' double buffer, Q, O of each key half) and
+//       issues the MMAs from one lane: S = Q C_K^T (M128 N64 K16 steps, A = Q in TMEM, B in
+//       shared memory) once K(t) is unpacked and S(t-1) has been read, and
+//       O_h += P'_h,hi V_h + P'_h,lo V_h per key half h (M128 ND K16, A in TMEM) once P'(t)
+//       is written.
+//     - warp 17: stages each key tile's records (one contiguous byte range of the stream)
+//       with bulk copies and orders the unpack tasks by width, three tiles ahead.
 //   All mbarrier waits are bounded; on a timeout the CTA records KVQ_ERR_DEVICE_CHECK,
 //   leaves its loops, waits (bounded) for its MMAs and frees its TMEM before returning.
 #include "kvq_internal.cuh"
@@ -33,23 +36,31 @@ namespace {
 
 constexpr int kQRows = 128;     // queries per tile (MMA M)
 constexpr int kKeys = 64;       // keys per key tile (QK MMA N, PV MMA K)
-// 16 warps: 0-3 softmax rows, 4-11 K/V unpack, 12 MMA issuer, 13 record stager (14-15 idle,
-// present so that the last warpgroup is whole for the register split below)
-constexpr int kTcThreads = 512;
+// 20 warps: 0-7 softmax (two per row, one per key half), 8-15 K/V unpack, 16 MMA issuer,
+// 17 record stager (18-19 idle, present so that the last warpgroup is whole for the register
+// split below)
+constexpr int kSoftmaxWarps = 8, kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kUnpackWarps = 8, kUnpackThreads = 32 * kUnpackWarps;
-constexpr int kMmaWarp = 4 + kUnpackWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + kUnpackWarps;
 constexpr int kStageWarp = kMmaWarp + 1;
+constexpr int kTcThreads = 32 * (kStageWarp + 3);
 constexpr int kQP = kUnpackThreads / 64;   // unpack threads per key (the tile's 64 keys)
-// Registers per thread after the split (launch: 128 x 512 threads = 65536): softmax 200,
-// unpack 96, MMA warpgroup 80: 128 x (200 + 2 x 96 + 80) = 60416 <= 65536.
-constexpr int kRegSoftmax = 200, kRegUnpack = 96, kRegMma = 80;
-static_assert(128 * (kRegSoftmax + 2 * kRegUnpack + kRegMma) <= 65536, "register split exceeds the launch");
+// Registers: the launch gives every thread kLaunchRegs (65536 / 640 rounded down to a
+// multiple of 8); setmaxnreg at the head of each role then moves them between warpgroups:
+// softmax kRegSoftmax, unpack kRegUnpack, MMA/stager warpgroup kRegMma per thread. The sum
+// stays within the launch's allocation; the host refuses to launch when the compiled
+// register count differs from kLaunchRegs.
+constexpr int kLaunchRegs = 96, kRegSoftmax = 144, kRegUnpack = 80, kRegMma = 32;
+static_assert(kTcThreads * kLaunchRegs <= 65536, "launch registers");
+static_assert(kSoftmaxThreads * kRegSoftmax + kUnpackThreads * kRegUnpack + 128 * kRegMma <= kTcThreads * kLaunchRegs,
+              "register split exceeds the launch");
 constexpr int kRawBufs = 3;     // record staging buffers: a key tile's records land up to three tiles ahead
+constexpr int kKvBufs = 3;      // unpacked K/V operand tiles in flight
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S double buffer at 0 and 64 (fp32), O at 128 (D columns), P' double buffer at
-// 256 and 320: each buffer holds P'_hi in 32 columns then P'_lo in 32 (fp16 pairs, the A
-// operand of the PV MMA)
-constexpr uint32_t kTmemS = 0, kTmemO = 128, kTmemP = 256;
+// TMEM columns: S (fp32, 64 keys) at 0; P' double buffer at 64 and 128, each holding per key
+// half h the fp16 pairs of P'_hi (16 columns) then P'_lo (16) at 32 h; Q (fp16 pairs, D / 2
+// columns) at 192; O of key half h (fp32, D columns) at 256 + h D.
+constexpr uint32_t kTmemS = 0, kTmemP = 64, kTmemQ = 192, kTmemO = 256;
 
 // ---- tcgen05 / UMMA helpers -------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), descriptor version 1.
@@ -156,6 +167,19 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
                  : "memory");
 }
 
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+                 "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                   "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+                   "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+                   "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+                   "r"(v[29]), "r"(v[30]), "r"(v[31])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16])
 {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -237,19 +261,20 @@ struct PfTile {
 
 template <int D>
 struct alignas(1024) PfSmem {
-    __half q[kQRows * D];             // K-major SW128, D/64 blocks of 128 rows x 128 B
-    __half k[2][kKeys * D];           // K-major SW128, D/64 blocks of 64 rows x 128 B
-    __half v[2][kKeys * D];           // MN-major SW128: atom (8 keys x 64 ch) at (key/8)*(D/64)+ch/64
+    __half k[kKvBufs][kKeys * D];     // K-major SW128, D/64 blocks of 64 rows x 128 B
+    __half v[kKvBufs][kKeys * D];     // MN-major SW128: atom (8 keys x 64 ch) at (key/8)*(D/64)+ch/64
     // side entries of key pairs (2j, 2j + 1), laid out for packed fp32 arithmetic:
-    float4 side_k[2][kKeys / 2];      // (s_K c, s_K c, z_K c, z_K c), c = log2(e)/sqrt(D)
-    float4 side_v[2][kKeys / 2];      // (s_V, s_V, z_V, z_V)
+    float4 side_k[kKvBufs][kKeys / 2];   // (s_K c, s_K c, z_K c, z_K c), c = log2(e)/sqrt(D)
+    float4 side_v[kKvBufs][kKeys / 2];   // (s_V, s_V, z_V, z_V)
     uint8_t raw[kRawBufs][kKeys * 4 * D];   // a key tile's records as stored (one contiguous range
                                             // of the stream; at most 64 keys x 2 x D fp16 values)
     // the tile's 256 conversion tasks (key, part), ordered by width class:
     // offset of the key's record in raw << 16 | class << 8 | key << 2 | part (class 4: no key)
     uint32_t task[kRawBufs][kUnpackThreads];
-    uint64_t raw_full[kRawBufs], raw_empty[kRawBufs];
-    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], drain;
+    float4 fin[2][kQRows];            // per key half: (running max, l, sum p z_V) of each row
+    float qpart[2][kQRows];           // per half of the channels: partial sums of each Q row
+    uint64_t raw_full[kRawBufs], raw_empty[kRawBufs], kv_full[kKvBufs], kv_empty[kKvBufs];
+    uint64_t s_full, s_free, p_full[2], pv_done[2], drain;
     uint32_t tmem_base;
     int32_t klo, khi, abort_flag;
 };
@@ -275,7 +300,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     const RecLoc stream = rec_loc(c, s, hk, 0);
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kKvBufs; ++i) {
             mbar_init(&sm.kv_full[i], kUnpackWarps);
             mbar_init(&sm.kv_empty[i], 1);
         }
@@ -283,12 +308,12 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             mbar_init(&sm.raw_full[i], 1);
             mbar_init(&sm.raw_empty[i], kUnpackWarps);
         }
-        mbar_init(&sm.s_full[0], 1);
-        mbar_init(&sm.s_full[1], 1);
-        mbar_init(&sm.p_full[0], 128);
-        mbar_init(&sm.p_full[1], 128);
-        mbar_init(&sm.pv_done[0], 1);
-        mbar_init(&sm.pv_done[1], 1);
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.s_free, kSoftmaxWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.p_full[i], kSoftmaxWarps);
+            mbar_init(&sm.pv_done[i], 1);
+        }
         mbar_init(&sm.drain, 1);
         sm.klo = INT32_MAX;
         sm.khi = -1;
@@ -301,96 +326,110 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
 
-    // ---- prologue: query rows (warps 0-3) ----
+    // ---- prologue: query rows (softmax warps; the two warps of a row load half the
+    // channels each into the Q columns of TMEM) ----
+    const int kh = warp / 4;                       // softmax: key half (and channel half of Q)
+    const int row = 32 * (warp & 3) + lane;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     int row_t = -1, row_lo = 0, row_i = -1;
-    float qsum = 0.f;
-    if (tid < kQRows) {
-        const int r = tid;
-        const bool valid = r < tile.count;
+    if (warp < kSoftmaxWarps) {
+        const bool valid = row < tile.count;
         if (valid) {
-            row_i = qidx[tile.start + r];
+            row_i = qidx[tile.start + row];
             row_t = pos0 + row_i;
             row_lo = (tile.mode == KVQ_MODE_LOCAL) ? max(0, row_t - w) : 0;
-            atomicMin(&sm.klo, row_lo);
-            atomicMax(&sm.khi, row_t);
+            if (kh == 0) {
+                atomicMin(&sm.klo, row_lo);
+                atomicMax(&sm.khi, row_t);
+            }
         }
-        const uint4 *src = reinterpret_cast<const uint4 *>(q + ((int64_t)(cu[s] + max(row_i, 0)) * H + h) * D);
+        const uint4 *src = reinterpret_cast<const uint4 *>(q + ((int64_t)(cu[s] + max(row_i, 0)) * H + h) * D) + kh * (D / 16);
+        uint32_t words[D / 4];
+        float part = 0.f;
 #pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch) {
-            uint4 x = valid ? src[ch] : make_uint4(0, 0, 0, 0);
+        for (int ch = 0; ch < D / 16; ++ch) {
+            const uint4 x = valid ? src[ch] : make_uint4(0, 0, 0, 0);
+            words[4 * ch] = x.x;
+            words[4 * ch + 1] = x.y;
+            words[4 * ch + 2] = x.z;
+            words[4 * ch + 3] = x.w;
             const __half2 *hx = reinterpret_cast<const __half2 *>(&x);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 f = __half22float2(hx[e]);
-                qsum += f.x + f.y;
+                part += f.x + f.y;
             }
-            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(sm.q) + (ch >> 3) * (kQRows * 128) +
-                                       kmajor_off(r, ch & 7)) = x;
         }
-        fence_async_smem();
+        if constexpr (D == 128) {
+            tmem_st32u(tmem + lane_base + kTmemQ + 32 * kh, words);
+        } else {
+            tmem_st16u(tmem + lane_base + kTmemQ + 16 * kh, words);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        sm.qpart[kh][row] = part;
+        tc_fence_before();
     }
     __syncthreads();
     tc_fence_after();
     const int klo = sm.klo, khi = sm.khi;
     const int n_kt = (khi >= klo) ? (khi - klo + kKeys) / kKeys : 0;
-    const uint32_t tmem = sm.tmem_base;
-    // Register split by warpgroup, at the head of each role: the softmax rows take what the
-    // unpack and MMA warpgroups give back (the sum stays within the launch's allocation,
-    // see kRegSoftmax).
     if (warp >= kMmaWarp) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegMma));
     }
     if (warp == kMmaWarp) {
         // ------------------------------- MMA issuer --------------------------------
-        // order: QK(0), then per tile t: QK(t+1) into the other S buffer, wait P(t), PV(t)
-        const uint32_t q0 = smem_u32(sm.q);
         constexpr uint32_t idesc_qk = umma_idesc(kKeys, false);
         constexpr uint32_t idesc_pv = umma_idesc(D, true);
         constexpr uint32_t v_sbo = (D / 64) * 1024;       // next 8 keys
         auto issue_qk = [&](int t) {
-            const int b = t & 1;
             tc_fence_after();
-            const uint32_t k0 = smem_u32(sm.k[b]);
+            const uint32_t k0 = smem_u32(sm.k[t % kKvBufs]);
             if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t da = umma_desc(q0 + (kk >> 2) * (kQRows * 128) + (kk & 3) * 32, 16, 1024);
                     const uint64_t db = umma_desc(k0 + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
-                    umma_f16(tmem + kTmemS + 64 * b, da, db, idesc_qk, kk > 0);
+                    umma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * kk, db, idesc_qk, kk > 0);
                 }
-                umma_commit(&sm.s_full[b]);
+                umma_commit(&sm.s_full);
             }
             __syncwarp();
         };
         auto issue_pv = [&](int t) {
             tc_fence_after();
-            const uint32_t v0 = smem_u32(sm.v[t & 1]);
+            const uint32_t v0 = smem_u32(sm.v[t % kKvBufs]);
             if (lane == 0) {
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    // P'_hi then P'_lo of buffer t & 1: 8 TMEM columns per 16 keys
-                    const uint32_t pa = tmem + kTmemP + 64 * (t & 1) + 32 * half;
 #pragma unroll
-                    for (int kk = 0; kk < kKeys / 16; ++kk) {
-                        const uint64_t db = umma_desc(v0 + 2 * kk * v_sbo, 1024, v_sbo);
-                        umma_f16_ts(tmem + kTmemO, pa + 8 * kk, db, idesc_pv, half > 0 || t > 0 || kk > 0);
+                    for (int part = 0; part < 2; ++part) {
+                        // P'_hi then P'_lo of key half `half`: 8 TMEM columns per 16 keys
+                        const uint32_t pa = tmem + kTmemP + 64 * (t & 1) + 32 * half + 16 * part;
+#pragma unroll
+                        for (int k2 = 0; k2 < 2; ++k2) {
+                            const int kk = 2 * half + k2;         // 16-key step of the tile
+                            const uint64_t db = umma_desc(v0 + 2 * kk * v_sbo, 1024, v_sbo);
+                            umma_f16_ts(tmem + kTmemO + half * D, pa + 8 * k2, db, idesc_pv, part > 0 || t > 0 || k2 > 0);
+                        }
                     }
                 }
                 umma_commit(&sm.pv_done[t & 1]);
-                umma_commit(&sm.kv_empty[t & 1]);
+                umma_commit(&sm.kv_empty[t % kKvBufs]);
             }
             __syncwarp();
         };
-        // Issue QK(t) as soon as K(t) is unpacked and PV(t) as soon as P(t) is written,
-        // whichever comes first. QK may run one tile ahead of PV (S is double buffered).
+        // Issue QK(t) once K(t) is unpacked and the softmax has read S(t-1), and PV(t) once
+        // P'(t) is written; QK first when both are ready (it feeds the softmax).
         bool alive = true;
         int next_qk = 0, next_pv = 0;
         uint64_t t_start = global_ns();
         while (next_pv < n_kt) {
             bool progressed = false;
-            if (next_qk < n_kt && next_qk <= next_pv + 1 &&
-                __all_sync(0xffffffffu, mbar_test(&sm.kv_full[next_qk & 1], (next_qk >> 1) & 1))) {
+            if (next_qk < n_kt &&
+                __all_sync(0xffffffffu, mbar_test(&sm.kv_full[next_qk % kKvBufs], (next_qk / kKvBufs) & 1) &&
+                                            (next_qk == 0 || mbar_test(&sm.s_free, (next_qk - 1) & 1)))) {
                 issue_qk(next_qk++);
                 progressed = true;
             }
@@ -409,7 +448,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 alive = false;
                 break;
             } else {
-                __nanosleep(64);          // leave the issue slots to the warps doing the work
+                __nanosleep(32);          // leave the issue slots to the warps doing the work
             }
         }
         if (!alive) sm.abort_flag = 1;
@@ -487,13 +526,13 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         // the copies of the last tiles (earlier ones were consumed before their buffer came back)
         for (int t = max(0, issued - kRawBufs); t < issued; ++t)
             mbar_wait(&sm.raw_full[t % kRawBufs], (t / kRawBufs) & 1, c.status);
-    } else if (warp >= 4 && warp < kMmaWarp) {
+    } else if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegUnpack));
         // ------------------------------ K/V unpack -----------------------------------
         // Thread = one conversion task of the tile (a key, a quarter of its channels), as
         // ordered by the stager; the side entry of its own key kj = u / 4 is loaded three
         // tiles ahead.
-        const int u = tid - 128;
+        const int u = tid - kSoftmaxThreads;
         const int kj = u / kQP, half = u % kQP;
         constexpr int CH = D / kQP;                  // channels per task
         auto load_side = [&](int t) -> float4 {
@@ -502,10 +541,10 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         };
         float4 sd_cur = load_side(0), sd_n1 = load_side(1), sd_n2 = load_side(2);
         for (int t = 0; t < n_kt; ++t) {
-            const int b = t & 1, st = t % kRawBufs;
+            const int b = t % kKvBufs, st = t % kRawBufs;
             const float4 sd_n3 = load_side(t + 3);
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.raw_full[st], (t / kRawBufs) & 1, c.status) &&
-                                             mbar_wait(&sm.kv_empty[b], ((t >> 1) & 1) ^ 1, c.status) &&
+                                             mbar_wait(&sm.kv_empty[b], ((t / kKvBufs) & 1) ^ 1, c.status) &&
                                              !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
                 sm.abort_flag = 1;
                 break;
@@ -547,79 +586,85 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             sd_n1 = sd_n2;
             sd_n2 = sd_n3;
         }
-    } else if (warp < 4) {
+    } else if (warp < kSoftmaxWarps) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
         // ------------------------------ softmax rows ---------------------------------
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // This thread: row `row`, keys 32 kh .. 32 kh + 31 of every tile.
+        const float qsum = sm.qpart[0][row] + sm.qpart[1][row];
+        const float2 qs2 = make_float2(qsum, qsum);
+        const uint32_t o_col = kTmemO + kh * D;
         float m_run = -INFINITY;
         float2 l_run = make_float2(0.f, 0.f), pz_run = make_float2(0.f, 0.f);   // even / odd keys
-        const float2 qs2 = make_float2(qsum, qsum);
         bool ok = true;
         for (int t = 0; t < n_kt; ++t) {
-            const int b = t & 1;
+            const int st = t % kKvBufs;
             // warp-uniform outcome: the TMEM accesses below are .sync.aligned
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], (t >> 1) & 1, c.status) &&
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full, t & 1, c.status) &&
                                              !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
                 sm.abort_flag = 1;
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int kt0 = klo + t * kKeys;
-            // the row's keys in this tile: [max(row_lo, kt0), min(row_t, kt0 + 63)]
-            const int c_lo = max(row_lo - kt0, 0), c_hi = min(row_t - kt0, kKeys - 1);
-            const bool interior = __all_sync(0xffffffffu, c_lo == 0 && c_hi == kKeys - 1);
+            float sv[32];
+            tmem_ld32(tmem + lane_base + kTmemS + 32 * kh, sv);
+            // S may now be overwritten by QK(t+1)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.s_free);
+            const int kt0 = klo + t * kKeys + 32 * kh;
+            // the row's keys in this half tile: [max(row_lo, kt0), min(row_t, kt0 + 31)]
+            const int c_lo = max(row_lo - kt0, 0), c_hi = min(row_t - kt0, 31);
+            const bool interior = __all_sync(0xffffffffu, c_lo == 0 && c_hi == 31);
             // Logits in log2 units relative to the running max, in one pass over key pairs:
-            // e = s_K c (q.c) + (z_K c Sum(q) - m). A row with no key yet uses m = 0.
+            // e = s_K c (q.c) + (z_K c Sum(q) - m). A half with no key yet uses m = 0.
             const float mref = (m_run == -INFINITY) ? 0.f : m_run;
             const float2 nm2 = make_float2(-mref, -mref);
-            float2 e[kKeys / 2];
+            const float4 *skp = &sm.side_k[st][16 * kh];
+            float2 e[16];
             float mx = -INFINITY;
-            {
-                float sv[kKeys];
-                tmem_ld64(tmem + lane_base + kTmemS + 64 * b, sv);
-                if (interior) {
+            if (interior) {
 #pragma unroll
-                    for (int j = 0; j < kKeys / 2; ++j) {
-                        const float4 sk = sm.side_k[b][j];
-                        e[j] = __ffma2_rn(make_float2(sk.x, sk.y), make_float2(sv[2 * j], sv[2 * j + 1]),
+                for (int j = 0; j < 16; ++j) {
+                    const float4 sk = skp[j];
+                    e[j] = __ffma2_rn(make_float2(sk.x, sk.y), make_float2(sv[2 * j], sv[2 * j + 1]),
+                                      __ffma2_rn(make_float2(sk.z, sk.w), qs2, nm2));
+                    mx = fmaxf(mx, fmaxf(e[j].x, e[j].y));
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float4 sk = skp[j];
+                    float2 x = __ffma2_rn(make_float2(sk.x, sk.y), make_float2(sv[2 * j], sv[2 * j + 1]),
                                           __ffma2_rn(make_float2(sk.z, sk.w), qs2, nm2));
-                        mx = fmaxf(mx, fmaxf(e[j].x, e[j].y));
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < kKeys / 2; ++j) {
-                        const float4 sk = sm.side_k[b][j];
-                        float2 x = __ffma2_rn(make_float2(sk.x, sk.y), make_float2(sv[2 * j], sv[2 * j + 1]),
-                                              __ffma2_rn(make_float2(sk.z, sk.w), qs2, nm2));
-                        x.x = (2 * j >= c_lo && 2 * j <= c_hi) ? x.x : -INFINITY;
-                        x.y = (2 * j + 1 >= c_lo && 2 * j + 1 <= c_hi) ? x.y : -INFINITY;
-                        e[j] = x;
-                        mx = fmaxf(mx, fmaxf(x.x, x.y));
-                    }
+                    x.x = (2 * j >= c_lo && 2 * j <= c_hi) ? x.x : -INFINITY;
+                    x.y = (2 * j + 1 >= c_lo && 2 * j + 1 <= c_hi) ? x.y : -INFINITY;
+                    e[j] = x;
+                    mx = fmaxf(mx, fmaxf(x.x, x.y));
                 }
             }
             /*TRACE_MAX*/
-            // Lazy rescaling: the row keeps its running max until a key exceeds it by more
+            // Lazy rescaling: the half keeps its running max until a key exceeds it by more
             // than 8 (so p <= 2^8 fits fp16 after the s_V scale); then the logits, O, l and
-            // pz move to the new max. The final O / l uses the same max, so the result is
-            // unchanged.
+            // pz move to the new max. The final merge uses each half's max, so the result
+            // is unchanged.
             const bool bump = (m_run == -INFINITY) ? (mx > -INFINITY) : (mx > 8.f);
             float corr = 1.f;
             if (__any_sync(0xffffffffu, bump)) {
                 const float d = bump ? mx : 0.f;
                 const float2 nd2 = make_float2(-d, -d);
 #pragma unroll
-                for (int j = 0; j < kKeys / 2; ++j) e[j] = __fadd2_rn(e[j], nd2);
+                for (int j = 0; j < 16; ++j) e[j] = __fadd2_rn(e[j], nd2);
                 if (bump) {
                     corr = (m_run == -INFINITY) ? 0.f : ex2(-mx);
                     m_run = mref + mx;
                 }
             }
+            const float4 *svp = &sm.side_v[st][16 * kh];
             float2 psum = make_float2(0.f, 0.f), pz = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < kKeys / 2; ++j) {
-                const float4 svz = sm.side_v[b][j];
+            for (int j = 0; j < 16; ++j) {
+                const float4 svz = svp[j];
                 const float2 p = make_float2(ex2(e[j].x), ex2(e[j].y));   // 2^-inf = 0: masked keys
                 psum = __fadd2_rn(psum, p);
                 pz = __ffma2_rn(p, make_float2(svz.z, svz.w), pz);
@@ -629,7 +674,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             l_run = __ffma2_rn(l_run, corr2, psum);
             pz_run = __ffma2_rn(pz_run, corr2, pz);
             /*TRACE_EXP*/
-            // P' buffer b was last read by PV(t-2); a rescale of O also needs PV(t-1) done
+            // P' buffer t & 1 was last read by PV(t-2); a rescale of O also needs PV(t-1) done
             // (the MMAs complete in issue order, so waiting for PV(t-1) covers PV(t-2))
             const bool rescale = t > 0 && __any_sync(0xffffffffu, bump);
             /*TRACE_RESC*/
@@ -643,59 +688,70 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 tc_fence_after();
             }
             /*TRACE_PVW*/
-            if (rescale) {                                  // rescale this warp's O rows
+            if (rescale) {                                  // rescale this half's O rows
 #pragma unroll
                 for (int cb = 0; cb < D / 32; ++cb) {
                     float ov[32];
-                    tmem_ld32(tmem + lane_base + kTmemO + cb * 32, ov);
+                    tmem_ld32(tmem + lane_base + o_col + cb * 32, ov);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) ov[i] *= corr;
-                    tmem_st32(tmem + lane_base + kTmemO + cb * 32, ov);
+                    tmem_st32(tmem + lane_base + o_col + cb * 32, ov);
                 }
             }
-            // P' = hi + lo, both fp16, row r of the TMEM A operand of buffer b: column j
-            // holds keys (2j, 2j + 1); hi in columns 0..31, lo in 32..63
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
+            // P' = hi + lo, both fp16: column j of this half's 16 holds keys (2j, 2j + 1)
+            {
                 uint32_t hw[16], lw[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float2 a = e[16 * hf + i];
+                    const float2 a = e[i];
                     const __half2 hv = __float22half2_rn(a);
                     const float2 hfv = __half22float2(hv);
                     const __half2 lv = __float22half2_rn(__fadd2_rn(a, make_float2(-hfv.x, -hfv.y)));
                     hw[i] = *reinterpret_cast<const uint32_t *>(&hv);
                     lw[i] = *reinterpret_cast<const uint32_t *>(&lv);
                 }
-                tmem_st16u(tmem + lane_base + kTmemP + 64 * b + 16 * hf, hw);
-                tmem_st16u(tmem + lane_base + kTmemP + 64 * b + 32 + 16 * hf, lw);
+                tmem_st16u(tmem + lane_base + kTmemP + 64 * (t & 1) + 32 * kh, hw);
+                tmem_st16u(tmem + lane_base + kTmemP + 64 * (t & 1) + 32 * kh + 16, lw);
             }
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
-            mbar_arrive(&sm.p_full[b]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.p_full[t & 1]);
         }
+        // ---- merge the two key halves of each row; each warp writes half the channels ----
         const int t_last = n_kt - 1;
         if (ok && n_kt > 0 &&
-            __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t_last & 1], (t_last >> 1) & 1, c.status))) {
-            tc_fence_after();
+            !__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t_last & 1], (t_last >> 1) & 1, c.status)))
+            ok = false;
+        tc_fence_after();
+        sm.fin[kh][row] = make_float4(m_run, l_run.x + l_run.y, pz_run.x + pz_run.y, 0.f);
+        // every softmax warp reaches this barrier, aborted or not
+        if (named_bar_or(1, kSoftmaxThreads, !ok)) {
+            if (row_t >= 0) sm.abort_flag = 1;
+        } else {
+            const float4 fa = sm.fin[0][row], fb = sm.fin[1][row];
+            const float m = fmaxf(fa.x, fb.x);
+            const float wa = (fa.x == -INFINITY) ? 0.f : ex2(fa.x - m);
+            const float wb = (fb.x == -INFINITY) ? 0.f : ex2(fb.x - m);
+            const float l = fa.y * wa + fb.y * wb, pzs = fa.z * wa + fb.z * wb;
+            const float inv = (l > 0.f) ? 1.0f / l : 0.f;
             const bool write = row_t >= 0;
-            const float l_sum = l_run.x + l_run.y, pz_sum = pz_run.x + pz_run.y;
-            const float inv = (l_sum > 0.f) ? 1.0f / l_sum : 0.f;
-            float *dst = out + ((int64_t)(cu[s] + max(row_i, 0)) * H + h) * D;
+            float *dst = out + ((int64_t)(cu[s] + max(row_i, 0)) * H + h) * D + kh * (D / 2);
 #pragma unroll
-            for (int cb = 0; cb < D / 32; ++cb) {
-                float ov[32];
-                tmem_ld32(tmem + lane_base + kTmemO + cb * 32, ov);
+            for (int cb = 0; cb < D / 64; ++cb) {
+                float oa[32], ob[32];
+                tmem_ld32(tmem + lane_base + kTmemO + kh * (D / 2) + cb * 32, oa);
+                tmem_ld32(tmem + lane_base + kTmemO + D + kh * (D / 2) + cb * 32, ob);
                 if (write) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
                         *reinterpret_cast<float4 *>(dst + cb * 32 + e) =
-                            make_float4((ov[e] + pz_sum) * inv, (ov[e + 1] + pz_sum) * inv,
-                                        (ov[e + 2] + pz_sum) * inv, (ov[e + 3] + pz_sum) * inv);
+                            make_float4((fmaf(oa[e], wa, ob[e] * wb) + pzs) * inv,
+                                        (fmaf(oa[e + 1], wa, ob[e + 1] * wb) + pzs) * inv,
+                                        (fmaf(oa[e + 2], wa, ob[e + 2] * wb) + pzs) * inv,
+                                        (fmaf(oa[e + 3], wa, ob[e + 3] * wb) + pzs) * inv);
                 }
             }
-        } else if (row_t >= 0) {
-            sm.abort_flag = 1;
         }
     }
 
@@ -868,6 +924,11 @@ cudaError_t run_tc(const kvq_cache *cache, const __half *q, const uint8_t *modes
     const size_t smem = sizeof(PfSmem<D>) + 1024;
     e = ensure_smem_attr((const void *)prefill_tc_kernel<D>, smem);
     if (e != cudaSuccess) return e;
+    // the register split inside the kernel assumes the launch's count per thread
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, (const void *)prefill_tc_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     profile_before(st);
     prefill_tc_kernel<D><<<(unsigned)max_tiles, kTcThreads, smem, st>>>(c, q, w, cu, ordered, cache->pf_count,
                                                                         cache->pf_qidx, out);
