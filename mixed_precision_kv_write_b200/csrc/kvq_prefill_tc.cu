@@ -36,13 +36,14 @@ namespace {
 
 constexpr int kQRows = 128;     // queries per tile (MMA M)
 constexpr int kKeys = 64;       // keys per key tile (QK MMA N, PV MMA K)
-// 20 warps: 0-7 softmax (two per row, one per key half), 8-15 K/V unpack, 16 MMA issuer,
-// 17 record stager (18-19 idle, present so that the last warpgroup is whole for the register
-// split below)
+// 20 warps: 0-7 softmax (two per row, one per key half), 8-15 K/V unpack, 16 QK issuer,
+// 17 record stager, 18 PV issuer (19 idle, present so that the last warpgroup is whole for the
+// register split below)
 constexpr int kSoftmaxWarps = 8, kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kUnpackWarps = 8, kUnpackThreads = 32 * kUnpackWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + kUnpackWarps;
 constexpr int kStageWarp = kMmaWarp + 1;
+constexpr int kPvWarp = kMmaWarp + 2;
 constexpr int kTcThreads = 32 * (kStageWarp + 3);
 constexpr int kQP = kUnpackThreads / 64;   // unpack threads per key (the tile's 64 keys)
 // Registers: the launch gives every thread kLaunchRegs (65536 / 640 rounded down to a
@@ -268,9 +269,9 @@ struct alignas(1024) PfSmem {
     float4 side_v[kKvBufs][kKeys / 2];   // (s_V, s_V, z_V, z_V)
     uint8_t raw[kRawBufs][kKeys * 4 * D];   // a key tile's records as stored (one contiguous range
                                             // of the stream; at most 64 keys x 2 x D fp16 values)
-    // the tile's 256 conversion tasks (key, part), ordered by width class:
-    // offset of the key's record in raw << 16 | class << 8 | key << 2 | part (class 4: no key)
-    uint32_t task[kRawBufs][kUnpackThreads];
+    // the tile's keys ordered by width class (class 4: no key):
+    // offset of the key's record in raw << 16 | class << 8 | key
+    uint32_t task[kRawBufs][kKeys];
     float4 fin[2][kQRows];            // per key half: (running max, l, sum p z_V) of each row
     float qpart[2][kQRows];           // per half of the channels: partial sums of each Q row
     uint64_t raw_full[kRawBufs], raw_empty[kRawBufs], kv_full[kKvBufs], kv_empty[kKvBufs];
@@ -314,7 +315,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             mbar_init(&sm.p_full[i], kSoftmaxWarps);
             mbar_init(&sm.pv_done[i], 1);
         }
-        mbar_init(&sm.drain, 1);
+        mbar_init(&sm.drain, 2);
         sm.klo = INT32_MAX;
         sm.khi = -1;
         sm.abort_flag = 0;
@@ -379,80 +380,73 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     if (warp >= kMmaWarp) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegMma));
     }
-    if (warp == kMmaWarp) {
-        // ------------------------------- MMA issuer --------------------------------
-        constexpr uint32_t idesc_qk = umma_idesc(kKeys, false);
-        constexpr uint32_t idesc_pv = umma_idesc(D, true);
-        constexpr uint32_t v_sbo = (D / 64) * 1024;       // next 8 keys
-        auto issue_qk = [&](int t) {
-            tc_fence_after();
-            const uint32_t k0 = smem_u32(sm.k[t % kKvBufs]);
-            if (lane == 0) {
+    // ---- MMA issue (warp 16: QK, warp 18: PV), one lane each ----
+    constexpr uint32_t idesc_qk = umma_idesc(kKeys, false);
+    constexpr uint32_t idesc_pv = umma_idesc(D, true);
+    constexpr uint32_t v_sbo = (D / 64) * 1024;       // next 8 keys
+    auto issue_qk = [&](int t) {
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(sm.k[t % kKvBufs]);
+        if (lane == 0) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t db = umma_desc(k0 + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
-                    umma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * kk, db, idesc_qk, kk > 0);
-                }
-                umma_commit(&sm.s_full);
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t db = umma_desc(k0 + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
+                umma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * kk, db, idesc_qk, kk > 0);
             }
-            __syncwarp();
-        };
-        auto issue_pv = [&](int t) {
-            tc_fence_after();
-            const uint32_t v0 = smem_u32(sm.v[t % kKvBufs]);
-            if (lane == 0) {
+            umma_commit(&sm.s_full);
+        }
+        __syncwarp();
+    };
+    auto issue_pv = [&](int t) {
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(sm.v[t % kKvBufs]);
+        if (lane == 0) {
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
+            for (int half = 0; half < 2; ++half) {
 #pragma unroll
-                    for (int part = 0; part < 2; ++part) {
-                        // P'_hi then P'_lo of key half `half`: 8 TMEM columns per 16 keys
-                        const uint32_t pa = tmem + kTmemP + 64 * (t & 1) + 32 * half + 16 * part;
+                for (int part = 0; part < 2; ++part) {
+                    // P'_hi then P'_lo of key half `half`: 8 TMEM columns per 16 keys
+                    const uint32_t pa = tmem + kTmemP + 64 * (t & 1) + 32 * half + 16 * part;
 #pragma unroll
-                        for (int k2 = 0; k2 < 2; ++k2) {
-                            const int kk = 2 * half + k2;         // 16-key step of the tile
-                            const uint64_t db = umma_desc(v0 + 2 * kk * v_sbo, 1024, v_sbo);
-                            umma_f16_ts(tmem + kTmemO + half * D, pa + 8 * k2, db, idesc_pv, part > 0 || t > 0 || k2 > 0);
-                        }
+                    for (int k2 = 0; k2 < 2; ++k2) {
+                        const int kk = 2 * half + k2;         // 16-key step of the tile
+                        const uint64_t db = umma_desc(v0 + 2 * kk * v_sbo, 1024, v_sbo);
+                        umma_f16_ts(tmem + kTmemO + half * D, pa + 8 * k2, db, idesc_pv, part > 0 || t > 0 || k2 > 0);
                     }
                 }
-                umma_commit(&sm.pv_done[t & 1]);
-                umma_commit(&sm.kv_empty[t % kKvBufs]);
             }
-            __syncwarp();
-        };
-        // Issue QK(t) once K(t) is unpacked and the softmax has read S(t-1), and PV(t) once
-        // P'(t) is written; QK first when both are ready (it feeds the softmax).
-        bool alive = true;
-        int next_qk = 0, next_pv = 0;
-        uint64_t t_start = global_ns();
-        while (next_pv < n_kt) {
-            bool progressed = false;
-            if (next_qk < n_kt &&
-                __all_sync(0xffffffffu, mbar_test(&sm.kv_full[next_qk % kKvBufs], (next_qk / kKvBufs) & 1) &&
-                                            (next_qk == 0 || mbar_test(&sm.s_free, (next_qk - 1) & 1)))) {
-                issue_qk(next_qk++);
-                progressed = true;
-            }
-            if (next_pv < next_qk &&
-                __all_sync(0xffffffffu, mbar_test(&sm.p_full[next_pv & 1], (next_pv >> 1) & 1))) {
-                issue_pv(next_pv++);
-                progressed = true;
-            }
-            if (progressed) {
-                t_start = global_ns();
-            } else if (global_ns() - t_start > 2000000000ull) {   // bounded: about two seconds
-                set_status(c.status, KVQ_ERR_DEVICE_CHECK);
-                alive = false;
-                break;
-            } else if (*reinterpret_cast<volatile int *>(&sm.abort_flag)) {
-                alive = false;
-                break;
-            } else {
-                __nanosleep(32);          // leave the issue slots to the warps doing the work
-            }
+            umma_commit(&sm.pv_done[t & 1]);
+            umma_commit(&sm.kv_empty[t % kKvBufs]);
         }
-        if (!alive) sm.abort_flag = 1;
-        // every MMA this CTA issued has completed before its TMEM is freed (bounded wait)
+        __syncwarp();
+    };
+    if (warp == kMmaWarp) {
+        // QK(t) once K(t) is unpacked and the softmax has read S(t-1); the PV MMAs come from
+        // their own warp. Both wait on their barriers (suspended, no polling).
+        for (int t = 0; t < n_kt; ++t) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.kv_full[t % kKvBufs], (t / kKvBufs) & 1, c.status) &&
+                                             (t == 0 || mbar_wait(&sm.s_free, (t - 1) & 1, c.status)) &&
+                                             !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
+                sm.abort_flag = 1;
+                break;
+            }
+            issue_qk(t);
+        }
+        // every MMA this warp issued has completed before the TMEM is freed (bounded wait)
+        if (lane == 0) umma_commit(&sm.drain);
+        __syncwarp();
+        mbar_wait(&sm.drain, 0, c.status);
+    } else if (warp == kPvWarp) {
+        // ------------------------------- PV issuer ---------------------------------
+        // PV(t) once P'(t) is in TMEM (which implies that QK(t) has completed)
+        for (int t = 0; t < n_kt; ++t) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_full[t & 1], (t >> 1) & 1, c.status) &&
+                                             !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
+                sm.abort_flag = 1;
+                break;
+            }
+            issue_pv(t);
+        }
         if (lane == 0) umma_commit(&sm.drain);
         __syncwarp();
         mbar_wait(&sm.drain, 0, c.status);
@@ -500,10 +494,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 if (cb == c2) pb = start + __popc(ba) + __popc(bb & lt);
                 start += __popc(ba) + __popc(bb);
             }
-            const uint32_t wa = ((ca < 4 ? (ma & ~15u) - base : 0u) << 16) | ((uint32_t)ca << 8) | ((uint32_t)lane << 2);
-            const uint32_t wb = ((cb < 4 ? (mb & ~15u) - base : 0u) << 16) | ((uint32_t)cb << 8) | ((uint32_t)(32 + lane) << 2);
-            *reinterpret_cast<uint4 *>(&sm.task[st][4 * pa]) = make_uint4(wa, wa | 1u, wa | 2u, wa | 3u);
-            *reinterpret_cast<uint4 *>(&sm.task[st][4 * pb]) = make_uint4(wb, wb | 1u, wb | 2u, wb | 3u);
+            sm.task[st][pa] = ((ca < 4 ? (ma & ~15u) - base : 0u) << 16) | ((uint32_t)ca << 8) | (uint32_t)lane;
+            sm.task[st][pb] = ((cb < 4 ? (mb & ~15u) - base : 0u) << 16) | ((uint32_t)cb << 8) | (uint32_t)(32 + lane);
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive_expect_tx(&sm.raw_full[st], end - base);
@@ -529,12 +521,15 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     } else if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegUnpack));
         // ------------------------------ K/V unpack -----------------------------------
-        // Thread = one conversion task of the tile (a key, a quarter of its channels), as
-        // ordered by the stager; the side entry of its own key kj = u / 4 is loaded three
-        // tiles ahead.
+        // Each warp converts 8 keys of the class-ordered list, D/8 lanes per key and one
+        // 8-channel chunk per lane, so that a quarter warp reads 128 consecutive staged bytes
+        // and writes eight distinct 16-byte slots of a swizzled row (no bank conflicts). The
+        // side entry of key kj = u / 4 is loaded three tiles ahead by one thread in four.
         const int u = tid - kSoftmaxThreads;
         const int kj = u / kQP, half = u % kQP;
-        constexpr int CH = D / kQP;                  // channels per task
+        constexpr int kCpr = D / 8;                  // 8-channel chunks per row
+        constexpr int kKpp = 32 / kCpr;              // keys per pass of a warp
+        const int uw = u >> 5, chunk = lane % kCpr, kslot = lane / kCpr;
         auto load_side = [&](int t) -> float4 {
             const int j = klo + t * kKeys + kj;
             return (half == 0 && t < n_kt && j <= khi) ? c.side[sbase + j] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -560,17 +555,14 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                 sv[0] = sd_cur.z;
                 sv[2] = sd_cur.w;
             }
-            const uint32_t task = sm.task[st][u];
-            const int cls = (int)((task >> 8) & 7u), tkj = (int)((task >> 2) & 63u), thalf = (int)(task & 3u);
-            const int bits = (cls < 4) ? (2 << cls) : 0;
-            const uint8_t *rec = sm.raw[st] + (task >> 16);
-            const uint8_t *ksrc = rec + thalf * (CH * bits / 8);
-            const uint8_t *vsrc = ksrc + bits * D / 8;
 #pragma unroll
-            for (int cc = 0; cc < CH / 8; ++cc) {
-                const int chunk = thalf * (CH / 8) + cc;      // 8-channel chunk of the row
-                const uint4 kx = bits ? unpack8(ksrc, bits, cc) : make_uint4(0, 0, 0, 0);
-                const uint4 vx = bits ? unpack8(vsrc, bits, cc) : make_uint4(0, 0, 0, 0);
+            for (int pass = 0; pass < 8 / kKpp; ++pass) {
+                const uint32_t task = sm.task[st][8 * uw + kKpp * pass + kslot];
+                const int cls = (int)((task >> 8) & 7u), tkj = (int)(task & 63u);
+                const int bits = (cls < 4) ? (2 << cls) : 0;
+                const uint8_t *ksrc = sm.raw[st] + (task >> 16);
+                const uint4 kx = bits ? unpack8(ksrc, bits, chunk) : make_uint4(0, 0, 0, 0);
+                const uint4 vx = bits ? unpack8(ksrc + bits * D / 8, bits, chunk) : make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4 *>(kb + (chunk >> 3) * (kKeys * 128) + kmajor_off(tkj, chunk & 7)) = kx;
                 const int n = chunk * 8;
                 const int atom = (tkj >> 3) * (D / 64) + (n >> 6);
