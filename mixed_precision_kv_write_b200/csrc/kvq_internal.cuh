@@ -208,15 +208,16 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
-// Wait until the barrier's phase `parity` has completed. The waiting thread may be
-// suspended by the hardware for up to ~0.1 ms per try (woken when the phase completes),
-// so waiting warps do not spin on issue slots. Bounded: gives up after `limit_ns` (about
-// two seconds by default), records KVQ_ERR_DEVICE_CHECK and returns false, so a logic
-// error ends the kernel with a status instead of hanging the GPU.
+// Wait until the barrier's phase `parity` has completed. Each try_wait lets the hardware
+// hold the thread for a short, implementation-defined time; a suspend-time hint
+// (KVQ_WAIT_HINT_NS > 0) would let it sleep longer but measured slower wake-ups on B200
+// (prefill and decode), so the default passes none. Bounded: gives up after `limit_ns`
+// (about two seconds by default), records KVQ_ERR_DEVICE_CHECK and returns false, so a
+// logic error ends the kernel with a status instead of hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 #ifndef KVQ_WAIT_HINT_NS
-#define KVQ_WAIT_HINT_NS 100000
+#define KVQ_WAIT_HINT_NS 0
 #endif
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
                                           uint64_t limit_ns = kWaitLimitNs)

@@ -20,9 +20,9 @@
 //     - warps 8-15: unpack each 64-key tile's K and V codes into exact fp16 operands (codes
 //       are integers <= 255; b = 16 keys are the fp16 values) in shared memory, three tiles
 //       in flight; K 128B-swizzled K-major, V 128B-swizzled MN-major.
-//     - warp 16: owns 512 TMEM columns (S, P' double buffer, Q, O of each key half) and
-//       issues the MMAs from one lane: S = Q C_K^T (M128 N64 K16 steps, A = Q in TMEM, B in
-//       shared memory) once K(t) is unpacked and S(t-1) has been read, and
+//     - warp 16: owns 512 TMEM columns (S double buffer, P', Q, O of each key half) and
+//       issues the QK MMAs from one lane: S = Q C_K^T (M128 N64 K16 steps, A = Q in TMEM, B
+//       in shared memory) once K(t) is unpacked and S(t-2) has been read; warp 18 issues
 //       O_h += P'_h,hi V_h + P'_h,lo V_h per key half h (M128 ND K16, A in TMEM) once P'(t)
 //       is written.
 //     - warp 17: stages each key tile's records (one contiguous byte range of the stream)
@@ -58,10 +58,12 @@ static_assert(kSoftmaxThreads * kRegSoftmax + kUnpackThreads * kRegUnpack + 128 
 constexpr int kRawBufs = 3;     // record staging buffers: a key tile's records land up to three tiles ahead
 constexpr int kKvBufs = 3;      // unpacked K/V operand tiles in flight
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S (fp32, 64 keys) at 0; P' double buffer at 64 and 128, each holding per key
-// half h the fp16 pairs of P'_hi (16 columns) then P'_lo (16) at 32 h; Q (fp16 pairs, D / 2
-// columns) at 192; O of key half h (fp32, D columns) at 256 + h D.
-constexpr uint32_t kTmemS = 0, kTmemP = 64, kTmemQ = 192, kTmemO = 256;
+// TMEM columns: S double buffer (fp32, 64 keys) at 0 and 64; P' at 128, holding per key half h
+// the fp16 pairs of P'_hi (16 columns) then P'_lo (16) at 32 h; Q (fp16 pairs, D / 2 columns)
+// at 192; O of key half h (fp32, D columns) at 256 + h D. S is double buffered so that QK(t+1)
+// never waits for the softmax of tile t; one P' buffer suffices because PV(t-1) has long
+// completed when the softmax of tile t writes P'(t).
+constexpr uint32_t kTmemS = 0, kTmemP = 128, kTmemQ = 192, kTmemO = 256;
 
 // ---- tcgen05 / UMMA helpers -------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), descriptor version 1.
@@ -275,7 +277,7 @@ struct alignas(1024) PfSmem {
     float4 fin[2][kQRows];            // per key half: (running max, l, sum p z_V) of each row
     float qpart[2][kQRows];           // per half of the channels: partial sums of each Q row
     uint64_t raw_full[kRawBufs], raw_empty[kRawBufs], kv_full[kKvBufs], kv_empty[kKvBufs];
-    uint64_t s_full, s_free, p_full[2], pv_done[2], drain;
+    uint64_t s_full[2], s_free[2], p_full, pv_done, drain;
     uint32_t tmem_base;
     int32_t klo, khi, abort_flag;
 };
@@ -309,12 +311,12 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             mbar_init(&sm.raw_full[i], 1);
             mbar_init(&sm.raw_empty[i], kUnpackWarps);
         }
-        mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.s_free, kSoftmaxWarps);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.p_full[i], kSoftmaxWarps);
-            mbar_init(&sm.pv_done[i], 1);
+            mbar_init(&sm.s_full[i], 1);
+            mbar_init(&sm.s_free[i], kSoftmaxWarps);
         }
+        mbar_init(&sm.p_full, kSoftmaxWarps);
+        mbar_init(&sm.pv_done, 1);
         mbar_init(&sm.drain, 2);
         sm.klo = INT32_MAX;
         sm.khi = -1;
@@ -391,9 +393,9 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint64_t db = umma_desc(k0 + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
-                umma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * kk, db, idesc_qk, kk > 0);
+                umma_f16_ts(tmem + kTmemS + 64 * (t & 1), tmem + kTmemQ + 8 * kk, db, idesc_qk, kk > 0);
             }
-            umma_commit(&sm.s_full);
+            umma_commit(&sm.s_full[t & 1]);
         }
         __syncwarp();
     };
@@ -406,7 +408,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
                     // P'_hi then P'_lo of key half `half`: 8 TMEM columns per 16 keys
-                    const uint32_t pa = tmem + kTmemP + 64 * (t & 1) + 32 * half + 16 * part;
+                    const uint32_t pa = tmem + kTmemP + 32 * half + 16 * part;
 #pragma unroll
                     for (int k2 = 0; k2 < 2; ++k2) {
                         const int kk = 2 * half + k2;         // 16-key step of the tile
@@ -415,17 +417,17 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                     }
                 }
             }
-            umma_commit(&sm.pv_done[t & 1]);
+            umma_commit(&sm.pv_done);
             umma_commit(&sm.kv_empty[t % kKvBufs]);
         }
         __syncwarp();
     };
     if (warp == kMmaWarp) {
-        // QK(t) once K(t) is unpacked and the softmax has read S(t-1); the PV MMAs come from
+        // QK(t) once K(t) is unpacked and the softmax has read S(t-2); the PV MMAs come from
         // their own warp. Both wait on their barriers (suspended, no polling).
         for (int t = 0; t < n_kt; ++t) {
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.kv_full[t % kKvBufs], (t / kKvBufs) & 1, c.status) &&
-                                             (t == 0 || mbar_wait(&sm.s_free, (t - 1) & 1, c.status)) &&
+                                             (t < 2 || mbar_wait(&sm.s_free[t & 1], ((t - 2) >> 1) & 1, c.status)) &&
                                              !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
                 sm.abort_flag = 1;
                 break;
@@ -440,7 +442,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         // ------------------------------- PV issuer ---------------------------------
         // PV(t) once P'(t) is in TMEM (which implies that QK(t) has completed)
         for (int t = 0; t < n_kt; ++t) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_full[t & 1], (t >> 1) & 1, c.status) &&
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_full, t & 1, c.status) &&
                                              !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
                 sm.abort_flag = 1;
                 break;
@@ -591,7 +593,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         for (int t = 0; t < n_kt; ++t) {
             const int st = t % kKvBufs;
             // warp-uniform outcome: the TMEM accesses below are .sync.aligned
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full, t & 1, c.status) &&
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t & 1], (t >> 1) & 1, c.status) &&
                                              !*reinterpret_cast<volatile int *>(&sm.abort_flag))) {
                 sm.abort_flag = 1;
                 ok = false;
@@ -599,11 +601,11 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             }
             tc_fence_after();
             float sv[32];
-            tmem_ld32(tmem + lane_base + kTmemS + 32 * kh, sv);
+            tmem_ld32(tmem + lane_base + kTmemS + 64 * (t & 1) + 32 * kh, sv);
             // S may now be overwritten by QK(t+1)
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_free);
+            if (lane == 0) mbar_arrive(&sm.s_free[t & 1]);
             const int kt0 = klo + t * kKeys + 32 * kh;
             // the row's keys in this half tile: [max(row_lo, kt0), min(row_t, kt0 + 31)]
             const int c_lo = max(row_lo - kt0, 0), c_hi = min(row_t - kt0, 31);
@@ -666,13 +668,11 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             l_run = __ffma2_rn(l_run, corr2, psum);
             pz_run = __ffma2_rn(pz_run, corr2, pz);
             /*TRACE_EXP*/
-            // P' buffer t & 1 was last read by PV(t-2); a rescale of O also needs PV(t-1) done
-            // (the MMAs complete in issue order, so waiting for PV(t-1) covers PV(t-2))
+            // P' was last read by PV(t-1), which a rescale of O also needs complete
             const bool rescale = t > 0 && __any_sync(0xffffffffu, bump);
             /*TRACE_RESC*/
-            const int t_wait = rescale ? t - 1 : t - 2;
-            if (t_wait >= 0) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t_wait & 1], (t_wait >> 1) & 1, c.status))) {
+            if (t > 0) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (t - 1) & 1, c.status))) {
                     sm.abort_flag = 1;
                     ok = false;
                     break;
@@ -702,18 +702,18 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
                     hw[i] = *reinterpret_cast<const uint32_t *>(&hv);
                     lw[i] = *reinterpret_cast<const uint32_t *>(&lv);
                 }
-                tmem_st16u(tmem + lane_base + kTmemP + 64 * (t & 1) + 32 * kh, hw);
-                tmem_st16u(tmem + lane_base + kTmemP + 64 * (t & 1) + 32 * kh + 16, lw);
+                tmem_st16u(tmem + lane_base + kTmemP + 32 * kh, hw);
+                tmem_st16u(tmem + lane_base + kTmemP + 32 * kh + 16, lw);
             }
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.p_full[t & 1]);
+            if (lane == 0) mbar_arrive(&sm.p_full);
         }
         // ---- merge the two key halves of each row; each warp writes half the channels ----
         const int t_last = n_kt - 1;
         if (ok && n_kt > 0 &&
-            !__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t_last & 1], (t_last >> 1) & 1, c.status)))
+            !__all_sync(0xffffffffu, mbar_wait(&sm.pv_done, t_last & 1, c.status)))
             ok = false;
         tc_fence_after();
         sm.fin[kh][row] = make_float4(m_run, l_run.x + l_run.y, pz_run.x + pz_run.y, 0.f);
