@@ -12,7 +12,7 @@
 //                         ranges, cut where the local window starts, so within an item
 //                         every active query reads every key. Ranges are cut into
 //                         near-equal items of at most 1152 keys. Each CTA reserves its items
-//                         with one atomic on a (call generation, count) word.
+//                         with one atomicAdd on the call's (generation, count) word.
 //   decode_splitk_kernel  three CTAs per SM, one producer and four consumer warps each. The
 //                         producer walks the CTA's items in stages of at most 128 keys and
 //                         24 KB of records: a ring of record-offset windows is bulk-copied
@@ -188,6 +188,8 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
     __shared__ int64_t u_sbase[kPlanThreads];
     pdl_wait();
     pdl_trigger();
+    // the previous call's kernels have completed: its count word becomes the next call's
+    if (blockIdx.x == 0 && threadIdx.x == 0) *wk.count_next = (unsigned long long)(gen + 1u) << 32;
     const int s = blockIdx.x;
     if (APPEND) append_seq<D>(c, ap.k, ap.v, ap.bits, ap.cu, ap.n_tok, ap.gen, ap.positions, s, bad_sh);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -243,23 +245,15 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
             tot += t;
         }
         if (tid == 0) {
-            // reserve [base, base + tot) in this call's list; the first CTA of a call to
-            // arrive resets the count left by the previous call
-            unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(wk.count), nw;
-            uint32_t base;
-            while (true) {
-                if ((uint32_t)(old >> 32) != gen) {
-                    base = 0;
-                    nw = ((unsigned long long)gen << 32) | (unsigned long long)tot;
-                } else {
-                    base = (uint32_t)old;
-                    nw = old + (unsigned long long)tot;
-                }
-                const unsigned long long prev = atomicCAS(wk.count, old, nw);
-                if (prev == old) break;
-                old = prev;
+            // reserve [base, base + tot) in this call's list (one atomic, no retries)
+            const unsigned long long old = atomicAdd(wk.count, (unsigned long long)tot);
+            const uint32_t tag = (uint32_t)(old >> 32);
+            if (tag != gen && tag != 0u) {           // stale word: list nothing
+                set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+                base_sh = 0xFFFFFFFFu;
+            } else {
+                base_sh = (uint32_t)old;
             }
-            base_sh = base;
             u_start[kPlanThreads] = tot;
         }
         const int rel = wpre + incl - cnt;            // the unit's first item within the pass
@@ -275,14 +269,16 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
             u_sbase[tid] = slot_of(c, s, hk, 0);
         }
         __syncthreads();
-        const int64_t base = base_sh;
+        const bool stale = base_sh == 0xFFFFFFFFu;
+        const int64_t base = stale ? 0 : base_sh;
         if (mine && u % nsub == 0) {                  // the KV head's items: its subgroups' runs
             int n_all = 0;
             for (int k = 0; k < nsub; ++k) n_all += cnt_sh[tid + k];
             wk.head_first[s * H + hk] = (int32_t)(base + rel);
-            wk.head_cnt[s * H + hk] = n_all;
+            wk.head_cnt[s * H + hk] = stale ? 0 : n_all;
         }
-        if (base + tot > wk.max_items) {
+        if (stale) {
+        } else if (base + tot > wk.max_items) {
             if (tid == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
         } else {
             // every thread writes items: item i of the pass belongs to the last unit whose
@@ -539,7 +535,9 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait();
     pdl_trigger();
-    const int n_items = (int)min((int64_t)(uint32_t)(*wk.count), wk.max_items);
+    const unsigned long long cw = *wk.count;
+    const uint32_t tag = (uint32_t)(cw >> 32);
+    const int n_items = (tag == wk.gen || tag == 0u) ? (int)min((int64_t)(uint32_t)cw, wk.max_items) : 0;
     const int HQ = c.H * c.G;
 
     if (tid == 0) {
@@ -1030,11 +1028,26 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const DecodeWork &wk, uint32
     return cudaGetLastError();
 }
 
+// wk.count points at the pair of count words; the call uses word gen & 1. `stale` is set when
+// a launch fails (a call whose planning kernel did not run leaves the next call's word
+// unprepared); the words are then cleared (tag 0, never used) before the next call.
 cudaError_t launch_any(const kvq_cache *cache, const DecodeWork &wk, uint32_t gen, const __half *q,
-                       const uint8_t *modes, int w, float *out, cudaStream_t st, const AppendArgs *ap)
+                       const uint8_t *modes, int w, float *out, cudaStream_t st, const AppendArgs *ap,
+                       bool &stale)
 {
-    if (cache->D == 128) return launch_decode_t<128>(cache, wk, gen, q, modes, w, out, st, ap);
-    return launch_decode_t<64>(cache, wk, gen, q, modes, w, out, st, ap);
+    if (stale) {
+        const cudaError_t e = cudaMemsetAsync(wk.count, 0, 2 * sizeof(unsigned long long), st);
+        if (e != cudaSuccess) return e;
+        stale = false;
+    }
+    DecodeWork cw = wk;
+    cw.count = wk.count + (gen & 1u);
+    cw.count_next = wk.count + ((gen + 1u) & 1u);
+    cw.gen = gen;
+    const cudaError_t e = (cache->D == 128) ? launch_decode_t<128>(cache, cw, gen, q, modes, w, out, st, ap)
+                                            : launch_decode_t<64>(cache, cw, gen, q, modes, w, out, st, ap);
+    if (e != cudaSuccess) stale = true;
+    return e;
 }
 
 } // namespace
@@ -1044,8 +1057,8 @@ cudaError_t launch_decode(const kvq_cache *cache, const __half *q, const uint8_t
 {
     kvq_cache *mc = const_cast<kvq_cache *>(cache);   // the call's generation id only
     uint32_t gen = ++mc->decode_gen;
-    if (gen == 0) gen = ++mc->decode_gen;             // 0 is the count word's initial generation
-    return launch_any(cache, cache->work, gen, q, modes, w, out, st, nullptr);
+    if (gen == 0) gen = ++mc->decode_gen;             // 0 tags a count word never used
+    return launch_any(cache, cache->work, gen, q, modes, w, out, st, nullptr, mc->work_stale);
 }
 
 cudaError_t launch_decode_step(kvq_cache *cache, const __half *q, const __half *k, const __half *v,
@@ -1056,7 +1069,7 @@ cudaError_t launch_decode_step(kvq_cache *cache, const __half *q, const __half *
     AppendArgs ap{k, v, bits, cu, positions, n_tok, ++cache->write_gen};
     uint32_t gen = ++cache->decode_gen;
     if (gen == 0) gen = ++cache->decode_gen;
-    return launch_any(cache, cache->work, gen, q, modes, w, out, st, &ap);
+    return launch_any(cache, cache->work, gen, q, modes, w, out, st, &ap, cache->work_stale);
 }
 
 } // namespace kvq
@@ -1078,7 +1091,8 @@ namespace {
 
 std::mutex g_scratch_mu;
 void *g_scratch_addr[256] = {};   // device address of g_decode_scratch, per device ordinal
-std::atomic<uint32_t> g_static_gen{0};
+std::atomic<uint32_t> g_static_gen[256];   // per device ordinal: generation of the last call
+bool g_static_stale[256] = {};             // per device ordinal: a launch failed (under g_scratch_mu)
 
 cudaError_t static_scratch(int dev, unsigned char **out)
 {
@@ -1144,12 +1158,15 @@ extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache,
     wk.partials = reinterpret_cast<float *>(base + o_part);
     wk.max_items = items;
     wk.qslots = qslots;
-    // a generation id no earlier call on the shared array used (never 0: the array starts
-    // zeroed, and the first planning CTA of this call resets the count it finds)
-    uint32_t gen = ++g_static_gen;
-    if (gen == 0) gen = ++g_static_gen;
+    // a generation id no earlier call on the shared array used (never 0, the tag of a word
+    // never used: the array starts zeroed)
+    uint32_t gen = ++g_static_gen[dev];
+    if (gen == 0) gen = ++g_static_gen[dev];
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    e = launch_any(cache, wk, gen, static_cast<const __half *>(q), modes, w, out, st, nullptr);
+    {
+        std::lock_guard<std::mutex> lock(g_scratch_mu);
+        e = launch_any(cache, wk, gen, static_cast<const __half *>(q), modes, w, out, st, nullptr, g_static_stale[dev]);
+    }
     if (e != cudaSuccess) return report_error(KVQ_ERR_CUDA, "routed_attn_decode_noalloc: kernel launch failed");
     return report_error(KVQ_OK, "");
 }

@@ -151,7 +151,14 @@ struct __align__(16) DecodeItem {
 
 struct DecodeWork {
     DecodeItem *items;   // [max_items]
-    unsigned long long *count; // [1]: call generation << 32 | items listed by the call
+    // Item counts, two words used by calls of alternating generation parity: a call of
+    // generation g reserves its items with atomicAdd on `count` (g << 32 | items; a word
+    // still tagged 0 has never been used) and prepares `count_next`, the word of call g + 1,
+    // as (g + 1) << 32. A word with any other tag is stale: the call lists nothing and
+    // reports KVQ_ERR_DEVICE_CHECK.
+    unsigned long long *count;
+    unsigned long long *count_next;
+    uint32_t gen;        // the call's generation
     int32_t *head_first; // [B*H] first item of (sequence, KV head)
     int32_t *head_cnt;   // [B*H] its items (all subgroups)
     float *partials;     // [max_items][qslots][D + 4]: (m, l, -, -, o[D])
@@ -332,6 +339,7 @@ struct kvq_cache {
     kvq::DecodeWork work;
     uint32_t write_gen;       // id of the last kvq_write call
     uint32_t decode_gen;      // id of the last decode call on the cache's own work list
+    bool work_stale;          // a decode launch failed: the count words are cleared before the next call
     void *pf_tiles;           // prefill tile lists (PfTile = 8 x int32): as listed, then ordered
     int32_t *pf_count;        // [1]
     int32_t *pf_qidx;         // [total_slots] per-(sequence, head) query lists
