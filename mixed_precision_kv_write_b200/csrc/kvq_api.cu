@@ -1,6 +1,8 @@
 // C ABI of the routed mixed-precision KV cache: argument checks, cache allocation,
 // small maintenance kernels (reset, truncate, lengths, export) and the status word.
-// The hot-path kernels live in kvq_write.cu, kvq_decode.cu and kvq_prefill.cu.
+// The hot-path kernels live in kvq_write.cu, kvq_decode.cu, kvq_prefill_tc.cu and
+// kvq_route.cu. Every compute entry point is an NVTX range (named after the call) for
+// timeline tools; without a tool attached a range costs a few nanoseconds.
 #include <algorithm>
 #include <cstdarg>
 #include <cstdio>
@@ -10,9 +12,16 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kvq_internal.cuh"
 
 namespace {
+
+struct ApiRange {                 // NVTX range around one API call
+    explicit ApiRange(const char *name) { nvtxRangePushA(name); }
+    ~ApiRange() { nvtxRangePop(); }
+};
 
 thread_local std::string g_err;
 
@@ -187,6 +196,7 @@ extern "C" {
 int kvq_route_argmax(const float *z_attn, const float *z_bits, int64_t n, uint8_t *modes,
                      uint8_t *bits, kvq_stream_t stream)
 {
+    const ApiRange range("kvq_route_argmax");
     if (n < 0) return fail(KVQ_ERR_ARG, "kvq_route_argmax: n = %lld < 0", (long long)n);
     if ((!z_attn) != (!modes)) return fail(KVQ_ERR_ARG, "kvq_route_argmax: z_attn and modes go together");
     if ((!z_bits) != (!bits)) return fail(KVQ_ERR_ARG, "kvq_route_argmax: z_bits and bits go together");
@@ -429,6 +439,7 @@ int kvq_cache_lengths(const kvq_cache *c, int32_t *lengths, kvq_stream_t stream)
 int kvq_write(const void *k, const void *v, const uint8_t *bits, const int32_t *cu_seqlens,
               int64_t n_tok, kvq_cache *c, kvq_stream_t stream)
 {
+    const ApiRange range("kvq_write");
     if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_write: bad cache");
     if (n_tok < 0 || n_tok > (int64_t)INT32_MAX / c->H)
         return fail(KVQ_ERR_ARG, "kvq_write: n_tok = %lld out of range", (long long)n_tok);
@@ -444,6 +455,7 @@ int kvq_write(const void *k, const void *v, const uint8_t *bits, const int32_t *
 int routed_attn_prefill(const void *q, const kvq_cache *c, const uint8_t *modes, int w,
                         const int32_t *cu_seqlens, int64_t n_tok, float *out, kvq_stream_t stream)
 {
+    const ApiRange range("routed_attn_prefill");
     if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "routed_attn_prefill: bad cache");
     if (w < 0) return fail(KVQ_ERR_ARG, "routed_attn_prefill: w = %d < 0", w);
     if (n_tok < 0 || n_tok > (int64_t)INT32_MAX / ((int64_t)c->H * c->view.G))
@@ -463,6 +475,7 @@ int routed_attn_prefill(const void *q, const kvq_cache *c, const uint8_t *modes,
 int routed_attn_decode(const void *q, const kvq_cache *c, const uint8_t *modes, int w, float *out,
                        kvq_stream_t stream)
 {
+    const ApiRange range("routed_attn_decode");
     if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "routed_attn_decode: bad cache");
     if (w < 0) return fail(KVQ_ERR_ARG, "routed_attn_decode: w = %d < 0", w);
     if (!q || !modes || !out) return fail(KVQ_ERR_ARG, "routed_attn_decode: q, modes or out is NULL");
@@ -477,6 +490,7 @@ int kvq_decode_step(const void *q, const void *k, const void *v, const uint8_t *
                     int64_t n_tok, const int32_t *positions, const uint8_t *modes, int w, kvq_cache *c,
                     float *out, kvq_stream_t stream)
 {
+    const ApiRange range("kvq_decode_step");
     if (!valid_cache(c)) return fail(KVQ_ERR_ARG, "kvq_decode_step: bad cache");
     if (w < 0) return fail(KVQ_ERR_ARG, "kvq_decode_step: w = %d < 0", w);
     if (n_tok < 0 || n_tok > (int64_t)INT32_MAX / c->H)

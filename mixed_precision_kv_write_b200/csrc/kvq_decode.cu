@@ -45,6 +45,8 @@
 #include <cstdio>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kvq_quant.cuh"
 
 namespace kvq {
@@ -1117,6 +1119,10 @@ extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache,
                                           int w, float *out, kvq_stream_t stream)
 {
     using namespace kvq;
+    struct Range {                 // NVTX range around the call
+        Range() { nvtxRangePushA("routed_attn_decode_noalloc"); }
+        ~Range() { nvtxRangePop(); }
+    } range;
     if (!cache || cache->B <= 0 || cache->H <= 0)
         return report_error(KVQ_ERR_ARG, "routed_attn_decode_noalloc: bad cache");
     if (w < 0) return report_error(KVQ_ERR_ARG, "routed_attn_decode_noalloc: w < 0");
