@@ -338,6 +338,8 @@ int kvq_cache_create_paged(kvq_cache **out, int batch, int heads, int query_grou
     c->pf_tiles = alloc(sizeof(int32_t) * 16 * (size_t)c->pf_max_tiles);    // two lists of 32-byte tiles
     c->pf_count = (int32_t *)alloc(sizeof(int32_t));
     c->pf_qidx = (int32_t *)alloc(sizeof(int32_t) * (size_t)slots * query_group);
+    c->scan_chunks = (max_cap + 1023) / 1024;
+    c->scan_flags = (uint64_t *)alloc(sizeof(uint64_t) * (size_t)BH * std::max(1, c->scan_chunks));
     for (int i = 0; i < c->n_allocs; ++i) okk = okk && c->allocs[i];
     if (!okk || c->n_allocs != n_tried) {
         kvq_cache_destroy(c);
@@ -371,6 +373,7 @@ int kvq_cache_create_paged(kvq_cache **out, int batch, int heads, int query_grou
     e = e ? e : cudaMemsetAsync(v.status, 0, sizeof(int32_t), st);
     e = e ? e : cudaMemsetAsync(v.meta, 0, sizeof(uint32_t) * (size_t)slots, st);
     e = e ? e : cudaMemsetAsync(wk.count, 0, 2 * sizeof(unsigned long long), st);
+    e = e ? e : cudaMemsetAsync(c->scan_flags, 0, sizeof(uint64_t) * (size_t)BH * std::max(1, c->scan_chunks), st);
     if (paged) {
         e = e ? e : cudaMemsetAsync(v.npages, 0, sizeof(int32_t) * BH, st);
         e = e ? e : cudaMemsetAsync(v.pool_next, 0, sizeof(int32_t), st);

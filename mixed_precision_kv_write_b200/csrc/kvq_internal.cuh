@@ -340,6 +340,8 @@ struct kvq_cache {
     uint32_t write_gen;       // id of the last kvq_write call
     uint32_t decode_gen;      // id of the last decode call on the cache's own work list
     bool work_stale;          // a decode launch failed: the count words are cleared before the next call
+    uint64_t *scan_flags;     // [B*H*scan_chunks]: the long write scan's per-chunk look-back words
+    int scan_chunks;          // chunks of 1024 tokens in the largest capacity
     void *pf_tiles;           // prefill tile lists (PfTile = 8 x int32): as listed, then ordered
     int32_t *pf_count;        // [1]
     int32_t *pf_qidx;         // [total_slots] per-(sequence, head) query lists

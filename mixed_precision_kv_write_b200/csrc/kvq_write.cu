@@ -130,6 +130,156 @@ write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *
     }
 }
 
+// Long calls: the same results as write_scan_kernel, with each (sequence, head) split into
+// chunks of 1024 tokens, one CTA of 256 threads per chunk, so that long sequences do not
+// leave most SMs idle. A CTA scans its chunk's record sizes, publishes the chunk's total
+// at once, and finds the bytes before its chunk by looking back over the totals (or the
+// running prefixes, once known) its predecessors published in a per-(sequence, head)
+// array of 64-bit words (call generation << 34 | state << 32 | bytes; state 1: the
+// chunk's total, 2: the prefix through the chunk). The look-back only waits on CTAs of
+// lower index, which start first; its wait is bounded. The last chunk of a (sequence,
+// head) records the write start and the new stream end.
+constexpr int kScanChunkThreads = 256, kScanChunkPer = 4, kScanChunk = kScanChunkThreads * kScanChunkPer;
+
+__device__ __forceinline__ void st_release_u64(uint64_t *p, uint64_t v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p)
+{
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(kScanChunkThreads)
+write_scan_chunk_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *__restrict__ cu,
+                        int64_t n_tok, uint32_t gen, uint64_t *__restrict__ flags, int n_chunks)
+{
+    __shared__ uint32_t wsum[kScanChunkThreads / 32];
+    __shared__ uint32_t excl_sh;
+    pdl_wait();
+    pdl_trigger();
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t gsh = blockIdx.x / n_chunks;
+    const int ck = (int)(blockIdx.x % n_chunks);
+    const int H = c.H;
+    if (gsh >= (int64_t)c.B * H) return;
+    const int s = (int)(gsh / H), h = (int)(gsh % H), sh = s * H + h;
+    const int64_t t0 = cu[s], t1 = cu[s + 1];
+    if (t0 < 0 || t1 < t0 || t1 > n_tok || (s == 0 && t0 != 0)) {
+        if (ck == 0 && tid == 0) {
+            set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+            c.wstart[sh] = -1;
+        }
+        return;
+    }
+    const int n = (int)(t1 - t0);
+    if (ck > 0 && ck * kScanChunk >= n) return;  // past this sequence's tokens
+    const int L0 = c.len[sh];
+    if ((int64_t)L0 + n > c.cap[s]) {
+        if (ck == 0 && tid == 0) {
+            set_status(c.status, KVQ_ERR_CAPACITY);
+            c.wstart[sh] = -1;
+        }
+        return;
+    }
+    const uint32_t off0 = c.end[sh];
+    const int nck = (n + kScanChunk - 1) / kScanChunk;
+    // this chunk's tokens: kScanChunkPer consecutive ones per thread
+    uint32_t sz[kScanChunkPer], wcs[kScanChunkPer], mine = 0;
+    bool bad = false;
+#pragma unroll
+    for (int e = 0; e < kScanChunkPer; ++e) {
+        const int i = ck * kScanChunk + tid * kScanChunkPer + e;
+        sz[e] = 0;
+        wcs[e] = 0;
+        if (i < n) {
+            const int b = bits[(t0 + i) * H + h];
+            const int wc = width_code(b);
+            if (wc < 0) bad = true;
+            else {
+                wcs[e] = (uint32_t)wc;
+                sz[e] = (uint32_t)(b * c.D / 4);
+            }
+        }
+        mine += sz[e];
+    }
+    uint32_t incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    if (lane == 31) wsum[wid] = incl;
+    __syncthreads();
+    uint32_t wpre = 0, agg = 0;
+#pragma unroll
+    for (int q = 0; q < kScanChunkThreads / 32; ++q) {
+        const uint32_t t = wsum[q];
+        if (q < wid) wpre += t;
+        agg += t;
+    }
+    if (tid == 0) {
+        uint64_t *fl = flags + gsh * n_chunks;
+        const uint32_t g30 = gen & 0x3FFFFFFFu;
+        const uint64_t tag = (uint64_t)g30 << 34;
+        uint32_t excl = off0;
+        if (ck == 0) {
+            st_release_u64(&fl[0], tag | (2ull << 32) | (uint64_t)(off0 + agg));
+        } else {
+            st_release_u64(&fl[ck], tag | (1ull << 32) | (uint64_t)agg);
+            excl = 0;
+            int j = ck - 1;
+            uint64_t t_begin = 0;
+            for (uint32_t it = 0;; ++it) {
+                const uint64_t wv = ld_acquire_u64(&fl[j]);
+                const uint32_t state = (uint32_t)(wv >> 32) & 3u;
+                if ((uint32_t)(wv >> 34) == g30 && state != 0u) {
+                    excl += (uint32_t)wv;
+                    if (state == 2u || j == 0) break;   // chunk 0 always publishes its prefix
+                    --j;
+                    continue;
+                }
+                if ((it & 63u) == 0) {                  // bounded: about two seconds
+                    const uint64_t tn = global_ns();
+                    if (t_begin == 0) t_begin = tn;
+                    else if (tn - t_begin > kWaitLimitNs) {
+                        set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+                        break;
+                    }
+                }
+            }
+            st_release_u64(&fl[ck], tag | (2ull << 32) | (uint64_t)(excl + agg));
+        }
+        excl_sh = excl;
+    }
+    __syncthreads();
+    const int64_t slot0 = slot_of(c, s, h, L0);
+    uint32_t o = excl_sh + wpre + incl - mine;
+#pragma unroll
+    for (int e = 0; e < kScanChunkPer; ++e) {
+        const int i = ck * kScanChunk + tid * kScanChunkPer + e;
+        if (i < n) c.meta[slot0 + i] = o | wcs[e];
+        o += sz[e];
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) {
+        c.bad[s] = gen;                          // same value from every writer
+        set_status(c.status, KVQ_ERR_BITS);
+    }
+    if (tid == 0 && (nck == 0 || ck == nck - 1)) {   // the last chunk (or an empty write)
+        const uint32_t end = excl_sh + agg;
+        if (map_pages(c, s, h, end)) {           // paged caches: pages for the new bytes
+            c.wstart[sh] = L0;
+            c.wend[sh] = end;
+        } else {
+            set_status(c.status, KVQ_ERR_CAPACITY);
+            c.wstart[sh] = -1;
+        }
+    }
+}
+
 // Staging of the quantize kernel: each CTA copies the fp16 K and V rows of T tokens x HG
 // heads (at most kWqHalves values per tensor) into shared memory with two bulk copies.
 #ifndef KVQ_WQ_THREADS
@@ -323,7 +473,12 @@ cudaError_t launch_write(kvq_cache *cache, const __half *k, const __half *v,
             const int64_t blocks = (groups + 7) / 8;
             le = launch_pdl(write_scan_kernel<32>, dim3((unsigned)blocks), dim3(256), 0, st, c, bits, cu, n_tok, gen);
         } else {
-            le = launch_pdl(write_scan_kernel<1024>, dim3((unsigned)groups), dim3(1024), 0, st, c, bits, cu, n_tok, gen);
+            // chunks of 1024 tokens per (sequence, head); no sequence has more chunks than
+            // the cache's largest capacity allows (a longer write fails its capacity check)
+            const int n_chunks = (int)std::max<int64_t>(1, std::min<int64_t>((n_tok + kScanChunk - 1) / kScanChunk,
+                                                                                 cache->scan_chunks));
+            le = launch_pdl(write_scan_chunk_kernel, dim3((unsigned)(groups * n_chunks)), dim3(kScanChunkThreads), 0, st,
+                            c, bits, cu, n_tok, gen, cache->scan_flags, n_chunks);
         }
         if (le != cudaSuccess) return le;
     }
