@@ -95,3 +95,41 @@ def test_decode_step_rollback_redecodes_exactly():
         for h in range(3):
             ref = oracle_decode(wl, k.cpu(), v.cpu(), bits.cpu(), q.cpu(), modes.cpu(), 100, s, h)
             assert_close_attn(first[s, h].cpu().numpy(), ref, f"s={s} h={h}")
+
+
+def test_decode_entry_points_interleaved():
+    # the three decode entry points alternate on one cache (the work-list counters of the
+    # cache and of the allocation-free scratch flip between two words per call): every call
+    # over the same cache state gives the same outputs
+    wl = synth.scaled(W["decode_1p3b"], seqlens=(900, 33, 2100, 1), heads=2)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    B = wl.batch
+    cu = synth.cu_seqlens(wl.seqlens).tolist()
+    cache = kvq.KVQCache(B, 2, 128, list(wl.seqlens))
+    pre = [L - 1 for L in wl.seqlens]
+    idx = torch.tensor(sum((_rows(cu, s, 0, pre[s]) for s in range(B)), []), device="cuda")
+    kvq.kvq_write(k[idx].contiguous(), v[idx].contiguous(), bits[idx].contiguous(),
+                  synth.cu_seqlens(pre, "cuda"), cache)
+    rows = torch.tensor([cu[s] + pre[s] for s in range(B)], device="cuda")
+    q, modes = synth.decode_queries(wl, "cuda")
+    one = synth.cu_seqlens([1] * B, "cuda")
+    pos = torch.tensor(pre, dtype=torch.int32, device="cuda")
+    kr, vr, br = k[rows].contiguous(), v[rows].contiguous(), bits[rows].contiguous()
+    first = kvq.decode_step(q, kr, vr, br, one, cache, modes, 64)
+    outs = []
+    for i in range(7):
+        which = i % 3
+        if which == 0:
+            outs.append(kvq.routed_attn_decode(q, cache, modes, 64))
+        elif which == 1:
+            outs.append(kvq.routed_attn_decode_noalloc(q, cache, modes, 64).clone())
+        else:
+            outs.append(kvq.decode_step(q, kr, vr, br, one, cache, modes, 64, positions=pos))
+        torch.cuda.synchronize()
+        cache.check()
+    for i, o in enumerate(outs):
+        assert torch.equal(o, first), f"call {i}"
+    for s in range(B):
+        for h in range(2):
+            ref = oracle_decode(wl, k.cpu(), v.cpu(), bits.cpu(), q.cpu(), modes.cpu(), 64, s, h)
+            assert_close_attn(first[s, h].cpu().numpy(), ref, f"s={s} h={h}")

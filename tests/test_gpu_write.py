@@ -180,3 +180,49 @@ def test_short_append_errors():
     assert e.value.code in (kvq.KVQ_ERR_BITS, kvq.KVQ_ERR_CAPACITY)
     assert cache.lengths().tolist() == [3, 2, 2, 3]
     check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), [(s, h) for s in (0, 3) for h in range(4)])
+
+
+def test_long_writes_in_several_calls_multi_chunk():
+    # each call is long (more than 64 tokens per sequence on average), so the record offsets
+    # are scanned in 1024-token chunks; the look-back of later calls must not read the flags
+    # that earlier calls left behind
+    wl = synth.scaled(W["ragged_prefill"], seqlens=(3000, 2600, 5), heads=3)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cache = kvq.KVQCache(wl.batch, wl.heads, wl.head_dim, list(wl.seqlens))
+    cu = synth.cu_seqlens(wl.seqlens).tolist()
+    pos = [0] * wl.batch
+    for cut in (1100, 2300, None):
+        counts = [(L if cut is None else min(cut, L)) - p for L, p in zip(wl.seqlens, pos)]
+        assert sum(counts) > 64 * wl.batch
+        kvq.kvq_write(*_append_rows(k, v, bits, cu, pos, counts), cache)
+        pos = [p + c for p, c in zip(pos, counts)]
+        cache.check()
+    assert cache.lengths().tolist() == list(wl.seqlens)
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(),
+                  [(s, h) for s in range(wl.batch) for h in range(wl.heads)])
+
+
+def test_long_write_errors_in_later_chunks():
+    # a long multi-chunk call where sequence 1 overflows its capacity and sequence 2 has a
+    # bad width in its third chunk: both are refused for every head, sequence 0 is written
+    wl = synth.scaled(W["ragged_prefill"], seqlens=(2500, 1500, 3100), heads=3)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    bits_bad = bits.clone()
+    cu = synth.cu_seqlens(wl.seqlens).tolist()
+    bits_bad[cu[2] + 2600, 1] = 5
+    cache = kvq.KVQCache(wl.batch, wl.heads, wl.head_dim, [2500, 1400, 3100])
+    kvq.kvq_write(k, v, bits_bad, synth.cu_seqlens(wl.seqlens, "cuda"), cache)
+    with pytest.raises(kvq.KVQError) as e:
+        cache.check()
+    assert e.value.code in (kvq.KVQ_ERR_BITS, kvq.KVQ_ERR_CAPACITY)
+    cache.check()  # cleared
+    assert cache.lengths().tolist() == [2500, 0, 0]
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), [(0, h) for h in range(wl.heads)])
+    # the refused sequences can be written afterwards (sequence 1 within its capacity)
+    kk, vv, bb, cus = _append_rows(k, v, bits, cu, [0, 0, 0], [0, 1400, 3100])
+    kvq.kvq_write(kk, vv, bb, cus, cache)
+    cache.check()
+    assert cache.lengths().tolist() == [2500, 1400, 3100]
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), [(2, h) for h in range(wl.heads)])
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), [(1, h) for h in range(wl.heads)],
+                  tok_ranges=(0, 1400))
