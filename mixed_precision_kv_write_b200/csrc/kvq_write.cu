@@ -167,7 +167,11 @@ write_scan_chunk_kernel(CacheView c, const uint8_t *__restrict__ bits, const int
     const int H = c.H;
     if (gsh >= (int64_t)c.B * H) return;
     const int s = (int)(gsh / H), h = (int)(gsh % H), sh = s * H + h;
+    // every load that does not depend on the token range goes out with cu
     const int64_t t0 = cu[s], t1 = cu[s + 1];
+    const int L0 = c.len[sh];
+    const int cap = c.cap[s];
+    const uint32_t off0 = c.end[sh];
     if (t0 < 0 || t1 < t0 || t1 > n_tok || (s == 0 && t0 != 0)) {
         if (ck == 0 && tid == 0) {
             set_status(c.status, KVQ_ERR_DEVICE_CHECK);
@@ -177,15 +181,13 @@ write_scan_chunk_kernel(CacheView c, const uint8_t *__restrict__ bits, const int
     }
     const int n = (int)(t1 - t0);
     if (ck > 0 && ck * kScanChunk >= n) return;  // past this sequence's tokens
-    const int L0 = c.len[sh];
-    if ((int64_t)L0 + n > c.cap[s]) {
+    if ((int64_t)L0 + n > cap) {
         if (ck == 0 && tid == 0) {
             set_status(c.status, KVQ_ERR_CAPACITY);
             c.wstart[sh] = -1;
         }
         return;
     }
-    const uint32_t off0 = c.end[sh];
     const int nck = (n + kScanChunk - 1) / kScanChunk;
     // this chunk's tokens: kScanChunkPer consecutive ones per thread
     uint32_t sz[kScanChunkPer], wcs[kScanChunkPer], mine = 0;
@@ -221,39 +223,53 @@ write_scan_chunk_kernel(CacheView c, const uint8_t *__restrict__ bits, const int
         if (q < wid) wpre += t;
         agg += t;
     }
-    if (tid == 0) {
+    if (wid == 0) {
+        // publish this chunk's total (chunk 0: its prefix), then warp 0 reads the words of
+        // up to 32 predecessors at once: the bytes before this chunk are the sum of the
+        // totals back to the nearest chunk whose prefix is known
         uint64_t *fl = flags + gsh * n_chunks;
         const uint32_t g30 = gen & 0x3FFFFFFFu;
         const uint64_t tag = (uint64_t)g30 << 34;
         uint32_t excl = off0;
         if (ck == 0) {
-            st_release_u64(&fl[0], tag | (2ull << 32) | (uint64_t)(off0 + agg));
+            if (lane == 0) st_release_u64(&fl[0], tag | (2ull << 32) | (uint64_t)(off0 + agg));
         } else {
-            st_release_u64(&fl[ck], tag | (1ull << 32) | (uint64_t)agg);
+            if (lane == 0) st_release_u64(&fl[ck], tag | (1ull << 32) | (uint64_t)agg);
             excl = 0;
-            int j = ck - 1;
+            int j0 = ck - 1;                      // the window's nearest predecessor
             uint64_t t_begin = 0;
             for (uint32_t it = 0;; ++it) {
-                const uint64_t wv = ld_acquire_u64(&fl[j]);
-                const uint32_t state = (uint32_t)(wv >> 32) & 3u;
-                if ((uint32_t)(wv >> 34) == g30 && state != 0u) {
-                    excl += (uint32_t)wv;
-                    if (state == 2u || j == 0) break;   // chunk 0 always publishes its prefix
-                    --j;
+                const int j = j0 - lane;
+                uint64_t wv = 0;
+                if (j >= 0) wv = ld_acquire_u64(&fl[j]);
+                const uint32_t state = ((uint32_t)(wv >> 34) == g30) ? (uint32_t)(wv >> 32) & 3u : 0u;
+                const uint32_t have = __ballot_sync(0xffffffffu, j >= 0 && state != 0u);
+                const uint32_t done = __ballot_sync(0xffffffffu, j >= 0 && state == 2u);
+                // chunk 0 always publishes its prefix, so a full window of published words
+                // either holds a known prefix or lies entirely past one
+                const int p = done ? __ffs(done) - 1 : 31;        // the last lane summed
+                const uint32_t need = (p == 31) ? 0xFFFFFFFFu : ((2u << p) - 1u);
+                if ((have & need) == need) {
+                    uint32_t v = (lane <= p) ? (uint32_t)wv : 0u;
+#pragma unroll
+                    for (int d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+                    excl += v;
+                    if (done) break;
+                    j0 -= 32;
                     continue;
                 }
-                if ((it & 63u) == 0) {                  // bounded: about two seconds
-                    const uint64_t tn = global_ns();
+                if ((it & 63u) == 0) {            // bounded: about two seconds (warp-uniform)
+                    const uint64_t tn = __shfl_sync(0xffffffffu, global_ns(), 0);
                     if (t_begin == 0) t_begin = tn;
                     else if (tn - t_begin > kWaitLimitNs) {
-                        set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+                        if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
                         break;
                     }
                 }
             }
-            st_release_u64(&fl[ck], tag | (2ull << 32) | (uint64_t)(excl + agg));
+            if (lane == 0) st_release_u64(&fl[ck], tag | (2ull << 32) | (uint64_t)(excl + agg));
         }
-        excl_sh = excl;
+        if (lane == 0) excl_sh = excl;
     }
     __syncthreads();
     const int64_t slot0 = slot_of(c, s, h, L0);
@@ -301,19 +317,216 @@ struct WqPair {                          // one (token, head) of the CTA
     int32_t pad;
 };
 
+#ifndef KVQ_WQ_MIXED_SUB
+#define KVQ_WQ_MIXED_SUB 1
+#endif
+
+// fl(x - z) for an fp16 x and an fp32 z: one instruction with the fp16 operand widened
+// exactly (sm_100 mixed-precision subtract), or the explicit conversion then the subtract.
+__device__ __forceinline__ float sub_h(uint32_t hbits, float z)
+{
+#if KVQ_WQ_MIXED_SUB
+    float d;
+    asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"((unsigned short)hbits), "f"(z));
+    return d;
+#else
+    return __fsub_rn(__half2float(__ushort_as_half((unsigned short)hbits)), z);
+#endif
+}
+
+// Codes of one chunk of 8 fp16 values (BITS = 2, 4, 8), packed LSB-first into w (BITS
+// bytes), with the arithmetic of quant_store: u = fl(x - z), Markstein's correctly rounded
+// quotient fl(u / s), rint by the 1.5 * 2^23 addition; `probe` sums the quotients.
+template <int BITS>
+__device__ __forceinline__ void chunk_codes(const uint4 &raw, float z, float2 y2, float2 ns2, float2 &probe,
+                                            uint32_t (&w)[2])
+{
+    const uint32_t hw[4] = {raw.x, raw.y, raw.z, raw.w};
+    const float2 mg2 = make_float2(kRoundMagic, kRoundMagic);
+    w[0] = w[1] = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {                     // values 2e, 2e + 1
+        const float2 u = make_float2(sub_h(hw[e] & 0xFFFFu, z), sub_h(hw[e] >> 16, z));
+        const float2 q0 = __fmul2_rn(u, y2);
+        const float2 r = __ffma2_rn(ns2, q0, u);      // u - s * q0, exact
+        const float2 q = __ffma2_rn(r, y2, q0);       // RN(u / s)
+        const float2 t = __fadd2_rn(q, mg2);
+        probe = __fadd2_rn(probe, q);
+        w[(2 * e * BITS) >> 5] += __float_as_uint(t.x) << ((2 * e * BITS) & 31);
+        w[((2 * e + 1) * BITS) >> 5] += __float_as_uint(t.y) << (((2 * e + 1) * BITS) & 31);
+    }
+    constexpr int kWordBits = BITS * 8 < 32 ? BITS * 8 : 32;
+    uint32_t magic = 0u;
+#pragma unroll
+    for (int sh = 0; sh < kWordBits; sh += BITS) magic += kRoundMagicBits << sh;
+    w[0] -= magic;
+    if (BITS == 8) w[1] -= magic;
+}
+
+// The plain formula for one chunk (taken only when a quotient was NaN: NaN or infinite
+// inputs), which gives code 0 for a NaN quotient.
+template <int BITS>
+__device__ __forceinline__ void chunk_codes_plain(const uint4 &raw, float z, float sc, uint32_t (&w)[2])
+{
+    const uint32_t hw[4] = {raw.x, raw.y, raw.z, raw.w};
+    const float top = (float)((1u << BITS) - 1u);
+    w[0] = w[1] = 0u;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float x = __half2float(__ushort_as_half((unsigned short)((e & 1) ? hw[e >> 1] >> 16 : hw[e >> 1] & 0xFFFFu)));
+        const float cv = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x, z), sc)), 0.0f), top);
+        w[(e * BITS) >> 5] |= __float2uint_rz(cv) << ((e * BITS) & 31);
+    }
+}
+
+// A record part's bytes [0, n): rel < split at p0 + rel, else at p1 + rel (a paged part
+// crosses at most one page boundary, never inside a 16-byte group; contiguous parts never
+// split).
+struct PartDst {
+    uint8_t *p0, *p1;
+    uint32_t split;
+    __device__ __forceinline__ uint8_t *at(uint32_t rel) const { return (rel < split ? p0 : p1) + rel; }
+};
+
+__device__ __forceinline__ PartDst part_dst(const RecLoc &L, uint32_t n)
+{
+    PartDst d;
+    d.p0 = L.at(0);
+    d.p1 = d.p0;
+    d.split = 0xFFFFFFFFu;
+    if (L.pt) {
+        const uint32_t page = 1u << L.shift;
+        const uint32_t room = page - (L.off & (page - 1u));
+        if (room < n) {
+            d.split = room;
+            d.p1 = L.at(room) - room;
+        }
+    }
+    return d;
+}
+
+__device__ __forceinline__ void swap_if(bool c, uint32_t &a, uint32_t &b)
+{
+    const uint32_t t = c ? b : a;
+    b = c ? a : b;
+    a = t;
+}
+
+// One lane writes the codes of one vector of D fp16 values held in shared memory, a
+// 16-byte group (16/BITS chunks of 8 values) per store. With x = lane mod 8, step j reads
+// chunk j ^ x: the eight lanes of a shared-memory phase read eight different bank groups
+// (every vector starts on a 128-byte boundary), and the G steps k*G .. k*G + G - 1 cover the
+// chunks of group k ^ (x / G), chunk slot i ^ (x mod G) filled at step k*G + i; the slots
+// are put in place by conditional swaps before the store. PLAIN selects the plain formula
+// (taken only when a quotient was NaN: NaN or infinite inputs). Returns the sum of the
+// quotients.
+template <int D, int BITS, bool PLAIN>
+__device__ __forceinline__ float lane_codes(const uint4 *src, float z, float sc, const PartDst &dst, int x)
+{
+    constexpr int NCH = D / 8, G = 16 / BITS, NG = NCH / G;
+    const float y = __frcp_rn(sc);
+    const float2 y2 = make_float2(y, y), ns2 = make_float2(-sc, -sc);
+    float2 probe = make_float2(0.0f, 0.0f);
+    const int m = x & (G - 1);
+#pragma unroll 1
+    for (int k = 0; k < NG; ++k) {
+        uint32_t o[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+            uint32_t w[2];
+            const uint4 raw = src[(k * G + i) ^ x];
+            if (PLAIN) chunk_codes_plain<BITS>(raw, z, sc, w);
+            else chunk_codes<BITS>(raw, z, y2, ns2, probe, w);
+            if (BITS == 8) {
+                o[2 * i] = w[0];
+                o[2 * i + 1] = w[1];
+            } else if (BITS == 4) {
+                o[i] = w[0];
+            } else {
+                o[i >> 1] |= (w[0] & 0xFFFFu) << (16 * (i & 1));
+            }
+        }
+        if (BITS == 8) {
+            swap_if(m & 1, o[0], o[2]);
+            swap_if(m & 1, o[1], o[3]);
+        } else if (BITS == 4) {
+            swap_if(m & 1, o[0], o[1]);
+            swap_if(m & 1, o[2], o[3]);
+            swap_if(m & 2, o[0], o[2]);
+            swap_if(m & 2, o[1], o[3]);
+        } else {
+            const uint32_t sel = (m & 1) ? 0x1032u : 0x3210u;     // halves swapped or kept
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = __byte_perm(o[e], 0u, sel);
+            swap_if(m & 2, o[0], o[1]);
+            swap_if(m & 2, o[2], o[3]);
+            swap_if(m & 4, o[0], o[2]);
+            swap_if(m & 4, o[1], o[3]);
+        }
+        *reinterpret_cast<uint4 *>(dst.at(16u * (uint32_t)(k ^ (x / G)))) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    return probe.x + probe.y;
+}
+
+template <int D, int BITS>
+__device__ __forceinline__ void lane_quant(const uint4 *src, float z, float sc, const PartDst &dst, int x)
+{
+    const float nan_probe = lane_codes<D, BITS, false>(src, z, sc, dst, x);
+    if (nan_probe != nan_probe) lane_codes<D, BITS, true>(src, z, sc, dst, x);   // same lane, same bytes
+}
+
+// One lane quantizes one vector: min/max, then the record part (the raw fp16 bits for
+// b = 16) and the (s, z) side entry.
+template <int D>
+__device__ __forceinline__ void lane_vector(const CacheView &c, const uint4 *src, int b, const RecLoc &L,
+                                            int64_t slot, int part, int x)
+{
+    constexpr int NCH = D / 8;
+    const PartDst dst = part_dst(L, (uint32_t)(b * D / 8));
+    float sc = 1.0f, z = 0.0f;
+    if (b == 16) {
+#pragma unroll 4
+        for (int j = 0; j < NCH; ++j) *reinterpret_cast<uint4 *>(dst.at(16u * (uint32_t)(j ^ x))) = src[j ^ x];
+    } else {
+        // min and max in fp16 (exact); -0 and +0 are one value, stored as +0 below
+        __half2 lo2 = *reinterpret_cast<const __half2 *>(&src[x].x), hi2 = lo2;
+#pragma unroll 4
+        for (int j = 0; j < NCH; ++j) {
+            const uint4 r = src[j ^ x];
+            const uint32_t hw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                lo2 = __hmin2(lo2, *reinterpret_cast<const __half2 *>(&hw[e]));
+                hi2 = __hmax2(hi2, *reinterpret_cast<const __half2 *>(&hw[e]));
+            }
+        }
+        const float mn = __half2float(__hmin(__low2half(lo2), __high2half(lo2)));
+        const float mx = __half2float(__hmax(__low2half(hi2), __high2half(hi2)));
+        const float top = (float)((1u << b) - 1u);
+        sc = __fadd_rn(__fdiv_rn(__fsub_rn(mx, mn), top), 0.0f);
+        z = __fadd_rn(mn, 0.0f);
+        if (sc != 0.0f) {
+            if (b == 8) lane_quant<D, 8>(src, z, sc, dst, x);
+            else if (b == 4) lane_quant<D, 4>(src, z, sc, dst, x);
+            else lane_quant<D, 2>(src, z, sc, dst, x);
+        } else {                                   // a constant vector: every code is 0
+            for (uint32_t o = 0; o < (uint32_t)(b * D / 8); o += 16u)
+                *reinterpret_cast<uint4 *>(dst.at(o)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    reinterpret_cast<float2 *>(&c.side[slot])[part] = make_float2(sc, z);
+}
+
 // One CTA per tile of T tokens x HG heads. Warp 0 starts two bulk copies (the tile's K and
 // V rows are contiguous when HG = H, else one copy per token and tensor); meanwhile every
 // thread resolves the destination of one (token, head): its sequence (binary search of
 // cu_seqlens), the call's verdict, the write start, and the record offset the scan kernel
-// assigned. Then each vector of D values is quantized by D/32 lanes from shared memory.
+// assigned. Then each vector of D values is quantized by one lane from shared memory.
 template <int D>
 __global__ void __launch_bounds__(kWqThreads)
 write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__restrict__ v,
                    const int32_t *__restrict__ cu, int64_t n_tok, uint32_t gen, int T, int HG)
 {
-    constexpr int NC = 4;                    // chunks of 8 values per lane
-    constexpr int VL = D / (8 * NC);         // lanes per vector
-    constexpr int VPW = 32 / VL;             // vectors per warp pass
     extern __shared__ __align__(128) uint8_t wq_smem[];
     __shared__ uint64_t bar;
     __shared__ WqPair pairs[kWqMaxPairs];
@@ -392,16 +605,16 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
         pairs[i] = pr;
     }
     __syncthreads();
-    // Sort the written pairs by width, so the lanes of a warp pass mostly share one code path.
+    // Sort the written pairs by width, so the lanes of a warp mostly share one code path.
     if (warp == 0) {
         const int n_pairs = Tc * HGc;
         int base = 0;
         for (int cls = 0; cls < 4; ++cls) {
             for (int i0 = 0; i0 < n_pairs; i0 += 32) {
-                const int i = i0 + lane;
-                const bool in = i < n_pairs && pairs[i].s >= 0 && (int)(pairs[i].meta & 3u) == cls;
+                const int ii = i0 + lane;
+                const bool in = ii < n_pairs && pairs[ii].s >= 0 && (int)(pairs[ii].meta & 3u) == cls;
                 const uint32_t m = __ballot_sync(0xffffffffu, in);
-                if (in) order[base + __popc(m & ((1u << lane) - 1u))] = (uint8_t)i;
+                if (in) order[base + __popc(m & ((1u << lane) - 1u))] = (uint8_t)ii;
                 base += __popc(m);
             }
         }
@@ -410,26 +623,16 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
     __syncthreads();
     if (!mbar_wait(&bar, 0, c.status)) return;
 
-    const int n_vec = 2 * n_written;         // vector vi: pair order[vi / 2], K (even) or V (odd)
-    const int li = lane % VL;
-    for (int vb = warp * VPW; vb < n_vec; vb += (kWqThreads / 32) * VPW) {
-        const int vi = vb + lane / VL;
-        const bool in_range = vi < n_vec;
-        const int pi = in_range ? order[vi >> 1] : 0, part = vi & 1;
-        uint4 raw[NC];
-#pragma unroll
-        for (int j = 0; j < NC; ++j) raw[j] = make_uint4(0u, 0u, 0u, 0u);
-        if (in_range) {
-            const uint4 *src = reinterpret_cast<const uint4 *>((part ? sv : sk) + pi * D);
-#pragma unroll
-            for (int j = 0; j < NC; ++j) raw[j] = src[j * VL + li];
-        }
-        const __half2 mm = vec_minmax<NC, VL>(raw);
-        if (!in_range) continue;
+    // one lane per vector: vector vi is pair order[vi / 2], K (even) or V (odd); the lanes of
+    // a warp take consecutive vectors of the width-sorted list
+    const int n_vec = 2 * n_written;
+    for (int vi = tid; vi < n_vec; vi += kWqThreads) {
+        const int pi = order[vi >> 1], part = vi & 1;
         const WqPair pr = pairs[pi];
         const int b = 2 << (pr.meta & 3u);
-        vec_store<NC, VL>(c, raw, mm, b, rec_loc(c, pr.s, pr.h, (pr.meta & ~15u) + part * (b * D / 8)), pr.slot,
-                          part, li);
+        const uint4 *src = reinterpret_cast<const uint4 *>((part ? sv : sk) + pi * D);
+        lane_vector<D>(c, src, b, rec_loc(c, pr.s, pr.h, (pr.meta & ~15u) + part * (b * D / 8)), pr.slot, part,
+                       lane & 7);
     }
 }
 
