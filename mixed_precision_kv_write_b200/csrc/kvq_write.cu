@@ -132,24 +132,27 @@ write_scan_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *
 
 // Long calls: the same results as write_scan_kernel, with each (sequence, head) split into
 // chunks of 1024 tokens, one CTA of 256 threads per chunk, so that long sequences do not
-// leave most SMs idle. A CTA scans its chunk's record sizes, publishes the chunk's total
-// at once, and finds the bytes before its chunk by looking back over the totals (or the
-// running prefixes, once known) its predecessors published in a per-(sequence, head)
-// array of 64-bit words (call generation << 34 | state << 32 | bytes; state 1: the
-// chunk's total, 2: the prefix through the chunk). The look-back only waits on CTAs of
-// lower index, which start first; its wait is bounded. The last chunk of a (sequence,
-// head) records the write start and the new stream end.
+// leave most SMs idle. A CTA scans its chunk's record sizes and sums those of the up to 16
+// chunks before it straight from the widths (their loads go out with its own), so most
+// CTAs wait on no other; a chunk further out adds the running prefix that the chunk 17
+// places back published in a per-(sequence, head) array of 64-bit words (call generation
+// << 34 | 2 << 32 | bytes through the chunk). That wait is on a CTA of lower index, which
+// starts first, and is bounded. The last chunk of a (sequence, head) records the write
+// start and the new stream end.
 constexpr int kScanChunkThreads = 256, kScanChunkPer = 4, kScanChunk = kScanChunkThreads * kScanChunkPer;
+constexpr int kScanDirect = 16;                  // chunks summed directly before the look-back
 
-__device__ __forceinline__ void st_release_u64(uint64_t *p, uint64_t v)
+// The look-back words carry their whole message (no other data is published with them),
+// so they are stored and polled with relaxed gpu-scope accesses: coherent in L2, no fence.
+__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v)
 {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p)
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p)
 {
     uint64_t v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(kScanChunkThreads)
 write_scan_chunk_kernel(CacheView c, const uint8_t *__restrict__ bits, const int32_t *__restrict__ cu,
                         int64_t n_tok, uint32_t gen, uint64_t *__restrict__ flags, int n_chunks)
 {
-    __shared__ uint32_t wsum[kScanChunkThreads / 32];
+    __shared__ uint32_t wsum[kScanChunkThreads / 32], wpre_sh[kScanChunkThreads / 32];
     __shared__ uint32_t excl_sh;
     pdl_wait();
     pdl_trigger();
@@ -208,68 +211,65 @@ write_scan_chunk_kernel(CacheView c, const uint8_t *__restrict__ bits, const int
         }
         mine += sz[e];
     }
+    // the bytes of the up to kScanDirect chunks before this one, summed from their widths
+    // directly (a bad width counts 0 bytes, as in its own chunk)
+    const int cd = max(0, ck - kScanDirect);
+    uint32_t pre = 0;
+    for (int cc = cd; cc < ck; ++cc) {
+#pragma unroll
+        for (int e = 0; e < kScanChunkPer; ++e) {
+            const int b = bits[(t0 + cc * kScanChunk + tid * kScanChunkPer + e) * H + h];
+            pre += width_code(b) >= 0 ? (uint32_t)(b * c.D / 4) : 0u;
+        }
+    }
     uint32_t incl = mine;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
         if (lane >= d) incl += y;
     }
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, d);
     if (lane == 31) wsum[wid] = incl;
+    if (lane == 0) wpre_sh[wid] = pre;
     __syncthreads();
-    uint32_t wpre = 0, agg = 0;
+    uint32_t wpre = 0, agg = 0, pre_all = 0;
 #pragma unroll
     for (int q = 0; q < kScanChunkThreads / 32; ++q) {
         const uint32_t t = wsum[q];
         if (q < wid) wpre += t;
         agg += t;
+        pre_all += wpre_sh[q];
     }
-    if (wid == 0) {
-        // publish this chunk's total (chunk 0: its prefix), then warp 0 reads the words of
-        // up to 32 predecessors at once: the bytes before this chunk are the sum of the
-        // totals back to the nearest chunk whose prefix is known
+    if (tid == 0) {
+        // chunks more than kScanDirect back: the running prefix that chunk ck - kScanDirect - 1
+        // publishes (gen << 34 | 2 << 32 | bytes through that chunk); every chunk publishes
+        // its own
         uint64_t *fl = flags + gsh * n_chunks;
         const uint32_t g30 = gen & 0x3FFFFFFFu;
         const uint64_t tag = (uint64_t)g30 << 34;
-        uint32_t excl = off0;
-        if (ck == 0) {
-            if (lane == 0) st_release_u64(&fl[0], tag | (2ull << 32) | (uint64_t)(off0 + agg));
-        } else {
-            if (lane == 0) st_release_u64(&fl[ck], tag | (1ull << 32) | (uint64_t)agg);
-            excl = 0;
-            int j0 = ck - 1;                      // the window's nearest predecessor
+        uint32_t excl = off0 + pre_all;
+        if (ck > kScanDirect) {
+            const int j = ck - kScanDirect - 1;
             uint64_t t_begin = 0;
             for (uint32_t it = 0;; ++it) {
-                const int j = j0 - lane;
-                uint64_t wv = 0;
-                if (j >= 0) wv = ld_acquire_u64(&fl[j]);
-                const uint32_t state = ((uint32_t)(wv >> 34) == g30) ? (uint32_t)(wv >> 32) & 3u : 0u;
-                const uint32_t have = __ballot_sync(0xffffffffu, j >= 0 && state != 0u);
-                const uint32_t done = __ballot_sync(0xffffffffu, j >= 0 && state == 2u);
-                // chunk 0 always publishes its prefix, so a full window of published words
-                // either holds a known prefix or lies entirely past one
-                const int p = done ? __ffs(done) - 1 : 31;        // the last lane summed
-                const uint32_t need = (p == 31) ? 0xFFFFFFFFu : ((2u << p) - 1u);
-                if ((have & need) == need) {
-                    uint32_t v = (lane <= p) ? (uint32_t)wv : 0u;
-#pragma unroll
-                    for (int d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
-                    excl += v;
-                    if (done) break;
-                    j0 -= 32;
-                    continue;
+                const uint64_t wv = ld_relaxed_u64(&fl[j]);
+                if ((uint32_t)(wv >> 34) == g30 && ((uint32_t)(wv >> 32) & 3u) == 2u) {
+                    excl = (uint32_t)wv + pre_all;
+                    break;
                 }
-                if ((it & 63u) == 0) {            // bounded: about two seconds (warp-uniform)
-                    const uint64_t tn = __shfl_sync(0xffffffffu, global_ns(), 0);
+                if ((it & 63u) == 0) {            // bounded: about two seconds
+                    const uint64_t tn = global_ns();
                     if (t_begin == 0) t_begin = tn;
                     else if (tn - t_begin > kWaitLimitNs) {
-                        if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+                        set_status(c.status, KVQ_ERR_DEVICE_CHECK);
                         break;
                     }
                 }
             }
-            if (lane == 0) st_release_u64(&fl[ck], tag | (2ull << 32) | (uint64_t)(excl + agg));
         }
-        if (lane == 0) excl_sh = excl;
+        st_relaxed_u64(&fl[ck], tag | (2ull << 32) | (uint64_t)(excl + agg));
+        excl_sh = excl;
     }
     __syncthreads();
     const int64_t slot0 = slot_of(c, s, h, L0);

@@ -226,3 +226,14 @@ def test_long_write_errors_in_later_chunks():
     check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), [(2, h) for h in range(wl.heads)])
     check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), [(1, h) for h in range(wl.heads)],
                   tok_ranges=(0, 1400))
+
+
+def test_long_write_beyond_direct_chunks():
+    # a 20000-token sequence: 20 scan chunks of 1024 tokens, so the last three add the
+    # running prefix published 17 chunks back to the 16 chunks they sum directly
+    wl = synth.scaled(W["prefill_160m"], seqlens=(20000, 300), heads=2)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cache = build_cache(wl, k, v, bits)
+    cache.check()
+    assert cache.lengths().tolist() == list(wl.seqlens)
+    check_records(cache, wl, k.cpu(), v.cpu(), bits.cpu(), [(s, h) for s in range(2) for h in range(2)])
