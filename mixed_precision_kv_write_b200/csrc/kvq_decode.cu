@@ -87,7 +87,7 @@ constexpr int kMetaWords = kWin + 8;
 // A consumer warp can run at most kStages items ahead of the slowest one (the stages are
 // shared and every item has at least one), so kStages + 1 merge slots never collide.
 constexpr int kMergeRing = kStages + 1;
-constexpr int kNewItem = 1, kLastSub = 2;         // stage flags
+constexpr int kNewItem = 1, kLastSub = 2, kStop = 4;   // stage flags (kStop: no more items)
 constexpr uint32_t kReadEndFromMeta = 0xFFFFFFFFu;
 constexpr uint32_t kValid = 0x80000000u;
 constexpr float kLazy = 8.f;                      // running-max slack, log2 units
@@ -191,7 +191,10 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
     pdl_wait();
     pdl_trigger();
     // the previous call's kernels have completed: its count word becomes the next call's
-    if (blockIdx.x == 0 && threadIdx.x == 0) *wk.count_next = (unsigned long long)(gen + 1u) << 32;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *wk.count_next = (unsigned long long)(gen + 1u) << 32;
+        *wk.cursor = 0u;                 // the split-K CTAs claim this call's items from 0
+    }
     const int s = blockIdx.x;
     if (APPEND) append_seq<D>(c, ap.k, ap.v, ap.bits, ap.cu, ap.n_tok, ap.gen, ap.positions, s, bad_sh);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -565,14 +568,19 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         // slot i (ja = the window's first key rounded down to a multiple of 4); lane l holds
         // slots KPL*l .. KPL*l + KPL - 1 (16-byte shared loads). Windows after an item's first
         // end on 4-aligned keys, so a window's keys fit slots [d, d + nwin) with
-        // d + nwin <= kWin. The next item's descriptor is loaded one item ahead.
-        int f_it = blockIdx.x;
-        if (f_it >= n_items) return;
-        DecodeItem f_d = wk.items[f_it];
-        DecodeItem f_nx = f_d;
-        if (f_it + (int)gridDim.x < n_items) f_nx = wk.items[f_it + gridDim.x];
+        // d + nwin <= kWin. Items are claimed one at a time from the call's cursor when the
+        // filler reaches them (CTAs that finish early take more); after the last one the
+        // producer marks a stage kStop.
+        auto claim = [&]() {
+            int v = 0;
+            if (lane == 0) v = (int)atomicAdd(wk.cursor, 1u);
+            return __shfl_sync(0xffffffffu, v, 0);
+        };
+        int f_it = claim();
+        bool f_valid = f_it < n_items, aborted = false;
+        DecodeItem f_d = wk.items[0];
+        if (f_valid) f_d = wk.items[f_it];
         int f_j = f_d.j0;
-        bool f_valid = true, aborted = false;
         int filled = 0, consumed = 0, issued = 0;
         auto pick = [](const uint32_t (&a)[KPL], int i) {       // a[i], i warp-uniform
             uint32_t v = a[0];
@@ -604,11 +612,10 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 ++filled;
                 f_j += nwin;
                 if (f_j >= f_d.j1) {
-                    f_it += gridDim.x;
+                    f_it = claim();
                     if (f_it < n_items) {
-                        f_d = f_nx;
+                        f_d = wk.items[f_it];
                         f_j = f_d.j0;
-                        if (f_it + (int)gridDim.x < n_items) f_nx = wk.items[f_it + gridDim.x];
                     } else {
                         f_valid = false;
                     }
@@ -765,6 +772,18 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 s0 = s1;
             }
         }
+        if (!aborted) {
+            // no more items: the next stage carries only the stop mark
+            const int stage = issued % kStages;
+            if (mbar_wait(&sm.empty[stage], ((uint32_t)(issued / kStages) & 1u) ^ 1u, c.status)) {
+                if (lane == 0) {
+                    sm.st[stage].info[2] = kStop;
+                    mbar_arrive(&sm.full[stage]);
+                }
+            } else {
+                aborted = true;
+            }
+        }
         if (aborted) {
             // no copy may still be writing this CTA's shared memory when it exits: wait
             // (bounded) for the last copy issued into each stage and each offset window
@@ -795,7 +814,16 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     QRegs Q;
     float qsum_l = 0.f;
     int ring = 0;                         // this item's merge slot
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ring = (ring + 1) % kMergeRing) {
+    for (;; ring = (ring + 1) % kMergeRing) {
+        // the item's first stage, or the producer's stop mark
+        if (dead) break;
+        if (*reinterpret_cast<volatile int32_t *>(&sm.abort_flag) || !mbar_wait(&sm.full[stage], phase, c.status)) {
+            sm.abort_flag = 1;
+            break;
+        }
+        if (sm.st[stage].info[2] & kStop) break;
+        const int it = sm.st[stage].info[0];
+        bool waited = true;                   // the first stage's wait is done
         KeyState ks;
         ks.m = kMInit;
         ks.l = 0.f;
@@ -805,12 +833,13 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         int nq = 1, rank = warp, nws = kConsumerWarps, qmask = 1;
         bool last = false;
         while (!last && !dead) {
-            if (*reinterpret_cast<volatile int32_t *>(&sm.abort_flag) ||
-                !mbar_wait(&sm.full[stage], phase, c.status)) {
+            if (!waited && (*reinterpret_cast<volatile int32_t *>(&sm.abort_flag) ||
+                            !mbar_wait(&sm.full[stage], phase, c.status))) {
                 dead = true;
                 sm.abort_flag = 1;
                 break;
             }
+            waited = false;
             Stage<D> &sg = sm.st[stage];
             const int flags = sg.info[2];
             last = (flags & kLastSub) != 0;
@@ -1030,21 +1059,23 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const DecodeWork &wk, uint32
     return cudaGetLastError();
 }
 
-// wk.count points at the pair of count words; the call uses word gen & 1. `stale` is set when
-// a launch fails (a call whose planning kernel did not run leaves the next call's word
-// unprepared); the words are then cleared (tag 0, never used) before the next call.
+// wk.count points at the pair of count words and the item cursor (a third word); the call
+// uses count word gen & 1. `stale` is set when a launch fails (a call whose planning kernel
+// did not run leaves the next call's word unprepared); the words are then cleared (tag 0,
+// never used) before the next call.
 cudaError_t launch_any(const kvq_cache *cache, const DecodeWork &wk, uint32_t gen, const __half *q,
                        const uint8_t *modes, int w, float *out, cudaStream_t st, const AppendArgs *ap,
                        bool &stale)
 {
     if (stale) {
-        const cudaError_t e = cudaMemsetAsync(wk.count, 0, 2 * sizeof(unsigned long long), st);
+        const cudaError_t e = cudaMemsetAsync(wk.count, 0, 3 * sizeof(unsigned long long), st);
         if (e != cudaSuccess) return e;
         stale = false;
     }
     DecodeWork cw = wk;
     cw.count = wk.count + (gen & 1u);
     cw.count_next = wk.count + ((gen + 1u) & 1u);
+    cw.cursor = reinterpret_cast<uint32_t *>(wk.count + 2);
     cw.gen = gen;
     const cudaError_t e = (cache->D == 128) ? launch_decode_t<128>(cache, cw, gen, q, modes, w, out, st, ap)
                                             : launch_decode_t<64>(cache, cw, gen, q, modes, w, out, st, ap);
@@ -1135,8 +1166,8 @@ extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache,
     if (dev != cache->device)
         return report_error(KVQ_ERR_ARG, "routed_attn_decode_noalloc: the cache's device is not the current device");
 
-    // scratch layout: count | head_first | head_cnt | items | partials, each 256-byte aligned,
-    // sized for the cache's worst case (every head full at capacity)
+    // scratch layout: count words and cursor | head_first | head_cnt | items | partials, each
+    // 256-byte aligned, sized for the cache's worst case (every head full at capacity)
     const int BH = cache->B * cache->H;                     // (sequence, KV head) units
     const int64_t items = cache->work.max_items;
     const int qslots = cache->work.qslots;

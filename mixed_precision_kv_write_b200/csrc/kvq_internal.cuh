@@ -158,6 +158,7 @@ struct DecodeWork {
     // reports KVQ_ERR_DEVICE_CHECK.
     unsigned long long *count;
     unsigned long long *count_next;
+    uint32_t *cursor;    // items claimed so far by the split-K CTAs (reset by the planning kernel)
     uint32_t gen;        // the call's generation
     int32_t *head_first; // [B*H] first item of (sequence, KV head)
     int32_t *head_cnt;   // [B*H] its items (all subgroups)
