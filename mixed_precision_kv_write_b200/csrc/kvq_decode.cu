@@ -14,8 +14,10 @@
 //                         near-equal items of at most 1152 keys. Each CTA reserves its items
 //                         with one atomicAdd on the call's (generation, count) word.
 //   decode_splitk_kernel  three CTAs per SM, one producer and four consumer warps each. The
-//                         producer walks the CTA's items in stages of at most 128 keys and
-//                         24 KB of records: a ring of record-offset windows is bulk-copied
+//                         producer claims items one at a time from the call's cursor (a CTA
+//                         that finishes early takes more) and walks each in stages of at
+//                         most 128 keys and 24 KB of records: a ring of record-offset
+//                         windows is bulk-copied
 //                         ahead, each stage's keys are sorted by width into chunks of one
 //                         width (8 keys at head_dim 128), and the stage's contiguous record
 //                         bytes, side entries and (for a new item) queries are bulk-copied
