@@ -545,7 +545,6 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     const unsigned long long cw = *wk.count;
     const uint32_t tag = (uint32_t)(cw >> 32);
     const int n_items = (tag == wk.gen || tag == 0u) ? (int)min((int64_t)(uint32_t)cw, wk.max_items) : 0;
-    const int HQ = c.H * c.G;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -692,23 +691,33 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 }
                 Stage<D> &sg = sm.st[stage];
                 if (lane == 0) {
-                    // the item's subgroup of queries: rows (s, hk * G + g0 ..) of q, contiguous
+                    // the item's subgroup of queries: rows sh * G + g0 .. of q (query head
+                    // hk * G + g of sequence s is row (s * H + hk) * G + g), contiguous
                     const int g0 = qinfo & 0xFF;
                     const int nq = min(kDecodeMaxQ, c.G - g0);
                     const uint32_t q_bytes = new_item ? (uint32_t)(2 * D * nq) : 0u;
-                    const int s_of = sh / c.H, hk = sh % c.H;
                     mbar_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
                     bulk_g2s(sg.side, c.side + sbase + ja + s0, 16u * n, &sm.full[stage]);
                     if (rec_bytes) {
-                        const RecLoc L = rec_loc(c, s_of, hk, 0);
-                        // a paged stream: one copy per page the stage's bytes touch
-                        const uint32_t n0 = L.pt ? min(rec_bytes, (((off0 >> c.page_shift) + 1u) << c.page_shift) - off0)
-                                                 : rec_bytes;
-                        bulk_g2s(sg.rec, L.at(off0), n0, &sm.full[stage]);
-                        if (rec_bytes > n0) bulk_g2s(sg.rec + n0, L.at(off0 + n0), rec_bytes - n0, &sm.full[stage]);
+                        if (!c.ptab) {
+                            // contiguous: the stream starts at its first slot * 4 * D bytes
+                            bulk_g2s(sg.rec, c.rec + sbase * (4 * D) + off0, rec_bytes, &sm.full[stage]);
+                        } else {
+                            // a paged stream: one copy per page the stage's bytes touch
+                            const uint32_t *pt = c.ptab + (size_t)sh * c.max_lpages;
+                            const uint32_t pm = (1u << c.page_shift) - 1u;
+                            const uint32_t n0 = min(rec_bytes, (pm + 1u) - (off0 & pm));
+                            bulk_g2s(sg.rec, c.rec + ((size_t)pt[off0 >> c.page_shift] << c.page_shift) + (off0 & pm),
+                                     n0, &sm.full[stage]);
+                            if (rec_bytes > n0) {
+                                const uint32_t o1 = off0 + n0;
+                                bulk_g2s(sg.rec + n0, c.rec + ((size_t)pt[o1 >> c.page_shift] << c.page_shift) + (o1 & pm),
+                                         rec_bytes - n0, &sm.full[stage]);
+                            }
+                        }
                     }
                     if (q_bytes)
-                        bulk_g2s(sg.q, q + ((int64_t)s_of * HQ + hk * c.G + g0) * D, q_bytes, &sm.full[stage]);
+                        bulk_g2s(sg.q, q + ((int64_t)sh * c.G + g0) * D, q_bytes, &sm.full[stage]);
                 }
                 // counting sort by width: per-lane counts of the four classes packed in one
                 // word (8 bits each), one warp prefix sum; each class's run padded to whole
