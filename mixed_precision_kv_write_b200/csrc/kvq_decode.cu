@@ -572,6 +572,8 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         // d + nwin <= kWin. Items are claimed one at a time from the call's cursor when the
         // filler reaches them (CTAs that finish early take more); after the last one the
         // producer marks a stage kStop.
+        // (Claiming the next item one item ahead, to hide the claim's latency, lengthened the
+        // tail more than it saved.)
         auto claim = [&]() {
             int v = 0;
             if (lane == 0) v = (int)atomicAdd(wk.cursor, 1u);
@@ -660,21 +662,29 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 // keys, and (paged caches) bytes in at most two pages
                 const uint32_t off0 = __shfl_sync(0xffffffffu, pick(m, s0 % KPL), s0 / KPL) & ~15u;
                 const uint32_t plast = (off0 >> c.page_shift) + 1u;
-                uint32_t cnt = 0;
+                int n;
+                uint32_t nxl;
+                if (dend - s0 <= 255 && bnd - off0 <= kStageRecBytes && bnd >= off0 &&
+                    ((bnd - 1u) >> c.page_shift) <= plast) {
+                    n = dend - s0;    // the rest of the window is one stage (the common case)
+                    nxl = bnd;
+                } else {
+                    uint32_t cnt = 0;
 #pragma unroll
-                for (int r = 0; r < KPL; ++r) {
-                    const int sl = KPL * lane + r;
-                    cnt += (sl >= s0 && sl < dend && sl < s0 + 255 && nx[r] - off0 <= kStageRecBytes &&
-                            ((nx[r] - 1u) >> c.page_shift) <= plast) ? 1u : 0u;
-                }
-                int n = (int)__reduce_add_sync(0xffffffffu, cnt);
-                if (n < 1) {          // only with corrupt offsets: flag it, keep making progress
-                    if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
-                    n = 1;
+                    for (int r = 0; r < KPL; ++r) {
+                        const int sl = KPL * lane + r;
+                        cnt += (sl >= s0 && sl < dend && sl < s0 + 255 && nx[r] - off0 <= kStageRecBytes &&
+                                ((nx[r] - 1u) >> c.page_shift) <= plast) ? 1u : 0u;
+                    }
+                    n = (int)__reduce_add_sync(0xffffffffu, cnt);
+                    if (n < 1) {      // only with corrupt offsets: flag it, keep making progress
+                        if (lane == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+                        n = 1;
+                    }
+                    const int kl = s0 + n - 1;
+                    nxl = __shfl_sync(0xffffffffu, pick(nx, kl % KPL), kl / KPL);
                 }
                 const int s1 = s0 + n;
-                const int kl = s1 - 1;
-                const uint32_t nxl = __shfl_sync(0xffffffffu, pick(nx, kl % KPL), kl / KPL);
                 const bool last = lastwin && s1 == dend;
                 const bool new_item = first && s0 == d;
                 uint32_t rec_bytes = nxl - off0;
@@ -690,34 +700,48 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     break;
                 }
                 Stage<D> &sg = sm.st[stage];
-                if (lane == 0) {
-                    // the item's subgroup of queries: rows sh * G + g0 .. of q (query head
-                    // hk * G + g of sequence s is row (s * H + hk) * G + g), contiguous
+                {
+                    // the stage's copies, one instruction on up to four lanes: side entries
+                    // (lane 0), record bytes (lane 1, and lane 2 for the part of a paged stream
+                    // on its next page), and for a new item the item's subgroup of queries
+                    // (lane 3): rows sh * G + g0 .. of q (query head hk * G + g of sequence s
+                    // is row (s * H + hk) * G + g), contiguous
                     const int g0 = qinfo & 0xFF;
                     const int nq = min(kDecodeMaxQ, c.G - g0);
                     const uint32_t q_bytes = new_item ? (uint32_t)(2 * D * nq) : 0u;
-                    mbar_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
-                    bulk_g2s(sg.side, c.side + sbase + ja + s0, 16u * n, &sm.full[stage]);
-                    if (rec_bytes) {
+                    if (lane == 0) mbar_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
+                    __syncwarp();
+                    const void *src = nullptr;
+                    void *dst = nullptr;
+                    uint32_t bytes = 0u;
+                    if (lane == 0) {
+                        src = c.side + sbase + ja + s0;
+                        dst = sg.side;
+                        bytes = 16u * n;
+                    } else if (lane == 3) {
+                        src = q + ((int64_t)sh * c.G + g0) * D;
+                        dst = sg.q;
+                        bytes = q_bytes;
+                    } else if (lane < 3 && rec_bytes) {
                         if (!c.ptab) {
                             // contiguous: the stream starts at its first slot * 4 * D bytes
-                            bulk_g2s(sg.rec, c.rec + sbase * (4 * D) + off0, rec_bytes, &sm.full[stage]);
+                            if (lane == 1) {
+                                src = c.rec + sbase * (4 * D) + off0;
+                                dst = sg.rec;
+                                bytes = rec_bytes;
+                            }
                         } else {
                             // a paged stream: one copy per page the stage's bytes touch
                             const uint32_t *pt = c.ptab + (size_t)sh * c.max_lpages;
                             const uint32_t pm = (1u << c.page_shift) - 1u;
                             const uint32_t n0 = min(rec_bytes, (pm + 1u) - (off0 & pm));
-                            bulk_g2s(sg.rec, c.rec + ((size_t)pt[off0 >> c.page_shift] << c.page_shift) + (off0 & pm),
-                                     n0, &sm.full[stage]);
-                            if (rec_bytes > n0) {
-                                const uint32_t o1 = off0 + n0;
-                                bulk_g2s(sg.rec + n0, c.rec + ((size_t)pt[o1 >> c.page_shift] << c.page_shift) + (o1 & pm),
-                                         rec_bytes - n0, &sm.full[stage]);
-                            }
+                            const uint32_t o = (lane == 1) ? off0 : off0 + n0;
+                            bytes = (lane == 1) ? n0 : rec_bytes - n0;
+                            if (bytes) src = c.rec + ((size_t)pt[o >> c.page_shift] << c.page_shift) + (o & pm);
+                            dst = sg.rec + (lane == 1 ? 0u : n0);
                         }
                     }
-                    if (q_bytes)
-                        bulk_g2s(sg.q, q + ((int64_t)sh * c.G + g0) * D, q_bytes, &sm.full[stage]);
+                    if (bytes) bulk_g2s(dst, src, bytes, &sm.full[stage]);
                 }
                 // counting sort by width: per-lane counts of the four classes packed in one
                 // word (8 bits each), one warp prefix sum; each class's run padded to whole
@@ -761,12 +785,15 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                         sg.perm[pos] = kValid | ((uint32_t)(sl - s0) << 16) | ro;
                     }
                 }
-                // padding entries repeat the first key of their class without the valid bit:
-                // the consumers read finite data of the right width there and weight it 0
+                // padding entries have no valid bit, so the consumers weight them 0; they must
+                // still read finite data: any bytes read as b-bit codes are finite (record 0
+                // of the stage will do), fp16 values are not, so the b = 16 run repeats its
+                // first key
                 __syncwarp();
 #pragma unroll
-                for (int cl = 0; cl < 4; ++cl)
-                    if (lane < pad_n[cl]) sg.perm[pad_at[cl] + lane] = sg.perm[cstart[cl]] & ~kValid;
+                for (int cl = 0; cl < 3; ++cl)
+                    if (lane < pad_n[cl]) sg.perm[pad_at[cl] + lane] = 0u;
+                if (lane < pad_n[3]) sg.perm[pad_at[3] + lane] = sg.perm[cstart[3]] & ~kValid;
                 if (lane == 0) {
                     sg.info[0] = it;
                     sg.info[1] = n;
@@ -835,6 +862,8 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         if (sm.st[stage].info[2] & kStop) break;
         const int it = sm.st[stage].info[0];
         bool waited = true;                   // the first stage's wait is done
+        rot = 0;                              // chunks dealt by the item's own stage count:
+                                              // results do not depend on the CTA's earlier items
         KeyState ks;
         ks.m = kMInit;
         ks.l = 0.f;

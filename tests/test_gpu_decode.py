@@ -135,3 +135,22 @@ def test_decode_full_size_sampled(name, n_check, n_rec):
     # skip heads are exact zeros everywhere
     skip = (mc.numpy() == 0)
     assert np.all(out[skip] == 0)
+
+
+def test_decode_bitwise_repeatable_with_many_items():
+    # more work items than split-K CTAs: which CTA takes which item varies from call to call
+    # (items are claimed dynamically), the outputs must not
+    wl = synth.scaled(W["decode_1p3b"], seqlens=(4096,) * 32, heads=4)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    cache = kvq.KVQCache(wl.batch, wl.heads, wl.head_dim, list(wl.seqlens))
+    kvq.kvq_write(k, v, bits, synth.cu_seqlens(wl.seqlens, "cuda"), cache)
+    del k, v
+    g = torch.Generator(device="cuda").manual_seed(5)
+    q = torch.randn((wl.batch, wl.heads, 128), generator=g, device="cuda").half()
+    modes = torch.full((wl.batch, wl.heads), 2, dtype=torch.uint8, device="cuda")
+    modes[::3, 1] = 1
+    outs = [kvq.routed_attn_decode(q, cache, modes, 300) for _ in range(4)]
+    outs.append(kvq.routed_attn_decode_noalloc(q, cache, modes, 300).clone())
+    cache.check()
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
