@@ -78,9 +78,9 @@ constexpr int kStages = KVQ_DECODE_STAGES;        // record stages in flight per
 #ifndef KVQ_DECODE_WINDOW
 #define KVQ_DECODE_WINDOW 128
 #endif
-constexpr int kWin = KVQ_DECODE_WINDOW;           // keys per window of record offsets (128 or 256)
+constexpr int kWin = KVQ_DECODE_WINDOW;           // keys per window of record offsets
 constexpr int KPL = kWin / 32;                    // window slots per producer lane
-static_assert(kWin == 128 || kWin == 256, "window of 128 or 256 keys");
+static_assert(kWin == 128, "windows of 128 keys: the width sort packs positions below 256 in bytes");
 constexpr uint32_t kStageRecBytes = KVQ_DECODE_STAGE_BYTES;   // record bytes per stage, at most
 constexpr int kPermSlots = kWin + 64;             // width-sorted keys padded to whole chunks
 constexpr int kMetaSlots = KVQ_DECODE_META_SLOTS; // windows of record offsets fetched ahead
@@ -743,14 +743,18 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     }
                     if (bytes) bulk_g2s(dst, src, bytes, &sm.full[stage]);
                 }
-                // counting sort by width: per-lane counts of the four classes packed in one
-                // word (8 bits each), one warp prefix sum; each class's run padded to whole
-                // chunks of KPS keys
-                uint32_t lc = 0;
+                // counting sort by width, four classes packed as bytes of one word: per-lane
+                // counts, one warp prefix sum; each class's run padded to whole chunks of KPS
+                // keys. Byte c of `cst` is class c's first position, of `run` this lane's
+                // next rank in class c (no byte overflows: at most 255 keys plus padding)
+                uint32_t lc = 0, shc[KPL];
+                bool inr[KPL];
 #pragma unroll
                 for (int r = 0; r < KPL; ++r) {
                     const int sl = KPL * lane + r;
-                    if (sl >= s0 && sl < s1) lc += 1u << (8 * (m[r] & 3u));
+                    inr[r] = sl >= s0 && sl < s1;
+                    shc[r] = (m[r] & 3u) << 3;
+                    if (inr[r]) lc += 1u << shc[r];
                 }
                 uint32_t incl = lc;
 #pragma unroll
@@ -759,41 +763,32 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     if (lane >= dd) incl += y;
                 }
                 const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
-                uint32_t run = incl - lc;               // this lane's first rank in each class
-                int cstart[4], pad_at[4], pad_n[4], pstart = 0;
-#pragma unroll
-                for (int cl = 0; cl < 4; ++cl) {
-                    const int tc = (int)((tot >> (8 * cl)) & 0xFFu);
-                    const int padded = (tc + KPS - 1) / KPS * KPS;
-                    cstart[cl] = pstart;
-                    pad_at[cl] = pstart + tc;
-                    pad_n[cl] = padded - tc;
-                    pstart += padded;
-                }
-
+                constexpr uint32_t kRound = 0x01010101u * (uint32_t)(KPS - 1);
+                const uint32_t padded = (tot + kRound) & ~kRound;      // run lengths, whole chunks
+                const uint32_t cst = (padded << 8) + (padded << 16) + (padded << 24);
+                const int pstart = (int)((cst >> 24) + (padded >> 24));
+                uint32_t run = cst + incl - lc;
 #pragma unroll
                 for (int r = 0; r < KPL; ++r) {
-                    const int sl = KPL * lane + r;
-                    if (sl >= s0 && sl < s1) {
-                        const uint32_t cl = m[r] & 3u;
-                        const int start = cl == 0 ? cstart[0] : cl == 1 ? cstart[1] : cl == 2 ? cstart[2] : cstart[3];
-                        const int pos = start + (int)((run >> (8 * cl)) & 0xFFu);
-                        run += 1u << (8 * cl);
+                    if (inr[r]) {
+                        const int pos = (int)((run >> shc[r]) & 0xFFu);
+                        run += 1u << shc[r];
                         // offset inside the stage; the clamp only bites on corrupt offsets and
                         // keeps every shared-memory read of the consumers inside the stage
-                        const uint32_t ro = min((m[r] & ~15u) - off0, kStageRecBytes - (uint32_t)(D * (2 << cl)) / 4u);
-                        sg.perm[pos] = kValid | ((uint32_t)(sl - s0) << 16) | ro;
+                        const uint32_t ro = min((m[r] & ~15u) - off0, kStageRecBytes - ((uint32_t)(D / 2) << (shc[r] >> 3)));
+                        sg.perm[pos] = kValid | ((uint32_t)(KPL * lane + r - s0) << 16) | ro;
                     }
                 }
                 // padding entries have no valid bit, so the consumers weight them 0; they must
                 // still read finite data: any bytes read as b-bit codes are finite (record 0
                 // of the stage will do), fp16 values are not, so the b = 16 run repeats its
                 // first key
+                const uint32_t pad_at = cst + tot, pad_n = padded - tot;
                 __syncwarp();
 #pragma unroll
                 for (int cl = 0; cl < 3; ++cl)
-                    if (lane < pad_n[cl]) sg.perm[pad_at[cl] + lane] = 0u;
-                if (lane < pad_n[3]) sg.perm[pad_at[3] + lane] = sg.perm[cstart[3]] & ~kValid;
+                    if (lane < (int)((pad_n >> (8 * cl)) & 0xFFu)) sg.perm[((pad_at >> (8 * cl)) & 0xFFu) + lane] = 0u;
+                if (lane < (int)(pad_n >> 24)) sg.perm[(pad_at >> 24) + lane] = sg.perm[cst >> 24] & ~kValid;
                 if (lane == 0) {
                     sg.info[0] = it;
                     sg.info[1] = n;
@@ -801,7 +796,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     sg.info[3] = pstart / KPS;
                     sg.info[4] = qinfo;
 #pragma unroll
-                    for (int cl = 0; cl < 4; ++cl) sg.cls_chunk[cl] = cstart[cl] / KPS;
+                    for (int cl = 0; cl < 4; ++cl) sg.cls_chunk[cl] = (int)((cst >> (8 * cl)) & 0xFFu) / KPS;
                     sg.cls_chunk[4] = pstart / KPS;
                 }
                 __syncwarp();
