@@ -700,48 +700,34 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                     break;
                 }
                 Stage<D> &sg = sm.st[stage];
-                {
-                    // the stage's copies, one instruction on up to four lanes: side entries
-                    // (lane 0), record bytes (lane 1, and lane 2 for the part of a paged stream
-                    // on its next page), and for a new item the item's subgroup of queries
-                    // (lane 3): rows sh * G + g0 .. of q (query head hk * G + g of sequence s
-                    // is row (s * H + hk) * G + g), contiguous
+                if (lane == 0) {
+                    // the item's subgroup of queries: rows sh * G + g0 .. of q (query head
+                    // hk * G + g of sequence s is row (s * H + hk) * G + g), contiguous
                     const int g0 = qinfo & 0xFF;
                     const int nq = min(kDecodeMaxQ, c.G - g0);
                     const uint32_t q_bytes = new_item ? (uint32_t)(2 * D * nq) : 0u;
-                    if (lane == 0) mbar_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
-                    __syncwarp();
-                    const void *src = nullptr;
-                    void *dst = nullptr;
-                    uint32_t bytes = 0u;
-                    if (lane == 0) {
-                        src = c.side + sbase + ja + s0;
-                        dst = sg.side;
-                        bytes = 16u * n;
-                    } else if (lane == 3) {
-                        src = q + ((int64_t)sh * c.G + g0) * D;
-                        dst = sg.q;
-                        bytes = q_bytes;
-                    } else if (lane < 3 && rec_bytes) {
+                    mbar_expect_tx(&sm.full[stage], 16u * n + rec_bytes + q_bytes);
+                    bulk_g2s(sg.side, c.side + sbase + ja + s0, 16u * n, &sm.full[stage]);
+                    if (rec_bytes) {
                         if (!c.ptab) {
                             // contiguous: the stream starts at its first slot * 4 * D bytes
-                            if (lane == 1) {
-                                src = c.rec + sbase * (4 * D) + off0;
-                                dst = sg.rec;
-                                bytes = rec_bytes;
-                            }
+                            bulk_g2s(sg.rec, c.rec + sbase * (4 * D) + off0, rec_bytes, &sm.full[stage]);
                         } else {
                             // a paged stream: one copy per page the stage's bytes touch
                             const uint32_t *pt = c.ptab + (size_t)sh * c.max_lpages;
                             const uint32_t pm = (1u << c.page_shift) - 1u;
                             const uint32_t n0 = min(rec_bytes, (pm + 1u) - (off0 & pm));
-                            const uint32_t o = (lane == 1) ? off0 : off0 + n0;
-                            bytes = (lane == 1) ? n0 : rec_bytes - n0;
-                            if (bytes) src = c.rec + ((size_t)pt[o >> c.page_shift] << c.page_shift) + (o & pm);
-                            dst = sg.rec + (lane == 1 ? 0u : n0);
+                            bulk_g2s(sg.rec, c.rec + ((size_t)pt[off0 >> c.page_shift] << c.page_shift) + (off0 & pm),
+                                     n0, &sm.full[stage]);
+                            if (rec_bytes > n0) {
+                                const uint32_t o1 = off0 + n0;
+                                bulk_g2s(sg.rec + n0, c.rec + ((size_t)pt[o1 >> c.page_shift] << c.page_shift) + (o1 & pm),
+                                         rec_bytes - n0, &sm.full[stage]);
+                            }
                         }
                     }
-                    if (bytes) bulk_g2s(dst, src, bytes, &sm.full[stage]);
+                    if (q_bytes)
+                        bulk_g2s(sg.q, q + ((int64_t)sh * c.G + g0) * D, q_bytes, &sm.full[stage]);
                 }
                 // counting sort by width, four classes packed as bytes of one word: per-lane
                 // counts, one warp prefix sum; each class's run padded to whole chunks of KPS
