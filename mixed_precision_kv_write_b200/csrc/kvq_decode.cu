@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kPlanThreads)
 decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, DecodeWork wk, uint32_t gen,
                    AppendArgs ap)
 {
-    __shared__ int bad_sh;
+    __shared__ AppendShared as;
     __shared__ int warp_tot[kPlanThreads / 32];
     __shared__ int cnt_sh[kPlanThreads];
     __shared__ uint32_t base_sh;
@@ -198,7 +198,7 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
         *wk.cursor = 0u;                 // the split-K CTAs claim this call's items from 0
     }
     const int s = blockIdx.x;
-    if (APPEND) append_seq<D>(c, ap.k, ap.v, ap.bits, ap.cu, ap.n_tok, ap.gen, ap.positions, s, bad_sh);
+    if (APPEND) append_seq<D>(c, ap.k, ap.v, ap.bits, ap.cu, ap.n_tok, ap.gen, ap.positions, s, as);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int H = c.H, G = c.G, HQ = H * G;
     const int nsub = (G + kDecodeMaxQ - 1) / kDecodeMaxQ;
@@ -211,7 +211,7 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
         if (mine) {
             hk = u / nsub;
             g0 = (u % nsub) * kDecodeMaxQ;
-            L = c.len[s * H + hk];
+            L = (APPEND && hk < kAppendHeads) ? as.len[hk] : c.len[s * H + hk];
             lo_loc = max(0, L - 1 - w);
             int full = 0, local = 0;
             for (int i = 0; i < kDecodeMaxQ && g0 + i < G; ++i) {
@@ -272,7 +272,7 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
         u_q[tid] = g0 | (mA << 8) | (mB << 12);
         u_L[tid] = L;
         if (mine && cnt > 0) {
-            u_end[tid] = c.end[s * H + hk];
+            u_end[tid] = (APPEND && hk < kAppendHeads) ? as.end[hk] : c.end[s * H + hk];
             u_sbase[tid] = slot_of(c, s, hk, 0);
         }
         __syncthreads();

@@ -136,39 +136,83 @@ __device__ __forceinline__ void vec_store(const CacheView &c, const uint4 (&raw)
     if (li == 0) reinterpret_cast<float2 *>(&c.side[slot])[part] = make_float2(sc, z);
 }
 
+// Per-head results of append_seq, in shared memory (heads beyond kAppendHeads use the
+// cache's arrays in global memory).
+constexpr int kAppendHeads = 64;
+constexpr int kAppendMeta = 512;                 // (token, head) record offsets kept on chip
+struct AppendShared {
+    int bad;                                     // a bad width in the sequence's new tokens
+    int32_t wstart[kAppendHeads];                // write start (-1: refused), per head
+    uint32_t wend[kAppendHeads];                 // stream end after the write, per head
+    int32_t len[kAppendHeads];                   // length on return, per head
+    uint32_t end[kAppendHeads];                  // stream end on return, per head
+    uint32_t meta[kAppendMeta];                  // token i, head h at i * H + h, when n * H fits
+};
+
 // Appends the call's tokens of sequence s (rows cu[s] .. cu[s+1]-1 of k, v, bits) for
 // every head; called by all threads of a block of 256 (it synchronizes the block).
-// Phase 1, a warp per head: the optional roll-back to positions[s] (the sequence keeps
-// its first min(len, positions[s]) tokens, as kvq_cache_truncate), then capacity, widths
-// and record offsets (warp prefix sum) of the new tokens. Phase 2, after the block has
-// seen every head's verdict: D/8 lanes per vector quantize straight from global memory.
-// A bad width refuses the sequence's write for every head; a capacity overflow refuses
-// that head. On return the new lengths and stream ends are committed and visible to the
-// whole block. Inconsistent cu_seqlens leave the sequence untouched (status set).
+// Every load that does not depend on another goes out first: the sequence's range,
+// roll-back position and slot geometry, each head's length and stream end, the first 32
+// widths of each head and this thread's first K/V chunks. Phase 1, a warp per head: the
+// optional roll-back to positions[s] (the sequence keeps its first min(len, positions[s])
+// tokens, as kvq_cache_truncate), then capacity, widths and record offsets (warp prefix
+// sum) of the new tokens. Phase 2, after the block has seen every head's verdict: D/8
+// lanes per vector quantize from the prefetched rows. A bad width refuses the sequence's
+// write for every head; a capacity overflow refuses that head. On return the new lengths
+// and stream ends are committed, visible to the whole block, and (heads below
+// kAppendHeads) also in `as`. Inconsistent cu_seqlens leave the sequence untouched (status
+// set; as.wstart[h] = -1).
 template <int D>
 __device__ __forceinline__ void append_seq(const CacheView &c, const __half *__restrict__ k,
                                            const __half *__restrict__ v, const uint8_t *__restrict__ bits,
                                            const int32_t *__restrict__ cu, int64_t n_tok, uint32_t gen,
-                                           const int32_t *__restrict__ positions, int s, int &bad_sh)
+                                           const int32_t *__restrict__ positions, int s, AppendShared &as)
 {
     constexpr int VL = D / 8, VPW = 32 / VL;
+    constexpr int kPre = 2;                      // vector passes whose rows are loaded up front
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = c.H;
     const int64_t t0 = cu[s], t1 = cu[s + 1];
+    const int roll = positions ? positions[s] : -1;
+    const int cap = c.cap[s];
+    const int64_t sbase = c.slot_base[s];
+    const int cpad = c.cap_pad[s];
     if (t0 < 0 || t1 < t0 || t1 > n_tok || (s == 0 && t0 != 0)) {   // block-uniform
         if (tid == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+        for (int h = tid; h < min(H, kAppendHeads); h += blockDim.x) {
+            as.wstart[h] = -1;
+            as.len[h] = c.len[s * H + h];
+            as.end[h] = c.end[s * H + h];
+        }
+        __syncthreads();
         return;
     }
     const int n = (int)(t1 - t0);
-    if (tid == 0) bad_sh = 0;
+    const int n_vec = 2 * n * H;                 // vector vi: pair vi / 2 = i * H + h, K or V
+    const int li = lane % VL;
+    const bool meta_on_chip = n * H <= kAppendMeta;
+    // this thread's first kPre vector chunks
+    uint4 pre[kPre];
+#pragma unroll
+    for (int p = 0; p < kPre; ++p) {
+        const int vi = warp * VPW + lane / VL + p * 8 * VPW;
+        pre[p] = make_uint4(0u, 0u, 0u, 0u);
+        if (vi < n_vec) {
+            const int pp = vi >> 1;
+            pre[p] = reinterpret_cast<const uint4 *>((vi & 1 ? v : k) + ((t0 + pp / H) * H + pp % H) * D)[li];
+        }
+    }
+    if (tid == 0) as.bad = 0;
     __syncthreads();
-    const int roll = positions ? positions[s] : -1;
     for (int h = warp; h < H; h += 8) {
         const int sh = s * H + h;
         int L0 = c.len[sh];
         uint32_t off = c.end[sh];
+        // the first 32 widths go out with the length
+        int b_first = 0;
+        if (lane < n) b_first = bits[(t0 + lane) * H + h];
         if (roll >= 0 && roll < L0) {             // roll back first (truncate semantics)
-            off = c.meta[slot_of(c, s, h, roll)] & ~15u;
+            off = c.meta[sbase + (int64_t)h * cpad + roll] & ~15u;
             L0 = roll;
         }
         __syncwarp();
@@ -176,19 +220,24 @@ __device__ __forceinline__ void append_seq(const CacheView &c, const __half *__r
             c.len[sh] = L0;
             c.end[sh] = off;
             c.wstart[sh] = -1;
+            if (h < kAppendHeads) {
+                as.wstart[h] = -1;
+                as.len[h] = L0;
+                as.end[h] = off;
+            }
         }
         if (n == 0) continue;
-        if ((int64_t)L0 + n > c.cap[s]) {
+        if ((int64_t)L0 + n > cap) {
             if (lane == 0) set_status(c.status, KVQ_ERR_CAPACITY);
             continue;
         }
-        const int64_t slot0 = slot_of(c, s, h, L0);
+        const int64_t slot0 = sbase + (int64_t)h * cpad + L0;
         bool bad = false;
         for (int base = 0; base < n; base += 32) {
             const int i = base + lane;
             uint32_t sz = 0, wc = 0;
             if (i < n) {
-                const int b = bits[(t0 + i) * H + h];
+                const int b = base == 0 ? b_first : bits[(t0 + i) * H + h];
                 const int wcode = width_code(b);
                 if (wcode < 0) bad = true;
                 else {
@@ -202,14 +251,22 @@ __device__ __forceinline__ void append_seq(const CacheView &c, const __half *__r
                 const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
                 if (lane >= d) incl += y;
             }
-            if (i < n) c.meta[slot0 + i] = (off + incl - sz) | wc;
+            if (i < n) {
+                const uint32_t m = (off + incl - sz) | wc;
+                c.meta[slot0 + i] = m;
+                if (meta_on_chip) as.meta[i * H + h] = m;
+            }
             off += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&bad_sh, 1);
+        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&as.bad, 1);
         if (lane == 0) {
             if (map_pages(c, s, h, off)) {       // paged caches: pages for the new bytes
                 c.wstart[sh] = L0;
                 c.wend[sh] = off;
+                if (h < kAppendHeads) {
+                    as.wstart[h] = L0;
+                    as.wend[h] = off;
+                }
             } else {
                 set_status(c.status, KVQ_ERR_CAPACITY);
             }
@@ -217,38 +274,49 @@ __device__ __forceinline__ void append_seq(const CacheView &c, const __half *__r
     }
     __syncthreads();
     if (n == 0) return;                          // block-uniform
-    if (bad_sh) {                                // the sequence's write is refused for every head
+    if (as.bad) {                                // the sequence's write is refused for every head
         if (tid == 0) {
             c.bad[s] = gen;
             set_status(c.status, KVQ_ERR_BITS);
         }
+        for (int h = tid; h < min(H, kAppendHeads); h += blockDim.x) as.wstart[h] = -1;
         __syncthreads();
         return;
     }
-    const int n_vec = 2 * n * H;                 // vector vi: pair vi / 2 = i * H + h, K or V
-    const int li = lane % VL;
-    for (int vb = warp * VPW; vb < n_vec; vb += 8 * VPW) {
+    int p = 0;
+    for (int vb = warp * VPW; vb < n_vec; vb += 8 * VPW, ++p) {
         const int vi = vb + lane / VL;
         const bool in_range = vi < n_vec;
-        const int p = vi >> 1, part = vi & 1;
-        const int i = p / H, h = p % H;
+        const int pp = vi >> 1, part = vi & 1;
+        const int i = pp / H, h = pp % H;
         uint4 raw[1] = {make_uint4(0u, 0u, 0u, 0u)};
-        if (in_range) raw[0] = reinterpret_cast<const uint4 *>((part ? v : k) + ((t0 + i) * H + h) * D)[li];
+        if (p < kPre) {
+#pragma unroll
+            for (int q = 0; q < kPre; ++q)
+                if (q == p) raw[0] = pre[q];
+        } else if (in_range) {
+            raw[0] = reinterpret_cast<const uint4 *>((part ? v : k) + ((t0 + i) * H + h) * D)[li];
+        }
         const __half2 mm = vec_minmax<1, VL>(raw);
         if (!in_range) continue;
-        const int st = c.wstart[s * H + h];
+        const int st = (h < kAppendHeads) ? as.wstart[h] : c.wstart[s * H + h];
         if (st < 0) continue;
-        const int64_t slot = slot_of(c, s, h, st + i);
-        const uint32_t meta = c.meta[slot];
+        const int64_t slot = sbase + (int64_t)h * cpad + st + i;
+        const uint32_t meta = meta_on_chip ? as.meta[i * H + h] : c.meta[slot];
         const int b = 2 << (meta & 3u);
         vec_store<1, VL>(c, raw, mm, b, rec_loc(c, s, h, (meta & ~15u) + part * (b * D / 8)), slot, part, li);
     }
     __syncthreads();
     for (int h = tid; h < H; h += blockDim.x) {  // commit the new lengths and stream ends
-        const int st = c.wstart[s * H + h];
+        const int st = (h < kAppendHeads) ? as.wstart[h] : c.wstart[s * H + h];
         if (st >= 0) {
+            const uint32_t e = (h < kAppendHeads) ? as.wend[h] : c.wend[s * H + h];
             c.len[s * H + h] = st + n;
-            c.end[s * H + h] = c.wend[s * H + h];
+            c.end[s * H + h] = e;
+            if (h < kAppendHeads) {
+                as.len[h] = st + n;
+                as.end[h] = e;
+            }
         }
     }
     __syncthreads();

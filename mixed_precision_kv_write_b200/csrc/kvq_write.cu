@@ -645,10 +645,10 @@ write_append_kernel(CacheView c, const __half *__restrict__ k, const __half *__r
                     const uint8_t *__restrict__ bits, const int32_t *__restrict__ cu, int64_t n_tok,
                     uint32_t gen)
 {
-    __shared__ int bad_sh;
+    __shared__ AppendShared as;
     pdl_wait();
     pdl_trigger();
-    append_seq<D>(c, k, v, bits, cu, n_tok, gen, nullptr, blockIdx.x, bad_sh);
+    append_seq<D>(c, k, v, bits, cu, n_tok, gen, nullptr, blockIdx.x, as);
 }
 
 } // namespace
