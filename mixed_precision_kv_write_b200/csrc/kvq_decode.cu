@@ -16,7 +16,7 @@
 //   decode_splitk_kernel  three CTAs per SM, one producer and four consumer warps each. The
 //                         producer claims items one at a time from the call's cursor (a CTA
 //                         that finishes early takes more) and walks each in stages of at
-//                         most 128 keys and 24 KB of records: a ring of record-offset
+//                         most 128 keys and 28 KB of records: a ring of record-offset
 //                         windows is bulk-copied
 //                         ahead, each stage's keys are sorted by width into chunks of one
 //                         width (8 keys at head_dim 128), and the stage's contiguous record
@@ -66,10 +66,10 @@ namespace {
 #define KVQ_DECODE_STAGES 2
 #endif
 #ifndef KVQ_DECODE_STAGE_BYTES
-#define KVQ_DECODE_STAGE_BYTES 24576
+#define KVQ_DECODE_STAGE_BYTES 28672
 #endif
 #ifndef KVQ_DECODE_META_SLOTS
-#define KVQ_DECODE_META_SLOTS 6
+#define KVQ_DECODE_META_SLOTS 4
 #endif
 constexpr int kConsumerWarps = KVQ_DECODE_CONSUMERS;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
