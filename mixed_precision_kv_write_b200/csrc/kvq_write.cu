@@ -298,13 +298,17 @@ write_scan_chunk_kernel(CacheView c, const uint8_t *__restrict__ bits, const int
 
 // Staging of the quantize kernel: each CTA copies the fp16 K and V rows of T tokens x HG
 // heads (at most kWqHalves values per tensor) into shared memory with two bulk copies.
+#ifndef KVQ_WQ_LPV
+#define KVQ_WQ_LPV 2
+#endif
 #ifndef KVQ_WQ_THREADS
-#define KVQ_WQ_THREADS 128
+#define KVQ_WQ_THREADS (128 * KVQ_WQ_LPV)
 #endif
 #ifndef KVQ_WQ_HALVES
 #define KVQ_WQ_HALVES 8192
 #endif
 constexpr int kWqThreads = KVQ_WQ_THREADS;
+constexpr int kWqLanesPerVec = KVQ_WQ_LPV;   // lanes per vector at head_dim 128 (64: one)
 constexpr int kWqHalves = KVQ_WQ_HALVES; // fp16 values of K (and of V) staged per CTA
 constexpr int kWqMaxPairs = kWqHalves / 64;
 static_assert(kWqMaxPairs <= kWqThreads, "one (token, head) pair per thread");
@@ -412,18 +416,21 @@ __device__ __forceinline__ void swap_if(bool c, uint32_t &a, uint32_t &b)
     a = t;
 }
 
-// One lane writes the codes of one vector of D fp16 values held in shared memory, a
-// 16-byte group (16/BITS chunks of 8 values) per store. With x = lane mod 8, step j reads
-// chunk j ^ x: the eight lanes of a shared-memory phase read eight different bank groups
-// (every vector starts on a 128-byte boundary), and the G steps k*G .. k*G + G - 1 cover the
-// chunks of group k ^ (x / G), chunk slot i ^ (x mod G) filled at step k*G + i; the slots
-// are put in place by conditional swaps before the store. PLAIN selects the plain formula
-// (taken only when a quotient was NaN: NaN or infinite inputs). Returns the sum of the
-// quotients.
-template <int D, int BITS, bool PLAIN>
-__device__ __forceinline__ float lane_codes(const uint4 *src, float z, float sc, const PartDst &dst, int x)
+// One lane writes the codes of NCHL chunks of 8 fp16 values held in shared memory (a whole
+// vector, or its half when two lanes share a vector), a 16-byte group (G = 16/BITS chunks)
+// per store at byte rel0 + 16 * group of the record part. With x = lane mod 8 (x < NCHL),
+// step j reads chunk j ^ x: the eight lanes of a shared-memory phase read eight different
+// bank groups (every vector starts on a 128-byte boundary), and the G steps k*G .. k*G + G - 1
+// cover the chunks of group k ^ (x / G), chunk slot i ^ (x mod G) filled at step k*G + i;
+// the slots are put in place by conditional swaps before the store. PLAIN selects the
+// plain formula (taken only when a quotient was NaN: NaN or infinite inputs). Returns the
+// sum of the quotients.
+template <int NCHL, int BITS, bool PLAIN>
+__device__ __forceinline__ float lane_codes(const uint4 *src, float z, float sc, const PartDst &dst, uint32_t rel0,
+                                            int x)
 {
-    constexpr int NCH = D / 8, G = 16 / BITS, NG = NCH / G;
+    constexpr int G = 16 / BITS, NG = NCHL / G;
+    static_assert(NCHL >= G, "a lane covers whole 16-byte groups");
     const float y = __frcp_rn(sc);
     const float2 y2 = make_float2(y, y), ns2 = make_float2(-sc, -sc);
     float2 probe = make_float2(0.0f, 0.0f);
@@ -463,35 +470,40 @@ __device__ __forceinline__ float lane_codes(const uint4 *src, float z, float sc,
             swap_if(m & 4, o[0], o[2]);
             swap_if(m & 4, o[1], o[3]);
         }
-        *reinterpret_cast<uint4 *>(dst.at(16u * (uint32_t)(k ^ (x / G)))) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4 *>(dst.at(rel0 + 16u * (uint32_t)(k ^ (x / G)))) = make_uint4(o[0], o[1], o[2], o[3]);
     }
     return probe.x + probe.y;
 }
 
-template <int D, int BITS>
-__device__ __forceinline__ void lane_quant(const uint4 *src, float z, float sc, const PartDst &dst, int x)
+template <int NCHL, int BITS>
+__device__ __forceinline__ void lane_quant(const uint4 *src, float z, float sc, const PartDst &dst, uint32_t rel0,
+                                           int x)
 {
-    const float nan_probe = lane_codes<D, BITS, false>(src, z, sc, dst, x);
-    if (nan_probe != nan_probe) lane_codes<D, BITS, true>(src, z, sc, dst, x);   // same lane, same bytes
+    const float nan_probe = lane_codes<NCHL, BITS, false>(src, z, sc, dst, rel0, x);
+    if (nan_probe != nan_probe) lane_codes<NCHL, BITS, true>(src, z, sc, dst, rel0, x);   // same lane, same bytes
 }
 
-// One lane quantizes one vector: min/max, then the record part (the raw fp16 bits for
-// b = 16) and the (s, z) side entry.
-template <int D>
-__device__ __forceinline__ void lane_vector(const CacheView &c, const uint4 *src, int b, const RecLoc &L,
-                                            int64_t slot, int part, int x)
+// LPV lanes (1 or 2, adjacent) quantize one vector: min/max (combined across the pair with
+// one shuffle), then each lane its share of the record part (the raw fp16 bits for
+// b = 16); the first lane writes the (s, z) side entry.
+template <int D, int LPV>
+__device__ __forceinline__ void lane_vector(const CacheView &c, const uint4 *vsrc, int b, const RecLoc &L,
+                                            int64_t slot, int part, int x, int half)
 {
-    constexpr int NCH = D / 8;
+    constexpr int NCHL = D / 8 / LPV;            // chunks per lane
     const PartDst dst = part_dst(L, (uint32_t)(b * D / 8));
+    const uint4 *src = vsrc + half * NCHL;
+    const uint32_t rel0 = (uint32_t)(half * (b * D / 8 / LPV));
     float sc = 1.0f, z = 0.0f;
     if (b == 16) {
 #pragma unroll 4
-        for (int j = 0; j < NCH; ++j) *reinterpret_cast<uint4 *>(dst.at(16u * (uint32_t)(j ^ x))) = src[j ^ x];
+        for (int j = 0; j < NCHL; ++j)
+            *reinterpret_cast<uint4 *>(dst.at(16u * (uint32_t)(half * NCHL + (j ^ x)))) = src[j ^ x];
     } else {
         // min and max in fp16 (exact); -0 and +0 are one value, stored as +0 below
         __half2 lo2 = *reinterpret_cast<const __half2 *>(&src[x].x), hi2 = lo2;
 #pragma unroll 4
-        for (int j = 0; j < NCH; ++j) {
+        for (int j = 0; j < NCHL; ++j) {
             const uint4 r = src[j ^ x];
             const uint32_t hw[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
@@ -500,21 +512,27 @@ __device__ __forceinline__ void lane_vector(const CacheView &c, const uint4 *src
                 hi2 = __hmax2(hi2, *reinterpret_cast<const __half2 *>(&hw[e]));
             }
         }
-        const float mn = __half2float(__hmin(__low2half(lo2), __high2half(lo2)));
-        const float mx = __half2float(__hmax(__low2half(hi2), __high2half(hi2)));
+        __half2 mm = __halves2half2(__hmin(__low2half(lo2), __high2half(lo2)),
+                                    __hneg(__hmax(__low2half(hi2), __high2half(hi2))));
+        if (LPV == 2) {                          // (min, -max) of the pair's halves
+            const unsigned pair = 3u << (threadIdx.x & 30);
+            const uint32_t o = __shfl_xor_sync(pair, *reinterpret_cast<uint32_t *>(&mm), 1);
+            mm = __hmin2(mm, *reinterpret_cast<const __half2 *>(&o));
+        }
+        const float mn = __low2float(mm), mx = -__high2float(mm);
         const float top = (float)((1u << b) - 1u);
         sc = __fadd_rn(__fdiv_rn(__fsub_rn(mx, mn), top), 0.0f);
         z = __fadd_rn(mn, 0.0f);
         if (sc != 0.0f) {
-            if (b == 8) lane_quant<D, 8>(src, z, sc, dst, x);
-            else if (b == 4) lane_quant<D, 4>(src, z, sc, dst, x);
-            else lane_quant<D, 2>(src, z, sc, dst, x);
+            if (b == 8) lane_quant<NCHL, 8>(src, z, sc, dst, rel0, x);
+            else if (b == 4) lane_quant<NCHL, 4>(src, z, sc, dst, rel0, x);
+            else lane_quant<NCHL, 2>(src, z, sc, dst, rel0, x);
         } else {                                   // a constant vector: every code is 0
-            for (uint32_t o = 0; o < (uint32_t)(b * D / 8); o += 16u)
-                *reinterpret_cast<uint4 *>(dst.at(o)) = make_uint4(0u, 0u, 0u, 0u);
+            for (uint32_t o = 0; o < (uint32_t)(b * D / 8 / LPV); o += 16u)
+                *reinterpret_cast<uint4 *>(dst.at(rel0 + o)) = make_uint4(0u, 0u, 0u, 0u);
         }
     }
-    reinterpret_cast<float2 *>(&c.side[slot])[part] = make_float2(sc, z);
+    if (half == 0) reinterpret_cast<float2 *>(&c.side[slot])[part] = make_float2(sc, z);
 }
 
 // One CTA per tile of T tokens x HG heads. Warp 0 starts two bulk copies (the tile's K and
@@ -623,16 +641,18 @@ write_quant_kernel(CacheView c, const __half *__restrict__ k, const __half *__re
     __syncthreads();
     if (!mbar_wait(&bar, 0, c.status)) return;
 
-    // one lane per vector: vector vi is pair order[vi / 2], K (even) or V (odd); the lanes of
-    // a warp take consecutive vectors of the width-sorted list
+    // LPV adjacent lanes per vector: vector vi is pair order[vi / 2], K (even) or V (odd);
+    // the lanes of a warp take consecutive vectors of the width-sorted list
+    constexpr int LPV = (D == 128) ? kWqLanesPerVec : 1;
     const int n_vec = 2 * n_written;
-    for (int vi = tid; vi < n_vec; vi += kWqThreads) {
+    for (int t = tid; t < n_vec * LPV; t += kWqThreads) {
+        const int vi = t / LPV, half = t % LPV;
         const int pi = order[vi >> 1], part = vi & 1;
         const WqPair pr = pairs[pi];
         const int b = 2 << (pr.meta & 3u);
         const uint4 *src = reinterpret_cast<const uint4 *>((part ? sv : sk) + pi * D);
-        lane_vector<D>(c, src, b, rec_loc(c, pr.s, pr.h, (pr.meta & ~15u) + part * (b * D / 8)), pr.slot, part,
-                       lane & 7);
+        lane_vector<D, LPV>(c, src, b, rec_loc(c, pr.s, pr.h, (pr.meta & ~15u) + part * (b * D / 8)), pr.slot, part,
+                            lane & 7, half);
     }
 }
 
