@@ -1027,7 +1027,18 @@ decode_combine_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
             idx_sh[k] = (p >= 0) ? (int32_t)(p / (D + 4)) : -1;
         }
         __syncthreads();
+        // 16 independent loads per round: a long item list costs few L2 round trips
         int k = 0;
+        for (; k + 16 <= n; k += 16) {
+            float v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int32_t ix = idx_sh[k + u];
+                v[u] = (ix >= 0) ? wk.partials[(int64_t)ix * (D + 4) + 4 + ch] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) acc = fmaf(v[u], f_sh[k + u], acc);
+        }
         for (; k + 4 <= n; k += 4) {
             float v[4];
 #pragma unroll
