@@ -42,6 +42,7 @@ constexpr int kKeys = 64;       // keys per key tile (QK MMA N, PV MMA K)
 constexpr int kSoftmaxWarps = 8, kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kUnpackWarps = 8, kUnpackThreads = 32 * kUnpackWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + kUnpackWarps;
+constexpr int kQReadyBar = 3;                   // named barrier: Q in TMEM (softmax warps + QK issuer)
 constexpr int kStageWarp = kMmaWarp + 1;
 constexpr int kPvWarp = kMmaWarp + 2;
 constexpr int kTcThreads = 32 * (kStageWarp + 3);
@@ -283,8 +284,16 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         mbar_init(&sm.p_full, kSoftmaxWarps);
         mbar_init(&sm.pv_done, 1);
         mbar_init(&sm.drain, 2);
+        // the tile's key range, from its first and last query: a tile's query list is
+        // monotonic (local queries ascending, full queries descending), so these hold the
+        // smallest and the largest position; each row checks its own range below
         sm.klo = INT32_MAX;
         sm.khi = -1;
+        if (tile.count > 0) {
+            const int ia = qidx[tile.start], ib = qidx[tile.start + tile.count - 1];
+            sm.khi = pos0 + max(ia, ib);
+            sm.klo = (tile.mode == KVQ_MODE_LOCAL) ? max(0, pos0 + min(ia, ib) - w) : 0;
+        }
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -298,7 +307,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     const uint32_t tmem = sm.tmem_base;
 
     // ---- prologue: query rows (softmax warps; the two warps of a row load half the
-    // channels each into the Q columns of TMEM) ----
+    // channels each into the Q columns of TMEM). The stager and the unpack warps start on
+    // the first key tiles meanwhile; the QK issuer waits for Q at a named barrier. ----
     const int kh = warp / 4;                       // softmax: key half (and channel half of Q)
     const int row = 32 * (warp & 3) + lane;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
@@ -309,10 +319,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
             row_i = qidx[tile.start + row];
             row_t = pos0 + row_i;
             row_lo = (tile.mode == KVQ_MODE_LOCAL) ? max(0, row_t - w) : 0;
-            if (kh == 0) {
-                atomicMin(&sm.klo, row_lo);
-                atomicMax(&sm.khi, row_t);
-            }
+            if (kh == 0 && (row_lo < sm.klo || row_t > sm.khi)) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
         }
         const uint4 *src = reinterpret_cast<const uint4 *>(q + ((int64_t)(cu[s] + max(row_i, 0)) * H + h) * D) + kh * (D / 16);
         uint32_t words[D / 4];
@@ -339,9 +346,8 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         sm.qpart[kh][row] = part;
         tc_fence_before();
+        named_bar_sync(kQReadyBar, kSoftmaxThreads + 32);   // Q in TMEM, with the QK issuer
     }
-    __syncthreads();
-    tc_fence_after();
     const int klo = sm.klo, khi = sm.khi;
     const int n_kt = (khi >= klo) ? (khi - klo + kKeys) / kKeys : 0;
     if (warp >= kMmaWarp) {
@@ -390,6 +396,7 @@ prefill_tc_kernel(CacheView c, const __half *__restrict__ q, int w, const int32_
     if (warp == kMmaWarp) {
         // QK(t) once K(t) is unpacked and the softmax has read S(t-2); the PV MMAs come from
         // their own warp. Both wait on their barriers (suspended, no polling).
+        named_bar_sync(kQReadyBar, kSoftmaxThreads + 32);       // the query rows are in TMEM
         for (int t = 0; t < n_kt; ++t) {
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.kv_full[t % kKvBufs], (t / kKvBufs) & 1, c.status) &&
                                              (t < 2 || mbar_wait(&sm.s_free[t & 1], ((t - 2) >> 1) & 1, c.status)) &&
