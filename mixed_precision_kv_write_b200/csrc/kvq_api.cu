@@ -330,9 +330,10 @@ int kvq_cache_create_paged(kvq_cache **out, int batch, int heads, int query_grou
     wk.max_items = max_items;
     wk.qslots = std::min(query_group, kvq::kDecodeMaxQ);
     wk.items = (kvq::DecodeItem *)alloc(sizeof(kvq::DecodeItem) * (size_t)max_items);
-    wk.count = (unsigned long long *)alloc(3 * sizeof(unsigned long long));   // two count words, the cursor
-    wk.head_first = (int32_t *)alloc(sizeof(int32_t) * BH);
-    wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * BH);
+    // the front pair of count words, the cursor, the back pair
+    wk.count = (unsigned long long *)alloc(kvq::kDecodeCountWords * sizeof(unsigned long long));
+    wk.head_first = (int32_t *)alloc(sizeof(int32_t) * 2 * BH);
+    wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * 2 * BH);
     wk.partials = (float *)alloc(sizeof(float) * (size_t)max_items * wk.qslots * (head_dim + 4));
     c->pf_max_tiles = slots * query_group / 128 + 2LL * BHQ;
     c->pf_tiles = alloc(sizeof(int32_t) * 16 * (size_t)c->pf_max_tiles);    // two lists of 32-byte tiles
@@ -372,7 +373,7 @@ int kvq_cache_create_paged(kvq_cache **out, int batch, int heads, int query_grou
     e = e ? e : cudaMemsetAsync(v.bad, 0, sizeof(uint32_t) * batch, st);
     e = e ? e : cudaMemsetAsync(v.status, 0, sizeof(int32_t), st);
     e = e ? e : cudaMemsetAsync(v.meta, 0, sizeof(uint32_t) * (size_t)slots, st);
-    e = e ? e : cudaMemsetAsync(wk.count, 0, 3 * sizeof(unsigned long long), st);
+    e = e ? e : cudaMemsetAsync(wk.count, 0, kvq::kDecodeCountWords * sizeof(unsigned long long), st);
     e = e ? e : cudaMemsetAsync(c->scan_flags, 0, sizeof(uint64_t) * (size_t)BH * std::max(1, c->scan_chunks), st);
     if (paged) {
         e = e ? e : cudaMemsetAsync(v.npages, 0, sizeof(int32_t) * BH, st);

@@ -11,11 +11,15 @@
 //                         every record read: the key range is the union of the subgroup's
 //                         ranges, cut where the local window starts, so within an item
 //                         every active query reads every key. Ranges are cut into
-//                         near-equal items of at most 1152 keys. Each CTA reserves its items
-//                         with one atomicAdd on the call's (generation, count) word.
+//                         near-equal items of at most 1152 keys. Items whose range is the
+//                         local window go to the back of the list, the others to the front;
+//                         each CTA reserves its items with one atomicAdd on each of the
+//                         call's (generation, count) words of the two regions.
 //   decode_splitk_kernel  three CTAs per SM, one producer and four consumer warps each. The
-//                         producer claims items one at a time from the call's cursor (a CTA
-//                         that finishes early takes more) and walks each in stages of at
+//                         producer claims items one at a time from the call's cursor, front
+//                         items first (a CTA that finishes early takes more; the short
+//                         window items come last and even out the CTAs' end times) and
+//                         walks each in stages of at
 //                         most 128 keys and 28 KB of records: a ring of record-offset
 //                         windows is bulk-copied
 //                         ahead, each stage's keys are sorted by width into chunks of one
@@ -174,33 +178,40 @@ __device__ __forceinline__ float h2f_hi(uint32_t w) { return __half2float(__usho
 
 // ------------------------------------------------------------------ planning
 // Appends the step's tokens of sequence blockIdx.x (APPEND), then lists the decode items of
-// its (KV head, subgroup) units.
+// its (KV head, subgroup) units: an item whose key range is the local window goes to the
+// back region of the list, every other item to the front region. The split-K CTAs claim
+// the front items first, so the short window items fill the end of the launch.
 template <int D, bool APPEND>
 __global__ void __launch_bounds__(kPlanThreads)
 decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, DecodeWork wk, uint32_t gen,
                    AppendArgs ap)
 {
     __shared__ AppendShared as;
-    __shared__ int warp_tot[kPlanThreads / 32];
-    __shared__ int cnt_sh[kPlanThreads];
-    __shared__ uint32_t base_sh;
-    // per unit of the pass: first item (relative to the pass), items of regions A and B,
-    // region sizes, query masks and subgroup, KV head, length, stream end, first slot
-    __shared__ int u_start[kPlanThreads + 1], u_cA[kPlanThreads], u_nA[kPlanThreads], u_nB[kPlanThreads];
+    // counts packed as front items | back items << 32 (a pass lists fewer than 2^31 of each)
+    __shared__ long long warp_tot[kPlanThreads / 32];
+    __shared__ long long cnt_sh[kPlanThreads];
+    __shared__ uint32_t base_sh[2];
+    // per unit of the pass: first front and first back item (relative to the pass), items of
+    // regions A and B, region sizes, query masks and subgroup, KV head, length, stream end,
+    // first slot
+    __shared__ int u_startF[kPlanThreads + 1], u_startB[kPlanThreads + 1];
+    __shared__ int u_cA[kPlanThreads], u_nA[kPlanThreads], u_nB[kPlanThreads];
     __shared__ int u_cB[kPlanThreads], u_q[kPlanThreads], u_L[kPlanThreads];
     __shared__ uint32_t u_end[kPlanThreads];
     __shared__ int64_t u_sbase[kPlanThreads];
     pdl_wait();
     pdl_trigger();
-    // the previous call's kernels have completed: its count word becomes the next call's
+    // the previous call's kernels have completed: its count words become the next call's
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *wk.count_next = (unsigned long long)(gen + 1u) << 32;
+        *wk.count_back_next = (unsigned long long)(gen + 1u) << 32;
         *wk.cursor = 0u;                 // the split-K CTAs claim this call's items from 0
     }
     const int s = blockIdx.x;
     if (APPEND) append_seq<D>(c, ap.k, ap.v, ap.bits, ap.cu, ap.n_tok, ap.gen, ap.positions, s, as);
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int H = c.H, G = c.G, HQ = H * G;
+    const int BH = c.B * H;
     const int nsub = (G + kDecodeMaxQ - 1) / kDecodeMaxQ;
     const int units = H * nsub;
     const int per_pass = (kPlanThreads / nsub) * nsub;      // whole KV heads per pass
@@ -208,6 +219,7 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
         const int u = u0 + tid;
         const bool mine = tid < per_pass && u < units;
         int L = 0, lo_loc = 0, nA = 0, nB = 0, mA = 0, mB = 0, g0 = 0, hk = 0;
+        bool win = false;                            // region B is the local window
         if (mine) {
             hk = u / nsub;
             g0 = (u % nsub) * kDecodeMaxQ;
@@ -220,6 +232,7 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
                 else if (m == KVQ_MODE_FULL) full |= 1 << i;
                 else if (m == KVQ_MODE_LOCAL) local |= 1 << i;
             }
+            win = local != 0;
             if (L > 0) {
                 if (local == 0 || full == 0) {       // one region: the mode set is the same throughout
                     mB = full | local;
@@ -234,74 +247,94 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
         }
         const int cA = (nA + kDecodeItemKeys - 1) / kDecodeItemKeys;
         const int cB = (nB + kDecodeItemKeys - 1) / kDecodeItemKeys;
-        const int cnt = cA + cB;
+        const long long cnt = (long long)(cA + (win ? 0 : cB)) | ((long long)(win ? cB : 0) << 32);
         cnt_sh[tid] = cnt;
-        int incl = cnt;
+        long long incl = cnt;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, d);
+            const long long y = __shfl_up_sync(0xffffffffu, incl, d);
             if (lane >= d) incl += y;
         }
         if (lane == 31) warp_tot[wid] = incl;
         __syncthreads();
-        int wpre = 0, tot = 0;
+        long long wpre = 0, tot = 0;
 #pragma unroll
         for (int qq = 0; qq < kPlanThreads / 32; ++qq) {
-            const int t = warp_tot[qq];
+            const long long t = warp_tot[qq];
             if (qq < wid) wpre += t;
             tot += t;
         }
+        const int totF = (int)(tot & 0xFFFFFFFFll), totB = (int)(tot >> 32);
         if (tid == 0) {
-            // reserve [base, base + tot) in this call's list (one atomic, no retries)
-            const unsigned long long old = atomicAdd(wk.count, (unsigned long long)tot);
-            const uint32_t tag = (uint32_t)(old >> 32);
-            if (tag != gen && tag != 0u) {           // stale word: list nothing
+            // reserve [base, base + tot) of this call's front and back regions (one atomic
+            // each, no retries)
+            const unsigned long long oF = atomicAdd(wk.count, (unsigned long long)totF);
+            const unsigned long long oB = atomicAdd(wk.count_back, (unsigned long long)totB);
+            const uint32_t tagF = (uint32_t)(oF >> 32), tagB = (uint32_t)(oB >> 32);
+            if ((tagF != gen && tagF != 0u) || (tagB != gen && tagB != 0u)) {   // stale: list nothing
                 set_status(c.status, KVQ_ERR_DEVICE_CHECK);
-                base_sh = 0xFFFFFFFFu;
+                base_sh[0] = 0xFFFFFFFFu;
             } else {
-                base_sh = (uint32_t)old;
+                base_sh[0] = (uint32_t)oF;
+                base_sh[1] = (uint32_t)oB;
             }
-            u_start[kPlanThreads] = tot;
+            u_startF[kPlanThreads] = totF;
+            u_startB[kPlanThreads] = totB;
         }
-        const int rel = wpre + incl - cnt;            // the unit's first item within the pass
-        u_start[tid] = rel;
+        const long long rel = wpre + incl - cnt;      // the unit's first items within the pass
+        u_startF[tid] = (int)(rel & 0xFFFFFFFFll);
+        u_startB[tid] = (int)(rel >> 32);
         u_cA[tid] = cA;
         u_cB[tid] = cB;
         u_nA[tid] = nA;
         u_nB[tid] = nB;
         u_q[tid] = g0 | (mA << 8) | (mB << 12);
         u_L[tid] = L;
-        if (mine && cnt > 0) {
+        if (mine && (cA + cB) > 0) {
             u_end[tid] = (APPEND && hk < kAppendHeads) ? as.end[hk] : c.end[s * H + hk];
             u_sbase[tid] = slot_of(c, s, hk, 0);
         }
         __syncthreads();
-        const bool stale = base_sh == 0xFFFFFFFFu;
-        const int64_t base = stale ? 0 : base_sh;
+        const bool stale = base_sh[0] == 0xFFFFFFFFu;
+        const int64_t baseF = stale ? 0 : base_sh[0], baseB = stale ? 0 : base_sh[1];
+        const bool over = !stale && (baseF + totF > wk.max_items || baseB + totB > wk.max_items);
         if (mine && u % nsub == 0) {                  // the KV head's items: its subgroups' runs
-            int n_all = 0;
-            for (int k = 0; k < nsub; ++k) n_all += cnt_sh[tid + k];
-            wk.head_first[s * H + hk] = (int32_t)(base + rel);
-            wk.head_cnt[s * H + hk] = stale ? 0 : n_all;
+            int nF = 0, nBk = 0;
+            for (int k = 0; k < nsub; ++k) {
+                nF += (int)(cnt_sh[tid + k] & 0xFFFFFFFFll);
+                nBk += (int)(cnt_sh[tid + k] >> 32);
+            }
+            const int unit = s * H + hk;
+            const bool none = stale || over;
+            wk.head_first[unit] = (int32_t)(baseF + (rel & 0xFFFFFFFFll));
+            wk.head_cnt[unit] = none ? 0 : nF;
+            // back items x .. x + nBk - 1 sit at max_items - 1 - x down to max_items - x - nBk
+            wk.head_first[BH + unit] = (int32_t)(wk.max_items - (baseB + (rel >> 32) + nBk));
+            wk.head_cnt[BH + unit] = none ? 0 : nBk;
         }
         if (stale) {
-        } else if (base + tot > wk.max_items) {
+        } else if (over) {
             if (tid == 0) set_status(c.status, KVQ_ERR_DEVICE_CHECK);
         } else {
-            // every thread writes items: item i of the pass belongs to the last unit whose
-            // first item is <= i (binary search over the pass's units)
+            // every thread writes items: item i of a region's pass belongs to the last unit
+            // whose first item in that region is <= i (binary search over the pass's units)
             const int n_units = min(per_pass, units - u0);
-            for (int i = tid; i < tot; i += kPlanThreads) {
-                int lo = 0, hi = n_units;                  // u_start[lo] <= i < u_start[hi]
+            for (int t = tid; t < totF + totB; t += kPlanThreads) {
+                const bool bk = t >= totF;
+                const int i = bk ? t - totF : t;
+                const int *ust = bk ? u_startB : u_startF;
+                int lo = 0, hi = n_units;                  // ust[lo] <= i < ust[hi]
                 while (hi - lo > 1) {
                     const int mid = (lo + hi) >> 1;
-                    if (u_start[mid] <= i) lo = mid;
+                    if (ust[mid] <= i) lo = mid;
                     else hi = mid;
                 }
-                while (lo + 1 < n_units && u_start[lo + 1] <= i) ++lo;   // skip units with no items
-                const int k0 = i - u_start[lo];
-                const bool inA = k0 < u_cA[lo];
-                const int k = inA ? k0 : k0 - u_cA[lo];
+                while (lo + 1 < n_units && ust[lo + 1] <= i) ++lo;   // skip units with no items
+                const int k0 = i - ust[lo];
+                // front: region A's items, then region B's when it is not the window; back:
+                // region B's items
+                const bool inA = !bk && k0 < u_cA[lo];
+                const int k = (inA || bk) ? k0 : k0 - u_cA[lo];
                 const int n = inA ? u_nA[lo] : u_nB[lo], ci = inA ? u_cA[lo] : u_cB[lo];
                 const int Lu = u_L[lo];
                 const int first_key = inA ? 0 : Lu - u_nB[lo];
@@ -318,7 +351,7 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
                 d.sbase = u_sbase[lo];
                 d.qinfo = (qv & 0xFF) | ((inA ? (qv >> 8) & 0xF : (qv >> 12) & 0xF) << 8);
                 d.pad = 0;
-                wk.items[base + i] = d;
+                wk.items[bk ? wk.max_items - 1 - (baseB + i) : baseF + i] = d;
             }
         }
         __syncthreads();                             // the per-unit arrays are reused by the next pass
@@ -542,9 +575,21 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait();
     pdl_trigger();
-    const unsigned long long cw = *wk.count;
-    const uint32_t tag = (uint32_t)(cw >> 32);
-    const int n_items = (tag == wk.gen || tag == 0u) ? (int)min((int64_t)(uint32_t)cw, wk.max_items) : 0;
+    // claim k < n_front is front item k; the rest come from the back of the list
+    int n_front = 0, n_items = 0;
+    {
+        const unsigned long long cf = *wk.count, cb = *wk.count_back;
+        const uint32_t tagF = (uint32_t)(cf >> 32), tagB = (uint32_t)(cb >> 32);
+        if ((tagF == wk.gen || tagF == 0u) && (tagB == wk.gen || tagB == 0u)) {
+            const int64_t nf = (uint32_t)cf, nb = (uint32_t)cb;
+            if (nf + nb <= wk.max_items) {
+                n_front = (int)nf;
+                n_items = (int)(nf + nb);
+            } else if (blockIdx.x == 0 && tid == 0) {
+                set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+            }
+        }
+    }
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -574,13 +619,15 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         // producer marks a stage kStop.
         // (Claiming the next item one item ahead, to hide the claim's latency, lengthened the
         // tail more than it saved.)
-        auto claim = [&]() {
+        auto claim = [&]() {                     // the claimed item's index, or -1 (none left)
             int v = 0;
             if (lane == 0) v = (int)atomicAdd(wk.cursor, 1u);
-            return __shfl_sync(0xffffffffu, v, 0);
+            v = __shfl_sync(0xffffffffu, v, 0);
+            if (v >= n_items) return -1;
+            return v < n_front ? v : (int)(wk.max_items - 1) - (v - n_front);
         };
         int f_it = claim();
-        bool f_valid = f_it < n_items, aborted = false;
+        bool f_valid = f_it >= 0, aborted = false;
         DecodeItem f_d = wk.items[0];
         if (f_valid) f_d = wk.items[f_it];
         int f_j = f_d.j0;
@@ -616,7 +663,7 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 f_j += nwin;
                 if (f_j >= f_d.j1) {
                     f_it = claim();
-                    if (f_it < n_items) {
+                    if (f_it >= 0) {
                         f_d = wk.items[f_it];
                         f_j = f_d.j0;
                     } else {
@@ -990,14 +1037,21 @@ decode_combine_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
     const int HQ = c.H * c.G;
     const int shq = blockIdx.x, ch = threadIdx.x, lane = ch & 31, wid = ch >> 5;
     const int s = shq / HQ, hq = shq % HQ, hk = hq / c.G, gq = hq % c.G;
-    const int unit = s * c.H + hk;
-    const int first = wk.head_first[unit], cnt = wk.head_cnt[unit];
+    const int unit = s * c.H + hk, BH = c.B * c.H;
+    // the KV head's front items, then its back items (a run outside the list is ignored:
+    // the planning kernel has reported it)
+    const int firstF = wk.head_first[unit], firstB = wk.head_first[BH + unit];
+    int cntF = wk.head_cnt[unit], cntB = wk.head_cnt[BH + unit];
+    if (firstF < 0 || cntF < 0 || firstF + (int64_t)cntF > wk.max_items) cntF = 0;
+    if (firstB < 0 || cntB < 0 || firstB + (int64_t)cntB > wk.max_items) cntB = 0;
+    const int cnt = cntF + cntB;
     const int QS = wk.qslots;
-    auto part_of = [&](int i) -> int64_t {      // this query's partial of item first + i, or -1
-        const int qinfo = wk.items[first + i].qinfo;
+    auto part_of = [&](int i) -> int64_t {      // this query's partial of the head's item i, or -1
+        const int ix = (i < cntF) ? firstF + i : firstB + (i - cntF);
+        const int qinfo = wk.items[ix].qinfo;
         const int d = gq - (qinfo & 0xFF);
         if (d < 0 || d >= kDecodeMaxQ || !((qinfo >> (8 + d)) & 1)) return -1;
-        return ((int64_t)(first + i) * QS + d) * (D + 4);
+        return ((int64_t)ix * QS + d) * (D + 4);
     };
     float M = kMInit;
     for (int i = ch; i < cnt; i += D) {
@@ -1091,8 +1145,8 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const DecodeWork &wk, uint32
     return cudaGetLastError();
 }
 
-// wk.count points at the pair of count words and the item cursor (a third word); the call
-// uses count word gen & 1. `stale` is set when a launch fails (a call whose planning kernel
+// wk.count points at kDecodeCountWords words: the pair of front count words, the item
+// cursor, the pair of back count words; the call uses the words of parity gen & 1. `stale` is set when a launch fails (a call whose planning kernel
 // did not run leaves the next call's word unprepared); the words are then cleared (tag 0,
 // never used) before the next call.
 cudaError_t launch_any(const kvq_cache *cache, const DecodeWork &wk, uint32_t gen, const __half *q,
@@ -1100,7 +1154,7 @@ cudaError_t launch_any(const kvq_cache *cache, const DecodeWork &wk, uint32_t ge
                        bool &stale)
 {
     if (stale) {
-        const cudaError_t e = cudaMemsetAsync(wk.count, 0, 3 * sizeof(unsigned long long), st);
+        const cudaError_t e = cudaMemsetAsync(wk.count, 0, kDecodeCountWords * sizeof(unsigned long long), st);
         if (e != cudaSuccess) return e;
         stale = false;
     }
@@ -1108,6 +1162,8 @@ cudaError_t launch_any(const kvq_cache *cache, const DecodeWork &wk, uint32_t ge
     cw.count = wk.count + (gen & 1u);
     cw.count_next = wk.count + ((gen + 1u) & 1u);
     cw.cursor = reinterpret_cast<uint32_t *>(wk.count + 2);
+    cw.count_back = wk.count + 3 + (gen & 1u);
+    cw.count_back_next = wk.count + 3 + ((gen + 1u) & 1u);
     cw.gen = gen;
     const cudaError_t e = (cache->D == 128) ? launch_decode_t<128>(cache, cw, gen, q, modes, w, out, st, ap)
                                             : launch_decode_t<64>(cache, cw, gen, q, modes, w, out, st, ap);
@@ -1204,8 +1260,8 @@ extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache,
     const int64_t items = cache->work.max_items;
     const int qslots = cache->work.qslots;
     const size_t o_first = 256;
-    const size_t o_cnt = o_first + align256(sizeof(int32_t) * (size_t)BH);
-    const size_t o_items = o_cnt + align256(sizeof(int32_t) * (size_t)BH);
+    const size_t o_cnt = o_first + align256(sizeof(int32_t) * 2 * (size_t)BH);
+    const size_t o_items = o_cnt + align256(sizeof(int32_t) * 2 * (size_t)BH);
     const size_t o_part = o_items + align256(sizeof(DecodeItem) * (size_t)items);
     const size_t need = o_part + sizeof(float) * (size_t)items * qslots * (cache->D + 4);
     if (need > kStaticScratchBytes) {

@@ -140,6 +140,7 @@ __device__ __forceinline__ void set_status(int32_t *status, int code)
 constexpr int kDecodeItemKeys = KVQ_DECODE_ITEM_KEYS;   // keys per split-K work item, at most (w + 1 = 513 fits one)
 constexpr int kDecodeWindowKeys = 128; // keys per window of record offsets inside an item
 constexpr int kDecodeMaxQ = 4;         // query heads served by one item (a subgroup of a GQA group)
+constexpr int kDecodeCountWords = 5;   // decode count words: front pair, item cursor, back pair
 
 struct __align__(16) DecodeItem {
     int32_t sh, j0, j1;  // (sequence, KV head) = s * H + hk, and key range [j0, j1)
@@ -151,17 +152,26 @@ struct __align__(16) DecodeItem {
 
 struct DecodeWork {
     DecodeItem *items;   // [max_items]
-    // Item counts, two words used by calls of alternating generation parity: a call of
-    // generation g reserves its items with atomicAdd on `count` (g << 32 | items; a word
-    // still tagged 0 has never been used) and prepares `count_next`, the word of call g + 1,
-    // as (g + 1) << 32. A word with any other tag is stale: the call lists nothing and
-    // reports KVQ_ERR_DEVICE_CHECK.
+    // The list has two regions: items whose key range is bounded by the local window fill
+    // it from the back (back item x sits at max_items - 1 - x), all others from the front,
+    // and the split-K CTAs claim the front ones first, so the short items come last.
+    // Item counts, a front and a back word per call, each pair used by calls of alternating
+    // generation parity: a call of generation g reserves its items with atomicAdd on `count`
+    // and `count_back` (g << 32 | items; a word still tagged 0 has never been used) and
+    // prepares `count_next` and `count_back_next`, the words of call g + 1, as (g + 1) << 32.
+    // A word with any other tag is stale: the call lists nothing and reports
+    // KVQ_ERR_DEVICE_CHECK.
     unsigned long long *count;
     unsigned long long *count_next;
+    unsigned long long *count_back;
+    unsigned long long *count_back_next;
     uint32_t *cursor;    // items claimed so far by the split-K CTAs (reset by the planning kernel)
     uint32_t gen;        // the call's generation
-    int32_t *head_first; // [B*H] first item of (sequence, KV head)
-    int32_t *head_cnt;   // [B*H] its items (all subgroups)
+    // [2 * B*H]: entry s * H + hk, the first front item of (sequence, KV head) and their
+    // number (all subgroups); entry B*H + s * H + hk, the same for its back items (the run
+    // [first, first + cnt) of item indices in both cases)
+    int32_t *head_first;
+    int32_t *head_cnt;
     float *partials;     // [max_items][qslots][D + 4]: (m, l, -, -, o[D])
     int64_t max_items;
     int qslots;          // min(G, kDecodeMaxQ)

@@ -154,3 +154,28 @@ def test_decode_bitwise_repeatable_with_many_items():
     cache.check()
     for o in outs[1:]:
         assert torch.equal(o, outs[0])
+
+
+@pytest.mark.parametrize("pattern", ["local", "full", "mixed"])
+def test_decode_list_regions(pattern):
+    # window items are listed at the back of the work list and the others at the front:
+    # only-local queries leave the front empty, only-full ones the back; mixed heads and
+    # queries fill both (a head's items can sit in both regions)
+    wl = synth.scaled(W["decode_1p3b"], seqlens=(3000, 2500, 700, 1), heads=4)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    g = torch.Generator(device="cuda").manual_seed(11)
+    q = torch.randn((wl.batch, 4, 128), generator=g, device="cuda").half()
+    fill = {"local": 1, "full": 2, "mixed": 2}[pattern]
+    modes = torch.full((wl.batch, 4), fill, dtype=torch.uint8, device="cuda")
+    if pattern == "mixed":
+        modes[:, 1] = 1
+        modes[1::2, 2] = 1
+        modes[2, 3] = 0
+    out, cache = _run_decode(wl, k, v, bits, q, modes, 300)
+    again = kvq.routed_attn_decode_noalloc(q, cache, modes, 300).cpu().numpy()
+    assert np.array_equal(again, out)
+    kc, vc, bc, qc, mc = k.cpu(), v.cpu(), bits.cpu(), q.cpu(), modes.cpu()
+    for s in range(wl.batch):
+        for h in range(4):
+            ref = oracle_decode(wl, kc, vc, bc, qc, mc, 300, s, h)
+            assert_close_attn(out[s, h], ref, f"{pattern} s={s} h={h} mode={int(mc[s, h])}")
