@@ -259,7 +259,7 @@ int kvq_cache_create_paged(kvq_cache **out, int batch, int heads, int query_grou
     }
     std::vector<int32_t> cap(batch), cap_pad(batch);
     std::vector<int64_t> slot_base(batch);
-    int64_t slots = 0, max_items = 0;
+    int64_t slots = 0, max_items = 0, mid_items = 0;
     int32_t max_cap = 0;
     for (int s = 0; s < batch; ++s) {
         const int64_t cp = capacity_tokens[s];
@@ -270,7 +270,8 @@ int kvq_cache_create_paged(kvq_cache **out, int batch, int heads, int query_grou
         cap_pad[s] = (int32_t)((cp + 4) & ~int64_t(3));    // >= cp + 1, multiple of 4
         slot_base[s] = slots;
         slots += (int64_t)heads * cap_pad[s];
-        max_items += (int64_t)heads * kvq::decode_max_items(cp, query_group);
+        max_items += (int64_t)heads * (kvq::decode_max_items(cp, query_group) + kvq::decode_mid_items(query_group));
+        mid_items += (int64_t)heads * kvq::decode_mid_items(query_group);
         max_cap = std::max(max_cap, cap[s]);
     }
     if (max_items > INT32_MAX / 2) return fail(KVQ_ERR_ARG, "kvq_cache_create: too many decode items");
@@ -328,12 +329,13 @@ int kvq_cache_create_paged(kvq_cache **out, int batch, int heads, int query_grou
     v.status = (int32_t *)alloc(sizeof(int32_t));
     kvq::DecodeWork &wk = c->work;
     wk.max_items = max_items;
+    wk.mid_base = max_items - mid_items;
     wk.qslots = std::min(query_group, kvq::kDecodeMaxQ);
     wk.items = (kvq::DecodeItem *)alloc(sizeof(kvq::DecodeItem) * (size_t)max_items);
-    // the front pair of count words, the cursor, the back pair
+    // the front pair of count words, the cursor, the back pair, the middle pair
     wk.count = (unsigned long long *)alloc(kvq::kDecodeCountWords * sizeof(unsigned long long));
-    wk.head_first = (int32_t *)alloc(sizeof(int32_t) * 2 * BH);
-    wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * 2 * BH);
+    wk.head_first = (int32_t *)alloc(sizeof(int32_t) * 3 * BH);
+    wk.head_cnt = (int32_t *)alloc(sizeof(int32_t) * 3 * BH);
     wk.partials = (float *)alloc(sizeof(float) * (size_t)max_items * wk.qslots * (head_dim + 4));
     c->pf_max_tiles = slots * query_group / 128 + 2LL * BHQ;
     c->pf_tiles = alloc(sizeof(int32_t) * 16 * (size_t)c->pf_max_tiles);    // two lists of 32-byte tiles

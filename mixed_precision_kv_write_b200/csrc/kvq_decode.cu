@@ -11,17 +11,17 @@
 //                         every record read: the key range is the union of the subgroup's
 //                         ranges, cut where the local window starts, so within an item
 //                         every active query reads every key. Ranges are cut into
-//                         near-equal items of at most 1152 keys. Items whose range is the
-//                         local window go to the back of the list, the others to the front;
-//                         each CTA reserves its items with one atomicAdd on each of the
-//                         call's (generation, count) words of the two regions.
+//                         near-equal pieces of at most 1152 keys: the local window's pieces
+//                         are back items, the other range's last piece a middle item and
+//                         its other pieces, two at a time, front items. Each CTA reserves
+//                         its items with one atomicAdd on each of the call's (generation,
+//                         count) words of the three regions.
 //   decode_splitk_kernel  three CTAs per SM, one producer and four consumer warps each. The
 //                         producer claims items one at a time from the call's cursor, front
-//                         items first (a CTA that finishes early takes more; the short
-//                         window items come last and even out the CTAs' end times) and
-//                         walks each in stages of at
-//                         most 128 keys and 28 KB of records: a ring of record-offset
-//                         windows is bulk-copied
+//                         items first, then middle, then back (a CTA that finishes early
+//                         takes more; the short items come last and even out the CTAs' end
+//                         times), and walks each in stages of at most 128 keys and 28 KB of
+//                         records: a ring of record-offset windows is bulk-copied
 //                         ahead, each stage's keys are sorted by width into chunks of one
 //                         width (8 keys at head_dim 128), and the stage's contiguous record
 //                         bytes, side entries and (for a new item) queries are bulk-copied
@@ -95,6 +95,14 @@ constexpr int kMetaWords = kWin + 8;
 constexpr int kMergeRing = kStages + 1;
 constexpr int kNewItem = 1, kLastSub = 2, kStop = 4;   // stage flags (kStop: no more items)
 constexpr uint32_t kReadEndFromMeta = 0xFFFFFFFFu;
+// DecodeItem.role of a front item: kPairHead, the next list entry is the following piece of
+// the same range; kPairTail, the entry before it is its head; kSolo, neither
+constexpr int kSolo = 0, kPairHead = 1, kPairTail = 2;
+// A call whose list has at least this many items per split-K CTA walks each pair of front
+// items as one item (fewer item starts and merges); a shorter list keeps the finer items
+#ifndef KVQ_DECODE_PAIR_ITEMS_PER_CTA
+#define KVQ_DECODE_PAIR_ITEMS_PER_CTA 6
+#endif
 constexpr uint32_t kValid = 0x80000000u;
 constexpr float kLazy = 8.f;                      // running-max slack, log2 units
 constexpr float kMInit = -1e30f;                  // running max before the first key
@@ -178,25 +186,31 @@ __device__ __forceinline__ float h2f_hi(uint32_t w) { return __half2float(__usho
 
 // ------------------------------------------------------------------ planning
 // Appends the step's tokens of sequence blockIdx.x (APPEND), then lists the decode items of
-// its (KV head, subgroup) units: an item whose key range is the local window goes to the
-// back region of the list, every other item to the front region. The split-K CTAs claim
-// the front items first, so the short window items fill the end of the launch.
+// its (KV head, subgroup) units. A unit's key range outside the local window (all of it
+// when no query of the subgroup is local) is cut into c near-equal pieces of at most
+// kDecodeItemKeys keys; pieces 0 .. c - 2 are front items (consecutive in the list, marked
+// as pairs (0, 1), (2, 3), ...), piece c - 1 a middle item; the window's pieces are back
+// items. The split-K CTAs claim front, then middle, then back items, so the long items
+// start first and the short ones even out the end of the launch. Which keys an item
+// covers, and which items pair up, depend on the unit alone (not on the order in which
+// the CTAs reserve), so the results do not depend on timing.
 template <int D, bool APPEND>
 __global__ void __launch_bounds__(kPlanThreads)
 decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, DecodeWork wk, uint32_t gen,
                    AppendArgs ap)
 {
     __shared__ AppendShared as;
-    // counts packed as front items | back items << 32 (a pass lists fewer than 2^31 of each)
+    // counts packed as front items | back items << 32 (a pass lists fewer than 2^31 of
+    // each), middle items apart
     __shared__ long long warp_tot[kPlanThreads / 32];
+    __shared__ int warp_totm[kPlanThreads / 32];
     __shared__ long long cnt_sh[kPlanThreads];
-    __shared__ uint32_t base_sh[2];
-    // per unit of the pass: first front and first back item (relative to the pass), items of
-    // regions A and B, region sizes, query masks and subgroup, KV head, length, stream end,
-    // first slot
-    __shared__ int u_startF[kPlanThreads + 1], u_startB[kPlanThreads + 1];
-    __shared__ int u_cA[kPlanThreads], u_nA[kPlanThreads], u_nB[kPlanThreads];
-    __shared__ int u_cB[kPlanThreads], u_q[kPlanThreads], u_L[kPlanThreads];
+    __shared__ int cntm_sh[kPlanThreads];
+    __shared__ uint32_t base_sh[3];
+    // per unit of the pass: first front, back and middle item (relative to the pass), keys
+    // outside and inside the window, query masks and subgroup, length, stream end, first slot
+    __shared__ int u_startF[kPlanThreads + 1], u_startB[kPlanThreads + 1], u_startM[kPlanThreads + 1];
+    __shared__ int u_nF[kPlanThreads], u_nW[kPlanThreads], u_q[kPlanThreads], u_L[kPlanThreads];
     __shared__ uint32_t u_end[kPlanThreads];
     __shared__ int64_t u_sbase[kPlanThreads];
     pdl_wait();
@@ -205,6 +219,7 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *wk.count_next = (unsigned long long)(gen + 1u) << 32;
         *wk.count_back_next = (unsigned long long)(gen + 1u) << 32;
+        *wk.count_mid_next = (unsigned long long)(gen + 1u) << 32;
         *wk.cursor = 0u;                 // the split-K CTAs claim this call's items from 0
     }
     const int s = blockIdx.x;
@@ -215,16 +230,16 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
     const int nsub = (G + kDecodeMaxQ - 1) / kDecodeMaxQ;
     const int units = H * nsub;
     const int per_pass = (kPlanThreads / nsub) * nsub;      // whole KV heads per pass
+    constexpr int K = kDecodeItemKeys;
     for (int u0 = 0; u0 < units; u0 += per_pass) {
         const int u = u0 + tid;
         const bool mine = tid < per_pass && u < units;
-        int L = 0, lo_loc = 0, nA = 0, nB = 0, mA = 0, mB = 0, g0 = 0, hk = 0;
-        bool win = false;                            // region B is the local window
+        int L = 0, nF = 0, nW = 0, mF = 0, mW = 0, g0 = 0, hk = 0;
         if (mine) {
             hk = u / nsub;
             g0 = (u % nsub) * kDecodeMaxQ;
             L = (APPEND && hk < kAppendHeads) ? as.len[hk] : c.len[s * H + hk];
-            lo_loc = max(0, L - 1 - w);
+            const int lo_loc = max(0, L - 1 - w);
             int full = 0, local = 0;
             for (int i = 0; i < kDecodeMaxQ && g0 + i < G; ++i) {
                 const int m = modes[(int64_t)s * HQ + hk * G + g0 + i];
@@ -232,85 +247,106 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
                 else if (m == KVQ_MODE_FULL) full |= 1 << i;
                 else if (m == KVQ_MODE_LOCAL) local |= 1 << i;
             }
-            win = local != 0;
             if (L > 0) {
-                if (local == 0 || full == 0) {       // one region: the mode set is the same throughout
-                    mB = full | local;
-                    nB = mB ? (local ? L - lo_loc : L) : 0;
-                } else {                             // full queries alone before the window
-                    mA = full;
-                    nA = lo_loc;
-                    mB = full | local;
-                    nB = L - lo_loc;
+                if (local) {                         // window [lo_loc, L): every active query;
+                    mW = full | local;               // keys before it: the full ones alone
+                    nW = L - lo_loc;
+                    mF = full;
+                    nF = full ? lo_loc : 0;
+                } else if (full) {                   // one range [0, L)
+                    mF = full;
+                    nF = L;
                 }
             }
         }
-        const int cA = (nA + kDecodeItemKeys - 1) / kDecodeItemKeys;
-        const int cB = (nB + kDecodeItemKeys - 1) / kDecodeItemKeys;
-        const long long cnt = (long long)(cA + (win ? 0 : cB)) | ((long long)(win ? cB : 0) << 32);
+        const int pieces = (nF + K - 1) / K;
+        const int cF = max(pieces - 1, 0), cM = pieces > 0 ? 1 : 0, cB = (nW + K - 1) / K;
+        const long long cnt = (long long)cF | ((long long)cB << 32);
         cnt_sh[tid] = cnt;
+        cntm_sh[tid] = cM;
         long long incl = cnt;
+        int inclm = cM;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const long long y = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += y;
+            const int ym = __shfl_up_sync(0xffffffffu, inclm, d);
+            if (lane >= d) {
+                incl += y;
+                inclm += ym;
+            }
         }
-        if (lane == 31) warp_tot[wid] = incl;
+        if (lane == 31) {
+            warp_tot[wid] = incl;
+            warp_totm[wid] = inclm;
+        }
         __syncthreads();
         long long wpre = 0, tot = 0;
+        int wprem = 0, totM = 0;
 #pragma unroll
         for (int qq = 0; qq < kPlanThreads / 32; ++qq) {
             const long long t = warp_tot[qq];
-            if (qq < wid) wpre += t;
+            const int tm = warp_totm[qq];
+            if (qq < wid) {
+                wpre += t;
+                wprem += tm;
+            }
             tot += t;
+            totM += tm;
         }
         const int totF = (int)(tot & 0xFFFFFFFFll), totB = (int)(tot >> 32);
         if (tid == 0) {
-            // reserve [base, base + tot) of this call's front and back regions (one atomic
-            // each, no retries)
+            // reserve [base, base + tot) of this call's front, back and middle regions (one
+            // atomic each, no retries)
             const unsigned long long oF = atomicAdd(wk.count, (unsigned long long)totF);
             const unsigned long long oB = atomicAdd(wk.count_back, (unsigned long long)totB);
-            const uint32_t tagF = (uint32_t)(oF >> 32), tagB = (uint32_t)(oB >> 32);
-            if ((tagF != gen && tagF != 0u) || (tagB != gen && tagB != 0u)) {   // stale: list nothing
-                set_status(c.status, KVQ_ERR_DEVICE_CHECK);
+            const unsigned long long oM = atomicAdd(wk.count_mid, (unsigned long long)totM);
+            const uint32_t tagF = (uint32_t)(oF >> 32), tagB = (uint32_t)(oB >> 32), tagM = (uint32_t)(oM >> 32);
+            if ((tagF != gen && tagF != 0u) || (tagB != gen && tagB != 0u) || (tagM != gen && tagM != 0u)) {
+                set_status(c.status, KVQ_ERR_DEVICE_CHECK);     // stale: list nothing
                 base_sh[0] = 0xFFFFFFFFu;
             } else {
                 base_sh[0] = (uint32_t)oF;
                 base_sh[1] = (uint32_t)oB;
+                base_sh[2] = (uint32_t)oM;
             }
             u_startF[kPlanThreads] = totF;
             u_startB[kPlanThreads] = totB;
+            u_startM[kPlanThreads] = totM;
         }
         const long long rel = wpre + incl - cnt;      // the unit's first items within the pass
+        const int relM = wprem + inclm - cM;
         u_startF[tid] = (int)(rel & 0xFFFFFFFFll);
         u_startB[tid] = (int)(rel >> 32);
-        u_cA[tid] = cA;
-        u_cB[tid] = cB;
-        u_nA[tid] = nA;
-        u_nB[tid] = nB;
-        u_q[tid] = g0 | (mA << 8) | (mB << 12);
+        u_startM[tid] = relM;
+        u_nF[tid] = nF;
+        u_nW[tid] = nW;
+        u_q[tid] = g0 | (mF << 8) | (mW << 12);
         u_L[tid] = L;
-        if (mine && (cA + cB) > 0) {
+        if (mine && (pieces + cB) > 0) {
             u_end[tid] = (APPEND && hk < kAppendHeads) ? as.end[hk] : c.end[s * H + hk];
             u_sbase[tid] = slot_of(c, s, hk, 0);
         }
         __syncthreads();
         const bool stale = base_sh[0] == 0xFFFFFFFFu;
-        const int64_t baseF = stale ? 0 : base_sh[0], baseB = stale ? 0 : base_sh[1];
-        const bool over = !stale && (baseF + totF > wk.max_items || baseB + totB > wk.max_items);
+        const int64_t baseF = stale ? 0 : base_sh[0], baseB = stale ? 0 : base_sh[1], baseM = stale ? 0 : base_sh[2];
+        const bool over = !stale && (baseF + totF > wk.mid_base || baseB + totB > wk.mid_base ||
+                                     baseM + totM > wk.max_items - wk.mid_base);
         if (mine && u % nsub == 0) {                  // the KV head's items: its subgroups' runs
-            int nF = 0, nBk = 0;
+            int nFi = 0, nBi = 0, nMi = 0;
             for (int k = 0; k < nsub; ++k) {
-                nF += (int)(cnt_sh[tid + k] & 0xFFFFFFFFll);
-                nBk += (int)(cnt_sh[tid + k] >> 32);
+                nFi += (int)(cnt_sh[tid + k] & 0xFFFFFFFFll);
+                nBi += (int)(cnt_sh[tid + k] >> 32);
+                nMi += cntm_sh[tid + k];
             }
             const int unit = s * H + hk;
             const bool none = stale || over;
             wk.head_first[unit] = (int32_t)(baseF + (rel & 0xFFFFFFFFll));
-            wk.head_cnt[unit] = none ? 0 : nF;
-            // back items x .. x + nBk - 1 sit at max_items - 1 - x down to max_items - x - nBk
-            wk.head_first[BH + unit] = (int32_t)(wk.max_items - (baseB + (rel >> 32) + nBk));
-            wk.head_cnt[BH + unit] = none ? 0 : nBk;
+            wk.head_cnt[unit] = none ? 0 : nFi;
+            // back items x .. x + nBi - 1 sit at mid_base - 1 - x down to mid_base - x - nBi
+            wk.head_first[BH + unit] = (int32_t)(wk.mid_base - (baseB + (rel >> 32) + nBi));
+            wk.head_cnt[BH + unit] = none ? 0 : nBi;
+            wk.head_first[2 * BH + unit] = (int32_t)(wk.mid_base + baseM + relM);
+            wk.head_cnt[2 * BH + unit] = none ? 0 : nMi;
         }
         if (stale) {
         } else if (over) {
@@ -319,10 +355,10 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
             // every thread writes items: item i of a region's pass belongs to the last unit
             // whose first item in that region is <= i (binary search over the pass's units)
             const int n_units = min(per_pass, units - u0);
-            for (int t = tid; t < totF + totB; t += kPlanThreads) {
-                const bool bk = t >= totF;
-                const int i = bk ? t - totF : t;
-                const int *ust = bk ? u_startB : u_startF;
+            for (int t = tid; t < totF + totM + totB; t += kPlanThreads) {
+                const int reg = (t < totF) ? 0 : (t < totF + totM) ? 1 : 2;   // front, middle, back
+                const int i = (reg == 0) ? t : (reg == 1) ? t - totF : t - totF - totM;
+                const int *ust = (reg == 0) ? u_startF : (reg == 1) ? u_startM : u_startB;
                 int lo = 0, hi = n_units;                  // ust[lo] <= i < ust[hi]
                 while (hi - lo > 1) {
                     const int mid = (lo + hi) >> 1;
@@ -330,28 +366,37 @@ decode_plan_kernel(CacheView c, const uint8_t *__restrict__ modes, int w, Decode
                     else hi = mid;
                 }
                 while (lo + 1 < n_units && ust[lo + 1] <= i) ++lo;   // skip units with no items
-                const int k0 = i - ust[lo];
-                // front: region A's items, then region B's when it is not the window; back:
-                // region B's items
-                const bool inA = !bk && k0 < u_cA[lo];
-                const int k = (inA || bk) ? k0 : k0 - u_cA[lo];
-                const int n = inA ? u_nA[lo] : u_nB[lo], ci = inA ? u_cA[lo] : u_cB[lo];
-                const int Lu = u_L[lo];
-                const int first_key = inA ? 0 : Lu - u_nB[lo];
-                const int per = n / ci, rem = n % ci;     // near-equal, non-empty items
-                const int qv = u_q[lo];
-                const int uu = u0 + lo;
+                const int k = i - ust[lo];
+                const int Lu = u_L[lo], qv = u_q[lo];
+                int j0, j1, mask, role = kSolo;
+                if (reg < 2) {                             // pieces of [0, nF)
+                    const int n = u_nF[lo], pc = (n + K - 1) / K;
+                    const int per = n / pc, rem = n % pc;  // near-equal, non-empty pieces
+                    const int pa = (reg == 0) ? k : pc - 1;
+                    j0 = pa * per + min(pa, rem);
+                    j1 = (pa + 1) * per + min(pa + 1, rem);
+                    mask = (qv >> 8) & 0xF;
+                    if (reg == 0) role = (k & 1) ? kPairTail : (k + 1 <= pc - 2) ? kPairHead : kSolo;
+                } else {                                   // pieces of the window [Lu - nW, Lu)
+                    const int n = u_nW[lo], pc = (n + K - 1) / K;
+                    const int per = n / pc, rem = n % pc;
+                    j0 = Lu - n + k * per + min(k, rem);
+                    j1 = j0 + per + (k < rem ? 1 : 0);
+                    mask = (qv >> 12) & 0xF;
+                }
                 DecodeItem d;
-                d.sh = s * H + uu / nsub;
-                d.j0 = first_key + k * per + min(k, rem);
-                d.j1 = d.j0 + per + (k < rem ? 1 : 0);
+                d.sh = s * H + (u0 + lo) / nsub;
+                d.j0 = j0;
+                d.j1 = j1;
                 // the stream end for the item ending at the last token; else the producer
                 // reads the offset of key j1 itself
-                d.end_off = (d.j1 < Lu) ? kReadEndFromMeta : u_end[lo];
+                d.end_off = (j1 < Lu) ? kReadEndFromMeta : u_end[lo];
                 d.sbase = u_sbase[lo];
-                d.qinfo = (qv & 0xFF) | ((inA ? (qv >> 8) & 0xF : (qv >> 12) & 0xF) << 8);
-                d.pad = 0;
-                wk.items[bk ? wk.max_items - 1 - (baseB + i) : baseF + i] = d;
+                d.qinfo = (qv & 0xFF) | (mask << 8);
+                d.role = role;
+                const int64_t ix = (reg == 0) ? baseF + i : (reg == 1) ? wk.mid_base + baseM + i
+                                                                       : wk.mid_base - 1 - (baseB + i);
+                wk.items[ix] = d;
             }
         }
         __syncthreads();                             // the per-unit arrays are reused by the next pass
@@ -575,16 +620,18 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait();
     pdl_trigger();
-    // claim k < n_front is front item k; the rest come from the back of the list
-    int n_front = 0, n_items = 0;
+    // claims 0 .. n_front - 1 are the front items, then come the middle items, then the back
+    // items from the end of the front/back zone down
+    int n_front = 0, n_fm = 0, n_items = 0;
     {
-        const unsigned long long cf = *wk.count, cb = *wk.count_back;
-        const uint32_t tagF = (uint32_t)(cf >> 32), tagB = (uint32_t)(cb >> 32);
-        if ((tagF == wk.gen || tagF == 0u) && (tagB == wk.gen || tagB == 0u)) {
-            const int64_t nf = (uint32_t)cf, nb = (uint32_t)cb;
-            if (nf + nb <= wk.max_items) {
+        const unsigned long long cf = *wk.count, cb = *wk.count_back, cm = *wk.count_mid;
+        const uint32_t tagF = (uint32_t)(cf >> 32), tagB = (uint32_t)(cb >> 32), tagM = (uint32_t)(cm >> 32);
+        if ((tagF == wk.gen || tagF == 0u) && (tagB == wk.gen || tagB == 0u) && (tagM == wk.gen || tagM == 0u)) {
+            const int64_t nf = (uint32_t)cf, nb = (uint32_t)cb, nm = (uint32_t)cm;
+            if (nf + nb <= wk.mid_base && nm <= wk.max_items - wk.mid_base) {
                 n_front = (int)nf;
-                n_items = (int)(nf + nb);
+                n_fm = (int)(nf + nm);
+                n_items = (int)(nf + nm + nb);
             } else if (blockIdx.x == 0 && tid == 0) {
                 set_status(c.status, KVQ_ERR_DEVICE_CHECK);
             }
@@ -614,22 +661,38 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
         // slot i (ja = the window's first key rounded down to a multiple of 4); lane l holds
         // slots KPL*l .. KPL*l + KPL - 1 (16-byte shared loads). Windows after an item's first
         // end on 4-aligned keys, so a window's keys fit slots [d, d + nwin) with
-        // d + nwin <= kWin. Items are claimed one at a time from the call's cursor when the
-        // filler reaches them (CTAs that finish early take more); after the last one the
-        // producer marks a stage kStop.
+        // d + nwin <= kWin. Items are claimed when the filler reaches them (CTAs that finish
+        // early take more); after the last one the producer marks a stage kStop.
         // (Claiming the next item one item ahead, to hide the claim's latency, lengthened the
         // tail more than it saved.)
-        auto claim = [&]() {                     // the claimed item's index, or -1 (none left)
-            int v = 0;
-            if (lane == 0) v = (int)atomicAdd(wk.cursor, 1u);
-            v = __shfl_sync(0xffffffffu, v, 0);
-            if (v >= n_items) return -1;
-            return v < n_front ? v : (int)(wk.max_items - 1) - (v - n_front);
+        // With a long list (a decision from the item count alone, the same in every CTA) a
+        // pair head's claimer walks both pieces as one item and marks the tail's partials
+        // empty (l = 0) for the combine; a claimed tail is then skipped.
+        const bool pairs = n_items >= KVQ_DECODE_PAIR_ITEMS_PER_CTA * (int)gridDim.x;
+        auto claim = [&](DecodeItem &d) {        // the next item's index (d: its range), or -1
+            for (;;) {
+                int v = 0;
+                if (lane == 0) v = (int)atomicAdd(wk.cursor, 1u);
+                v = __shfl_sync(0xffffffffu, v, 0);
+                if (v >= n_items) return -1;
+                const int it = v < n_front ? v
+                             : v < n_fm    ? (int)wk.mid_base + (v - n_front)
+                                           : (int)wk.mid_base - 1 - (v - n_fm);
+                d = wk.items[it];
+                if (!pairs || v >= n_front || d.role == kSolo) return it;
+                if (d.role == kPairTail) continue;
+                const DecodeItem d2 = wk.items[it + 1];     // the head's tail (a front item)
+                d.j1 = d2.j1;
+                d.end_off = d2.end_off;
+                const int slot_q = lane;                  // lanes 0..3: the query slots
+                if (slot_q < wk.qslots && ((d2.qinfo >> (8 + slot_q)) & 1))
+                    wk.partials[((int64_t)(it + 1) * wk.qslots + slot_q) * (D + 4) + 1] = 0.f;
+                return it;
+            }
         };
-        int f_it = claim();
-        bool f_valid = f_it >= 0, aborted = false;
         DecodeItem f_d = wk.items[0];
-        if (f_valid) f_d = wk.items[f_it];
+        int f_it = claim(f_d);
+        bool f_valid = f_it >= 0, aborted = false;
         int f_j = f_d.j0;
         int filled = 0, consumed = 0, issued = 0;
         auto pick = [](const uint32_t (&a)[KPL], int i) {       // a[i], i warp-uniform
@@ -662,9 +725,8 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
                 ++filled;
                 f_j += nwin;
                 if (f_j >= f_d.j1) {
-                    f_it = claim();
+                    f_it = claim(f_d);
                     if (f_it >= 0) {
-                        f_d = wk.items[f_it];
                         f_j = f_d.j0;
                     } else {
                         f_valid = false;
@@ -1038,25 +1100,35 @@ decode_combine_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
     const int shq = blockIdx.x, ch = threadIdx.x, lane = ch & 31, wid = ch >> 5;
     const int s = shq / HQ, hq = shq % HQ, hk = hq / c.G, gq = hq % c.G;
     const int unit = s * c.H + hk, BH = c.B * c.H;
-    // the KV head's front items, then its back items (a run outside the list is ignored:
-    // the planning kernel has reported it)
-    const int firstF = wk.head_first[unit], firstB = wk.head_first[BH + unit];
-    int cntF = wk.head_cnt[unit], cntB = wk.head_cnt[BH + unit];
-    if (firstF < 0 || cntF < 0 || firstF + (int64_t)cntF > wk.max_items) cntF = 0;
-    if (firstB < 0 || cntB < 0 || firstB + (int64_t)cntB > wk.max_items) cntB = 0;
-    const int cnt = cntF + cntB;
+    // the KV head's front, back and middle items (a run outside the list is ignored: the
+    // planning kernel has reported it)
+    int first[3], run[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+        first[r] = wk.head_first[r * BH + unit];
+        run[r] = wk.head_cnt[r * BH + unit];
+        if (first[r] < 0 || run[r] < 0 || first[r] + (int64_t)run[r] > wk.max_items) run[r] = 0;
+    }
+    const int cnt = run[0] + run[1] + run[2];
     const int QS = wk.qslots;
     auto part_of = [&](int i) -> int64_t {      // this query's partial of the head's item i, or -1
-        const int ix = (i < cntF) ? firstF + i : firstB + (i - cntF);
+        const int ix = (i < run[0]) ? first[0] + i
+                     : (i < run[0] + run[1]) ? first[1] + (i - run[0]) : first[2] + (i - run[0] - run[1]);
         const int qinfo = wk.items[ix].qinfo;
         const int d = gq - (qinfo & 0xFF);
         if (d < 0 || d >= kDecodeMaxQ || !((qinfo >> (8 + d)) & 1)) return -1;
         return ((int64_t)ix * QS + d) * (D + 4);
     };
+    // (m, l) of a partial; l = 0 marks a pair tail that the split-K kernel walked with its
+    // head (a walked item has l >= 1): it takes no part
+    auto ml_of = [&](int64_t p) { return *reinterpret_cast<const float2 *>(wk.partials + p); };
     float M = kMInit;
     for (int i = ch; i < cnt; i += D) {
         const int64_t p = part_of(i);
-        if (p >= 0) M = fmaxf(M, wk.partials[p]);
+        if (p >= 0) {
+            const float2 ml = ml_of(p);
+            if (ml.y > 0.f) M = fmaxf(M, ml.x);
+        }
     }
 #pragma unroll
     for (int dd = 16; dd >= 1; dd >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, dd));
@@ -1071,11 +1143,16 @@ decode_combine_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
     for (int i0 = 0; i0 < cnt; i0 += kCombineChunk) {
         const int n = min(cnt - i0, kCombineChunk);
         for (int k = ch; k < n; k += D) {
-            const int64_t p = part_of(i0 + k);
+            int64_t p = part_of(i0 + k);
             float f = 0.f;
             if (p >= 0) {
-                f = ex2(wk.partials[p] - M);
-                L = fmaf(wk.partials[p + 1], f, L);
+                const float2 ml = ml_of(p);
+                if (ml.y > 0.f) {
+                    f = ex2(ml.x - M);
+                    L = fmaf(ml.y, f, L);
+                } else {
+                    p = -1;
+                }
             }
             f_sh[k] = f;
             idx_sh[k] = (p >= 0) ? (int32_t)(p / (D + 4)) : -1;
@@ -1146,7 +1223,8 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const DecodeWork &wk, uint32
 }
 
 // wk.count points at kDecodeCountWords words: the pair of front count words, the item
-// cursor, the pair of back count words; the call uses the words of parity gen & 1. `stale` is set when a launch fails (a call whose planning kernel
+// cursor, the pair of back count words, the pair of middle count words; the call uses the
+// words of parity gen & 1. `stale` is set when a launch fails (a call whose planning kernel
 // did not run leaves the next call's word unprepared); the words are then cleared (tag 0,
 // never used) before the next call.
 cudaError_t launch_any(const kvq_cache *cache, const DecodeWork &wk, uint32_t gen, const __half *q,
@@ -1164,6 +1242,8 @@ cudaError_t launch_any(const kvq_cache *cache, const DecodeWork &wk, uint32_t ge
     cw.cursor = reinterpret_cast<uint32_t *>(wk.count + 2);
     cw.count_back = wk.count + 3 + (gen & 1u);
     cw.count_back_next = wk.count + 3 + ((gen + 1u) & 1u);
+    cw.count_mid = wk.count + 5 + (gen & 1u);
+    cw.count_mid_next = wk.count + 5 + ((gen + 1u) & 1u);
     cw.gen = gen;
     const cudaError_t e = (cache->D == 128) ? launch_decode_t<128>(cache, cw, gen, q, modes, w, out, st, ap)
                                             : launch_decode_t<64>(cache, cw, gen, q, modes, w, out, st, ap);
@@ -1260,8 +1340,8 @@ extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache,
     const int64_t items = cache->work.max_items;
     const int qslots = cache->work.qslots;
     const size_t o_first = 256;
-    const size_t o_cnt = o_first + align256(sizeof(int32_t) * 2 * (size_t)BH);
-    const size_t o_items = o_cnt + align256(sizeof(int32_t) * 2 * (size_t)BH);
+    const size_t o_cnt = o_first + align256(sizeof(int32_t) * 3 * (size_t)BH);
+    const size_t o_items = o_cnt + align256(sizeof(int32_t) * 3 * (size_t)BH);
     const size_t o_part = o_items + align256(sizeof(DecodeItem) * (size_t)items);
     const size_t need = o_part + sizeof(float) * (size_t)items * qslots * (cache->D + 4);
     if (need > kStaticScratchBytes) {
@@ -1282,6 +1362,7 @@ extern "C" int routed_attn_decode_noalloc(const void *q, const kvq_cache *cache,
     wk.items = reinterpret_cast<DecodeItem *>(base + o_items);
     wk.partials = reinterpret_cast<float *>(base + o_part);
     wk.max_items = items;
+    wk.mid_base = cache->work.mid_base;
     wk.qslots = qslots;
     // a generation id no earlier call on the shared array used (never 0, the tag of a word
     // never used: the array starts zeroed)

@@ -140,50 +140,57 @@ __device__ __forceinline__ void set_status(int32_t *status, int code)
 constexpr int kDecodeItemKeys = KVQ_DECODE_ITEM_KEYS;   // keys per split-K work item, at most (w + 1 = 513 fits one)
 constexpr int kDecodeWindowKeys = 128; // keys per window of record offsets inside an item
 constexpr int kDecodeMaxQ = 4;         // query heads served by one item (a subgroup of a GQA group)
-constexpr int kDecodeCountWords = 5;   // decode count words: front pair, item cursor, back pair
+constexpr int kDecodeCountWords = 7;   // decode count words: front pair, item cursor, back pair, middle pair
 
 struct __align__(16) DecodeItem {
     int32_t sh, j0, j1;  // (sequence, KV head) = s * H + hk, and key range [j0, j1)
     uint32_t end_off;    // byte offset of key j1 in the stream (the stream end if j1 = len)
     int64_t sbase;       // slot of key 0 of (sequence, KV head)
     int32_t qinfo;       // first query g0 of the subgroup | active-query mask << 8 (bit i: g0 + i)
-    int32_t pad;
+    int32_t role;        // front items: pair role (kSolo, kPairHead, kPairTail); 0 otherwise
 };
 
 struct DecodeWork {
     DecodeItem *items;   // [max_items]
-    // The list has two regions: items whose key range is bounded by the local window fill
-    // it from the back (back item x sits at max_items - 1 - x), all others from the front,
-    // and the split-K CTAs claim the front ones first, so the short items come last.
-    // Item counts, a front and a back word per call, each pair used by calls of alternating
-    // generation parity: a call of generation g reserves its items with atomicAdd on `count`
-    // and `count_back` (g << 32 | items; a word still tagged 0 has never been used) and
-    // prepares `count_next` and `count_back_next`, the words of call g + 1, as (g + 1) << 32.
-    // A word with any other tag is stale: the call lists nothing and reports
-    // KVQ_ERR_DEVICE_CHECK.
+    // The list has three regions. [0, mid_base) holds the front items, filled from the
+    // start, and the back items (the local window's keys), filled from the end (back item x
+    // sits at mid_base - 1 - x); [mid_base, max_items) holds the middle items (the last
+    // piece of each range outside the window). The split-K CTAs claim front, middle, then
+    // back items, so the long items come first and the short ones last.
+    // Item counts, a pair of words per region, used by calls of alternating generation
+    // parity: a call of generation g reserves its items with atomicAdd on `count`,
+    // `count_back` and `count_mid` (g << 32 | items; a word still tagged 0 has never been
+    // used) and prepares the `_next` words, those of call g + 1, as (g + 1) << 32. A word
+    // with any other tag is stale: the call lists nothing and reports KVQ_ERR_DEVICE_CHECK.
     unsigned long long *count;
     unsigned long long *count_next;
     unsigned long long *count_back;
     unsigned long long *count_back_next;
+    unsigned long long *count_mid;
+    unsigned long long *count_mid_next;
     uint32_t *cursor;    // items claimed so far by the split-K CTAs (reset by the planning kernel)
     uint32_t gen;        // the call's generation
-    // [2 * B*H]: entry s * H + hk, the first front item of (sequence, KV head) and their
-    // number (all subgroups); entry B*H + s * H + hk, the same for its back items (the run
-    // [first, first + cnt) of item indices in both cases)
+    // [3 * B*H]: entry r * B*H + s * H + hk, the first item of (sequence, KV head) in region
+    // r (0 front, 1 back, 2 middle) and their number (all subgroups): the run
+    // [first, first + cnt) of item indices
     int32_t *head_first;
     int32_t *head_cnt;
     float *partials;     // [max_items][qslots][D + 4]: (m, l, -, -, o[D])
     int64_t max_items;
+    int64_t mid_base;    // first index of the middle region
     int qslots;          // min(G, kDecodeMaxQ)
 };
 
-// Upper bound of the items a decode call lists for a cache: per (sequence, KV head) and
-// subgroup of at most kDecodeMaxQ query heads, ceil(cap / kDecodeItemKeys) + 1 (the key
-// range may be cut once where the local window starts).
+// Upper bound of the front and back items a decode call lists for a cache: per (sequence,
+// KV head) and subgroup of at most kDecodeMaxQ query heads, ceil(cap / kDecodeItemKeys) + 1
+// (the key range may be cut once where the local window starts).
 inline int64_t decode_max_items(int64_t cap, int G)
 {
     return (int64_t)((G + kDecodeMaxQ - 1) / kDecodeMaxQ) * ((cap + kDecodeItemKeys - 1) / kDecodeItemKeys + 1);
 }
+
+// Middle items per (sequence, KV head): at most one per subgroup.
+inline int64_t decode_mid_items(int G) { return (G + kDecodeMaxQ - 1) / kDecodeMaxQ; }
 
 // ---- PTX helpers -----------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p)

@@ -138,9 +138,10 @@ def test_decode_full_size_sampled(name, n_check, n_rec):
 
 
 def test_decode_bitwise_repeatable_with_many_items():
-    # more work items than split-K CTAs: which CTA takes which item varies from call to call
-    # (items are claimed dynamically), the outputs must not
-    wl = synth.scaled(W["decode_1p3b"], seqlens=(4096,) * 32, heads=4)
+    # several times more work items than split-K CTAs: which CTA takes which item, and
+    # where in the list a sequence's items land, vary from call to call (items are reserved
+    # and claimed dynamically), the outputs must not
+    wl = synth.scaled(W["decode_1p3b"], seqlens=(4096,) * 64, heads=8)
     k, v, bits = synth.kv_tokens(wl, "cuda")
     cache = kvq.KVQCache(wl.batch, wl.heads, wl.head_dim, list(wl.seqlens))
     kvq.kvq_write(k, v, bits, synth.cu_seqlens(wl.seqlens, "cuda"), cache)
@@ -158,9 +159,10 @@ def test_decode_bitwise_repeatable_with_many_items():
 
 @pytest.mark.parametrize("pattern", ["local", "full", "mixed"])
 def test_decode_list_regions(pattern):
-    # window items are listed at the back of the work list and the others at the front:
-    # only-local queries leave the front empty, only-full ones the back; mixed heads and
-    # queries fill both (a head's items can sit in both regions)
+    # window pieces are listed at the back of the work list, the last piece of each other
+    # range in the middle and its other pieces, two at a time, at the front: only-local
+    # queries leave the front and middle empty, only-full ones the back; mixed heads and
+    # queries fill all three (a head's items can sit in every region)
     wl = synth.scaled(W["decode_1p3b"], seqlens=(3000, 2500, 700, 1), heads=4)
     k, v, bits = synth.kv_tokens(wl, "cuda")
     g = torch.Generator(device="cuda").manual_seed(11)
