@@ -138,10 +138,11 @@ def test_decode_full_size_sampled(name, n_check, n_rec):
 
 
 def test_decode_bitwise_repeatable_with_many_items():
-    # several times more work items than split-K CTAs: which CTA takes which item, and
-    # where in the list a sequence's items land, vary from call to call (items are reserved
-    # and claimed dynamically), the outputs must not
-    wl = synth.scaled(W["decode_1p3b"], seqlens=(4096,) * 64, heads=8)
+    # several times more work items than split-K CTAs (about 4,000, enough for front items
+    # to be walked in pairs): which CTA takes which item, and where in the list a
+    # sequence's items land, vary from call to call (items are reserved and claimed
+    # dynamically), the outputs must not
+    wl = synth.scaled(W["decode_1p3b"], seqlens=(4096,) * 64, heads=16)
     k, v, bits = synth.kv_tokens(wl, "cuda")
     cache = kvq.KVQCache(wl.batch, wl.heads, wl.head_dim, list(wl.seqlens))
     kvq.kvq_write(k, v, bits, synth.cu_seqlens(wl.seqlens, "cuda"), cache)
