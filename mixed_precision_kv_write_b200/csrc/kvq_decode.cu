@@ -34,7 +34,9 @@
 //                         the last warp to do so merges them into a partial per (item,
 //                         query), while the others go on with the next item.
 //   decode_combine_kernel log-sum-exp merge of the partials of each (sequence, query head),
-//                         one thread per channel; zeros for skip heads and empty sequences.
+//                         one thread per channel (decode_combine_warp_kernel, a warp per
+//                         output, when there are at least 4 outputs per SM); zeros for skip
+//                         heads and empty sequences.
 //
 // Arithmetic. With codes c, scale s and zero z (Eq. 4):
 //   q . deq(k_j) = s_j * (q . c_j) + z_j * sum(q)         (one dot product on integer codes)
@@ -1080,7 +1082,133 @@ decode_splitk_kernel(CacheView c, const __half *__restrict__ q, DecodeWork wk)
     }
 }
 
-// One CTA of D threads per (sequence, query head). The query's partials are those of its
+// Calls with many (sequence, query head) outputs: one warp per output, kCombineWarps warps
+// per CTA, D/32 channels per lane. The query's partials are those of its KV head's items whose subgroup holds it as an
+// active query. The lanes share the per-item work (the maximum, then each item's weight
+// 2^(m_i - M) and the sum of the l_i weights, 32 items a round); then every lane sums the
+// weighted o_i of its channels over the round's items, in item order, with independent
+// loads. No block barrier.
+constexpr int kCombineWarps = 4;
+constexpr int kCombineThreads = 32 * kCombineWarps;
+constexpr int kCombineWarpMinPerSm = 4;      // outputs per SM from which the warp form is used
+
+template <int D>
+__global__ void __launch_bounds__(kCombineThreads)
+decode_combine_warp_kernel(CacheView c, DecodeWork wk, float *__restrict__ out)
+{
+    constexpr int CPL = D / 32;                   // channels per lane
+    static_assert(CPL == 2 || CPL == 4, "head_dim 64 or 128");
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int HQ = c.H * c.G;
+    const int shq = blockIdx.x * kCombineWarps + (int)(threadIdx.x >> 5);
+    if (shq >= c.B * HQ) return;                  // warp-uniform
+    const int s = shq / HQ, hq = shq % HQ, hk = hq / c.G, gq = hq % c.G;
+    const int unit = s * c.H + hk, BH = c.B * c.H;
+    // the KV head's front, back and middle items (a run outside the list is ignored: the
+    // planning kernel has reported it)
+    int first[3], run[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+        first[r] = wk.head_first[r * BH + unit];
+        run[r] = wk.head_cnt[r * BH + unit];
+        if (first[r] < 0 || run[r] < 0 || first[r] + (int64_t)run[r] > wk.max_items) run[r] = 0;
+    }
+    const int cnt = run[0] + run[1] + run[2];
+    const int QS = wk.qslots;
+    auto part_of = [&](int i) -> int64_t {      // this query's partial of the head's item i, or -1
+        const int ix = (i < run[0]) ? first[0] + i
+                     : (i < run[0] + run[1]) ? first[1] + (i - run[0]) : first[2] + (i - run[0] - run[1]);
+        const int qinfo = wk.items[ix].qinfo;
+        const int d = gq - (qinfo & 0xFF);
+        if (d < 0 || d >= kDecodeMaxQ || !((qinfo >> (8 + d)) & 1)) return -1;
+        return ((int64_t)ix * QS + d) * (D + 4);
+    };
+    // (m, l) of a partial; l = 0 marks a pair tail that the split-K kernel walked with its
+    // head (a walked item has l >= 1): it takes no part
+    auto ml_of = [&](int64_t p) { return *reinterpret_cast<const float2 *>(wk.partials + p); };
+    auto o_of = [&](int64_t p, float (&v)[CPL]) {  // this lane's channels of o
+        const float *src = wk.partials + p + 4 + CPL * lane;
+        if constexpr (CPL == 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(src);
+            v[0] = x.x;
+            v[1] = x.y;
+            v[2] = x.z;
+            v[3] = x.w;
+        } else {
+            const float2 x = *reinterpret_cast<const float2 *>(src);
+            v[0] = x.x;
+            v[1] = x.y;
+        }
+    };
+    float M = kMInit;
+    for (int i = lane; i < cnt; i += 32) {
+        const int64_t p = part_of(i);
+        if (p >= 0) {
+            const float2 ml = ml_of(p);
+            if (ml.y > 0.f) M = fmaxf(M, ml.x);
+        }
+    }
+#pragma unroll
+    for (int dd = 16; dd >= 1; dd >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, dd));
+    // (the summation order is fixed: results do not depend on thread timing)
+    float L = 0.f, acc[CPL];
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) acc[k] = 0.f;
+    for (int i0 = 0; i0 < cnt; i0 += 32) {
+        float f = 0.f;
+        int64_t pi = -1;
+        if (i0 + lane < cnt) {
+            const int64_t p = part_of(i0 + lane);
+            if (p >= 0) {
+                const float2 ml = ml_of(p);
+                if (ml.y > 0.f) {
+                    f = ex2(ml.x - M);
+                    L = fmaf(ml.y, f, L);
+                    pi = p;
+                }
+            }
+        }
+        const int n = min(32, cnt - i0);
+        int k = 0;
+        for (; k + 8 <= n; k += 8) {               // 8 independent loads per round
+            float v[8][CPL], fk[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t pu = __shfl_sync(0xffffffffu, pi, k + u);
+                fk[u] = __shfl_sync(0xffffffffu, f, k + u);
+                if (pu >= 0) o_of(pu, v[u]);
+                else {
+#pragma unroll
+                    for (int q = 0; q < CPL; ++q) v[u][q] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                for (int q = 0; q < CPL; ++q) acc[q] = fmaf(v[u][q], fk[u], acc[q]);
+        }
+        for (; k < n; ++k) {
+            const int64_t pu = __shfl_sync(0xffffffffu, pi, k);
+            const float fu = __shfl_sync(0xffffffffu, f, k);
+            if (pu >= 0) {
+                float v[CPL];
+                o_of(pu, v);
+#pragma unroll
+                for (int q = 0; q < CPL; ++q) acc[q] = fmaf(v[q], fu, acc[q]);
+            }
+        }
+    }
+#pragma unroll
+    for (int dd = 16; dd >= 1; dd >>= 1) L += __shfl_xor_sync(0xffffffffu, L, dd);
+    float *dst = out + (int64_t)shq * D + CPL * lane;
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) dst[q] = (L > 0.f) ? acc[q] / L : 0.f;
+}
+
+// Calls with few outputs (long contexts over few heads, many items per output): one CTA of D
+// threads per (sequence, query head). The query's partials are those of its
 // KV head's items whose subgroup holds it as an active query. The threads first share the
 // per-item work (the maximum, then each item's weight 2^(m_i - M) and the sum of l_i
 // weights, kept in shared memory for a chunk of items), then thread = channel sums the
@@ -1217,7 +1345,15 @@ cudaError_t launch_decode_t(const kvq_cache *cache, const DecodeWork &wk, uint32
     e = launch_pdl(decode_splitk_kernel<D>, dim3(grid), dim3(kThreads), smem, st, c, q, wk);
     if (e != cudaSuccess) return e;
     profile_after(st);
-    e = launch_pdl(decode_combine_kernel<D>, dim3(c.B * c.H * c.G), dim3(D), 0, st, c, wk, out);
+    // a warp per output once there are enough outputs to fill the GPU with warps (measured:
+    // decode_1p3b's 1024 outputs 0.9 us faster per step; decode_long's 128 outputs of about
+    // 60 items each 4 us slower than with a CTA per output)
+    const int n_out = c.B * c.H * c.G;
+    if (n_out >= kCombineWarpMinPerSm * num_sms())
+        e = launch_pdl(decode_combine_warp_kernel<D>, dim3((n_out + kCombineWarps - 1) / kCombineWarps),
+                       dim3(kCombineThreads), 0, st, c, wk, out);
+    else
+        e = launch_pdl(decode_combine_kernel<D>, dim3(n_out), dim3(D), 0, st, c, wk, out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -182,3 +182,22 @@ def test_decode_list_regions(pattern):
         for h in range(4):
             ref = oracle_decode(wl, kc, vc, bc, qc, mc, 300, s, h)
             assert_close_attn(out[s, h], ref, f"{pattern} s={s} h={h} mode={int(mc[s, h])}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_many_outputs(D):
+    # at least 4 (sequence, query head) outputs per SM: the combine runs one warp per output
+    # (fewer outputs take a CTA each, as in the small cases above)
+    base = W["decode_1p3b"] if D == 128 else W["prefill_160m"]
+    heads = 12
+    wl = synth.scaled(base, seqlens=tuple(40 + 37 * i for i in range(64)), heads=heads)
+    k, v, bits = synth.kv_tokens(wl, "cuda")
+    g = torch.Generator(device="cuda").manual_seed(17 + D)
+    q = torch.randn((wl.batch, heads, D), generator=g, device="cuda").half()
+    modes = torch.randint(0, 3, (wl.batch, heads), generator=g, device="cuda").to(torch.uint8)
+    out, _ = _run_decode(wl, k, v, bits, q, modes, 50)
+    kc, vc, bc, qc, mc = k.cpu(), v.cpu(), bits.cpu(), q.cpu(), modes.cpu()
+    for s in range(0, wl.batch, 7):
+        for h in range(0, heads, 5):
+            ref = oracle_decode(wl, kc, vc, bc, qc, mc, 50, s, h)
+            assert_close_attn(out[s, h], ref, f"D={D} s={s} h={h} mode={int(mc[s, h])}")
