@@ -543,7 +543,8 @@ def run_ours(args):
     if not args.no_prefill:
         extra["prefill"] = prefill_measure("ragged_prefill", dev, pk, pk_kind, route=True,
                                            profiles=("prefill_tc_ragged_prefill.md", "write_quant_ragged_prefill.md"))
-        extra["prefill_160m"] = prefill_measure("prefill_160m", dev, pk, pk_kind)
+        extra["prefill_160m"] = prefill_measure("prefill_160m", dev, pk, pk_kind,
+                                                profiles=("prefill_tc_prefill_160m.md", "write_quant_prefill_160m.md"))
         extra["decode_long"] = decode_workload_measure("decode_long", dev, pk, pk_kind)
         gq = decode_workload_measure("decode_1p3b", dev, pk, pk_kind, group=4)
         gq["workload"] = ("decode_1p3b with grouped-query attention: 16 query heads in groups of 4 over "
